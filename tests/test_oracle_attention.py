@@ -1,0 +1,158 @@
+"""Pins of the oracle's quantised attention.
+
+* With the e4m3 rounding of P switched off, the tiled online softmax (the
+  QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV sequence of "Sage2
+  SM89 Temporal Pair Experiment", Candidate) must equal plain fp64 softmax
+  over the dequantised operands, for many tiles, ragged tails, causal masks
+  and GQA.
+* With one key tile the running max is the row max, so P8 has a closed form;
+  it is checked with torch's own float8 conversion.
+* Special cases: L = 1 (softmax = 1), identical keys (mean of V rows), rows
+  with no visible key.
+* The whole method stays within the accuracy gate against unquantised fp64
+  attention (cosine >= 0.998) on the small workloads, and a planted mistake
+  (dropping K smoothing) is caught by that gate on an outlier workload.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+
+def _bits(t):
+    return workloads.bits_u16(t)
+
+
+def _dequant_reference(oracle_mod, qk, v8t, vs, Lq, Lk, blk_q, blk_k, scale, causal, D, H, Hk):
+    """fp64 softmax(Sq Sk^T * scale / D) (V8 * vs) from the quantised operands."""
+    B = qk["q8"].shape[0]
+    out = np.zeros((B, H, Lq, D))
+    for b in range(B):
+        for h in range(H):
+            hk = h // (H // Hk)
+            qd = qk["q8"][b, h, :Lq].astype(np.float64) * np.repeat(qk["qs"][b, h], blk_q)[:Lq, None]
+            kd = qk["k8"][b, hk, :Lk].astype(np.float64) * np.repeat(qk["ks"][b, hk], blk_k)[:Lk, None]
+            vd = oracle_mod.e4m3_decode(v8t[b, hk, :, :Lk]).T * vs[b, hk][None, :].astype(np.float64)
+            s = (qd @ kd.T) * (scale / D)
+            if causal:
+                i = np.arange(Lq)[:, None]
+                j = np.arange(Lk)[None, :]
+                s = np.where(j <= i + (Lk - Lq), s, -np.inf)
+            mx = s.max(axis=1, keepdims=True)
+            ok = np.isfinite(mx)
+            e = np.where(ok, np.exp(s - np.where(ok, mx, 0)), 0.0)
+            den = e.sum(axis=1, keepdims=True)
+            out[b, h] = np.where(den > 0, (e @ vd) / np.where(den > 0, den, 1), 0.0)
+    return out
+
+
+@pytest.mark.parametrize("Lq,Lk,causal,H,Hk,D,blk_q,blk_k", [
+    (256, 256, False, 2, 2, 64, 64, 64),
+    (300, 555, False, 2, 1, 64, 128, 64),
+    (383, 383, True, 2, 2, 128, 128, 64),
+    (129, 400, True, 4, 2, 64, 64, 128),
+    (500, 130, True, 1, 1, 64, 64, 64),      # Lq > Lk: leading rows see no key
+])
+def test_online_softmax_equals_exact_without_p_rounding(oracle_mod, Lq, Lk, causal, H, Hk, D,
+                                                         blk_q, blk_k):
+    g = torch.Generator().manual_seed(Lq * 7 + Lk)
+    q = (torch.randn((1, H, Lq, D), generator=g) * 2).to(torch.bfloat16)
+    k = (torch.randn((1, Hk, Lk, D), generator=g) * 2 + 1).to(torch.bfloat16)
+    v = torch.randn((1, Hk, Lk, D), generator=g).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(D)
+    qk = oracle_mod.quant_qk(_bits(q), _bits(k), blk_q, blk_k)
+    v8t, vs = oracle_mod.quant_v(_bits(v))
+    _, got = oracle_mod.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, Lq, Lk, blk_q, blk_k,
+                             scale, causal, quantize_p=False, want_f64=True)
+    ref = _dequant_reference(oracle_mod, qk, v8t, vs, Lq, Lk, blk_q, blk_k, scale, causal, D, H, Hk)
+    assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    if causal and Lq > Lk:
+        assert (got[:, :, :Lq - Lk] == 0).all()
+
+
+def test_single_tile_p8_closed_form(oracle_mod):
+    """Lk <= 128: P8 = e4m3(448 * exp(x - rowmax)), d = sum exp(x - rowmax)."""
+    Lq, Lk, D, H = 64, 100, 64, 2
+    g = torch.Generator().manual_seed(99)
+    q = torch.randn((1, H, Lq, D), generator=g).to(torch.bfloat16)
+    k = (torch.randn((1, H, Lk, D), generator=g) + 2).to(torch.bfloat16)
+    v = torch.randn((1, H, Lk, D), generator=g).to(torch.bfloat16)
+    scale = 0.125
+    qk = oracle_mod.quant_qk(_bits(q), _bits(k), 64, 64)
+    v8t, vs = oracle_mod.quant_v(_bits(v))
+    _, got = oracle_mod.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, Lq, Lk, 64, 64,
+                             scale, False, want_f64=True)
+    for h in range(H):
+        acc = qk["q8"][0, h, :Lq].astype(np.int64) @ qk["k8"][0, h, :Lk].astype(np.int64).T
+        x = acc * qk["qs"][0, h, 0].astype(np.float64) * np.repeat(qk["ks"][0, h], 64)[None, :Lk] \
+            * (scale / D)
+        p = np.exp(x - x.max(axis=1, keepdims=True))
+        p8 = torch.from_numpy(p * 448.0).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        vdec = oracle_mod.e4m3_decode(v8t[0, h, :, :Lk]).T
+        ref = (p8 @ vdec) * vs[0, h][None, :] / (448.0 * p.sum(axis=1, keepdims=True))
+        assert np.abs(got[0, h] - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_length_one_returns_dequantised_v(oracle_mod):
+    D = 64
+    g = torch.Generator().manual_seed(1)
+    q = torch.randn((1, 1, 1, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((1, 1, 1, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((1, 1, 1, D), generator=g).to(torch.bfloat16)
+    out, _, v8t, vs = oracle_mod.sage_attention(_bits(q), _bits(k), _bits(v), 64, 64, 0.125, False)
+    ref = oracle_mod.e4m3_decode(v8t[0, 0, :, 0]) * vs[0, 0].astype(np.float64)
+    assert np.array_equal(out[0, 0, 0], oracle_mod.f64_to_bf16(ref))
+    # and the dequantised V row is the V row itself within e4m3 precision
+    vf = oracle_mod.bf16_to_f32(_bits(v))[0, 0, 0]
+    assert np.abs(ref - vf).max() <= 2.0 ** -4 * np.abs(vf).max()
+
+
+def test_identical_keys_give_mean_of_v(oracle_mod):
+    L, D = 300, 64
+    g = torch.Generator().manual_seed(2)
+    q = torch.randn((1, 1, L, D), generator=g).to(torch.bfloat16)
+    k = torch.randn((1, 1, 1, D), generator=g).expand(1, 1, L, D).to(torch.bfloat16).contiguous()
+    v = torch.randn((1, 1, L, D), generator=g).to(torch.bfloat16)
+    out, _, v8t, vs = oracle_mod.sage_attention(_bits(q), _bits(k), _bits(v), 64, 64, 0.125, False)
+    vdec = oracle_mod.e4m3_decode(v8t[0, 0, :, :L]) * vs[0, 0][:, None].astype(np.float64)
+    ref = oracle_mod.f64_to_bf16(vdec.mean(axis=1))
+    # smoothed identical keys are all zero -> every logit is 0 -> p = 1
+    for i in range(L):
+        assert np.array_equal(out[0, 0, i], ref)
+
+
+def _cosine(a, b):
+    a = a.ravel().astype(np.float64)
+    b = b.ravel().astype(np.float64)
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+
+def test_method_accuracy_gate_c1(oracle_mod):
+    cfg, q, k, v = workloads.make_prefill_config("c1")
+    out, _, _, _ = oracle_mod.sage_attention(_bits(q), _bits(k), _bits(v), cfg["blk_q"],
+                                             cfg["blk_k"], cfg["softmax_scale"], cfg["causal"])
+    exact = oracle_mod.attn_exact(_bits(q), _bits(k), _bits(v), cfg["softmax_scale"], cfg["causal"])
+    assert _cosine(oracle_mod.bf16_to_f32(out), exact) >= 0.998
+
+
+def test_method_accuracy_gate_outliers_and_planted_mistake(oracle_mod):
+    """A C2-like workload (outlier K channels, large K bias) on fewer tokens:
+    the method passes the gate; without K smoothing it does not."""
+    q, k, v = workloads.make_prefill(B=1, H=2, Hk=2, L=512, D=128, seed=21, kbias_std=30.0,
+                                     outlier_channels=4, outlier_mult=20.0)
+    scale = 1.0 / math.sqrt(128)
+    rows = np.arange(0, 512, 7, dtype=np.int32)
+    out, qk, v8t, vs = oracle_mod.sage_attention(_bits(q), _bits(k), _bits(v), 128, 64, scale,
+                                                 False, rows=rows)
+    exact = oracle_mod.attn_exact(_bits(q), _bits(k), _bits(v), scale, False, rows=rows)
+    good = _cosine(oracle_mod.bf16_to_f32(out), exact)
+    assert good >= 0.998
+    # planted mistake: quantise K without subtracting its mean
+    k8n, ksn = oracle_mod._quant_i8(_bits(k), None, 64, None)
+    bad_out = oracle_mod.attn(qk["q8"], qk["qs"], k8n, ksn, v8t, vs, 512, 512, 128, 64, scale,
+                              False, rows=rows)
+    bad = _cosine(oracle_mod.bf16_to_f32(bad_out), exact)
+    assert bad < good and bad < 0.998

@@ -1,0 +1,104 @@
+"""Pins of the oracle's paged FP8 decode.
+
+* The sliding-window convention (each of the MTP query tokens attends to the
+  `window` keys ending at its own position) reproduces the window-tile counts
+  the FlyDSL pa_decode page prints (tests/golden/window_tiles.txt).
+* The oracle's paged, GQA, per-token-scaled decode equals a brute-force
+  computation over the un-paged cache that uses torch's float8 conversion for
+  the query quantisation and scipy's Hadamard matrix for the rotation.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_tiles():
+    rows = []
+    for line in open(os.path.join(GOLDEN, "window_tiles.txt")):
+        if line.strip() and not line.startswith("#"):
+            rows.append(tuple(int(x) for x in line.split()))
+    return rows
+
+
+def _attended_keys(ctx, T, window):
+    """Union of the keys that the T last positions attend to (our reading)."""
+    keys = set()
+    for t in range(T):
+        p = ctx - T + t
+        keys.update(range(max(0, p - window + 1), p + 1))
+    return keys
+
+
+@pytest.mark.parametrize("window,mtp,tile,tiles", _golden_tiles())
+def test_window_convention_reproduces_page_tile_counts(window, mtp, tile, tiles):
+    assert (window + mtp - 2 + tile - 1) // tile + 1 == tiles
+    worst = 0
+    for ctx in range(window + mtp, window + mtp + 2 * tile):
+        keys = _attended_keys(ctx, mtp, window)
+        assert len(keys) == window + mtp - 1
+        worst = max(worst, len({j // tile for j in keys}))
+    assert worst == tiles
+
+
+def _brute_decode(oracle_mod, d, window, scale):
+    q = d["q"].float().numpy()                          # [B, T, H, D]
+    B, T, H, D = q.shape
+    Hk, page = d["k_cache"].shape[1], d["k_cache"].shape[2]
+    Hmat = scipy.linalg.hadamard(D).astype(np.float64)
+    kdec = oracle_mod.e4m3_decode(d["k_cache"].numpy())
+    vdec = oracle_mod.e4m3_decode(d["v_cache"].numpy())
+    out = np.zeros((B, T, H, D))
+    for b in range(B):
+        ctx = int(d["ctx_lens"][b])
+        pages = d["page_table"][b].numpy()
+        toks = np.arange(ctx)
+        phys = pages[toks // page]
+        slot = toks % page
+        for h in range(H):
+            hk = h // (H // Hk)
+            K = kdec[phys, hk, slot]                    # [ctx, D]
+            V = vdec[phys, hk, slot]
+            ks = d["k_scale"].numpy()[phys, hk, slot].astype(np.float64)
+            vs = d["v_scale"].numpy()[phys, hk, slot].astype(np.float64)
+            for t in range(T):
+                qh = oracle_mod.fwht_f32(q[b, t, h][None, :])[0]
+                assert np.abs(qh - q[b, t, h] @ Hmat).max() <= 1e-4 * np.abs(q[b, t, h]).sum()
+                a = np.abs(qh).max()
+                s = np.float32(a) / np.float32(448.0)
+                r = np.float32(448.0) / np.float32(a)
+                q8 = torch.from_numpy((qh * r).astype(np.float32)).to(torch.float8_e4m3fn)
+                q8 = q8.to(torch.float64).numpy()
+                p = ctx - T + t
+                lo = max(0, p - window + 1)
+                sl = slice(lo, p + 1)
+                logits = (K[sl] @ q8) * float(s) * ks[sl] * (scale / D)
+                w = np.exp(logits - logits.max())
+                w /= w.sum()
+                out[b, t, h] = (w * vs[sl]) @ V[sl]
+    return out
+
+
+@pytest.mark.parametrize("B,T,H,Hk,D,page,lo,hi,window", [
+    (3, 4, 8, 2, 64, 16, 40, 90, 32),
+    (2, 1, 4, 1, 128, 128, 100, 300, 512),      # window >= ctx: whole context
+    (2, 4, 16, 1, 128, 128, 300, 700, 256),
+])
+def test_decode_matches_brute_force(oracle_mod, B, T, H, Hk, D, page, lo, hi, window):
+    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=D, page=page, ctx_lo=lo, ctx_hi=hi,
+                              seed=B * 100 + D)
+    scale = 1.0 / math.sqrt(D)
+    out, o64 = oracle_mod.decode(workloads.bits_u16(d["q"]), d["k_cache"].numpy(),
+                                 d["v_cache"].numpy(), d["k_scale"].numpy(), d["v_scale"].numpy(),
+                                 d["page_table"].numpy(), d["ctx_lens"].numpy(), window, scale,
+                                 want_f64=True)
+    ref = _brute_decode(oracle_mod, d, window, scale)
+    assert np.abs(o64 - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    assert np.array_equal(out, oracle_mod.f64_to_bf16(o64))
