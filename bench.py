@@ -1,0 +1,347 @@
+#!/usr/bin/env python
+"""Throughput of the quantised attention path on B200.
+
+One step = the whole hot path on one batch of seeded synthetic inputs that
+already sit in HBM: sage_quant_qk (K mean, smoothing, Hadamard rotation, INT8
+Q/K) + sage_quant_v (e4m3 V) + sage_attn_fwd (INT8 QK^T, online softmax, e4m3
+PV, bf16 out). Workload: non-causal video-DiT prefill B=1 H=24 L=4096 D=128
+(Q blocks 128 tokens, K blocks 64). Metric: TOPS = 4 B H L^2 D / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sage|reference]
+
+N > 1 runs under torchrun: every rank runs its own replica of the workload
+(the path has no exchange step), timing is the max over ranks, and `value`
+counts the work of all ranks. `--impl reference` times the CPU oracle on the
+host cores on a bounded sample of the same workload (rank 0 only).
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-attn TOPS (4*B*H*L^2*D/t) and % of B200 INT8/FP8 tensor peak"
+UNIT = "TOPS"
+INT8_OVER_BF16 = 2.0        # nominal dense INT8/FP8 : BF16 tensor ratio (4.5 : 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
+    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "c4"])
+    ap.add_argument("--sets", type=int, default=4, help="rotating input sets (L2 defeat)")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def work_ops(cfg):
+    ops = 4.0 * cfg["B"] * cfg["H"] * cfg["L"] * cfg["L"] * cfg["D"]
+    return ops / 2 if cfg["causal"] else ops
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index, enabled=True):
+        self.gpu = gpu_index
+        self.proc = None
+        self.enabled = enabled
+        self.path = None
+
+    def __enter__(self):
+        if self.enabled:
+            fd, self.path = tempfile.mkstemp(prefix="clocks", suffix=".csv")
+            os.close(fd)
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                     "--format=csv,noheader,nounits", "-lms", "100"],
+                    stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                time.sleep(0.3)
+            except OSError:
+                self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+def cpu_baseline(cfg, seconds):
+    """The oracle as it stands, on the host cores, on whole heads of the same
+    workload until about `seconds` of CPU time has run."""
+    import numpy as np
+    import oracle
+    import workloads
+
+    cores = os.cpu_count() or 1
+    _, q, k, v = workloads.make_prefill_config(cfg["key"])
+    b = workloads.bits_u16
+    qb, kb, vb = b(q), b(k), b(v)
+    L, D = cfg["L"], cfg["D"]
+
+    def run(heads):
+        t = time.perf_counter()
+        qk = oracle.quant_qk(qb[:, :heads], kb[:, :heads], cfg["blk_q"], cfg["blk_k"], threads=cores)
+        v8t, vs = oracle.quant_v(vb[:, :heads], threads=cores)
+        oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, L, L, cfg["blk_q"],
+                    cfg["blk_k"], cfg["softmax_scale"], cfg["causal"], threads=cores)
+        return time.perf_counter() - t
+
+    t1 = run(1)
+    heads = int(max(1, min(cfg["H"], math.floor(seconds / max(t1, 1e-3)))))
+    if heads > 1:
+        t1 = run(heads)
+    ops = work_ops(dict(cfg, H=heads, B=1))
+    return {"value": ops / t1 / 1e12, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": "B=1, %d of %d heads, all %d query rows (quantise Q/K/V + attention), %.1f s"
+                      % (heads, cfg["H"], L, t1)}
+
+
+def run_reference(args):
+    import workloads
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = dict(workloads.PREFILL[args.workload], key=args.workload)
+    vals = []
+    cb = None
+    for _ in range(max(1, args.steps)):
+        cb = cpu_baseline(cfg, min(args.cpu_seconds, 20.0))
+        vals.append(cb["value"])
+        if len(vals) >= 3:
+            break
+    value = statistics.median(vals)
+    cb["value"] = value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": len(vals), "warmup": 0,
+        "ms_per_step": work_ops(dict(cfg)) / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3",
+        "data": "synthetic", "config": {"workload": cfg["name"], "B": cfg["B"], "H": cfg["H"],
+                                        "L": cfg["L"], "D": cfg["D"]},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def run_sage(args):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_attention_smoothing_b200 as sage
+    import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    cfg = dict(workloads.PREFILL[args.workload], key=args.workload)
+    B, H, Hk, L, D = cfg["B"], cfg["H"], cfg["Hk"], cfg["L"], cfg["D"]
+    blk_q, blk_k, scale, causal = cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"], cfg["causal"]
+    _, q, k, v = workloads.make_prefill_config(args.workload)
+
+    h = sage.Hadamard(D)
+    stream = torch.cuda.current_stream()
+    sets = []
+    for _ in range(args.sets):
+        qs, ks, vs_ = q.cuda(), k.cuda(), v.cuda()          # [B,H,L,D] views of [B,L,H,D]
+        bufs = sage.QuantBuffers(B, H, Hk, L, L, D, blk_q, blk_k)
+        out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
+        sets.append((qs, ks, vs_, bufs, out))
+    set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + 2 * q.numel() * 2
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+
+    def step(i, timed):
+        qs, ks, vs_, bufs, out = sets[i % len(sets)]
+        sage.sage_quant_qk(h, qs, ks, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                           bufs.k_mean, bufs.ws, stream)
+        sage.sage_quant_v(vs_, bufs.v8_t, bufs.v_scale, bufs.ws, stream)
+        if timed:
+            ev[i][0].record(stream)
+        sage.sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
+                           B, H, Hk, L, L, D, blk_q, blk_k, scale, causal, out, None, stream)
+        if timed:
+            ev[i][1].record(stream)
+
+    for i in range(args.warmup):
+        step(i, False)
+    torch.cuda.synchronize()
+    if sage.sage_device_error(stream) != sage.SAGE_OK:
+        raise RuntimeError("device error during warm-up")
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local, enabled=not args.no_clocks) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i, True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    if sage.sage_device_error(stream) != sage.SAGE_OK:
+        raise RuntimeError("device error during the timed steps")
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1))
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ops = work_ops(cfg)
+    value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    pk, pk_src = peaks()
+    peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
+    achieved = ops / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved, "peak": peak_tops,
+                "unit": "TFLOP/s", "frac": achieved / peak_tops, "traffic": None,
+                "peak_source": "%s bf16 burst x %.0f (INT8/FP8 : BF16 nominal)" % (pk_src, INT8_OVER_BF16),
+                "frac_of_sustained": achieved / (pk["bf16_tflops_sustained"] * INT8_OVER_BF16),
+                "attn_ms": attn_ms}
+
+    # end to end through the public API: pinned host inputs -> device ->
+    # quantise + attention -> result back to pinned host memory, every step
+    qh = q.permute(0, 2, 1, 3).contiguous().pin_memory()      # [B, L, H, D] host buffers
+    kh = k.permute(0, 2, 1, 3).contiguous().pin_memory()
+    vh = v.permute(0, 2, 1, 3).contiguous().pin_memory()
+    oh = torch.empty((B, L, H, D), dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = (torch.empty_like(x, device="cuda") for x in (qh, kh, vh))
+    od = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda")
+    ebufs = sets[0][3]
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        sage.sage_attention(h, qd.permute(0, 2, 1, 3), kd.permute(0, 2, 1, 3),
+                            vd.permute(0, 2, 1, 3), blk_q, blk_k, scale, causal,
+                            out=od.permute(0, 2, 1, 3), bufs=ebufs, stream=stream)
+        oh.copy_(od, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e = {"value": world * ops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+           "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
+           "d2h_bytes_per_step": oh.numel() * oh.element_size(),
+           "ms_per_step": e2e_ms / args.e2e_steps}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(cfg, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8+e4m3", "data": "synthetic",
+            "config": {"workload": cfg["name"], "B": B, "H": H, "L": L, "D": D,
+                       "blk_q": blk_q, "blk_k": blk_k, "causal": causal,
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "%d rotating input sets of %.0f MB (> 126 MB L2)"
+                             % (len(sets), set_bytes / 1e6)},
+            "roofline": roofline,
+            "cpu_baseline": cb,
+            "e2e": e2e,
+            "gpu_launches": 5 * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_sage(args)
+
+
+if __name__ == "__main__":
+    main()

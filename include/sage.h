@@ -1,0 +1,212 @@
+/*
+ * sage.h -- C ABI of libsage, a B200 (sm_100a) implementation of
+ * SageAttention-style quantized attention with K smoothing.
+ *
+ * The path, in call order:
+ *   sage_hadamard_init   once per head dimension: the rotation is fixed once
+ *                        and reused for every call ("Sage v2 improvements":
+ *                        the Hadamard matrix is created once and reused).
+ *   sage_quant_qk        K smoothing (subtract K's per-(b,h) mean over the
+ *                        sequence), Hadamard rotation of Q and K along the
+ *                        head dim, INT8 quantisation with one absmax scale
+ *                        per token block ("perf(dsv4): qproj wq_b transpose +
+ *                        serving contract; ...", sequence diagram: Hadamard
+ *                        transform -> per-head amax -> dequant scale -> INT8
+ *                        rows).
+ *   sage_quant_v         FP8 e4m3 quantisation of V with one scale per
+ *                        channel ("Sage2 SM89 Temporal Pair Experiment",
+ *                        Candidate: the kernel fuses a per-channel V scale).
+ *   sage_attn_fwd        S = Q8 K8^T in INT8, dequantised, online softmax in
+ *                        128-key tiles with the per-tile order QK ->
+ *                        update_mdo -> accumulate_d -> RS_32_to_8 -> PV
+ *                        ("Sage2 SM89 Temporal Pair Experiment", Candidate),
+ *                        P cast to e4m3 after scaling by FP8_MAX = 448, PV in
+ *                        FP8, epilogue x 1/FP8_MAX ("[FlyDSL] [Misc] pa_decode:
+ *                        key the tile kernel on FlyDSL dtypes and drop the
+ *                        batch-first plan grid", Changes), bf16 output.
+ *   sage_attn_decode     paged FP8-KV decode (same page: window-family
+ *                        workload, per-token FP8 K/V scales, MTP, GQA).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers on the device that is current
+ *     for the calling thread, owned by the caller; the library never
+ *     allocates, frees or copies them, never synchronises the stream (except
+ *     sage_device_error) and never makes a contiguous copy ("Sage v2
+ *     improvements": the forced .contiguous() was the bottleneck; "sage_attn3"
+ *     API page: preprocess_qkv / postprocess_output permute-and-copy).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream. Work is enqueued on it and the call returns at once.
+ *   - Views (sage_cview4 / sage_view4) describe logical [B, H, L, D] tensors
+ *     with sizes and strides counted in ELEMENTS (bf16), any non-negative
+ *     strides; layouts that allow 16-byte vector access (unit D stride,
+ *     other strides multiples of 8, 16-byte-aligned base) take the vector
+ *     path, any other layout takes the scalar path with identical results.
+ *   - Validation happens on the host before anything is launched; on error
+ *     nothing is enqueued. Bad pointers/sizes/strides -> SAGE_ERR_INVALID_ARG,
+ *     valid but unsupported shapes or formats -> SAGE_ERR_UNSUPPORTED (the
+ *     FlyDSL page refuses unsupported dtypes the same two ways), a workspace
+ *     that is too small -> SAGE_ERR_WORKSPACE, a failed CUDA launch ->
+ *     SAGE_ERR_CUDA. Nothing aborts or traps.
+ *   - Inputs must be finite; NaN/Inf inputs are outside the contract.
+ *   - Every device wait inside the kernels is bounded; a wait that expires
+ *     records an error word that sage_device_error reports as
+ *     SAGE_ERR_TIMEOUT.
+ *
+ * Quantised buffer layouts (part of the contract; produced by the quant
+ * entry points, consumed by sage_attn_fwd). Lpad(L) = L rounded up to 128.
+ *   q8      int8   [B, H,  Lpad(Lq), D]  contiguous, rows >= Lq zero
+ *   q_scale fp32   [B, H,  ceil(Lq / blk_q)]
+ *   k8      int8   [B, Hk, Lpad(Lk), D]  contiguous, rows >= Lk zero
+ *   k_scale fp32   [B, Hk, ceil(Lk / blk_k)]
+ *   k_mean  fp32   [B, Hk, D]
+ *   v8_t    e4m3   [B, Hk, D, Lpad(Lk)]  contiguous (V transposed: keys are
+ *                                       the contiguous dim), columns >= Lk 0
+ *   v_scale fp32   [B, Hk, D]
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sage_status {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,  /* null pointer, negative size/stride, bad handle */
+    SAGE_ERR_UNSUPPORTED = 2,  /* valid but not supported (D, block size, page size, ...) */
+    SAGE_ERR_ALIGNMENT = 3,    /* a quantised buffer is not 16-byte aligned */
+    SAGE_ERR_WORKSPACE = 4,    /* workspace missing or smaller than *_workspace() */
+    SAGE_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed */
+    SAGE_ERR_TIMEOUT = 6       /* a bounded device wait expired (see sage_device_error) */
+} sage_status;
+
+/* Read-only logical [B, H, L, D] view; sizes and strides in elements. */
+typedef struct sage_cview4 {
+    const void* ptr;
+    int64_t size[4];
+    int64_t stride[4];
+} sage_cview4;
+
+/* Writable logical [B, H, L, D] view; sizes and strides in elements. */
+typedef struct sage_view4 {
+    void* ptr;
+    int64_t size[4];
+    int64_t stride[4];
+} sage_view4;
+
+/* Opaque, immutable after init; usable from any stream and thread. */
+typedef struct sage_hadamard_s* sage_hadamard;
+
+/* Build the Sylvester Hadamard rotation H_D (entries +-1, H H^T = D I) for
+ * head_dim D in {64, 128} once, on host and on `device` ("Sage v2
+ * improvements": created once, reused by every call). The kernels apply it
+ * as the fp32 butterfly x -> x H (stages h = 1, 2, ..., D/2, each output one
+ * IEEE add or subtract), unnormalised; the 1/D that Q H (K H)^T carries is
+ * folded into the logit scale by sage_attn_fwd. *out receives the handle.
+ * Errors: INVALID_ARG (out NULL, device < 0), UNSUPPORTED (other D),
+ * CUDA (device not usable). */
+sage_status sage_hadamard_init(int head_dim, int device, sage_hadamard* out);
+
+/* Free a handle from sage_hadamard_init (NULL is accepted). */
+sage_status sage_hadamard_destroy(sage_hadamard h);
+
+/* Copy H (row-major D x D, int8 +-1) to host memory `host_out` (D*D bytes)
+ * and/or report D through `head_dim` (either may be NULL). */
+sage_status sage_hadamard_matrix(sage_hadamard h, int8_t* host_out, int* head_dim);
+
+/* Bytes of device workspace sage_quant_qk needs (fp64 partial sums of K). */
+size_t sage_quant_qk_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
+
+/* Smooth, rotate and INT8-quantise Q and K.
+ *   q_bf16: [B, H, Lq, D] bf16 view;  k_bf16: [B, Hk, Lk, D] bf16 view;
+ *   H % Hk == 0, D == handle's D, blk_q, blk_k in {32, 64, 128}.
+ * Computes, per (b, h):
+ *   mean_K[d] = fp32( (fp64 sum over the Lk tokens of K) / Lk )
+ *   K_s = K - mean_K (fp32); Q is not smoothed;
+ *   x_hat = butterfly(x) for every row of Q and K_s (fp32);
+ *   per block of blk tokens: a = max|x_hat|, scale = a / 127,
+ *   code = clamp(round_half_even(x_hat * (127 / a)), -127, 127) (a = 0 gives
+ *   scale 0 and zero codes).
+ * Writes q8, q_scale, k8, k_scale in the layouts above and, if k_mean is not
+ * NULL, mean_K [B, Hk, D]. ws: device workspace of at least
+ * sage_quant_qk_workspace(...) bytes, 256-byte aligned; its contents on
+ * entry do not matter. Quantised outputs must be 16-byte aligned.
+ * Results are bit-identical for any input strides. */
+sage_status sage_quant_qk(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16, int blk_q,
+                          int blk_k, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
+                          float* k_mean, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sage_quant_v needs (per-chunk channel maxima). */
+size_t sage_quant_v_workspace(int B, int Hk, int L, int D);
+
+/* FP8 e4m3 (OCP e4m3fn, max 448) per-channel quantisation of V.
+ *   v_bf16: [B, Hk, L, D] bf16 view, D in {64, 128}.
+ * Per (b, h, d): a = max over the L tokens of |v|, scale = a / 448,
+ * code = e4m3_round_nearest_even_saturating(v * (448 / a)) (a = 0 gives
+ * scale 0 and zero codes). Writes v8_t [B, Hk, D, Lpad(L)] (transposed) and
+ * v_scale [B, Hk, D]. ws as for sage_quant_qk. */
+sage_status sage_quant_v(sage_cview4 v_bf16, uint8_t* v8_t, float* v_scale, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sage_attn_fwd needs (0 in this version). */
+size_t sage_attn_fwd_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
+
+/* Quantised attention forward on the buffers written by the quant calls.
+ * For query row i of head h (kv head h / (H / Hk)) and key j, with
+ * c = softmax_scale / D:
+ *   x_ij = (sum_d q8[i,d] k8[j,d]) * q_scale[i / blk_q] * k_scale[j / blk_k] * c
+ *   causal != 0 masks j > i + (Lk - Lq) (bottom-right aligned).
+ * Keys are processed in tiles of 128 in ascending order; per tile the
+ * running max m and denominator d of each row are updated, P8 =
+ * e4m3(448 * exp(x - m)) feeds an FP8 PV product, d sums the unquantised
+ * probabilities, and out = bf16(O * v_scale / (448 * d)); a row that sees no
+ * key is written as zeros. out_bf16: [B, H, Lq, D] bf16 view of any strides.
+ * Supported: D in {64, 128}, blk_q and blk_k in {32, 64, 128}, Lq, Lk >= 1.
+ * Pointers q8, k8, v8_t must be 16-byte aligned. ws may be NULL. */
+sage_status sage_attn_fwd(const int8_t* q8, const float* q_scale, const int8_t* k8,
+                          const float* k_scale, const uint8_t* v8_t, const float* v_scale, int B,
+                          int H, int Hk, int Lq, int Lk, int D, int blk_q, int blk_k,
+                          float softmax_scale, int causal, sage_view4 out_bf16, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sage_attn_decode needs (split-KV partials). */
+size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window);
+
+/* Paged FP8-KV decode with MTP query tokens and a sliding window.
+ *   q_bf16: [B, T, H, D] bf16 view (the T query tokens are the last T
+ *   positions of each sequence); k_cache, v_cache: e4m3 codes
+ *   [num_pages, Hk, page_size, D] contiguous; k_scale, v_scale: fp32 per
+ *   token [num_pages, Hk, page_size]; page_table: int32 [B, max_pages]
+ *   logical -> physical page; ctx_lens: int32 [B], T <= ctx <= max_pages *
+ *   page_size. The cache holds keys already in the rotated domain.
+ * For token t (position p = ctx - T + t) and head h: q_hat = butterfly(q)
+ * (fp32), per-(t, h) e4m3 quantisation with scale max|q_hat| / 448; keys j in
+ * [max(0, p - window + 1), p]; S_j = (q8 . k8_j) * s_q * k_scale_j *
+ * softmax_scale / D; softmax; out = sum_j p_j v_scale_j v8_j -> bf16.
+ * out_bf16: [B, T, H, D] bf16 view. Supported: D == 128, page_size in
+ * {16, 32, 64, 128}, H % Hk == 0, H / Hk <= 16, T * (H / Hk) <= 64,
+ * window >= 1. ws: at least sage_attn_decode_workspace(...) bytes. */
+sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
+                             const uint8_t* v_cache, const float* k_scale, const float* v_scale,
+                             const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
+                             int H, int Hk, int D, int page_size, int max_pages, int num_pages,
+                             int window, float softmax_scale, sage_view4 out_bf16, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sage_status_string(sage_status s);
+
+/* Synchronise `stream`, then read and clear the library's device error
+ * words on the current device: SAGE_ERR_TIMEOUT if a bounded wait expired
+ * since the last call, SAGE_ERR_CUDA if the stream reports a CUDA error,
+ * SAGE_OK otherwise. */
+sage_status sage_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H_ */

@@ -1,0 +1,258 @@
+"""Python binding of libsage, the sm_100a quantized-attention library.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+behind the C ABI declared in ``include/sage.h``; there is no CPU or PyTorch
+fallback, and a missing or unloadable ``libsage.so`` raises at once.
+
+The functions keep the C names. Tensors are torch tensors on the current
+CUDA device; views are passed with their own strides (no ``.contiguous()``).
+``stream`` defaults to torch's current stream.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage.so")
+
+SAGE_OK = 0
+SAGE_ERR_INVALID_ARG = 1
+SAGE_ERR_UNSUPPORTED = 2
+SAGE_ERR_ALIGNMENT = 3
+SAGE_ERR_WORKSPACE = 4
+SAGE_ERR_CUDA = 5
+SAGE_ERR_TIMEOUT = 6
+
+EXPORTS = (
+    "sage_hadamard_init", "sage_hadamard_destroy", "sage_hadamard_matrix",
+    "sage_quant_qk_workspace", "sage_quant_qk", "sage_quant_v_workspace", "sage_quant_v",
+    "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_decode_workspace",
+    "sage_attn_decode", "sage_status_string", "sage_device_error",
+)
+
+
+class SageError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s failed: %s" % (where, status_string(status)))
+
+
+class CView4(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("size", ctypes.c_int64 * 4),
+                ("stride", ctypes.c_int64 * 4)]
+
+
+class View4(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("size", ctypes.c_int64 * 4),
+                ("stride", ctypes.c_int64 * 4)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libsage.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise OSError("libsage.so not built: run `python -m quantized_attention_smoothing_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.sage_status_string.restype = ctypes.c_char_p
+    L.sage_status_string.argtypes = [i32]
+    L.sage_hadamard_init.restype = i32
+    L.sage_hadamard_init.argtypes = [i32, i32, ctypes.POINTER(vp)]
+    L.sage_hadamard_destroy.restype = i32
+    L.sage_hadamard_destroy.argtypes = [vp]
+    L.sage_hadamard_matrix.restype = i32
+    L.sage_hadamard_matrix.argtypes = [vp, vp, ctypes.POINTER(i32)]
+    L.sage_quant_qk_workspace.restype = sz
+    L.sage_quant_qk_workspace.argtypes = [i32] * 6
+    L.sage_quant_qk.restype = i32
+    L.sage_quant_qk.argtypes = [vp, CView4, CView4, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.sage_quant_v_workspace.restype = sz
+    L.sage_quant_v_workspace.argtypes = [i32] * 4
+    L.sage_quant_v.restype = i32
+    L.sage_quant_v.argtypes = [CView4, vp, vp, vp, sz, vp]
+    L.sage_attn_fwd_workspace.restype = sz
+    L.sage_attn_fwd_workspace.argtypes = [i32] * 6
+    L.sage_attn_fwd.restype = i32
+    L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp] + [i32] * 8 + [f32, i32, View4, vp, sz, vp]
+    L.sage_attn_decode_workspace.restype = sz
+    L.sage_attn_decode_workspace.argtypes = [i32] * 6
+    L.sage_attn_decode.restype = i32
+    L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 10 + \
+        [f32, View4, vp, sz, vp]
+    L.sage_device_error.restype = i32
+    L.sage_device_error.argtypes = [vp]
+    _lib = L
+    return L
+
+
+def status_string(status):
+    return lib().sage_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != SAGE_OK:
+        raise SageError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _view(t, cls):
+    if t.dim() != 4:
+        raise ValueError("expected a 4-d tensor view, got shape %s" % (tuple(t.shape),))
+    v = cls()
+    v.ptr = t.data_ptr()
+    for i in range(4):
+        v.size[i] = t.shape[i]
+        v.stride[i] = t.stride(i)
+    return v
+
+
+class Hadamard:
+    """Owns a sage_hadamard handle (built once per head dim and device)."""
+
+    def __init__(self, head_dim, device=None):
+        if device is None:
+            device = torch.cuda.current_device()
+        h = ctypes.c_void_p()
+        _check(lib().sage_hadamard_init(int(head_dim), int(device), ctypes.byref(h)),
+               "sage_hadamard_init")
+        self.handle = h
+        self.head_dim = int(head_dim)
+        self.device = int(device)
+
+    def matrix(self):
+        import numpy as np
+        out = np.zeros((self.head_dim, self.head_dim), dtype=np.int8)
+        d = ctypes.c_int()
+        _check(lib().sage_hadamard_matrix(self.handle, out.ctypes.data_as(ctypes.c_void_p),
+                                          ctypes.byref(d)), "sage_hadamard_matrix")
+        return out
+
+    def close(self):
+        if self.handle is not None and _lib is not None:
+            _lib.sage_hadamard_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def sage_hadamard_init(head_dim, device=None):
+    return Hadamard(head_dim, device)
+
+
+def sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D):
+    return int(lib().sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D))
+
+
+def sage_quant_v_workspace(B, Hk, L, D):
+    return int(lib().sage_quant_v_workspace(B, Hk, L, D))
+
+
+def sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D):
+    return int(lib().sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D))
+
+
+def sage_attn_decode_workspace(B, T, H, Hk, D, window):
+    return int(lib().sage_attn_decode_workspace(B, T, H, Hk, D, window))
+
+
+def sage_quant_qk(h, q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean=None, ws=None,
+                  stream=None):
+    _check(lib().sage_quant_qk(h.handle, _view(q, CView4), _view(k, CView4), int(blk_q),
+                               int(blk_k), _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale),
+                               _ptr(k_mean), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                               _stream(stream)), "sage_quant_qk")
+
+
+def sage_quant_v(v, v8_t, v_scale, ws=None, stream=None):
+    _check(lib().sage_quant_v(_view(v, CView4), _ptr(v8_t), _ptr(v_scale), _ptr(ws),
+                              0 if ws is None else ws.numel() * ws.element_size(),
+                              _stream(stream)), "sage_quant_v")
+
+
+def sage_attn_fwd(q8, q_scale, k8, k_scale, v8_t, v_scale, B, H, Hk, Lq, Lk, D, blk_q, blk_k,
+                  softmax_scale, causal, out, ws=None, stream=None):
+    _check(lib().sage_attn_fwd(_ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale), _ptr(v8_t),
+                               _ptr(v_scale), B, H, Hk, Lq, Lk, D, blk_q, blk_k,
+                               float(softmax_scale), int(bool(causal)), _view(out, View4),
+                               _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                               _stream(stream)), "sage_attn_fwd")
+
+
+def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_lens, page_size,
+                     num_pages, window, softmax_scale, out, ws=None, stream=None):
+    B, T, H, D = q.shape
+    Hk = k_cache.shape[1]
+    max_pages = page_table.shape[1]
+    _check(lib().sage_attn_decode(h.handle, _view(q, CView4), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(k_scale), _ptr(v_scale), _ptr(page_table), _ptr(ctx_lens),
+                                  B, T, H, Hk, D, int(page_size), int(max_pages), int(num_pages),
+                                  int(window), float(softmax_scale), _view(out, View4), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(),
+                                  _stream(stream)), "sage_attn_decode")
+
+
+def sage_device_error(stream=None):
+    return int(lib().sage_device_error(_stream(stream)))
+
+
+# ---------------------------------------------------------------- convenience
+
+def round_up(x, m):
+    return (x + m - 1) // m * m
+
+
+class QuantBuffers:
+    """Device buffers of the quantised operands for one [B, H(k), L, D] shape."""
+
+    def __init__(self, B, H, Hk, Lq, Lk, D, blk_q, blk_k, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+        self.shape = (B, H, Hk, Lq, Lk, D, blk_q, blk_k)
+        self.q8 = torch.empty((B, H, round_up(Lq, 128), D), dtype=torch.int8, device=dev)
+        self.q_scale = torch.empty((B, H, math.ceil(Lq / blk_q)), dtype=torch.float32, device=dev)
+        self.k8 = torch.empty((B, Hk, round_up(Lk, 128), D), dtype=torch.int8, device=dev)
+        self.k_scale = torch.empty((B, Hk, math.ceil(Lk / blk_k)), dtype=torch.float32, device=dev)
+        self.k_mean = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
+        self.v8_t = torch.empty((B, Hk, D, round_up(Lk, 128)), dtype=torch.uint8, device=dev)
+        self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
+        ws = max(sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D), sage_quant_v_workspace(B, Hk, Lk, D),
+                 sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D), 16)
+        self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev)
+
+
+def sage_attention(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, out=None, bufs=None,
+                   stream=None):
+    """Quantise Q/K/V and run the quantised attention; q, k, v are [B, H(k),
+    L, D] bf16 views. Returns (out, bufs); out defaults to a [B, H, L, D]
+    view of a [B, L, H, D] tensor (the video-DiT layout)."""
+    B, H, Lq, D = q.shape
+    Hk, Lk = k.shape[1], k.shape[2]
+    if bufs is None:
+        bufs = QuantBuffers(B, H, Hk, Lq, Lk, D, blk_q, blk_k, q.device.index)
+    if out is None:
+        out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=q.device).permute(0, 2, 1, 3)
+    sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                  bufs.k_mean, bufs.ws, stream)
+    sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws, stream)
+    sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale, B, H, Hk,
+                  Lq, Lk, D, blk_q, blk_k, softmax_scale, causal, out, None, stream)
+    return out, bufs

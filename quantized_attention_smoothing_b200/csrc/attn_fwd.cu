@@ -1,0 +1,478 @@
+// attn_fwd.cu -- quantised attention forward for sm_100a.
+//
+// One CTA owns two 128-row query tiles of one (b, h) and streams the key
+// axis in 128-key tiles. Roles (320 threads):
+//   warps 0-3   softmax for query tile 0 (thread = query row = TMEM lane)
+//   warps 4-7   softmax for query tile 1
+//   warp 8      TMA producer: both Q tiles once, then a ring of K / V^T stages
+//   warp 9      MMA issuer (one thread): tcgen05 kind::i8 S = Q8 K8^T into
+//               TMEM (int32), tcgen05 kind::f8f6f4 O += P8 V8 into TMEM (fp32)
+// TMEM (512 columns): S_w at [128 w, 128 w + 128), O_w at [256 + 128 w, +D).
+// The MMA warp issues S(t) for both tiles before PV(t-1), so the tensor pipe
+// works on the next scores while the softmax warps convert the current ones
+// (the overlap "Sage2 SM89 Temporal Pair Experiment" (Candidate) obtains with
+// warp pairs on sm_89).
+//
+// Per 128-key tile the softmax warps follow the page's sequence
+//   QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV
+// with m, d per row in registers, y = acc * (q_scale * k_scale *
+// softmax_scale / D * log2 e) (base-2 logits), m' = max(m, max y),
+// alpha = 2^(m - m'), d = alpha d + sum 2^(y - m') (before the FP8 cast),
+// P8 = e4m3(448 * 2^(y - m')) written to shared memory in the UMMA 128B-swizzled
+// K-major layout, and O *= alpha in TMEM whenever alpha != 1 for some row of
+// the warp. The epilogue writes bf16(O * v_scale / (448 d)) through the
+// caller's strides ("[FlyDSL] [Misc] pa_decode: ...", Changes: P scaled by
+// FP8_MAX before the cast, epilogue x 1/FP8_MAX; "sage_attn3" API page: the
+// output is written straight into a [B, L, H, D] layout without a copy).
+//
+// Every mbarrier wait is bounded (see mbar_wait): on timeout the CTA records
+// an error word, raises a CTA-wide abort flag, drains its own MMAs and
+// returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "sage_internal.h"
+#include "sage_ptx.cuh"
+
+namespace sage {
+namespace {
+
+__device__ unsigned g_attn_err;
+
+constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
+constexpr int BN = 128;          // keys per tile
+constexpr int QT = 2;            // query tiles per CTA
+constexpr int kThreads = 320;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+    static constexpr int kStages = D == 128 ? 4 : 6;
+    static constexpr int kQBytes = BM * D;
+    static constexpr int kKBytes = BN * D;
+    static constexpr int kVBytes = D * BN;
+    static constexpr int kPBytes = BM * BN;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + QT * kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKBytes;
+    static constexpr int kOffP = kOffV + kStages * kVBytes;
+    static constexpr int kOffBar = kOffP + QT * kPBytes;
+    static constexpr int kBarQ = 0;
+    static constexpr int kBarKFull = 1;
+    static constexpr int kBarKEmpty = kBarKFull + kStages;
+    static constexpr int kBarVFull = kBarKEmpty + kStages;
+    static constexpr int kBarVEmpty = kBarVFull + kStages;
+    static constexpr int kBarSFull = kBarVEmpty + kStages;   // [QT]
+    static constexpr int kBarSEmpty = kBarSFull + QT;        // [QT], 4 warp arrivals
+    static constexpr int kBarPFull = kBarSEmpty + QT;        // [QT], 4 warp arrivals
+    static constexpr int kBarODone = kBarPFull + QT;         // [QT]
+    static constexpr int kBarFinal = kBarODone + QT;
+    static constexpr int kNumBars = kBarFinal + 1;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + runtime 1024-B alignment
+    static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "alignment");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+struct Params {
+    const float* q_scale;
+    const float* k_scale;
+    const float* v_scale;
+    __nv_bfloat16* out;
+    int64_t os0, os1, os2, os3;
+    int H, Hk, Lq, Lk, LpadQ, LpadK, blk_q, blk_k, nbq, nbk;
+    float logit_scale_log2;        // softmax_scale / D * log2(e)
+    int heavy_first;
+    int out_vec;
+};
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+template <int D, int NKB, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    int bh, qt;
+    if (p.heavy_first) {
+        bh = blockIdx.x;
+        qt = gridDim.y - 1 - blockIdx.y;
+    } else {
+        qt = blockIdx.x;
+        bh = blockIdx.y;
+    }
+    const int b = bh / p.H, h = bh % p.H;
+    const int bhk = b * p.Hk + h / (p.H / p.Hk);
+    const int q_row0 = qt * (QT * BM);
+
+    int kv_end = p.Lk;
+    if (CAUSAL) {
+        const int lim = q_row0 + QT * BM + (p.Lk - p.Lq);     // last visible key + 1
+        kv_end = max(0, min(kv_end, lim));
+    }
+    const int n_tiles = (kv_end + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kNumBars; ++i) {
+            const bool four = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
+                              (i >= C::kBarPFull && i < C::kBarPFull + QT);
+            mbar_init(&bars[i], four ? 4u : 1u);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(&bars[C::kBarQ], QT * C::kQBytes);
+            for (int w = 0; w < QT; ++w)
+                tma_load_2d(smem + C::kOffQ + w * C::kQBytes, &tmQ, &bars[C::kBarQ], 0,
+                            bh * p.LpadQ + q_row0 + w * BM);
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % C::kStages;
+                const uint32_t ph = (t / C::kStages) & 1;
+                if (!mbar_wait(&bars[C::kBarKEmpty + s], ph ^ 1, abort_flag, &g_attn_err, 1)) break;
+                mbar_arrive_expect_tx(&bars[C::kBarKFull + s], C::kKBytes);
+                tma_load_2d(smem + C::kOffK + s * C::kKBytes, &tmK, &bars[C::kBarKFull + s], 0,
+                            bhk * p.LpadK + t * BN);
+                if (!mbar_wait(&bars[C::kBarVEmpty + s], ph ^ 1, abort_flag, &g_attn_err, 2)) break;
+                mbar_arrive_expect_tx(&bars[C::kBarVFull + s], C::kVBytes);
+                tma_load_2d(smem + C::kOffV + s * C::kVBytes, &tmV, &bars[C::kBarVFull + s],
+                            t * BN, bhk * D);
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t kIdescQK = umma_idesc(2, 1, BM, BN);   // s8 x s8 -> s32
+            constexpr uint32_t kIdescPV = umma_idesc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
+            const uint32_t sQ = smem_u32(smem + C::kOffQ);
+            const uint32_t sK = smem_u32(smem + C::kOffK);
+            const uint32_t sV = smem_u32(smem + C::kOffV);
+            const uint32_t sP = smem_u32(smem + C::kOffP);
+
+            auto issue_pv = [&](int u) -> bool {
+                const int s = u % C::kStages;
+                const uint32_t ph = (u / C::kStages) & 1;
+                if (!mbar_wait(&bars[C::kBarVFull + s], ph, abort_flag, &g_attn_err, 3)) return false;
+                tc_fence_after();
+                const uint64_t vdesc = umma_desc_kmajor(sV + s * C::kVBytes, 128);
+                for (int w = 0; w < QT; ++w) {
+                    if (!mbar_wait(&bars[C::kBarPFull + w], u & 1, abort_flag, &g_attn_err, 4))
+                        return false;
+                    tc_fence_after();
+                    const uint64_t pdesc = umma_desc_kmajor(sP + w * C::kPBytes, 128);
+#pragma unroll
+                    for (int kk = 0; kk < BN / 32; ++kk)
+                        mma_f8_ss(tmem + 256 + w * BM, pdesc + 2 * kk, vdesc + 2 * kk, kIdescPV,
+                                  (u > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bars[C::kBarODone + w]);
+                }
+                mma_commit(&bars[C::kBarVEmpty + s]);
+                return true;
+            };
+
+            bool ok = mbar_wait(&bars[C::kBarQ], 0, abort_flag, &g_attn_err, 5);
+            tc_fence_after();
+            for (int t = 0; ok && t < n_tiles; ++t) {
+                const int s = t % C::kStages;
+                const uint32_t ph = (t / C::kStages) & 1;
+                if (!(ok = mbar_wait(&bars[C::kBarKFull + s], ph, abort_flag, &g_attn_err, 6))) break;
+                tc_fence_after();
+                const uint64_t kdesc = umma_desc_kmajor(sK + s * C::kKBytes, D);
+                for (int w = 0; w < QT && ok; ++w) {
+                    if (t > 0) {
+                        ok = mbar_wait(&bars[C::kBarSEmpty + w], (t - 1) & 1, abort_flag,
+                                       &g_attn_err, 7);
+                        if (!ok) break;
+                        tc_fence_after();
+                    }
+                    const uint64_t qdesc = umma_desc_kmajor(sQ + w * C::kQBytes, D);
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK,
+                                  kk > 0 ? 1u : 0u);
+                    mma_commit(&bars[C::kBarSFull + w]);
+                }
+                if (!ok) break;
+                mma_commit(&bars[C::kBarKEmpty + s]);
+                if (t > 0) ok = issue_pv(t - 1);
+            }
+            if (ok) issue_pv(n_tiles - 1);
+            // drain every MMA this thread issued before TMEM is released
+            mma_commit(&bars[C::kBarFinal]);
+            mbar_wait(&bars[C::kBarFinal], 0, abort_flag, &g_attn_err, 8);
+        }
+    } else {
+        // ---------------------------------------------------------- softmax
+        const int w = warp >> 2, ww = warp & 3;
+        const int r = ww * 32 + lane;
+        const int i = q_row0 + w * BM + r;
+        const bool valid = i < p.Lq;
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(ww * 32) << 16);
+        const uint32_t s_col = w * BN;
+        const uint32_t o_col = 256 + w * BM;
+        const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + i / p.blk_q]) : 0.0f;
+        const float arow = qsc * p.logit_scale_log2;
+        int jlim = valid ? p.Lk - 1 : -1;
+        if (CAUSAL && valid) jlim = min(jlim, i + (p.Lk - p.Lq));
+        uint8_t* sP = smem + C::kOffP + w * C::kPBytes;
+        const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
+
+        float m = -INFINITY, dsum = 0.0f;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            ok = warp_all(mbar_wait(&bars[C::kBarSFull + w], t & 1, abort_flag, &g_attn_err, 9));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[4][32];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(lane_addr + s_col + 32 * c4, sv[c4]);
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) tmem_wait_ld(sv[c4]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
+
+            const int j0 = t * BN;
+            float ksc[NKB];
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
+                const int bi = min((j0 + kb * (BN / NKB)) / p.blk_k, p.nbk - 1);
+                ksc[kb] = __ldg(&ksrow[bi]) * arow;
+            }
+            // QK: dequantised base-2 logits, masked; row max
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                const float acc = static_cast<float>(static_cast<int>(sv[c / 32][c % 32]));
+                float y = acc * ksc[c / (BN / NKB)];
+                y = (j0 + c <= jlim) ? y : -INFINITY;
+                sv[c / 32][c % 32] = __float_as_uint(y);
+                mt = fmaxf(mt, y);
+            }
+            // update_mdo (max part), accumulate_d, RS_32_to_8
+            const float m_new = fmaxf(m, mt);
+            const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
+            const float alpha = ex2_approx(m - msub);
+            float rowsum = 0.0f;
+            uint32_t pk[BN / 4];
+#pragma unroll
+            for (int c = 0; c < BN; c += 4) {
+                float e[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    e[k] = ex2_approx(__uint_as_float(sv[(c + k) / 32][(c + k) % 32]) - msub);
+                    rowsum += e[k];
+                }
+                const uint32_t lo = e4m3x2_rn_satfinite(e[0] * 448.0f, e[1] * 448.0f);
+                const uint32_t hi = e4m3x2_rn_satfinite(e[2] * 448.0f, e[3] * 448.0f);
+                pk[c / 4] = lo | (hi << 16);
+            }
+            dsum = dsum * alpha + rowsum;
+
+            if (t > 0) {
+                // PV(t-1) must be complete before O is rescaled and P is overwritten
+                ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (t - 1) & 1, abort_flag,
+                                        &g_attn_err, 10));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        uint32_t o[32];
+                        tmem_ld32(lane_addr + o_col + 32 * c4, o);
+                        tmem_wait_ld(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(lane_addr + o_col + 32 * c4, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P8 row -> shared memory, 128B swizzle (16-byte chunk c of row r at c ^ (r & 7))
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(sP + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarPFull + w]);
+            m = m_new;
+        }
+
+        // epilogue: out = O * v_scale / (448 d) -> bf16, through the caller's strides
+        const float* vsrow = p.v_scale + (int64_t)bhk * D;
+        __nv_bfloat16* orow = p.out + b * p.os0 + h * p.os1 + (int64_t)i * p.os2;
+        if (ok && n_tiles > 0) {
+            ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (n_tiles - 1) & 1, abort_flag,
+                                    &g_attn_err, 11));
+            if (ok) {
+                tc_fence_after();
+                const float inv = dsum > 0.0f ? 1.0f / (448.0f * dsum) : 0.0f;
+#pragma unroll
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_addr + o_col + 32 * c4, o);
+                    tmem_wait_ld(o);
+                    if (valid) {
+                        uint32_t packed[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float v0 = __uint_as_float(o[e]) * (__ldg(&vsrow[32 * c4 + e]) * inv);
+                            const float v1 = __uint_as_float(o[e + 1]) * (__ldg(&vsrow[32 * c4 + e + 1]) * inv);
+                            const __nv_bfloat162 pr = __floats2bfloat162_rn(v0, v1);
+                            packed[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+                        }
+                        if (p.out_vec) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1],
+                                                     packed[4 * q4 + 2], packed[4 * q4 + 3]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) {
+                                const uint16_t bits = (e & 1) ? (packed[e / 2] >> 16) : (packed[e / 2] & 0xFFFFu);
+                                *reinterpret_cast<uint16_t*>(orow + (int64_t)(32 * c4 + e) * p.os3) = bits;
+                            }
+                        }
+                    }
+                }
+            }
+        } else if (n_tiles == 0 && valid) {
+            for (int d = 0; d < D; ++d) orow[(int64_t)d * p.os3] = __float2bfloat16_rn(0.0f);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2-D uint8 tensor map: `rows` rows of `cols` bytes (row pitch = cols), box
+// {box_cols, box_rows}, swizzle matching the row length of the box.
+bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows,
+                  uint32_t box_cols, uint32_t box_rows) {
+    auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw =
+        box_cols == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int NKB, bool CAUSAL>
+cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const Params& p, dim3 grid, cudaStream_t s) {
+    auto kern = attn_fwd_kernel<D, NKB, CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+template <int D, int NKB>
+cudaError_t launch_c(bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                     const CUtensorMap& tv, const Params& p, dim3 grid, cudaStream_t s) {
+    return causal ? launch_t<D, NKB, true>(tq, tk, tv, p, grid, s)
+                  : launch_t<D, NKB, false>(tq, tk, tv, p, grid, s);
+}
+
+template <int D>
+cudaError_t launch_d(int nkb, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
+                     const CUtensorMap& tv, const Params& p, dim3 grid, cudaStream_t s) {
+    switch (nkb) {
+        case 1: return launch_c<D, 1>(causal, tq, tk, tv, p, grid, s);
+        case 2: return launch_c<D, 2>(causal, tq, tk, tv, p, grid, s);
+        default: return launch_c<D, 4>(causal, tq, tk, tv, p, grid, s);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
+    const int LpadQ = static_cast<int>(round_up(a.Lq, kTile));
+    const int LpadK = static_cast<int>(round_up(a.Lk, kTile));
+    CUtensorMap tq, tk, tv;
+    if (!encode_u8_2d(&tq, a.q8, a.D, (uint64_t)a.B * a.H * LpadQ, a.D, BM) ||
+        !encode_u8_2d(&tk, a.k8, a.D, (uint64_t)a.B * a.Hk * LpadK, a.D, BN) ||
+        !encode_u8_2d(&tv, a.v8t, LpadK, (uint64_t)a.B * a.Hk * a.D, BN, a.D))
+        return cudaErrorInvalidValue;
+    Params p;
+    p.q_scale = a.q_scale;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.os0 = a.out_stride[0];
+    p.os1 = a.out_stride[1];
+    p.os2 = a.out_stride[2];
+    p.os3 = a.out_stride[3];
+    p.H = a.H;
+    p.Hk = a.Hk;
+    p.Lq = a.Lq;
+    p.Lk = a.Lk;
+    p.LpadQ = LpadQ;
+    p.LpadK = LpadK;
+    p.blk_q = a.blk_q;
+    p.blk_k = a.blk_k;
+    p.nbq = static_cast<int>(ceil_div(a.Lq, a.blk_q));
+    p.nbk = static_cast<int>(ceil_div(a.Lk, a.blk_k));
+    p.logit_scale_log2 = a.softmax_scale / static_cast<float>(a.D) * kLog2e;
+    p.heavy_first = a.causal ? 1 : 0;
+    p.out_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 8 == 0 && a.out_stride[1] % 8 == 0 &&
+                 a.out_stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.out) % 16 == 0)
+                    ? 1
+                    : 0;
+    const int nqt = static_cast<int>(ceil_div(a.Lq, QT * BM));
+    const dim3 grid = a.causal ? dim3(a.B * a.H, nqt) : dim3(nqt, a.B * a.H);
+    const int nkb = BN / a.blk_k;
+    return a.D == 128 ? launch_d<128>(nkb, a.causal != 0, tq, tk, tv, p, grid, s)
+                      : launch_d<64>(nkb, a.causal != 0, tq, tk, tv, p, grid, s);
+}
+
+unsigned read_clear_attn_error() {
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_err, sizeof v) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_attn_err, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace sage

@@ -1,0 +1,359 @@
+// quant.cu -- K smoothing statistics, fused smooth + Hadamard + INT8
+// quantisation of Q and K, and FP8 e4m3 per-channel quantisation of V.
+//
+// Numerics are a fixed operation graph so that results are bit-identical
+// to a plain sequential evaluation (this TU is compiled with -fmad=false,
+// and every rounding step uses an explicit _rn intrinsic):
+//   mean_K = fp32(fp64 sum / L)           (fp64 partial sums per 512-token
+//                                          chunk, then chunks in order)
+//   x_s    = x - mean_K                   (fp32, K only)
+//   x_hat  = butterfly(x_s)               (fp32, stages h = 1, 2, ..., D/2)
+//   a      = max |x_hat| over the block;  s = a / 127;  r = 127 / a
+//   code   = clamp(rne(x_hat * r), +-127)
+//   V:  a = max |v| per channel; s = a / 448; code = e4m3_rn_sat(v * (448/a))
+// Sources: "Sage v2 improvements" (Hadamard built once, any-stride inputs);
+// "perf(dsv4): qproj wq_b transpose + serving contract; sparse_attn/indexer
+// tuning", sequence diagram (Hadamard -> per-head amax -> scale -> INT8);
+// "Sage2 SM89 Temporal Pair Experiment", Candidate (per-channel V scale);
+// "[FlyDSL] [Misc] pa_decode: ...", Changes (FP8_MAX of e4m3 = 448).
+#include <type_traits>
+
+#include <cuda_bf16.h>
+
+#include "sage_internal.h"
+#include "sage_ptx.cuh"
+
+namespace sage {
+namespace {
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
+    return __uint_as_float(bits16 << 16);
+}
+
+// Load 8 consecutive (along D) bf16 values of one token row as raw bits.
+// VEC: one 16-byte load (caller guarantees alignment); else 8 scalar loads.
+__device__ __forceinline__ uint4 load_row8(const uint16_t* base, int64_t off, int64_t sd,
+                                           bool vec) {
+    if (vec) return __ldg(reinterpret_cast<const uint4*>(base + off));
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t lo = __ldg(base + off + (2 * i) * sd);
+        uint32_t hi = __ldg(base + off + (2 * i + 1) * sd);
+        w[i] = lo | (hi << 16);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        x[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+}
+
+// ---------------------------------------------------------------- stats
+// grid (chunks, B*Hh), 256 threads. MODE 0: fp64 column sums (K mean);
+// MODE 1: fp32 column absmax (V scale). One output row of D values per
+// (b, h, chunk).
+template <int D, int MODE>
+__global__ void __launch_bounds__(256) column_stats_kernel(View4 x, int L, void* partial,
+                                                           int vec) {
+    constexpr int TPR = D / 8;           // threads per token row
+    constexpr int RPI = 256 / TPR;       // token rows per iteration
+    using Acc = typename std::conditional<MODE == 0, double, float>::type;
+    __shared__ Acc red[RPI][D];
+
+    const int Hh = static_cast<int>(x.size[1]);
+    const int bh = blockIdx.y;
+    const int b = bh / Hh, h = bh % Hh;
+    const int tid = threadIdx.x;
+    const int cg = tid % TPR, rg = tid / TPR;
+    const int l0 = blockIdx.x * kStatRows;
+    const int l1 = min(L, l0 + kStatRows);
+    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
+    const int64_t row0 = b * x.stride[0] + h * x.stride[1] + (int64_t)(cg * 8) * x.stride[3];
+
+    Acc acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = Acc(0);
+    for (int l = l0 + rg; l < l1; l += RPI) {
+        float v[8];
+        unpack8(load_row8(base, row0 + (int64_t)l * x.stride[2], x.stride[3], vec != 0), v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (MODE == 0) acc[i] = __dadd_rn(acc[i], (double)v[i]);
+            else acc[i] = fmaxf(acc[i], fabsf(v[i]));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[rg][cg * 8 + i] = acc[i];
+    __syncthreads();
+    if (tid < D) {
+        Acc s = red[0][tid];
+        for (int r = 1; r < RPI; ++r) {
+            if (MODE == 0) s = __dadd_rn(s, red[r][tid]);
+            else s = fmaxf(s, red[r][tid]);
+        }
+        static_cast<Acc*>(partial)[((int64_t)bh * gridDim.x + blockIdx.x) * D + tid] = s;
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void butterfly(float (&x)[D]) {
+    // stage h pairs (j, j + h) for j = (k / h) * 2h + k % h, k = 0 .. D/2 - 1
+#pragma unroll
+    for (int lg = 0; (1 << lg) < D; ++lg) {
+        const int h = 1 << lg;
+#pragma unroll
+        for (int k = 0; k < D / 2; ++k) {
+            const int j = ((k >> lg) << (lg + 1)) + (k & (h - 1));
+            const float a = x[j], c = x[j + h];
+            x[j] = __fadd_rn(a, c);
+            x[j + h] = __fsub_rn(a, c);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- Q/K int8
+// One CTA of 128 threads per (tensor, b, h, 128-token tile); thread = token.
+template <int D>
+__global__ void __launch_bounds__(128) qk_quant_kernel(
+    View4 q, View4 k, int blk_q, int blk_k, int n_qtiles, const double* __restrict__ ksum,
+    int kchunks, int8_t* __restrict__ q8, float* __restrict__ q_scale, int8_t* __restrict__ k8,
+    float* __restrict__ k_scale, float* __restrict__ k_mean, int qvec, int kvec) {
+    constexpr int RS = D + 8;                    // staging row stride (bf16), 16 B aligned
+    __shared__ __align__(16) uint16_t stage[kTile * RS];
+    __shared__ float mean_s[D];
+    __shared__ float wmax[4];
+
+    const bool isK = blockIdx.x >= (unsigned)n_qtiles;
+    const View4& x = isK ? k : q;
+    const int tile_lin = isK ? blockIdx.x - n_qtiles : blockIdx.x;
+    const int L = static_cast<int>(x.size[2]);
+    const int Hh = static_cast<int>(x.size[1]);
+    const int ntiles = static_cast<int>(ceil_div(L, kTile));
+    const int bh = tile_lin / ntiles, tl = tile_lin % ntiles;
+    const int b = bh / Hh, h = bh % Hh;
+    const int blk = isK ? blk_k : blk_q;
+    const int nb = static_cast<int>(ceil_div(L, blk));
+    const bool vec = (isK ? kvec : qvec) != 0;
+    const int tid = threadIdx.x;
+
+    if (isK && tid < D) {
+        const double* p = ksum + (int64_t)bh * kchunks * D + tid;
+        double s = p[0];
+        for (int c = 1; c < kchunks; ++c) s = __dadd_rn(s, p[(int64_t)c * D]);
+        const float m = __double2float_rn(__ddiv_rn(s, (double)L));
+        mean_s[tid] = m;
+        if (tl == 0 && k_mean != nullptr) k_mean[(int64_t)bh * D + tid] = m;
+    }
+
+    // coalesced staging of the 128 x D bf16 tile (rows beyond L are zero)
+    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
+    const int64_t hoff = b * x.stride[0] + h * x.stride[1];
+    for (int c = tid; c < kTile * (D / 8); c += 128) {
+        const int r = c / (D / 8), cc = c % (D / 8);
+        const int l = tl * kTile + r;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (l < L) u = load_row8(base, hoff + (int64_t)l * x.stride[2] + (int64_t)(cc * 8) * x.stride[3],
+                                 x.stride[3], vec);
+        *reinterpret_cast<uint4*>(&stage[r * RS + cc * 8]) = u;
+    }
+    __syncthreads();
+
+    const int l = tl * kTile + tid;
+    const bool valid = l < L;
+    float v[D];
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        float t8[8];
+        unpack8(*reinterpret_cast<const uint4*>(&stage[tid * RS + c * 8]), t8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[c * 8 + i] = t8[i];
+    }
+    if (isK && valid) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) v[d] = __fsub_rn(v[d], mean_s[d]);
+    }
+    butterfly<D>(v);
+
+    float a = 0.0f;
+#pragma unroll
+    for (int d = 0; d < D; ++d) a = fmaxf(a, fabsf(v[d]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    const int warp = tid >> 5;
+    if ((tid & 31) == 0) wmax[warp] = a;
+    __syncthreads();           // also: everyone finished reading `stage`
+    float amax;
+    if (blk == 32) amax = wmax[warp];
+    else if (blk == 64) amax = fmaxf(wmax[warp & ~1], wmax[warp | 1]);
+    else amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    float s = 0.0f, r = 0.0f;
+    if (amax != 0.0f) {
+        s = __fdiv_rn(amax, 127.0f);
+        r = __fdiv_rn(127.0f, amax);
+    }
+    if (valid && (l % blk) == 0) {
+        float* scales = isK ? k_scale : q_scale;
+        scales[(int64_t)bh * nb + l / blk] = s;
+    }
+
+    // codes -> byte staging (row stride D + 16 bytes) -> contiguous tile store
+    uint8_t* cst = reinterpret_cast<uint8_t*>(stage);
+    constexpr int CS = D + 16;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int bi = 0; bi < 4; ++bi) {
+                int code = __float2int_rn(__fmul_rn(v[c * 16 + wi * 4 + bi], r));
+                code = max(-127, min(127, code));
+                word |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * bi);
+            }
+            w[wi] = word;
+        }
+        *reinterpret_cast<uint4*>(&cst[tid * CS + c * 16]) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncthreads();
+    int8_t* dst = (isK ? k8 : q8) + ((int64_t)bh * ntiles * kTile + (int64_t)tl * kTile) * D;
+    for (int c = tid; c < kTile * (D / 16); c += 128) {
+        const int rr = c / (D / 16), cc = c % (D / 16);
+        *reinterpret_cast<uint4*>(dst + (int64_t)rr * D + cc * 16) =
+            *reinterpret_cast<const uint4*>(&cst[rr * CS + cc * 16]);
+    }
+}
+
+// ---------------------------------------------------------------- V e4m3
+// One CTA of 128 threads per (b, h, 128-token tile). Writes V transposed:
+// v8t[b, h, d, token].
+template <int D>
+__global__ void __launch_bounds__(128) v_quant_kernel(View4 x, const float* __restrict__ vmax,
+                                                      int vchunks, uint8_t* __restrict__ v8t,
+                                                      float* __restrict__ v_scale, int vec) {
+    constexpr int RS = D + 8;
+    constexpr int OS = kTile + 16;               // output staging row stride (bytes)
+    static_assert(D * OS <= kTile * RS * 2, "output staging reuses the input buffer");
+    __shared__ __align__(16) uint16_t stage[kTile * RS];
+    __shared__ float rmul[D];
+
+    const int L = static_cast<int>(x.size[2]);
+    const int Hh = static_cast<int>(x.size[1]);
+    const int ntiles = static_cast<int>(ceil_div(L, kTile));
+    const int bh = blockIdx.x / ntiles, tl = blockIdx.x % ntiles;
+    const int b = bh / Hh, h = bh % Hh;
+    const int tid = threadIdx.x;
+
+    if (tid < D) {
+        const float* p = vmax + (int64_t)bh * vchunks * D + tid;
+        float a = p[0];
+        for (int c = 1; c < vchunks; ++c) a = fmaxf(a, p[(int64_t)c * D]);
+        float s = 0.0f, r = 0.0f;
+        if (a != 0.0f) {
+            s = __fdiv_rn(a, 448.0f);
+            r = __fdiv_rn(448.0f, a);
+        }
+        rmul[tid] = r;
+        if (tl == 0) v_scale[(int64_t)bh * D + tid] = s;
+    }
+    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
+    const int64_t hoff = b * x.stride[0] + h * x.stride[1];
+    for (int c = tid; c < kTile * (D / 8); c += 128) {
+        const int r = c / (D / 8), cc = c % (D / 8);
+        const int l = tl * kTile + r;
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (l < L) u = load_row8(base, hoff + (int64_t)l * x.stride[2] + (int64_t)(cc * 8) * x.stride[3],
+                                 x.stride[3], vec != 0);
+        *reinterpret_cast<uint4*>(&stage[r * RS + cc * 8]) = u;
+    }
+    __syncthreads();
+    uint32_t w[kTile / 4];
+    if (tid < D) {
+        const float r = rmul[tid];
+#pragma unroll
+        for (int wi = 0; wi < kTile / 4; ++wi) {
+            float y[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                y[i] = __fmul_rn(bf16_bits_to_f32(stage[(wi * 4 + i) * RS + tid]), r);
+            const uint32_t lo = e4m3x2_rn_satfinite(y[0], y[1]);
+            const uint32_t hi = e4m3x2_rn_satfinite(y[2], y[3]);
+            w[wi] = lo | (hi << 16);
+        }
+    }
+    __syncthreads();
+    uint8_t* ost = reinterpret_cast<uint8_t*>(stage);
+    if (tid < D) {
+#pragma unroll
+        for (int c = 0; c < kTile / 16; ++c)
+            *reinterpret_cast<uint4*>(&ost[tid * OS + c * 16]) =
+                make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+    }
+    __syncthreads();
+    const int64_t Lpad = (int64_t)ntiles * kTile;
+    uint8_t* dst = v8t + (int64_t)bh * D * Lpad + (int64_t)tl * kTile;
+    for (int c = tid; c < D * (kTile / 16); c += 128) {
+        const int d = c / (kTile / 16), cc = c % (kTile / 16);
+        *reinterpret_cast<uint4*>(dst + (int64_t)d * Lpad + cc * 16) =
+            *reinterpret_cast<const uint4*>(&ost[d * OS + cc * 16]);
+    }
+}
+
+}  // namespace
+
+size_t quant_qk_ws_bytes(int B, int Hk, int Lk, int D) {
+    return (size_t)B * Hk * stat_chunks(Lk) * D * sizeof(double);
+}
+
+size_t quant_v_ws_bytes(int B, int Hk, int L, int D) {
+    return (size_t)B * Hk * stat_chunks(L) * D * sizeof(float);
+}
+
+cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
+                            float* q_scale, int8_t* k8, float* k_scale, float* k_mean, void* ws,
+                            cudaStream_t s) {
+    const int B = (int)q.size[0], H = (int)q.size[1], Lq = (int)q.size[2], D = (int)q.size[3];
+    const int Hk = (int)k.size[1], Lk = (int)k.size[2];
+    const int kchunks = stat_chunks(Lk);
+    const int kvec = view_vec8(k), qvec = view_vec8(q);
+    double* ksum = static_cast<double*>(ws);
+    const dim3 sgrid(kchunks, B * Hk);
+    const int n_qtiles = B * H * (int)ceil_div(Lq, kTile);
+    const int n_ktiles = B * Hk * (int)ceil_div(Lk, kTile);
+    if (D == 128) {
+        column_stats_kernel<128, 0><<<sgrid, 256, 0, s>>>(k, Lk, ksum, kvec);
+        qk_quant_kernel<128><<<n_qtiles + n_ktiles, 128, 0, s>>>(
+            q, k, blk_q, blk_k, n_qtiles, ksum, kchunks, q8, q_scale, k8, k_scale, k_mean, qvec, kvec);
+    } else {
+        column_stats_kernel<64, 0><<<sgrid, 256, 0, s>>>(k, Lk, ksum, kvec);
+        qk_quant_kernel<64><<<n_qtiles + n_ktiles, 128, 0, s>>>(
+            q, k, blk_q, blk_k, n_qtiles, ksum, kchunks, q8, q_scale, k8, k_scale, k_mean, qvec, kvec);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,
+                           cudaStream_t s) {
+    const int B = (int)v.size[0], Hk = (int)v.size[1], L = (int)v.size[2], D = (int)v.size[3];
+    const int chunks = stat_chunks(L);
+    const int vec = view_vec8(v);
+    float* vmax = static_cast<float*>(ws);
+    const dim3 sgrid(chunks, B * Hk);
+    const int ntiles = B * Hk * (int)ceil_div(L, kTile);
+    if (D == 128) {
+        column_stats_kernel<128, 1><<<sgrid, 256, 0, s>>>(v, L, vmax, vec);
+        v_quant_kernel<128><<<ntiles, 128, 0, s>>>(v, vmax, chunks, v8t, v_scale, vec);
+    } else {
+        column_stats_kernel<64, 1><<<sgrid, 256, 0, s>>>(v, L, vmax, vec);
+        v_quant_kernel<64><<<ntiles, 128, 0, s>>>(v, vmax, chunks, v8t, v_scale, vec);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace sage

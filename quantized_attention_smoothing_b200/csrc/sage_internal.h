@@ -1,0 +1,84 @@
+// sage_internal.h -- declarations shared between the C-ABI layer and the
+// kernel translation units of libsage. Not installed, not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace sage {
+
+// Plain copy of a caller's view (element sizes / strides), passed by value
+// to kernels.
+struct View4 {
+    const void* ptr;
+    int64_t size[4];
+    int64_t stride[4];
+};
+
+// 16-byte vector access is possible: unit innermost stride, the other
+// strides multiples of 8 elements, 16-byte aligned base.
+inline bool view_vec8(const View4& v) {
+    return v.stride[3] == 1 && (v.stride[0] % 8) == 0 && (v.stride[1] % 8) == 0 &&
+           (v.stride[2] % 8) == 0 && (reinterpret_cast<uintptr_t>(v.ptr) % 16) == 0;
+}
+
+constexpr int kTile = 128;                  // token tile of every kernel
+constexpr unsigned kErrTimeoutCode = 1u;    // low byte of a device error word
+constexpr int kStatRows = 512;              // tokens per statistics chunk
+
+__host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+__host__ __device__ inline int64_t ceil_div(int64_t x, int64_t m) { return (x + m - 1) / m; }
+inline int stat_chunks(int L) { return static_cast<int>(ceil_div(L, kStatRows)); }
+
+// ---- quantisation (quant.cu)
+size_t quant_qk_ws_bytes(int B, int Hk, int Lk, int D);
+size_t quant_v_ws_bytes(int B, int Hk, int L, int D);
+cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
+                            float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
+                            void* ws, cudaStream_t s);
+cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,
+                           cudaStream_t s);
+
+// ---- attention forward (attn_fwd.cu)
+struct AttnArgs {
+    const int8_t* q8;
+    const float* q_scale;
+    const int8_t* k8;
+    const float* k_scale;
+    const uint8_t* v8t;
+    const float* v_scale;
+    int B, H, Hk, Lq, Lk, D, blk_q, blk_k;
+    float softmax_scale;
+    int causal;
+    void* out;
+    int64_t out_size[4];
+    int64_t out_stride[4];
+};
+cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s);
+unsigned read_clear_attn_error();
+
+// ---- decode (decode.cu)
+struct DecodeArgs {
+    View4 q;                   // [B, T, H, D] bf16
+    const uint8_t* k_cache;
+    const uint8_t* v_cache;
+    const float* k_scale;
+    const float* v_scale;
+    const int32_t* page_table;
+    const int32_t* ctx_lens;
+    int B, T, H, Hk, D, page_size, max_pages, num_pages, window;
+    float softmax_scale;
+    void* out;
+    int64_t out_stride[4];
+    void* ws;
+};
+size_t decode_ws_bytes(int B, int T, int H, int Hk, int D, int window);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+unsigned read_clear_decode_error();
+
+// ---- driver entry point for tensor-map encoding (sage_api.cu)
+void* tensor_map_encoder();
+
+}  // namespace sage

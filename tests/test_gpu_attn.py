@@ -1,0 +1,109 @@
+"""GPU parity of the quantised attention forward (tcgen05 kernel) against
+the CPU oracle. Element-wise on small shapes spanning several 128-key tiles
+with ragged tails, causal masks (bottom-right aligned), GQA, both head dims
+and all block sizes; on sampled rows at the full workload sizes. The oracle
+quantises the original inputs itself (nothing it uses comes from the GPU)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_smoothing_b200 as sage
+import workloads
+from gpu_helpers import bits, compare_output, sample_rows, to_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def handles():
+    from quantized_attention_smoothing_b200 import build
+    build.build()
+    return {64: sage.Hadamard(64), 128: sage.Hadamard(128)}
+
+
+def _run(handles, q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True):
+    D = q.shape[3]
+    out, _ = sage.sage_attention(handles[D], to_gpu(q), to_gpu(k), to_gpu(v), blk_q, blk_k, scale,
+                                 causal)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    gpu = bits(out)                                     # [B, H, Lq, D]
+    qk = oracle.quant_qk(bits(q), bits(k), blk_q, blk_k)
+    v8t, vs = oracle.quant_v(bits(v))
+    _, ref = oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, q.shape[2], k.shape[2],
+                         blk_q, blk_k, scale, causal, rows=rows, want_f64=True)
+    ex = oracle.attn_exact(bits(q), bits(k), bits(v), scale, causal, rows=rows) if exact else None
+    if rows is not None:
+        gpu = gpu[:, :, rows]
+    return gpu, ref, ex
+
+
+SHAPES = [
+    # B, H, Hk, Lq, Lk, D, blk_q, blk_k, causal
+    (1, 2, 2, 256, 256, 64, 64, 64, False),          # the small config
+    (1, 2, 2, 300, 300, 128, 128, 64, False),        # ragged tail
+    (1, 2, 2, 383, 383, 128, 128, 64, True),         # causal, ragged
+    (2, 4, 2, 257, 513, 64, 64, 32, False),          # GQA, Lq != Lk
+    (1, 2, 1, 129, 1000, 128, 128, 128, True),       # causal with Lq < Lk
+    (1, 1, 1, 500, 130, 64, 64, 64, True),           # causal with Lq > Lk: early rows see nothing
+    (1, 1, 1, 1, 1, 128, 32, 32, False),             # single token
+    (1, 3, 3, 640, 640, 128, 64, 128, False),        # 5 key tiles, 3 CTAs (odd q-tile count)
+]
+
+
+@pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,blk_q,blk_k,causal", SHAPES)
+def test_attn_matches_oracle_elementwise(handles, B, H, Hk, Lq, Lk, D, blk_q, blk_k, causal):
+    g = torch.Generator().manual_seed(Lq * 31 + Lk + D)
+    q = torch.randn((B, Lq, H, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    k = (torch.randn((B, Lk, Hk, D), generator=g) + torch.randn((B, 1, Hk, D), generator=g) * 2)
+    k = k.to(torch.bfloat16).permute(0, 2, 1, 3)
+    v = torch.randn((B, Lk, Hk, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    scale = 1.0 / math.sqrt(D)
+    gpu, ref, ex = _run(handles, q, k, v, blk_q, blk_k, scale, causal)
+    compare_output(gpu, ref, ex, label=str((B, H, Hk, Lq, Lk, D, causal)))
+    if causal and Lq > Lk:
+        assert (gpu[:, :, :Lq - Lk] == 0).all()
+
+
+def test_attn_c1_config(handles):
+    cfg, q, k, v = workloads.make_prefill_config("c1")
+    gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
+                        cfg["causal"])
+    compare_output(gpu, ref, ex, label="c1")
+
+
+def test_attn_output_strides(handles):
+    """Contiguous [B,H,L,D] output, the [B,L,H,D] view, and a scalar-path view."""
+    q, k, v = workloads.make_prefill(B=1, H=2, Hk=2, L=300, D=128, seed=8, kbias_std=2.0)
+    h = handles[128]
+    qg, kg, vg = to_gpu(q), to_gpu(k), to_gpu(v)
+    outs = []
+    o1 = torch.empty((1, 2, 300, 128), dtype=torch.bfloat16, device="cuda")
+    o2 = torch.empty((1, 300, 2, 128), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
+    o3 = torch.empty((1, 2, 300, 131), dtype=torch.bfloat16, device="cuda")[..., :128]
+    for o in (o1, o2, o3):
+        sage.sage_attention(h, qg, kg, vg, 128, 64, 0.1, False, out=o)
+        outs.append(o.contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+def test_attn_deterministic(handles):
+    cfg, q, k, v = workloads.make_prefill_config("c1")
+    h = handles[64]
+    a, _ = sage.sage_attention(h, to_gpu(q), to_gpu(k), to_gpu(v), 64, 64, 0.125, False)
+    b, _ = sage.sage_attention(h, to_gpu(q), to_gpu(k), to_gpu(v), 64, 64, 0.125, False)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("key,nrows", [("c2", 24), ("c3", 8), ("c4", 4)])
+def test_attn_full_size_sampled_rows(handles, key, nrows):
+    cfg, q, k, v = workloads.make_prefill_config(key)
+    rows = sample_rows(cfg["L"], nrows, seed=cfg["H"])
+    gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
+                        cfg["causal"], rows=rows, exact=True)
+    compare_output(gpu, ref, ex, label=key)
