@@ -28,6 +28,8 @@
 // Every mbarrier wait is bounded (see mbar_wait): on timeout the CTA records
 // an error word, raises a CTA-wide abort flag, drains its own MMAs and
 // returns.
+#include <climits>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -44,6 +46,9 @@ constexpr int BN = 128;          // keys per tile
 constexpr int QT = 2;            // query tiles per CTA
 constexpr int kThreads = 320;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;   // log2(FP8_MAX of e4m3)
+constexpr int kMagicI = 0x4B400000;               // bit pattern of 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;            // 1.5 * 2^23
 
 template <int D>
 struct Cfg {
@@ -93,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const Params p) {
     using C = Cfg<D>;
+    constexpr int kKeysPerBlk = BN / NKB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -240,6 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sP = smem + C::kOffP + w * C::kPBytes;
         const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
 
+        float ks_next[NKB];
+#pragma unroll
+        for (int kb = 0; kb < NKB; ++kb)
+            ks_next[kb] = __ldg(&ksrow[min((kb * kKeysPerBlk) / p.blk_k, p.nbk - 1)]);
         float m = -INFINITY, dsum = 0.0f;
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
@@ -256,66 +266,119 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
 
             const int j0 = t * BN;
+            // tiles that reach past this row's last visible key need masking
+            const bool need_mask = __any_sync(0xffffffffu, j0 + BN - 1 > jlim);
             float ksc[NKB];
 #pragma unroll
             for (int kb = 0; kb < NKB; ++kb) {
-                const int bi = min((j0 + kb * (BN / NKB)) / p.blk_k, p.nbk - 1);
-                ksc[kb] = __ldg(&ksrow[bi]) * arow;
+                ksc[kb] = ks_next[kb] * arow;
+                // prefetch the next tile's key-block scales
+                const int bi = min((j0 + BN + kb * kKeysPerBlk) / p.blk_k, p.nbk - 1);
+                ks_next[kb] = __ldg(&ksrow[bi]);
             }
-            // QK: dequantised base-2 logits, masked; row max
+            // QK, update_mdo (max part): the logit y = acc * ksc is monotonic in
+            // the integer accumulator (ksc >= 0), so the row max is taken on
+            // the raw int32 values of each key block, in 8 independent chains.
             float mt = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const float acc = static_cast<float>(static_cast<int>(sv[c / 32][c % 32]));
-                float y = acc * ksc[c / (BN / NKB)];
-                y = (j0 + c <= jlim) ? y : -INFINITY;
-                sv[c / 32][c % 32] = __float_as_uint(y);
-                mt = fmaxf(mt, y);
+            for (int kb = 0; kb < NKB; ++kb) {
+                int mx[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) mx[u] = INT_MIN;
+#pragma unroll
+                for (int c = 0; c < kKeysPerBlk; ++c) {
+                    const int col = kb * kKeysPerBlk + c;
+                    int a = static_cast<int>(sv[col / 32][col % 32]);
+                    if (need_mask) a = (j0 + col <= jlim) ? a : INT_MIN;
+                    mx[c % 8] = max(mx[c % 8], a);
+                }
+                const int kmx = max(max(max(mx[0], mx[1]), max(mx[2], mx[3])),
+                                    max(max(mx[4], mx[5]), max(mx[6], mx[7])));
+                if (kmx != INT_MIN) mt = fmaxf(mt, static_cast<float>(kmx) * ksc[kb]);
             }
-            // update_mdo (max part), accumulate_d, RS_32_to_8
             const float m_new = fmaxf(m, mt);
             const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
             const float alpha = ex2_approx(m - msub);
-            float rowsum = 0.0f;
-            uint32_t pk[BN / 4];
-#pragma unroll
-            for (int c = 0; c < BN; c += 4) {
-                float e[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    e[k] = ex2_approx(__uint_as_float(sv[(c + k) / 32][(c + k) % 32]) - msub);
-                    rowsum += e[k];
-                }
-                const uint32_t lo = e4m3x2_rn_satfinite(e[0] * 448.0f, e[1] * 448.0f);
-                const uint32_t hi = e4m3x2_rn_satfinite(e[2] * 448.0f, e[3] * 448.0f);
-                pk[c / 4] = lo | (hi << 16);
-            }
-            dsum = dsum * alpha + rowsum;
-
             if (t > 0) {
                 // PV(t-1) must be complete before O is rescaled and P is overwritten
                 ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (t - 1) & 1, abort_flag,
                                         &g_attn_err, 10));
                 if (!ok) break;
                 tc_fence_after();
+            }
+            // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m'). The int32
+            // accumulator becomes fp32 exactly through the 1.5 * 2^23 bias
+            // (|acc| < 2^21): float(acc) = as_float(acc + bias) - 1.5 * 2^23;
+            // then one FMA per element: arg = float(acc) * ksc + (log2(448) - m').
+            // Pairs of keys share a key block, so both steps run as f32x2.
+            // Each 16-key chunk of P8 goes straight to shared memory in the
+            // 128B-swizzled K-major layout (chunk c of row r at c ^ (r & 7)).
+            uint64_t ksc2[NKB];
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) ksc2[kb] = f2_pack(ksc[kb], ksc[kb]);
+            const float cofs = kLog2_448 - msub;
+            const uint64_t cofs2 = f2_pack(cofs, cofs);
+            const uint64_t nmag2 = f2_pack(-kMagicF, -kMagicF);
+            uint64_t acc2[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int ch = 0; ch < BN / 16; ++ch) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int c = ch * 16 + q4 * 4;
+                    float e[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k += 2) {
+                        const int col = c + k;
+                        const float f0 = __int_as_float(static_cast<int>(sv[col / 32][col % 32]) + kMagicI);
+                        const float f1 = __int_as_float(static_cast<int>(sv[(col + 1) / 32][(col + 1) % 32]) + kMagicI);
+                        const uint64_t x2 = f2_add(f2_pack(f0, f1), nmag2);
+                        float a0, a1;
+                        f2_unpack(f2_fma(x2, ksc2[col / kKeysPerBlk], cofs2), a0, a1);
+                        if (need_mask) {
+                            a0 = (j0 + col <= jlim) ? a0 : -INFINITY;
+                            a1 = (j0 + col + 1 <= jlim) ? a1 : -INFINITY;
+                        }
+                        e[k] = ex2_approx(a0);
+                        e[k + 1] = ex2_approx(a1);
+                    }
+                    acc2[q4] = f2_add(acc2[q4], f2_add(f2_pack(e[0], e[1]), f2_pack(e[2], e[3])));
+                    const uint32_t lo = e4m3x2_rn_satfinite(e[0], e[1]);
+                    const uint32_t hi = e4m3x2_rn_satfinite(e[2], e[3]);
+                    pk[q4] = lo | (hi << 16);
+                }
+                *reinterpret_cast<uint4*>(sP + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            {
+                const uint64_t a01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+                float r0, r1;
+                f2_unpack(a01, r0, r1);
+                dsum = dsum * alpha + (r0 + r1);
+            }
+            if (t > 0) {
+                // update_mdo (rescale part): O *= alpha, skipped when no row of the
+                // warp changed its max (alpha == 1 exactly)
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                    const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         uint32_t o[32];
                         tmem_ld32(lane_addr + o_col + 32 * c4, o);
                         tmem_wait_ld(o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        for (int e = 0; e < 32; e += 2) {
+                            float x0, x1;
+                            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2),
+                                      x0, x1);
+                            o[e] = __float_as_uint(x0);
+                            o[e + 1] = __float_as_uint(x1);
+                        }
                         tmem_st32(lane_addr + o_col + 32 * c4, o);
                     }
                     tmem_wait_st();
                 }
             }
-            // P8 row -> shared memory, 128B swizzle (16-byte chunk c of row r at c ^ (r & 7))
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(sP + r * 128 + ((ch ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -331,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     &g_attn_err, 11));
             if (ok) {
                 tc_fence_after();
-                const float inv = dsum > 0.0f ? 1.0f / (448.0f * dsum) : 0.0f;
+                const float inv = dsum > 0.0f ? 1.0f / dsum : 0.0f;     // dsum carries the 448
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];

@@ -79,13 +79,23 @@ __global__ void __launch_bounds__(256) column_stats_kernel(View4 x, int L, void*
     Acc acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = Acc(0);
-    for (int l = l0 + rg; l < l1; l += RPI) {
-        float v[8];
-        unpack8(load_row8(base, row0 + (int64_t)l * x.stride[2], x.stride[3], vec != 0), v);
+    for (int l = l0 + rg; l < l1; l += 4 * RPI) {
+        uint4 u[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (MODE == 0) acc[i] = __dadd_rn(acc[i], (double)v[i]);
-            else acc[i] = fmaxf(acc[i], fabsf(v[i]));
+        for (int k = 0; k < 4; ++k) {
+            const int ll = l + k * RPI;
+            u[k] = ll < l1 ? load_row8(base, row0 + (int64_t)ll * x.stride[2], x.stride[3], vec != 0)
+                           : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float v[8];
+            unpack8(u[k], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (MODE == 0) acc[i] = __dadd_rn(acc[i], (double)v[i]);
+                else acc[i] = fmaxf(acc[i], fabsf(v[i]));
+            }
         }
     }
 #pragma unroll
@@ -118,16 +128,22 @@ __device__ __forceinline__ void butterfly(float (&x)[D]) {
 }
 
 // ---------------------------------------------------------------- Q/K int8
-// One CTA of 128 threads per (tensor, b, h, 128-token tile); thread = token.
+// One CTA per (tensor, b, h, 128-token tile); D/32 threads per token, each
+// holding 32 consecutive channels. The butterfly stages h < 32 run inside a
+// thread; h = 32 and h = 64 pair lanes (lane ^ 1, lane ^ 2) and every output
+// is still the single fp32 add (lower + upper) or subtract (lower - upper)
+// of the same two values as in a sequential evaluation.
 template <int D>
-__global__ void __launch_bounds__(128) qk_quant_kernel(
+__global__ void __launch_bounds__(kTile * (D / 32)) qk_quant_kernel(
     View4 q, View4 k, int blk_q, int blk_k, int n_qtiles, const double* __restrict__ ksum,
     int kchunks, int8_t* __restrict__ q8, float* __restrict__ q_scale, int8_t* __restrict__ k8,
     float* __restrict__ k_scale, float* __restrict__ k_mean, int qvec, int kvec) {
-    constexpr int RS = D + 8;                    // staging row stride (bf16), 16 B aligned
-    __shared__ __align__(16) uint16_t stage[kTile * RS];
+    constexpr int TPR = D / 32;                   // threads per token row
+    constexpr int NT = kTile * TPR;
+    constexpr int NW = NT / 32;                   // warps
+    constexpr int RPW = 32 / TPR;                 // rows per warp
     __shared__ float mean_s[D];
-    __shared__ float wmax[4];
+    __shared__ float wmax[NW];
 
     const bool isK = blockIdx.x >= (unsigned)n_qtiles;
     const View4& x = isK ? k : q;
@@ -141,93 +157,89 @@ __global__ void __launch_bounds__(128) qk_quant_kernel(
     const int nb = static_cast<int>(ceil_div(L, blk));
     const bool vec = (isK ? kvec : qvec) != 0;
     const int tid = threadIdx.x;
+    const int r = tid / TPR, c = tid % TPR;
+    const int l = tl * kTile + r;
+    const bool valid = l < L;
+
+    // issue the row loads first (32 channels = 64 bytes per thread)
+    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
+    const int64_t off = b * x.stride[0] + h * x.stride[1] + (int64_t)l * x.stride[2] +
+                        (int64_t)(32 * c) * x.stride[3];
+    uint4 raw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        raw[i] = valid ? load_row8(base, off + (int64_t)(8 * i) * x.stride[3], x.stride[3], vec)
+                       : make_uint4(0, 0, 0, 0);
 
     if (isK && tid < D) {
         const double* p = ksum + (int64_t)bh * kchunks * D + tid;
         double s = p[0];
-        for (int c = 1; c < kchunks; ++c) s = __dadd_rn(s, p[(int64_t)c * D]);
+        for (int ch = 1; ch < kchunks; ++ch) s = __dadd_rn(s, p[(int64_t)ch * D]);
         const float m = __double2float_rn(__ddiv_rn(s, (double)L));
         mean_s[tid] = m;
         if (tl == 0 && k_mean != nullptr) k_mean[(int64_t)bh * D + tid] = m;
     }
-
-    // coalesced staging of the 128 x D bf16 tile (rows beyond L are zero)
-    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
-    const int64_t hoff = b * x.stride[0] + h * x.stride[1];
-    for (int c = tid; c < kTile * (D / 8); c += 128) {
-        const int r = c / (D / 8), cc = c % (D / 8);
-        const int l = tl * kTile + r;
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (l < L) u = load_row8(base, hoff + (int64_t)l * x.stride[2] + (int64_t)(cc * 8) * x.stride[3],
-                                 x.stride[3], vec);
-        *reinterpret_cast<uint4*>(&stage[r * RS + cc * 8]) = u;
-    }
     __syncthreads();
 
-    const int l = tl * kTile + tid;
-    const bool valid = l < L;
-    float v[D];
+    float v[32];
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
+    for (int i = 0; i < 4; ++i) {
         float t8[8];
-        unpack8(*reinterpret_cast<const uint4*>(&stage[tid * RS + c * 8]), t8);
+        unpack8(raw[i], t8);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[c * 8 + i] = t8[i];
+        for (int j = 0; j < 8; ++j) v[8 * i + j] = t8[j];
     }
     if (isK && valid) {
 #pragma unroll
-        for (int d = 0; d < D; ++d) v[d] = __fsub_rn(v[d], mean_s[d]);
+        for (int j = 0; j < 32; ++j) v[j] = __fsub_rn(v[j], mean_s[32 * c + j]);
     }
-    butterfly<D>(v);
+    butterfly<32>(v);
+#pragma unroll
+    for (int hb = 1; hb < TPR; hb <<= 1) {       // stages h = 32 * hb across lanes
+        const bool upper = (c & hb) != 0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[j], hb);
+            v[j] = upper ? __fsub_rn(o, v[j]) : __fadd_rn(v[j], o);
+        }
+    }
 
     float a = 0.0f;
 #pragma unroll
-    for (int d = 0; d < D; ++d) a = fmaxf(a, fabsf(v[d]));
+    for (int j = 0; j < 32; ++j) a = fmaxf(a, fabsf(v[j]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     const int warp = tid >> 5;
     if ((tid & 31) == 0) wmax[warp] = a;
-    __syncthreads();           // also: everyone finished reading `stage`
-    float amax;
-    if (blk == 32) amax = wmax[warp];
-    else if (blk == 64) amax = fmaxf(wmax[warp & ~1], wmax[warp | 1]);
-    else amax = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    float s = 0.0f, r = 0.0f;
+    __syncthreads();
+    const int wpb = max(1, blk / RPW);            // warps per quantisation block
+    const int w0 = (warp / wpb) * wpb;
+    float amax = 0.0f;
+    for (int w = w0; w < w0 + wpb; ++w) amax = fmaxf(amax, wmax[w]);
+    float s = 0.0f, rr = 0.0f;
     if (amax != 0.0f) {
         s = __fdiv_rn(amax, 127.0f);
-        r = __fdiv_rn(127.0f, amax);
+        rr = __fdiv_rn(127.0f, amax);
     }
-    if (valid && (l % blk) == 0) {
+    if (valid && c == 0 && (l % blk) == 0) {
         float* scales = isK ? k_scale : q_scale;
         scales[(int64_t)bh * nb + l / blk] = s;
     }
-
-    // codes -> byte staging (row stride D + 16 bytes) -> contiguous tile store
-    uint8_t* cst = reinterpret_cast<uint8_t*>(stage);
-    constexpr int CS = D + 16;
+    uint32_t w[8];
 #pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-        uint32_t w[4];
+    for (int wi = 0; wi < 8; ++wi) {
+        uint32_t word = 0;
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int bi = 0; bi < 4; ++bi) {
-                int code = __float2int_rn(__fmul_rn(v[c * 16 + wi * 4 + bi], r));
-                code = max(-127, min(127, code));
-                word |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * bi);
-            }
-            w[wi] = word;
+        for (int bi = 0; bi < 4; ++bi) {
+            int code = __float2int_rn(__fmul_rn(v[4 * wi + bi], rr));
+            code = max(-127, min(127, code));
+            word |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * bi);
         }
-        *reinterpret_cast<uint4*>(&cst[tid * CS + c * 16]) = make_uint4(w[0], w[1], w[2], w[3]);
+        w[wi] = word;
     }
-    __syncthreads();
-    int8_t* dst = (isK ? k8 : q8) + ((int64_t)bh * ntiles * kTile + (int64_t)tl * kTile) * D;
-    for (int c = tid; c < kTile * (D / 16); c += 128) {
-        const int rr = c / (D / 16), cc = c % (D / 16);
-        *reinterpret_cast<uint4*>(dst + (int64_t)rr * D + cc * 16) =
-            *reinterpret_cast<const uint4*>(&cst[rr * CS + cc * 16]);
-    }
+    int8_t* dst = (isK ? k8 : q8) + ((int64_t)bh * ntiles * kTile + l) * D + 32 * c;
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
 }
 
 // ---------------------------------------------------------------- V e4m3
@@ -328,11 +340,11 @@ cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k
     const int n_ktiles = B * Hk * (int)ceil_div(Lk, kTile);
     if (D == 128) {
         column_stats_kernel<128, 0><<<sgrid, 256, 0, s>>>(k, Lk, ksum, kvec);
-        qk_quant_kernel<128><<<n_qtiles + n_ktiles, 128, 0, s>>>(
+        qk_quant_kernel<128><<<n_qtiles + n_ktiles, kTile * 4, 0, s>>>(
             q, k, blk_q, blk_k, n_qtiles, ksum, kchunks, q8, q_scale, k8, k_scale, k_mean, qvec, kvec);
     } else {
         column_stats_kernel<64, 0><<<sgrid, 256, 0, s>>>(k, Lk, ksum, kvec);
-        qk_quant_kernel<64><<<n_qtiles + n_ktiles, 128, 0, s>>>(
+        qk_quant_kernel<64><<<n_qtiles + n_ktiles, kTile * 2, 0, s>>>(
             q, k, blk_q, blk_k, n_qtiles, ksum, kchunks, q8, q_scale, k8, k_scale, k_mean, qvec, kvec);
     }
     return cudaGetLastError();
