@@ -41,6 +41,20 @@ namespace {
 
 __device__ unsigned g_attn_err;
 
+#ifdef SAGE_ATTN_TRACE
+// Development-only phase timestamps (clock64) of CTA (0, 0): rows 0/1 are
+// softmax warps 0 and 4 (lane 0), row 2 the MMA thread; 16 tiles x 12 marks.
+__device__ long long g_attn_trace[3][16][12];
+#define SAGE_MARK(row, t, k)                                                         \
+    do {                                                                             \
+        if (trace_on && (t) < 16) g_attn_trace[row][t][k] = clock64();               \
+    } while (0)
+#else
+#define SAGE_MARK(row, t, k) \
+    do {                     \
+    } while (0)
+#endif
+
 constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;          // keys per tile
 constexpr int QT = 2;            // query tiles per CTA
@@ -49,6 +63,16 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(FP8_MAX of e4m3)
 constexpr int kMagicI = 0x4B400000;               // bit pattern of 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;            // 1.5 * 2^23
+// every kPolyEvery-th key pair takes its exponential from exp2_poly_x2
+// instead of the MUFU unit (0 = never)
+#ifndef SAGE_POLY_EVERY
+#define SAGE_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = SAGE_POLY_EVERY;
+
+// K block scales of one head staged in shared memory (larger heads read the
+// rest from global memory)
+constexpr int kKsSmem = 1024;
 
 template <int D>
 struct Cfg {
@@ -74,7 +98,8 @@ struct Cfg {
     static constexpr int kBarFinal = kBarODone + QT;
     static constexpr int kNumBars = kBarFinal + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + runtime 1024-B alignment
+    static constexpr int kOffKs = kOffMisc + 16;             // K block scales of the head
+    static constexpr int kSmemBytes = kOffKs + kKsSmem * 4 + 1024;  // + runtime alignment
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -86,6 +111,7 @@ struct Params {
     __nv_bfloat16* out;
     int64_t os0, os1, os2, os3;
     int H, Hk, Lq, Lk, LpadQ, LpadK, blk_q, blk_k, nbq, nbk;
+    int lg_blk_q, lg_blk_k;        // log2 of the (power-of-two) block sizes
     float logit_scale_log2;        // softmax_scale / D * log2(e)
     int heavy_first;
     int out_vec;
@@ -126,6 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         kv_end = max(0, min(kv_end, lim));
     }
     const int n_tiles = (kv_end + BN - 1) / BN;
+#ifdef SAGE_ATTN_TRACE
+    const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0;
+#endif
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
@@ -139,6 +168,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 9) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
+    }
+    float* ks_s = reinterpret_cast<float*>(smem + C::kOffKs);
+    {
+        const float* ksrc = p.k_scale + (int64_t)bhk * p.nbk;
+        const int nks = min(p.nbk, kKsSmem);
+        for (int i = threadIdx.x; i < nks; i += kThreads) ks_s[i] = __ldg(&ksrc[i]);
     }
     tc_fence_before();
     __syncthreads();
@@ -204,26 +239,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = 0; ok && t < n_tiles; ++t) {
                 const int s = t % C::kStages;
                 const uint32_t ph = (t / C::kStages) & 1;
+                SAGE_MARK(2, t, 0);
                 if (!(ok = mbar_wait(&bars[C::kBarKFull + s], ph, abort_flag, &g_attn_err, 6))) break;
+                SAGE_MARK(2, t, 1);
                 tc_fence_after();
                 const uint64_t kdesc = umma_desc_kmajor(sK + s * C::kKBytes, D);
                 for (int w = 0; w < QT && ok; ++w) {
-                    if (t > 0) {
-                        ok = mbar_wait(&bars[C::kBarSEmpty + w], (t - 1) & 1, abort_flag,
-                                       &g_attn_err, 7);
-                        if (!ok) break;
-                        tc_fence_after();
-                    }
+                    // S_w holds the 1.5 * 2^23 bias (written by the softmax warps
+                    // after their last read, phase t of s_empty); the MMA adds onto it
+                    ok = mbar_wait(&bars[C::kBarSEmpty + w], t & 1, abort_flag, &g_attn_err, 7);
+                    if (!ok) break;
+                    tc_fence_after();
                     const uint64_t qdesc = umma_desc_kmajor(sQ + w * C::kQBytes, D);
 #pragma unroll
                     for (int kk = 0; kk < D / 32; ++kk)
-                        mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK,
-                                  kk > 0 ? 1u : 0u);
+                        mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, 1u);
                     mma_commit(&bars[C::kBarSFull + w]);
+                    SAGE_MARK(2, t, 2 + w);
                 }
                 if (!ok) break;
                 mma_commit(&bars[C::kBarKEmpty + s]);
                 if (t > 0) ok = issue_pv(t - 1);
+                SAGE_MARK(2, t, 4);
             }
             if (ok) issue_pv(n_tiles - 1);
             // drain every MMA this thread issued before TMEM is released
@@ -239,152 +276,177 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(ww * 32) << 16);
         const uint32_t s_col = w * BN;
         const uint32_t o_col = 256 + w * BM;
-        const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + i / p.blk_q]) : 0.0f;
+        const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + (i >> p.lg_blk_q)]) : 0.0f;
         const float arow = qsc * p.logit_scale_log2;
         int jlim = valid ? p.Lk - 1 : -1;
         if (CAUSAL && valid) jlim = min(jlim, i + (p.Lk - p.Lq));
         uint8_t* sP = smem + C::kOffP + w * C::kPBytes;
         const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
 
-        float ks_next[NKB];
-#pragma unroll
-        for (int kb = 0; kb < NKB; ++kb)
-            ks_next[kb] = __ldg(&ksrow[min((kb * kKeysPerBlk) / p.blk_k, p.nbk - 1)]);
+        // S_w starts as the bias 1.5 * 2^23 in every column: int32 accumulation
+        // onto it leaves bits that read directly as the fp32 value 1.5 * 2^23 +
+        // acc (exact, |acc| < 2^21)
+#pragma unroll 1
+        for (int ch = 0; ch < BN / 32; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
+
         float m = -INFINITY, dsum = 0.0f;
         bool ok = true;
+#ifdef SAGE_ATTN_TRACE
+        const bool tr = trace_on && lane == 0 && ww == 0;
+#define SMARK(k) SAGE_MARK(w, t, k)
+#define trace_on tr
+#else
+#define SMARK(k)
+#endif
+        // The score tile is read from TMEM twice, 32 columns at a time: pass 1
+        // takes the row max, pass 2 the exponentials. Rolled loops keep the
+        // code small (instruction-cache resident) and the live state at one
+        // 32-column chunk.
         for (int t = 0; t < n_tiles; ++t) {
+            SMARK(0);
             ok = warp_all(mbar_wait(&bars[C::kBarSFull + w], t & 1, abort_flag, &g_attn_err, 9));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[4][32];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(lane_addr + s_col + 32 * c4, sv[c4]);
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_wait_ld(sv[c4]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
-
+            SMARK(1);
             const int j0 = t * BN;
             // tiles that reach past this row's last visible key need masking
             const bool need_mask = __any_sync(0xffffffffu, j0 + BN - 1 > jlim);
-            float ksc[NKB];
-#pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) {
-                ksc[kb] = ks_next[kb] * arow;
-                // prefetch the next tile's key-block scales
-                const int bi = min((j0 + BN + kb * kKeysPerBlk) / p.blk_k, p.nbk - 1);
-                ks_next[kb] = __ldg(&ksrow[bi]);
-            }
-            // QK, update_mdo (max part): the logit y = acc * ksc is monotonic in
-            // the integer accumulator (ksc >= 0), so the row max is taken on
-            // the raw int32 values of each key block, in 8 independent chains.
+            SMARK(2);
+
+            // QK and update_mdo (max part). The biased accumulators are fp32
+            // values 1.5 * 2^23 + acc (exact); y = acc * ksc is monotonic in acc
+            // (ksc >= 0), so each 32-key chunk's max is taken on the raw values
+            // (three-input max) and unbiased and scaled once.
             float mt = -INFINITY;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + s_col + 32 * ch, v);
+                tmem_wait_ld(v);
+                SMARK(8 + ch);
+                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) {
-                int mx[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) mx[u] = INT_MIN;
-#pragma unroll
-                for (int c = 0; c < kKeysPerBlk; ++c) {
-                    const int col = kb * kKeysPerBlk + c;
-                    int a = static_cast<int>(sv[col / 32][col % 32]);
-                    if (need_mask) a = (j0 + col <= jlim) ? a : INT_MIN;
-                    mx[c % 8] = max(mx[c % 8], a);
+                for (int i = 0; i < 16; ++i) {
+                    float x0 = __uint_as_float(v[2 * i]);
+                    float x1 = __uint_as_float(v[2 * i + 1]);
+                    if (need_mask) {
+                        const int jc = j0 + 32 * ch + 2 * i;
+                        x0 = (jc <= jlim) ? x0 : -INFINITY;
+                        x1 = (jc + 1 <= jlim) ? x1 : -INFINITY;
+                    }
+                    mx[i & 3] = fmax3(mx[i & 3], x0, x1);
                 }
-                const int kmx = max(max(max(mx[0], mx[1]), max(mx[2], mx[3])),
-                                    max(max(mx[4], mx[5]), max(mx[6], mx[7])));
-                if (kmx != INT_MIN) mt = fmaxf(mt, static_cast<float>(kmx) * ksc[kb]);
+                const float cm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                const int bi = min((j0 + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
+                const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
+                if (cm != -INFINITY) mt = fmaxf(mt, (cm - kMagicF) * kc);
             }
             const float m_new = fmaxf(m, mt);
             const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
             const float alpha = ex2_approx(m - msub);
+            SMARK(3);
             if (t > 0) {
-                // PV(t-1) must be complete before O is rescaled and P is overwritten
+                // PV(t-1) must be complete before P is overwritten and O rescaled
                 ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (t - 1) & 1, abort_flag,
                                         &g_attn_err, 10));
                 if (!ok) break;
                 tc_fence_after();
             }
-            // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m'). The int32
-            // accumulator becomes fp32 exactly through the 1.5 * 2^23 bias
-            // (|acc| < 2^21): float(acc) = as_float(acc + bias) - 1.5 * 2^23;
-            // then one FMA per element: arg = float(acc) * ksc + (log2(448) - m').
-            // Pairs of keys share a key block, so both steps run as f32x2.
-            // Each 16-key chunk of P8 goes straight to shared memory in the
-            // 128B-swizzled K-major layout (chunk c of row r at c ^ (r & 7)).
-            uint64_t ksc2[NKB];
-#pragma unroll
-            for (int kb = 0; kb < NKB; ++kb) ksc2[kb] = f2_pack(ksc[kb], ksc[kb]);
+            SMARK(4);
+            // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m') =
+            // 2^(acc * ksc + log2(448) - m'), one FMA per key; the exponential
+            // runs on the MUFU unit, except for every kPolyEvery-th key pair
+            // which takes the FMA-pipe polynomial (the MUFU unit is the
+            // bottleneck of this loop). Each chunk's 32 P8 bytes go to shared
+            // memory in the 128B-swizzled K-major layout (16-byte chunk c of
+            // row r at c ^ (r & 7)).
             const float cofs = kLog2_448 - msub;
             const uint64_t cofs2 = f2_pack(cofs, cofs);
             const uint64_t nmag2 = f2_pack(-kMagicF, -kMagicF);
-            uint64_t acc2[4] = {0, 0, 0, 0};
+            uint64_t acc2 = 0;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + s_col + 32 * ch, v);
+                const int bi = min((j0 + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
+                const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
+                const uint64_t kc2 = f2_pack(kc, kc);
+                tmem_wait_ld(v);
+                uint32_t pk[8];
 #pragma unroll
-            for (int ch = 0; ch < BN / 16; ++ch) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int c = ch * 16 + q4 * 4;
-                    float e[4];
-#pragma unroll
-                    for (int k = 0; k < 4; k += 2) {
-                        const int col = c + k;
-                        const float f0 = __int_as_float(static_cast<int>(sv[col / 32][col % 32]) + kMagicI);
-                        const float f1 = __int_as_float(static_cast<int>(sv[(col + 1) / 32][(col + 1) % 32]) + kMagicI);
-                        const uint64_t x2 = f2_add(f2_pack(f0, f1), nmag2);
-                        float a0, a1;
-                        f2_unpack(f2_fma(x2, ksc2[col / kKeysPerBlk], cofs2), a0, a1);
-                        if (need_mask) {
-                            a0 = (j0 + col <= jlim) ? a0 : -INFINITY;
-                            a1 = (j0 + col + 1 <= jlim) ? a1 : -INFINITY;
-                        }
-                        e[k] = ex2_approx(a0);
-                        e[k + 1] = ex2_approx(a1);
+                for (int i = 0; i < 16; ++i) {
+                    const uint64_t x2 = f2_add(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                                               nmag2);
+                    float a0, a1;
+                    f2_unpack(f2_fma(x2, kc2, cofs2), a0, a1);
+                    if (need_mask) {
+                        const int jc = j0 + 32 * ch + 2 * i;
+                        a0 = (jc <= jlim) ? a0 : -INFINITY;
+                        a1 = (jc + 1 <= jlim) ? a1 : -INFINITY;
                     }
-                    acc2[q4] = f2_add(acc2[q4], f2_add(f2_pack(e[0], e[1]), f2_pack(e[2], e[3])));
-                    const uint32_t lo = e4m3x2_rn_satfinite(e[0], e[1]);
-                    const uint32_t hi = e4m3x2_rn_satfinite(e[2], e[3]);
-                    pk[q4] = lo | (hi << 16);
+                    float e0, e1;
+                    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
+                        exp2_poly_x2(a0, a1, e0, e1);
+                    } else {
+                        e0 = ex2_approx(a0);
+                        e1 = ex2_approx(a1);
+                    }
+                    acc2 = f2_add(acc2, f2_pack(e0, e1));
+                    const uint32_t pr = e4m3x2_rn_satfinite(e0, e1);
+                    if (i & 1) pk[i / 2] |= pr << 16;
+                    else pk[i / 2] = pr;
                 }
-                *reinterpret_cast<uint4*>(sP + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                uint8_t* prow = sP + r * 128;
+                *reinterpret_cast<uint4*>(prow + (((2 * ch) ^ (r & 7)) << 4)) =
                     make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4*>(prow + (((2 * ch + 1) ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
+            // the score tile has been read for the last time: put the bias back
+            // for the next tile's accumulation and hand the buffer to the MMA
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
             {
-                const uint64_t a01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
                 float r0, r1;
-                f2_unpack(a01, r0, r1);
+                f2_unpack(acc2, r0, r1);
                 dsum = dsum * alpha + (r0 + r1);
             }
+            SMARK(5);
             if (t > 0) {
                 // update_mdo (rescale part): O *= alpha, skipped when no row of the
                 // warp changed its max (alpha == 1 exactly)
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                    const uint64_t a2 = f2_pack(alpha, alpha);
-#pragma unroll
+#pragma unroll 1
                     for (int c4 = 0; c4 < D / 32; ++c4) {
                         uint32_t o[32];
                         tmem_ld32(lane_addr + o_col + 32 * c4, o);
                         tmem_wait_ld(o);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float x0, x1;
-                            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2),
-                                      x0, x1);
-                            o[e] = __float_as_uint(x0);
-                            o[e + 1] = __float_as_uint(x1);
-                        }
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                         tmem_st32(lane_addr + o_col + 32 * c4, o);
                     }
                     tmem_wait_st();
                 }
             }
+            SMARK(6);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[C::kBarPFull + w]);
+            SMARK(7);
             m = m_new;
         }
+#ifdef SAGE_ATTN_TRACE
+#undef trace_on
+#endif
 
         // epilogue: out = O * v_scale / (448 d) -> bf16, through the caller's strides
         const float* vsrow = p.v_scale + (int64_t)bhk * D;
@@ -395,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) {
                 tc_fence_after();
                 const float inv = dsum > 0.0f ? 1.0f / dsum : 0.0f;     // dsum carries the 448
-#pragma unroll
+#pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(lane_addr + o_col + 32 * c4, o);
@@ -518,6 +580,8 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
     p.blk_k = a.blk_k;
     p.nbq = static_cast<int>(ceil_div(a.Lq, a.blk_q));
     p.nbk = static_cast<int>(ceil_div(a.Lk, a.blk_k));
+    p.lg_blk_q = __builtin_ctz(static_cast<unsigned>(a.blk_q));
+    p.lg_blk_k = __builtin_ctz(static_cast<unsigned>(a.blk_k));
     p.logit_scale_log2 = a.softmax_scale / static_cast<float>(a.D) * kLog2e;
     p.heavy_first = a.causal ? 1 : 0;
     p.out_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 8 == 0 && a.out_stride[1] % 8 == 0 &&
@@ -530,6 +594,12 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
     return a.D == 128 ? launch_d<128>(nkb, a.causal != 0, tq, tk, tv, p, grid, s)
                       : launch_d<64>(nkb, a.causal != 0, tq, tk, tv, p, grid, s);
 }
+
+#ifdef SAGE_ATTN_TRACE
+extern "C" __attribute__((visibility("default"))) int sage_debug_attn_trace(long long* host) {
+    return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : -1;
+}
+#endif
 
 unsigned read_clear_attn_error() {
     unsigned v = 0, zero = 0;

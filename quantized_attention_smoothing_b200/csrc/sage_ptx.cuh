@@ -239,6 +239,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// Write `value` into 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t value) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1};" ::"r"(taddr),
+        "r"(value)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -286,6 +296,41 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
     return r;
+}
+
+
+// Three-input fp32 max (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// 2^a for two arguments on the FMA pipe. a is clamped to >= -125 (the result
+// stays a normal float; exact values there are below 2^-125), split as
+// a = n + f with n = rint(a) (1.5 * 2^23 rounding bias) and f in [-0.5, 0.5];
+// 2^f is a degree-5 polynomial (Chebyshev interpolation of 2^f on
+// [-0.5, 0.5], fit for this library: relative error <= 2.2e-7 in fp32 Horner
+// form over a in [-125, 9]) and 2^n is added into the exponent field.
+__device__ __forceinline__ void exp2_poly_x2(float a0, float a1, float& e0, float& e1) {
+    a0 = fmaxf(a0, -125.0f);
+    a1 = fmaxf(a1, -125.0f);
+    const uint64_t a2 = f2_pack(a0, a1);
+    const uint64_t t2 = f2_add(a2, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n2 = f2_add(t2, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f2 = f2_fma(n2, f2_pack(-1.0f, -1.0f), a2);
+    uint64_t p2 = f2_pack(0x1.5f089p-10f, 0x1.5f089p-10f);
+    p2 = f2_fma(p2, f2, f2_pack(0x1.3d107p-7f, 0x1.3d107p-7f));
+    p2 = f2_fma(p2, f2, f2_pack(0x1.c6af6cp-5f, 0x1.c6af6cp-5f));
+    p2 = f2_fma(p2, f2, f2_pack(0x1.ebf906p-3f, 0x1.ebf906p-3f));
+    p2 = f2_fma(p2, f2, f2_pack(0x1.62e43p-1f, 0x1.62e43p-1f));
+    p2 = f2_fma(p2, f2, f2_pack(0x1.000002p+0f, 0x1.000002p+0f));
+    float p0, p1, t0, t1;
+    f2_unpack(p2, p0, p1);
+    f2_unpack(t2, t0, t1);
+    // the bias bits of t vanish when shifted into the exponent field
+    e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 }  // namespace sage
