@@ -132,12 +132,34 @@ size_t sage_quant_qk_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
  *   scale 0 and zero codes).
  * Writes q8, q_scale, k8, k_scale in the layouts above and, if k_mean is not
  * NULL, mean_K [B, Hk, D]. ws: device workspace of at least
- * sage_quant_qk_workspace(...) bytes, 256-byte aligned; its contents on
+ * sage_quant_qk_workspace(...) bytes, 16-byte aligned; its contents on
  * entry do not matter. Quantised outputs must be 16-byte aligned.
  * Results are bit-identical for any input strides. */
 sage_status sage_quant_qk(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16, int blk_q,
                           int blk_k, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale,
                           float* k_mean, void* ws, size_t ws_bytes, void* stream);
+
+/* The same computation and outputs as sage_quant_qk, for callers that cannot
+ * allocate device memory when they quantise (for example a serving loop whose
+ * device memory is budgeted once at start-up, or code that must not risk the
+ * implicit device synchronisation cudaMalloc / cudaFree can cause). The
+ * paper has no counterpart to this entry point; it is a property of this
+ * library.
+ * The scratch that sage_quant_qk takes as `ws` comes instead from a fixed
+ * 8 MiB array built into the library; every GPU that loads the library holds
+ * it until the process exits. Calls whose sage_quant_qk_workspace(...) exceeds
+ * 8 MiB are rejected with SAGE_ERR_WORKSPACE before anything is launched
+ * (8 MiB covers, e.g., B * Hk * ceil(Lk / 256) * D <= 1 Mi).
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture. Every call on a device shares the one array and leaves
+ * its last contents there (each call writes every scratch entry it reads, so no
+ * clearing is needed): calls that may run concurrently on the GPU (different
+ * streams without ordering between them) race on it and must be serialised by
+ * the caller. Allocates nothing; errors as for sage_quant_qk. */
+sage_status sage_quant_qk_noalloc(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16,
+                                  int blk_q, int blk_k, int8_t* q8, float* q_scale, int8_t* k8,
+                                  float* k_scale, float* k_mean, void* stream);
 
 /* Bytes of device workspace sage_quant_v needs (per-chunk channel maxima). */
 size_t sage_quant_v_workspace(int B, int Hk, int L, int D);

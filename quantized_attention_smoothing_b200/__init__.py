@@ -27,7 +27,8 @@ SAGE_ERR_TIMEOUT = 6
 
 EXPORTS = (
     "sage_hadamard_init", "sage_hadamard_destroy", "sage_hadamard_matrix",
-    "sage_quant_qk_workspace", "sage_quant_qk", "sage_quant_v_workspace", "sage_quant_v",
+    "sage_quant_qk_workspace", "sage_quant_qk", "sage_quant_qk_noalloc",
+    "sage_quant_v_workspace", "sage_quant_v",
     "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_decode_workspace",
     "sage_attn_decode", "sage_status_string", "sage_device_error",
 )
@@ -73,6 +74,8 @@ def lib():
     L.sage_quant_qk_workspace.argtypes = [i32] * 6
     L.sage_quant_qk.restype = i32
     L.sage_quant_qk.argtypes = [vp, CView4, CView4, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.sage_quant_qk_noalloc.restype = i32
+    L.sage_quant_qk_noalloc.argtypes = [vp, CView4, CView4, i32, i32, vp, vp, vp, vp, vp, vp]
     L.sage_quant_v_workspace.restype = sz
     L.sage_quant_v_workspace.argtypes = [i32] * 4
     L.sage_quant_v.restype = i32
@@ -181,6 +184,17 @@ def sage_quant_qk(h, q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean=None, 
                                int(blk_k), _ptr(q8), _ptr(q_scale), _ptr(k8), _ptr(k_scale),
                                _ptr(k_mean), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                _stream(stream)), "sage_quant_qk")
+
+
+def sage_quant_qk_noalloc(h, q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean=None,
+                          stream=None):
+    """sage_quant_qk without a caller workspace: for callers that cannot
+    allocate device memory at the call (scratch comes from a fixed array in
+    the library; see include/sage.h for its limit and the sharing rules)."""
+    _check(lib().sage_quant_qk_noalloc(h.handle, _view(q, CView4), _view(k, CView4), int(blk_q),
+                                       int(blk_k), _ptr(q8), _ptr(q_scale), _ptr(k8),
+                                       _ptr(k_scale), _ptr(k_mean), _stream(stream)),
+           "sage_quant_qk_noalloc")
 
 
 def sage_quant_v(v, v8_t, v_scale, ws=None, stream=None):

@@ -369,3 +369,63 @@ cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* w
 }
 
 }  // namespace sage
+
+// ---------------------------------------------------------------- no-allocation variant
+// sage_quant_qk_noalloc: the same Q/K smoothing + rotation + INT8 quantisation
+// as sage_quant_qk, for callers that cannot allocate device memory at the
+// point of the call -- for instance a serving loop whose device memory is
+// budgeted once at start-up, or code that must not risk the implicit device
+// synchronisation that cudaMalloc / cudaFree can cause. Its scratch (the fp64
+// per-chunk column sums of K) lives in the fixed array below instead of a
+// caller workspace.
+#include <mutex>
+
+#include "../../include/sage.h"
+
+namespace {
+
+// Largest scratch the no-allocation entry point supports. Every GPU that
+// loads libsage holds this array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;    // 8 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_qk_noalloc_scratch[kNoAllocScratchBytes];
+
+// Host code cannot use g_qk_noalloc_scratch directly: on the host the name
+// stands for a host-side shadow, not a device address. The device address is
+// looked up once per device (with that device current) and cached.
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+sage_status noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return SAGE_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_qk_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return SAGE_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SAGE_OK;
+}
+
+}  // namespace
+
+extern "C" sage_status sage_quant_qk_noalloc(sage_hadamard h, sage_cview4 q_bf16,
+                                             sage_cview4 k_bf16, int blk_q, int blk_k, int8_t* q8,
+                                             float* q_scale, int8_t* k8, float* k_scale,
+                                             float* k_mean, void* stream) {
+    if (!h || !k_bf16.ptr) return SAGE_ERR_INVALID_ARG;
+    const int64_t B = k_bf16.size[0], Hk = k_bf16.size[1], Lk = k_bf16.size[2], D = k_bf16.size[3];
+    if (B < 1 || Hk < 1 || Lk < 1 || D < 1 || Lk > (int64_t(1) << 31) - 1) return SAGE_ERR_INVALID_ARG;
+    const size_t need = sage::quant_qk_ws_bytes((int)B, (int)Hk, (int)Lk, (int)D);
+    if (need > kNoAllocScratchBytes) return SAGE_ERR_WORKSPACE;     // beyond the fixed scratch
+    void* scratch = nullptr;
+    const sage_status st = noalloc_scratch(&scratch);
+    if (st != SAGE_OK) return st;
+    return sage_quant_qk(h, q_bf16, k_bf16, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, scratch,
+                         kNoAllocScratchBytes, stream);
+}
