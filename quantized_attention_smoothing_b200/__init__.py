@@ -87,7 +87,7 @@ def lib():
     L.sage_attn_decode_workspace.restype = sz
     L.sage_attn_decode_workspace.argtypes = [i32] * 6
     L.sage_attn_decode.restype = i32
-    L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 10 + \
+    L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 9 + \
         [f32, View4, vp, sz, vp]
     L.sage_device_error.restype = i32
     L.sage_device_error.argtypes = [vp]

@@ -131,3 +131,21 @@ def test_hadamard_init_argument_checks(L):
     assert L.sage_hadamard_init(128, -1, ctypes.byref(h)) == sage.SAGE_ERR_INVALID_ARG
     assert L.sage_hadamard_init(96, 0, ctypes.byref(h)) == sage.SAGE_ERR_UNSUPPORTED
     assert L.sage_hadamard_destroy(None) == sage.SAGE_OK
+
+
+def test_decode_validation_without_gpu(L):
+    """Argument marshalling of the decode entry point and its refusals."""
+    p = ctypes.c_void_p(0x10000)
+    q = _cview(size=(2, 4, 16, 128))
+    out = _view(0x20000, (2, 4, 16, 128))
+    args = [q, p, p, p, p, p, p, 2, 4, 16, 1, 128, 128, 64, 100, 4096, 0.088, out, p, 1 << 30, None]
+    # null handle
+    assert L.sage_attn_decode(None, *args) == sage.SAGE_ERR_INVALID_ARG
+    # the Python wrapper passes the same argument count as the C declaration
+    class FakeHandle:
+        handle = None
+    qt = __import__("torch").zeros((2, 4, 16, 128), dtype=__import__("torch").bfloat16)
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_attn_decode(FakeHandle(), qt, qt, qt, qt, qt, qt, qt, 128, 100, 4096, 0.088, qt,
+                              None, stream=0)
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARG

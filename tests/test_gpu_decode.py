@@ -1,0 +1,81 @@
+"""GPU parity of the paged FP8 decode (sage_attn_decode) against the CPU
+oracle, element-wise: the MTP4 / GQA16 / page-128 / window-4096 workload of
+the FlyDSL pa_decode page's window family, and small shapes covering other
+page sizes, short contexts, windows wider than the context, padded row
+grids (T * H / Hk < 64) and strided query/output views."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_smoothing_b200 as sage
+import workloads
+from gpu_helpers import bits, compare_output
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def h128():
+    from quantized_attention_smoothing_b200 import build
+    build.build()
+    return sage.Hadamard(128)
+
+
+def _run(h, d, window, scale, q_layout="btHd", out_layout="btHd"):
+    q = d["q"]
+    B, T, H, D = q.shape
+    if q_layout == "strided":           # [B, T, H, D] view of a [B, H, T, D+8] buffer
+        buf = torch.zeros((B, H, T, D + 8), dtype=torch.bfloat16)
+        buf[..., :D] = q.permute(0, 2, 1, 3)
+        qg = buf.cuda().permute(0, 2, 1, 3)[..., :D]
+    else:
+        qg = q.cuda()
+    if out_layout == "strided":
+        og = torch.empty((B, H, T, D + 8), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)[..., :D]
+    else:
+        og = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((max(16, sage.sage_attn_decode_workspace(B, T, H, d["k_cache"].shape[1], D,
+                                                               window)),),
+                     dtype=torch.uint8, device="cuda")
+    sage.sage_attn_decode(h, qg, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(),
+                          d["v_scale"].cuda(), d["page_table"].cuda(), d["ctx_lens"].cuda(),
+                          d["k_cache"].shape[2], d["num_pages"], window, scale, og, ws)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    _, ref = oracle.decode(workloads.bits_u16(q), d["k_cache"].numpy(), d["v_cache"].numpy(),
+                           d["k_scale"].numpy(), d["v_scale"].numpy(), d["page_table"].numpy(),
+                           d["ctx_lens"].numpy(), window, scale, want_f64=True)
+    return bits(og.contiguous()), ref
+
+
+def test_decode_window_family_workload(h128):
+    cfg, d = workloads.make_decode_config("c5")
+    gpu, ref = _run(h128, d, cfg["window"], cfg["softmax_scale"])
+    stats = compare_output(gpu, ref, None, label="c5")
+    assert stats["cos_oracle"] >= 0.9999
+
+
+@pytest.mark.parametrize("B,T,H,Hk,page,lo,hi,window", [
+    (3, 4, 8, 2, 16, 40, 90, 32),        # page 16, window < ctx, R = 16
+    (2, 1, 8, 1, 128, 100, 300, 512),    # T = 1, window >= ctx, R = 8 (padded rows)
+    (2, 2, 16, 2, 64, 257, 700, 256),    # page 64, R = 16
+    (4, 4, 16, 1, 32, 4, 30, 4096),      # tiny contexts
+    (1, 3, 12, 3, 128, 1000, 1000, 300), # T = 3, G = 4
+])
+def test_decode_shapes(h128, B, T, H, Hk, page, lo, hi, window):
+    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=128, page=page, ctx_lo=lo, ctx_hi=hi,
+                              seed=B * 1000 + page + window)
+    gpu, ref = _run(h128, d, window, 1.0 / math.sqrt(128))
+    compare_output(gpu, ref, None, label=str((B, T, H, Hk, page, window)))
+
+
+def test_decode_strided_views(h128):
+    d = workloads.make_decode(B=2, T=4, H=16, Hk=1, D=128, page=128, ctx_lo=600, ctx_hi=900,
+                              seed=77)
+    a, ref = _run(h128, d, 512, 0.08)
+    b, _ = _run(h128, d, 512, 0.08, q_layout="strided", out_layout="strided")
+    assert np.array_equal(a, b)
+    compare_output(a, ref, None, label="strided")
