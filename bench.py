@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the paged-decode measurement and print its object")
     return ap.parse_args()
 
 
@@ -56,6 +58,26 @@ def peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attn_traffic():
+    """DRAM bytes per attn_fwd launch from the committed ncu summary, if the
+    kernel source is unchanged since the capture (else None)."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_dit_prefill_b1_h24_l4096_d128.md")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    m_sha = re.search(r"^source_sha256: ([0-9a-f]+)", text, flags=re.M)
+    m_b = re.search(r"^dram_bytes_per_launch: (\d+)", text, flags=re.M)
+    if not m_sha or not m_b:
+        return None
+    src = b"".join(open(os.path.join(ROOT, "quantized_attention_smoothing_b200", "csrc", f), "rb").read()
+                   for f in ("attn_fwd.cu", "sage_ptx.cuh"))
+    if hashlib.sha256(src).hexdigest()[:len(m_sha.group(1))] != m_sha.group(1):
+        return None
+    return int(m_b.group(1))
 
 
 def work_ops(cfg):
@@ -326,7 +348,7 @@ def run_sage(args):
     peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
     achieved = ops / (attn_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved, "peak": peak_tops,
-                "unit": "TFLOP/s", "frac": achieved / peak_tops, "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peak_tops, "traffic": attn_traffic(),
                 "peak_source": "%s bf16 burst x %.0f (INT8/FP8 : BF16 nominal)" % (pk_src, INT8_OVER_BF16),
                 "frac_of_sustained": achieved / (pk["bf16_tflops_sustained"] * INT8_OVER_BF16),
                 "attn_ms": attn_ms}
@@ -400,6 +422,11 @@ def run_sage(args):
 
 def main():
     args = parse()
+    if args.decode_only:
+        import torch
+        import quantized_attention_smoothing_b200 as sage
+        print(json.dumps(bench_decode(sage, torch, torch.cuda.current_stream())))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
