@@ -58,7 +58,10 @@ __device__ long long g_attn_trace[3][16][12];
 constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;          // keys per tile
 constexpr int QT = 2;            // query tiles per CTA
-constexpr int kThreads = 320;
+constexpr int kSoftWarps = 16;   // 2 query tiles x 2 column halves x 4 lane quarters
+constexpr int kTmaWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int kThreads = 32 * (kSoftWarps + 2);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(FP8_MAX of e4m3)
 constexpr int kMagicI = 0x4B400000;               // bit pattern of 1.5 * 2^23
@@ -92,14 +95,18 @@ struct Cfg {
     static constexpr int kBarVFull = kBarKEmpty + kStages;
     static constexpr int kBarVEmpty = kBarVFull + kStages;
     static constexpr int kBarSFull = kBarVEmpty + kStages;   // [QT]
-    static constexpr int kBarSEmpty = kBarSFull + QT;        // [QT], 4 warp arrivals
-    static constexpr int kBarPFull = kBarSEmpty + QT;        // [QT], 4 warp arrivals
+    static constexpr int kBarSEmpty = kBarSFull + QT;        // [QT], 8 warp arrivals
+    static constexpr int kBarPFull = kBarSEmpty + QT;        // [QT], 8 warp arrivals
     static constexpr int kBarODone = kBarPFull + QT;         // [QT]
-    static constexpr int kBarFinal = kBarODone + QT;
+    static constexpr int kBarMax = kBarODone + QT;           // [QT], 8 warp arrivals
+    static constexpr int kBarSum = kBarMax + QT;             // [QT], 8 warp arrivals
+    static constexpr int kBarFinal = kBarSum + QT;
     static constexpr int kNumBars = kBarFinal + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffKs = kOffMisc + 16;             // K block scales of the head
-    static constexpr int kSmemBytes = kOffKs + kKsSmem * 4 + 1024;  // + runtime alignment
+    static constexpr int kOffXmax = kOffKs + kKsSmem * 4;    // [2][QT][2][BM] half-row maxima
+    static constexpr int kOffXsum = kOffXmax + 2 * QT * 2 * BM * 4;   // [QT][2][BM] half-row sums
+    static constexpr int kSmemBytes = kOffXsum + QT * 2 * BM * 4 + 1024;  // + runtime alignment
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -118,6 +125,54 @@ struct Params {
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// Max of one 32-key chunk of biased scores (fp32 values 1.5 * 2^23 + acc).
+// MASK: keys jc0 + k > jlim count as -inf. Instantiated twice so that the
+// unmasked (common) case carries no per-key compare / select.
+template <bool MASK>
+__device__ __forceinline__ float chunk_max(const uint32_t (&v)[32], int jc0, int jlim) {
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        float x0 = __uint_as_float(v[2 * k]);
+        float x1 = __uint_as_float(v[2 * k + 1]);
+        if (MASK) {
+            x0 = (jc0 + 2 * k <= jlim) ? x0 : -INFINITY;
+            x1 = (jc0 + 2 * k + 1 <= jlim) ? x1 : -INFINITY;
+        }
+        mx[k & 3] = fmax3(mx[k & 3], x0, x1);
+    }
+    return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// Exponentials of one 32-key chunk: p448 = 2^((x - bias) * kc + cofs) as
+// f32x2 pairs, row-sum into acc2, e4m3 codes into pk (4 keys per word).
+template <bool MASK>
+__device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], uint64_t kc2, uint64_t cofs2,
+                                          int jc0, int jlim, uint64_t& acc2, uint32_t (&pk)[8]) {
+    const uint64_t nmag2 = f2_pack(-kMagicF, -kMagicF);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+        const uint64_t x2 = f2_add(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), nmag2);
+        float a0, a1;
+        f2_unpack(f2_fma(x2, kc2, cofs2), a0, a1);
+        if (MASK) {
+            a0 = (jc0 + 2 * k <= jlim) ? a0 : -INFINITY;
+            a1 = (jc0 + 2 * k + 1 <= jlim) ? a1 : -INFINITY;
+        }
+        float e0, e1;
+        if (kPolyEvery > 0 && k % kPolyEvery == kPolyEvery - 1) {
+            exp2_poly_x2(a0, a1, e0, e1);
+        } else {
+            e0 = ex2_approx(a0);
+            e1 = ex2_approx(a1);
+        }
+        acc2 = f2_add(acc2, f2_pack(e0, e1));
+        const uint32_t pr = e4m3x2_rn_satfinite(e0, e1);
+        if (k & 1) pk[k / 2] |= pr << 16;
+        else pk[k / 2] = pr;
+    }
+}
 
 template <int D, int NKB, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -158,14 +213,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
-            const bool four = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
-                              (i >= C::kBarPFull && i < C::kBarPFull + QT);
-            mbar_init(&bars[i], four ? 4u : 1u);
+            const bool eight = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
+                               (i >= C::kBarPFull && i < C::kBarPFull + QT) ||
+                               (i >= C::kBarMax && i < C::kBarMax + QT) ||
+                               (i >= C::kBarSum && i < C::kBarSum + QT);
+            mbar_init(&bars[i], eight ? 8u : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
@@ -180,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0 && n_tiles > 0) {
             tma_prefetch_desc(&tmQ);
@@ -203,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             t * BN, bhk * D);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t kIdescQK = umma_idesc(2, 1, BM, BN);   // s8 x s8 -> s32
@@ -269,25 +326,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------- softmax
-        const int w = warp >> 2, ww = warp & 3;
+        // Two threads per query row: warp = tile (w) x column half (hf) x
+        // lane quarter (ww); the thread owns TMEM lane 32 ww + lane (its row)
+        // and key columns [64 hf, 64 hf + 64) of the score tile, and output
+        // columns [hf D/2, (hf + 1) D/2) of the accumulator. The two halves of
+        // a row exchange their maxima (and, at the end, their sums) through
+        // shared memory.
+        const int w = warp >> 3, hf = (warp >> 2) & 1, ww = warp & 3;
         const int r = ww * 32 + lane;
         const int i = q_row0 + w * BM + r;
         const bool valid = i < p.Lq;
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(ww * 32) << 16);
-        const uint32_t s_col = w * BN;
-        const uint32_t o_col = 256 + w * BM;
+        const uint32_t s_col = w * BN + hf * (BN / 2);
+        const uint32_t o_col = 256 + w * BM + hf * (D / 2);
         const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + (i >> p.lg_blk_q)]) : 0.0f;
         const float arow = qsc * p.logit_scale_log2;
         int jlim = valid ? p.Lk - 1 : -1;
         if (CAUSAL && valid) jlim = min(jlim, i + (p.Lk - p.Lq));
         uint8_t* sP = smem + C::kOffP + w * C::kPBytes;
         const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
+        float* xmax = reinterpret_cast<float*>(smem + C::kOffXmax);   // [2][QT][2][BM]
+        float* xsum = reinterpret_cast<float*>(smem + C::kOffXsum);   // [QT][2][BM]
+        constexpr int kHalfChunks = BN / 64;                           // 32-key chunks per half
 
         // S_w starts as the bias 1.5 * 2^23 in every column: int32 accumulation
         // onto it leaves bits that read directly as the fp32 value 1.5 * 2^23 +
         // acc (exact, |acc| < 2^21)
 #pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
+        for (int ch = 0; ch < kHalfChunks; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -296,16 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = -INFINITY, dsum = 0.0f;
         bool ok = true;
 #ifdef SAGE_ATTN_TRACE
-        const bool tr = trace_on && lane == 0 && ww == 0;
+        const bool tr = trace_on && lane == 0 && ww == 0 && hf == 0;
 #define SMARK(k) SAGE_MARK(w, t, k)
 #define trace_on tr
 #else
 #define SMARK(k)
 #endif
-        // The score tile is read from TMEM twice, 32 columns at a time: pass 1
-        // takes the row max, pass 2 the exponentials. Rolled loops keep the
-        // code small (instruction-cache resident) and the live state at one
-        // 32-column chunk.
         for (int t = 0; t < n_tiles; ++t) {
             SMARK(0);
             ok = warp_all(mbar_wait(&bars[C::kBarSFull + w], t & 1, abort_flag, &g_attn_err, 9));
@@ -313,38 +375,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             SMARK(1);
             const int j0 = t * BN;
-            // tiles that reach past this row's last visible key need masking
-            const bool need_mask = __any_sync(0xffffffffu, j0 + BN - 1 > jlim);
-            SMARK(2);
+            const int jh = j0 + hf * (BN / 2);          // first key of this half
+            // halves that reach past this row's last visible key need masking
+            const bool need_mask = __any_sync(0xffffffffu, jh + BN / 2 - 1 > jlim);
 
-            // QK and update_mdo (max part). The biased accumulators are fp32
-            // values 1.5 * 2^23 + acc (exact); y = acc * ksc is monotonic in acc
-            // (ksc >= 0), so each 32-key chunk's max is taken on the raw values
-            // (three-input max) and unbiased and scaled once.
+            // QK and update_mdo (max part), on this half's columns. The biased
+            // accumulators are fp32 values 1.5 * 2^23 + acc (exact); y = acc * ksc
+            // is monotonic in acc (ksc >= 0), so each 32-key chunk's max is taken
+            // on the raw values (three-input max), then unbiased and scaled.
             float mt = -INFINITY;
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
+            for (int ch = 0; ch < kHalfChunks; ++ch) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + s_col + 32 * ch, v);
                 tmem_wait_ld(v);
-                SMARK(8 + ch);
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float x0 = __uint_as_float(v[2 * i]);
-                    float x1 = __uint_as_float(v[2 * i + 1]);
-                    if (need_mask) {
-                        const int jc = j0 + 32 * ch + 2 * i;
-                        x0 = (jc <= jlim) ? x0 : -INFINITY;
-                        x1 = (jc + 1 <= jlim) ? x1 : -INFINITY;
-                    }
-                    mx[i & 3] = fmax3(mx[i & 3], x0, x1);
-                }
-                const float cm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                const int bi = min((j0 + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
+                const float cm = need_mask ? chunk_max<true>(v, jh + 32 * ch, jlim)
+                                           : chunk_max<false>(v, jh + 32 * ch, jlim);
+                const int bi = min((jh + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
                 const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
                 if (cm != -INFINITY) mt = fmaxf(mt, (cm - kMagicF) * kc);
             }
+            // combine with the other half of the row
+            float* xm = xmax + ((t & 1) * QT + w) * 2 * BM;
+            xm[hf * BM + r] = mt;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarMax + w]);
+            ok = warp_all(mbar_wait(&bars[C::kBarMax + w], t & 1, abort_flag, &g_attn_err, 13));
+            if (!ok) break;
+            mt = fmaxf(mt, xm[(hf ^ 1) * BM + r]);
             const float m_new = fmaxf(m, mt);
             const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
             const float alpha = ex2_approx(m - msub);
@@ -358,58 +416,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             SMARK(4);
             // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m') =
-            // 2^(acc * ksc + log2(448) - m'), one FMA per key; the exponential
-            // runs on the MUFU unit, except for every kPolyEvery-th key pair
-            // which takes the FMA-pipe polynomial (the MUFU unit is the
-            // bottleneck of this loop). Each chunk's 32 P8 bytes go to shared
-            // memory in the 128B-swizzled K-major layout (16-byte chunk c of
-            // row r at c ^ (r & 7)).
+            // 2^(acc * ksc + log2(448) - m'), one FMA per key (f32x2); the
+            // exponential runs on the MUFU unit, except for every kPolyEvery-th
+            // key pair (FMA-pipe polynomial). Each 32-key chunk of P8 goes to
+            // shared memory in the 128B-swizzled K-major layout (16-byte chunk c
+            // of row r at c ^ (r & 7)).
             const float cofs = kLog2_448 - msub;
             const uint64_t cofs2 = f2_pack(cofs, cofs);
-            const uint64_t nmag2 = f2_pack(-kMagicF, -kMagicF);
             uint64_t acc2 = 0;
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) {
+            for (int ch = 0; ch < kHalfChunks; ++ch) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + s_col + 32 * ch, v);
-                const int bi = min((j0 + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
+                const int cg = hf * kHalfChunks + ch;      // 32-key chunk of the tile
+                const int bi = min((j0 + 32 * cg) >> p.lg_blk_k, p.nbk - 1);
                 const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
                 const uint64_t kc2 = f2_pack(kc, kc);
                 tmem_wait_ld(v);
                 uint32_t pk[8];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint64_t x2 = f2_add(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
-                                               nmag2);
-                    float a0, a1;
-                    f2_unpack(f2_fma(x2, kc2, cofs2), a0, a1);
-                    if (need_mask) {
-                        const int jc = j0 + 32 * ch + 2 * i;
-                        a0 = (jc <= jlim) ? a0 : -INFINITY;
-                        a1 = (jc + 1 <= jlim) ? a1 : -INFINITY;
-                    }
-                    float e0, e1;
-                    if (kPolyEvery > 0 && i % kPolyEvery == kPolyEvery - 1) {
-                        exp2_poly_x2(a0, a1, e0, e1);
-                    } else {
-                        e0 = ex2_approx(a0);
-                        e1 = ex2_approx(a1);
-                    }
-                    acc2 = f2_add(acc2, f2_pack(e0, e1));
-                    const uint32_t pr = e4m3x2_rn_satfinite(e0, e1);
-                    if (i & 1) pk[i / 2] |= pr << 16;
-                    else pk[i / 2] = pr;
-                }
+                if (need_mask) chunk_exp<true>(v, kc2, cofs2, j0 + 32 * cg, jlim, acc2, pk);
+                else chunk_exp<false>(v, kc2, cofs2, j0 + 32 * cg, jlim, acc2, pk);
                 uint8_t* prow = sP + r * 128;
-                *reinterpret_cast<uint4*>(prow + (((2 * ch) ^ (r & 7)) << 4)) =
+                *reinterpret_cast<uint4*>(prow + (((2 * cg) ^ (r & 7)) << 4)) =
                     make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(prow + (((2 * ch + 1) ^ (r & 7)) << 4)) =
+                *reinterpret_cast<uint4*>(prow + (((2 * cg + 1) ^ (r & 7)) << 4)) =
                     make_uint4(pk[4], pk[5], pk[6], pk[7]);
             }
-            // the score tile has been read for the last time: put the bias back
-            // for the next tile's accumulation and hand the buffer to the MMA
+            // this half of the score tile has been read for the last time: put
+            // the bias back for the next tile's accumulation and release it
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 32; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
+            for (int ch = 0; ch < kHalfChunks; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -417,15 +453,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 float r0, r1;
                 f2_unpack(acc2, r0, r1);
-                dsum = dsum * alpha + (r0 + r1);
+                dsum = dsum * alpha + (r0 + r1);       // this half's share of d
             }
             SMARK(5);
             if (t > 0) {
-                // update_mdo (rescale part): O *= alpha, skipped when no row of the
-                // warp changed its max (alpha == 1 exactly)
+                // update_mdo (rescale part): O *= alpha on this half's output
+                // columns, skipped when no row of the warp changed its max
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                    for (int c4 = 0; c4 < D / 64; ++c4) {
                         uint32_t o[32];
                         tmem_ld32(lane_addr + o_col + 32 * c4, o);
                         tmem_wait_ld(o);
@@ -448,53 +484,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 #undef trace_on
 #endif
 
-        // epilogue: out = O * v_scale / (448 d) -> bf16, through the caller's strides
-        const float* vsrow = p.v_scale + (int64_t)bhk * D;
-        __nv_bfloat16* orow = p.out + b * p.os0 + h * p.os1 + (int64_t)i * p.os2;
+        // epilogue: out = O * v_scale / (448 d) -> bf16 (d = both halves' sums;
+        // 448 is inside the exponent), this half's columns, caller's strides
+        const float* vsrow = p.v_scale + (int64_t)bhk * D + hf * (D / 2);
+        __nv_bfloat16* orow = p.out + b * p.os0 + h * p.os1 + (int64_t)i * p.os2 +
+                              (int64_t)(hf * (D / 2)) * p.os3;
         if (ok && n_tiles > 0) {
-            ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (n_tiles - 1) & 1, abort_flag,
-                                    &g_attn_err, 11));
+            float* xs = xsum + w * 2 * BM;
+            xs[hf * BM + r] = dsum;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarSum + w]);
+            ok = warp_all(mbar_wait(&bars[C::kBarSum + w], 0, abort_flag, &g_attn_err, 14));
             if (ok) {
-                tc_fence_after();
-                const float inv = dsum > 0.0f ? 1.0f / dsum : 0.0f;     // dsum carries the 448
+                const float dtot = dsum + xs[(hf ^ 1) * BM + r];
+                ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (n_tiles - 1) & 1, abort_flag,
+                                        &g_attn_err, 11));
+                if (ok) {
+                    tc_fence_after();
+                    const float inv = dtot > 0.0f ? 1.0f / dtot : 0.0f;
 #pragma unroll 1
-                for (int c4 = 0; c4 < D / 32; ++c4) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_addr + o_col + 32 * c4, o);
-                    tmem_wait_ld(o);
-                    if (valid) {
-                        uint32_t packed[16];
+                    for (int c4 = 0; c4 < D / 64; ++c4) {
+                        uint32_t o[32];
+                        tmem_ld32(lane_addr + o_col + 32 * c4, o);
+                        tmem_wait_ld(o);
+                        if (valid) {
+                            uint32_t packed[16];
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float v0 = __uint_as_float(o[e]) * (__ldg(&vsrow[32 * c4 + e]) * inv);
-                            const float v1 = __uint_as_float(o[e + 1]) * (__ldg(&vsrow[32 * c4 + e + 1]) * inv);
-                            const __nv_bfloat162 pr = __floats2bfloat162_rn(v0, v1);
-                            packed[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
-                        }
-                        if (p.out_vec) {
-                            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+                            for (int e = 0; e < 32; e += 2) {
+                                const float v0 = __uint_as_float(o[e]) * (__ldg(&vsrow[32 * c4 + e]) * inv);
+                                const float v1 = __uint_as_float(o[e + 1]) * (__ldg(&vsrow[32 * c4 + e + 1]) * inv);
+                                const __nv_bfloat162 pr = __floats2bfloat162_rn(v0, v1);
+                                packed[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+                            }
+                            if (p.out_vec) {
+                                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
 #pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4)
-                                dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1],
-                                                     packed[4 * q4 + 2], packed[4 * q4 + 3]);
-                        } else {
+                                for (int q4 = 0; q4 < 4; ++q4)
+                                    dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1],
+                                                         packed[4 * q4 + 2], packed[4 * q4 + 3]);
+                            } else {
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const uint16_t bits = (e & 1) ? (packed[e / 2] >> 16) : (packed[e / 2] & 0xFFFFu);
-                                *reinterpret_cast<uint16_t*>(orow + (int64_t)(32 * c4 + e) * p.os3) = bits;
+                                for (int e = 0; e < 32; ++e) {
+                                    const uint16_t bits16 = (e & 1) ? (packed[e / 2] >> 16) : (packed[e / 2] & 0xFFFFu);
+                                    *reinterpret_cast<uint16_t*>(orow + (int64_t)(32 * c4 + e) * p.os3) = bits16;
+                                }
                             }
                         }
                     }
                 }
             }
         } else if (n_tiles == 0 && valid) {
-            for (int d = 0; d < D; ++d) orow[(int64_t)d * p.os3] = __float2bfloat16_rn(0.0f);
+            for (int d = 0; d < D / 2; ++d) orow[(int64_t)d * p.os3] = __float2bfloat16_rn(0.0f);
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
@@ -598,6 +644,12 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
 #ifdef SAGE_ATTN_TRACE
 extern "C" __attribute__((visibility("default"))) int sage_debug_attn_trace(long long* host) {
     return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : -1;
+}
+extern "C" __attribute__((visibility("default"))) unsigned long long sage_debug_wait_polls(int reset) {
+    unsigned long long v = 0, z = 0;
+    cudaMemcpyFromSymbol(&v, g_wait_polls, sizeof v);
+    if (reset) cudaMemcpyToSymbol(g_wait_polls, &z, sizeof z);
+    return v;
 }
 #endif
 

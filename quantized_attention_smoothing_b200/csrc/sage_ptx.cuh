@@ -26,6 +26,10 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // ------------------------------------------------------------ mbarrier
 
+#ifdef SAGE_ATTN_TRACE
+__device__ unsigned long long g_wait_polls;   // development-only poll counter
+#endif
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");
@@ -85,6 +89,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
+#ifdef SAGE_ATTN_TRACE
+        atomicAdd(&g_wait_polls, 1ull);
+#endif
         if (mbar_try_wait_sleep(a, parity, 200000u)) return true;
         if (*abort_flag) return false;
         if (global_timer_ns() - t0 > kWaitTimeoutNs) {
