@@ -26,11 +26,9 @@ inline bool view_vec8(const View4& v) {
 
 constexpr int kTile = 128;                  // token tile of every kernel
 constexpr unsigned kErrTimeoutCode = 1u;    // low byte of a device error word
-constexpr int kStatRows = 256;              // tokens per statistics chunk
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 __host__ __device__ inline int64_t ceil_div(int64_t x, int64_t m) { return (x + m - 1) / m; }
-inline int stat_chunks(int L) { return static_cast<int>(ceil_div(L, kStatRows)); }
 
 // ---- quantisation (quant.cu)
 size_t quant_qk_ws_bytes(int B, int Hk, int Lk, int D);
@@ -40,6 +38,7 @@ cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k
                             void* ws, cudaStream_t s);
 cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,
                            cudaStream_t s);
+unsigned read_clear_quant_error();
 
 // ---- attention forward (attn_fwd.cu)
 struct AttnArgs {

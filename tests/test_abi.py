@@ -53,9 +53,9 @@ def test_status_strings(L):
 
 
 def test_workspace_sizes_are_host_only(L):
-    # K column sums: fp64 per (b, h, 256-token chunk, d)
-    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 16 * 128 * 8
-    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 128 * 128 * 4
+    # K: the fp32 mean per (b, kv head, d); V: the fp32 multiplier 448 / a per (b, h, d)
+    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 128 * 4
+    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 128 * 4
     assert L.sage_attn_fwd_workspace(1, 24, 24, 4096, 4096, 128) == 0
     assert L.sage_quant_qk_workspace(0, 1, 1, 1, 1, 64) == 0
 

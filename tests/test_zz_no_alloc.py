@@ -66,11 +66,11 @@ def test_no_alloc_matches_workspace_entry_point_twice():
 
 def test_no_alloc_rejects_sizes_beyond_its_scratch():
     h = sage.Hadamard(128)
-    # 8 Mi tokens of K over 2 heads needs 2 * 32768 * 128 * 8 B = 64 MiB of scratch
+    # 32768 kv heads of D = 128 need 32768 * 128 * 4 B = 16 MiB of K means
     big = sage.CView4()
     big.ptr = 0x10000
-    sizes = (1, 2, 8 << 20, 128)
-    strides = (2 * (8 << 20) * 128, (8 << 20) * 128, 128, 1)
+    sizes = (1, 32768, 1, 128)
+    strides = (32768 * 128, 128, 128, 1)
     for i in range(4):
         big.size[i] = sizes[i]
         big.stride[i] = strides[i]
