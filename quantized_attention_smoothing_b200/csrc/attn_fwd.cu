@@ -1,17 +1,30 @@
 // attn_fwd.cu -- quantised attention forward for sm_100a.
 //
 // One CTA owns two 128-row query tiles of one (b, h) and streams the key
-// axis in 128-key tiles. Roles (320 threads):
+// axis in 128-key tiles. Roles (384 threads):
 //   warps 0-3   softmax for query tile 0 (thread = query row = TMEM lane)
 //   warps 4-7   softmax for query tile 1
 //   warp 8      TMA producer: both Q tiles once, then a ring of K / V^T stages
 //   warp 9      MMA issuer (one thread): tcgen05 kind::i8 S = Q8 K8^T into
 //               TMEM (int32), tcgen05 kind::f8f6f4 O += P8 V8 into TMEM (fp32)
+//   warps 10-11 idle (they complete the register warpgroup of warps 8-9)
 // TMEM (512 columns): S_w at [128 w, 128 w + 128), O_w at [256 + 128 w, +D).
-// The MMA warp issues S(t) for both tiles before PV(t-1), so the tensor pipe
-// works on the next scores while the softmax warps convert the current ones
-// (the overlap "Sage2 SM89 Temporal Pair Experiment" (Candidate) obtains with
-// warp pairs on sm_89).
+// Registers: the CTA launches at 168 per thread; the producer warpgroup
+// (warps 8-11) drops to 40 and the softmax warpgroups rise to 232, so a
+// thread can hold its whole 128-key score row.
+//
+// A softmax thread reads its whole score row (128 keys) from TMEM into
+// registers and hands the S columns straight back, so the tensor pipe
+// computes the next tile's scores while the current ones are converted.
+// P8 goes to shared memory (double buffered per query tile), which lets
+// PV(t) run while tile t + 1 is converted. MMA issue order per tile t:
+//   QK_0(t+1), QK_1(t+1), PV_0(t), PV_1(t)
+// so each query tile depends only on its own softmax warps. The two tiles'
+// exponential phases take turns (a token passed between the softmax
+// warpgroups through bounded mbarriers), so one tile's TMEM traffic, max and
+// rescale overlap the other's MUFU work on the SM sub-partitions (the overlap
+// "Sage2 SM89 Temporal Pair Experiment" (Candidate) obtains with warp pairs
+// on sm_89).
 //
 // Per 128-key tile the softmax warps follow the page's sequence
 //   QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV
@@ -58,10 +71,16 @@ __device__ long long g_attn_trace[3][16][12];
 constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;          // keys per tile
 constexpr int QT = 2;            // query tiles per CTA
-constexpr int kSoftWarps = 16;   // 2 query tiles x 2 column halves x 4 lane quarters
-constexpr int kTmaWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int kThreads = 32 * (kSoftWarps + 2);
+constexpr int kSoftWarps = 8;    // 2 query tiles x 4 lane quarters
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 32 * (kSoftWarps + 4);
+// per-thread registers after the split; 128 * (2 * kSoftRegs + kProdRegs) must
+// not exceed kThreads * (registers at launch, 168) or the increase never
+// completes
+constexpr int kSoftRegs = 232;
+constexpr int kProdRegs = 40;
+static_assert(128 * (2 * kSoftRegs + kProdRegs) <= kThreads * 168, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(FP8_MAX of e4m3)
 constexpr int kMagicI = 0x4B400000;               // bit pattern of 1.5 * 2^23
@@ -79,34 +98,33 @@ constexpr int kKsSmem = 1024;
 
 template <int D>
 struct Cfg {
-    static constexpr int kStages = D == 128 ? 4 : 6;
+    static constexpr int kStages = D == 128 ? 3 : 6;
     static constexpr int kQBytes = BM * D;
     static constexpr int kKBytes = BN * D;
     static constexpr int kVBytes = D * BN;
     static constexpr int kPBytes = BM * BN;
+    static constexpr int kPBufs = 2;                         // P double buffer per query tile
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + QT * kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKBytes;
-    static constexpr int kOffP = kOffV + kStages * kVBytes;
-    static constexpr int kOffBar = kOffP + QT * kPBytes;
+    static constexpr int kOffP = kOffV + kStages * kVBytes;  // [QT][kPBufs] tiles
+    static constexpr int kOffBar = kOffP + QT * kPBufs * kPBytes;
     static constexpr int kBarQ = 0;
     static constexpr int kBarKFull = 1;
     static constexpr int kBarKEmpty = kBarKFull + kStages;
     static constexpr int kBarVFull = kBarKEmpty + kStages;
     static constexpr int kBarVEmpty = kBarVFull + kStages;
     static constexpr int kBarSFull = kBarVEmpty + kStages;   // [QT]
-    static constexpr int kBarSEmpty = kBarSFull + QT;        // [QT], 8 warp arrivals
-    static constexpr int kBarPFull = kBarSEmpty + QT;        // [QT], 8 warp arrivals
+    static constexpr int kBarSEmpty = kBarSFull + QT;        // [QT], 4 warp arrivals
+    static constexpr int kBarPFull = kBarSEmpty + QT;        // [QT], 4 warp arrivals
     static constexpr int kBarODone = kBarPFull + QT;         // [QT]
-    static constexpr int kBarMax = kBarODone + QT;           // [QT], 8 warp arrivals
-    static constexpr int kBarSum = kBarMax + QT;             // [QT], 8 warp arrivals
-    static constexpr int kBarFinal = kBarSum + QT;
+    static constexpr int kBarTok = kBarODone + QT;           // [QT], 4 warp arrivals
+    static constexpr int kBarFinal = kBarTok + QT;
     static constexpr int kNumBars = kBarFinal + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffKs = kOffMisc + 16;             // K block scales of the head
-    static constexpr int kOffXmax = kOffKs + kKsSmem * 4;    // [2][QT][2][BM] half-row maxima
-    static constexpr int kOffXsum = kOffXmax + 2 * QT * 2 * BM * 4;   // [QT][2][BM] half-row sums
-    static constexpr int kSmemBytes = kOffXsum + QT * 2 * BM * 4 + 1024;  // + runtime alignment
+    static constexpr int kOffVs = kOffKs + kKsSmem * 4;      // V channel scales of the head
+    static constexpr int kSmemBytes = kOffVs + D * 4 + 1024; // + runtime alignment
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -126,52 +144,96 @@ struct Params {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
-// Max of one 32-key chunk of biased scores (fp32 values 1.5 * 2^23 + acc).
-// MASK: keys jc0 + k > jlim count as -inf. Instantiated twice so that the
-// unmasked (common) case carries no per-key compare / select.
-template <bool MASK>
-__device__ __forceinline__ float chunk_max(const uint32_t (&v)[32], int jc0, int jlim) {
+// View 32 consecutive registers of a larger per-thread array as one
+// tcgen05.ld / st operand.
+__device__ __forceinline__ uint32_t (&slice32(uint32_t* base))[32] {
+    return *reinterpret_cast<uint32_t(*)[32]>(base);
+}
+
+// Four e4m3 codes (RN, satfinite) of e0..e3 in one word, e0 in byte 0.
+__device__ __forceinline__ uint32_t e4m3x4(float e0, float e1, float e2, float e3) {
+    uint32_t w;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+        "mov.b32 %0, {lo, hi};\n\t}"
+        : "=r"(w)
+        : "f"(e0), "f"(e1), "f"(e2), "f"(e3));
+    return w;
+}
+
+// Max of n consecutive biased scores s[0..n) (fp32 values 1.5 * 2^23 + acc).
+// MASK: keys j0 + k > jlim count as -inf.
+template <int N, bool MASK>
+__device__ __forceinline__ float block_max(const uint32_t* s, int j0, int jlim) {
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        float x0 = __uint_as_float(v[2 * k]);
-        float x1 = __uint_as_float(v[2 * k + 1]);
+    for (int k = 0; k < N / 2; ++k) {
+        float x0 = __uint_as_float(s[2 * k]);
+        float x1 = __uint_as_float(s[2 * k + 1]);
         if (MASK) {
-            x0 = (jc0 + 2 * k <= jlim) ? x0 : -INFINITY;
-            x1 = (jc0 + 2 * k + 1 <= jlim) ? x1 : -INFINITY;
+            x0 = (j0 + 2 * k <= jlim) ? x0 : -INFINITY;
+            x1 = (j0 + 2 * k + 1 <= jlim) ? x1 : -INFINITY;
         }
         mx[k & 3] = fmax3(mx[k & 3], x0, x1);
     }
     return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
 }
 
-// Exponentials of one 32-key chunk: p448 = 2^((x - bias) * kc + cofs) as
-// f32x2 pairs, row-sum into acc2, e4m3 codes into pk (4 keys per word).
-template <bool MASK>
-__device__ __forceinline__ void chunk_exp(const uint32_t (&v)[32], uint64_t kc2, uint64_t cofs2,
-                                          int jc0, int jlim, uint64_t& acc2, uint32_t (&pk)[8]) {
+// accumulate_d and RS_32_to_8 for a whole 128-key score row, in three
+// sweeps of independent instructions (so a single warp keeps the MUFU unit
+// fed): logits in place, exponentials in place, then row sum, e4m3 packing
+// and the P8 row store (128B-swizzled K-major: 16-byte chunk c of row r at
+// c ^ (r & 7)). Returns the sum of the unquantised exponentials.
+template <int NKB, bool MASK>
+__device__ __forceinline__ float row_exp(uint32_t (&s)[BN], const float (&kc)[NKB], float cofs,
+                                         int j0, int jlim, uint8_t* prow, int r) {
+    constexpr int kKeysPerBlk = BN / NKB;
     const uint64_t nmag2 = f2_pack(-kMagicF, -kMagicF);
+    const uint64_t cofs2 = f2_pack(cofs, cofs);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        const uint64_t x2 = f2_add(f2_pack(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1])), nmag2);
+    for (int k = 0; k < BN / 2; ++k) {
+        const float kcc = kc[(2 * k) / kKeysPerBlk];
+        const uint64_t x2 = f2_add(f2_pack(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), nmag2);
         float a0, a1;
-        f2_unpack(f2_fma(x2, kc2, cofs2), a0, a1);
+        f2_unpack(f2_fma(x2, f2_pack(kcc, kcc), cofs2), a0, a1);
         if (MASK) {
-            a0 = (jc0 + 2 * k <= jlim) ? a0 : -INFINITY;
-            a1 = (jc0 + 2 * k + 1 <= jlim) ? a1 : -INFINITY;
+            a0 = (j0 + 2 * k <= jlim) ? a0 : -INFINITY;
+            a1 = (j0 + 2 * k + 1 <= jlim) ? a1 : -INFINITY;
         }
+        s[2 * k] = __float_as_uint(a0);
+        s[2 * k + 1] = __float_as_uint(a1);
+    }
+#pragma unroll
+    for (int k = 0; k < BN / 2; ++k) {
         float e0, e1;
         if (kPolyEvery > 0 && k % kPolyEvery == kPolyEvery - 1) {
-            exp2_poly_x2(a0, a1, e0, e1);
+            exp2_poly_x2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1]), e0, e1);
         } else {
-            e0 = ex2_approx(a0);
-            e1 = ex2_approx(a1);
+            e0 = ex2_approx(__uint_as_float(s[2 * k]));
+            e1 = ex2_approx(__uint_as_float(s[2 * k + 1]));
         }
-        acc2 = f2_add(acc2, f2_pack(e0, e1));
-        const uint32_t pr = e4m3x2_rn_satfinite(e0, e1);
-        if (k & 1) pk[k / 2] |= pr << 16;
-        else pk[k / 2] = pr;
+        s[2 * k] = __float_as_uint(e0);
+        s[2 * k + 1] = __float_as_uint(e1);
     }
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int c = 0; c < BN / 16; ++c) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t* e = s + 16 * c + 4 * q;
+            acc[q] = f2_add(acc[q], f2_pack(__uint_as_float(e[0]), __uint_as_float(e[1])));
+            acc[q] = f2_add(acc[q], f2_pack(__uint_as_float(e[2]), __uint_as_float(e[3])));
+            pk[q] = e4m3x4(__uint_as_float(e[0]), __uint_as_float(e[1]), __uint_as_float(e[2]),
+                           __uint_as_float(e[3]));
+        }
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    const uint64_t t2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+    float r0, r1;
+    f2_unpack(t2, r0, r1);
+    return r0 + r1;
 }
 
 template <int D, int NKB, bool CAUSAL>
@@ -201,23 +263,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int bhk = b * p.Hk + h / (p.H / p.Hk);
     const int q_row0 = qt * (QT * BM);
 
-    int kv_end = p.Lk;
-    if (CAUSAL) {
-        const int lim = q_row0 + QT * BM + (p.Lk - p.Lq);     // last visible key + 1
-        kv_end = max(0, min(kv_end, lim));
+    // key tiles each query tile visits: all of them, or (causal, bottom-right
+    // aligned) up to the last key its last row sees; none for a tile wholly
+    // past Lq
+    int n_w[QT];
+#pragma unroll
+    for (int w = 0; w < QT; ++w) {
+        int kv_end = p.Lk;
+        if (CAUSAL) kv_end = max(0, min(kv_end, q_row0 + (w + 1) * BM + (p.Lk - p.Lq)));
+        n_w[w] = q_row0 + w * BM < p.Lq ? (kv_end + BN - 1) / BN : 0;
     }
-    const int n_tiles = (kv_end + BN - 1) / BN;
+    const int n_max = max(n_w[0], n_w[1]);
 #ifdef SAGE_ATTN_TRACE
     const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0;
 #endif
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
-            const bool eight = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
-                               (i >= C::kBarPFull && i < C::kBarPFull + QT) ||
-                               (i >= C::kBarMax && i < C::kBarMax + QT) ||
-                               (i >= C::kBarSum && i < C::kBarSum + QT);
-            mbar_init(&bars[i], eight ? 8u : 1u);
+            const bool four = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
+                              (i >= C::kBarPFull && i < C::kBarPFull + QT) ||
+                              (i >= C::kBarTok && i < C::kBarTok + QT);
+            mbar_init(&bars[i], four ? 4u : 1u);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -227,19 +293,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_relinquish();
     }
     float* ks_s = reinterpret_cast<float*>(smem + C::kOffKs);
+    float* vs_s = reinterpret_cast<float*>(smem + C::kOffVs);
     {
         const float* ksrc = p.k_scale + (int64_t)bhk * p.nbk;
         const int nks = min(p.nbk, kKsSmem);
         for (int i = threadIdx.x; i < nks; i += kThreads) ks_s[i] = __ldg(&ksrc[i]);
+        for (int i = threadIdx.x; i < D; i += kThreads) vs_s[i] = __ldg(&p.v_scale[(int64_t)bhk * D + i]);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == kTmaWarp) {
+    if (warp >= kSoftWarps) {
+      reg_dealloc<kProdRegs>();
+      if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0 && n_max > 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
@@ -247,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int w = 0; w < QT; ++w)
                 tma_load_2d(smem + C::kOffQ + w * C::kQBytes, &tmQ, &bars[C::kBarQ], 0,
                             bh * p.LpadQ + q_row0 + w * BM);
-            for (int t = 0; t < n_tiles; ++t) {
+            for (int t = 0; t < n_max; ++t) {
                 const int s = t % C::kStages;
                 const uint32_t ph = (t / C::kStages) & 1;
                 if (!mbar_wait(&bars[C::kBarKEmpty + s], ph ^ 1, abort_flag, &g_attn_err, 1)) break;
@@ -262,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0 && n_tiles > 0) {
+        if (lane == 0 && n_max > 0) {
             constexpr uint32_t kIdescQK = umma_idesc(2, 1, BM, BN);   // s8 x s8 -> s32
             constexpr uint32_t kIdescPV = umma_idesc(1, 0, BM, D);    // e4m3 x e4m3 -> f32
             const uint32_t sQ = smem_u32(smem + C::kOffQ);
@@ -270,22 +340,50 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sV = smem_u32(smem + C::kOffV);
             const uint32_t sP = smem_u32(smem + C::kOffP);
 
-            auto issue_pv = [&](int u) -> bool {
-                const int s = u % C::kStages;
-                const uint32_t ph = (u / C::kStages) & 1;
-                if (!mbar_wait(&bars[C::kBarVFull + s], ph, abort_flag, &g_attn_err, 3)) return false;
+            // QK_w(t) for every query tile that visits key tile t. S_w holds
+            // the 1.5 * 2^23 bias (written back by the softmax warps as they
+            // release it); the MMA accumulates onto it.
+            auto issue_qk = [&](int t) -> bool {
+                const int s = t % C::kStages;
+                const uint32_t ph = (t / C::kStages) & 1;
+                if (!mbar_wait(&bars[C::kBarKFull + s], ph, abort_flag, &g_attn_err, 6)) return false;
                 tc_fence_after();
-                const uint64_t vdesc = umma_desc_kmajor(sV + s * C::kVBytes, 128);
+                const uint64_t kdesc = umma_desc_kmajor(sK + s * C::kKBytes, D);
                 for (int w = 0; w < QT; ++w) {
-                    if (!mbar_wait(&bars[C::kBarPFull + w], u & 1, abort_flag, &g_attn_err, 4))
+                    if (t >= n_w[w]) continue;
+                    if (!mbar_wait(&bars[C::kBarSEmpty + w], t & 1, abort_flag, &g_attn_err, 7))
                         return false;
                     tc_fence_after();
-                    const uint64_t pdesc = umma_desc_kmajor(sP + w * C::kPBytes, 128);
+                    const uint64_t qdesc = umma_desc_kmajor(sQ + w * C::kQBytes, D);
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; ++kk)
+                        mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, 1u);
+                    mma_commit(&bars[C::kBarSFull + w]);
+                    SAGE_MARK(2, t, 1 + w);
+                }
+                mma_commit(&bars[C::kBarKEmpty + s]);
+                return true;
+            };
+            // PV_w(t): O_w += P_w(t) V(t), once softmax w has written P_w(t)
+            // and rescaled O_w for tile t (P_full).
+            auto issue_pv = [&](int t) -> bool {
+                const int s = t % C::kStages;
+                const uint32_t ph = (t / C::kStages) & 1;
+                if (!mbar_wait(&bars[C::kBarVFull + s], ph, abort_flag, &g_attn_err, 3)) return false;
+                const uint64_t vdesc = umma_desc_kmajor(sV + s * C::kVBytes, 128);
+                for (int w = 0; w < QT; ++w) {
+                    if (t >= n_w[w]) continue;
+                    if (!mbar_wait(&bars[C::kBarPFull + w], t & 1, abort_flag, &g_attn_err, 4))
+                        return false;
+                    tc_fence_after();
+                    const uint64_t pdesc =
+                        umma_desc_kmajor(sP + (w * C::kPBufs + (t & 1)) * C::kPBytes, 128);
 #pragma unroll
                     for (int kk = 0; kk < BN / 32; ++kk)
                         mma_f8_ss(tmem + 256 + w * BM, pdesc + 2 * kk, vdesc + 2 * kk, kIdescPV,
-                                  (u > 0 || kk > 0) ? 1u : 0u);
+                                  (t > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&bars[C::kBarODone + w]);
+                    SAGE_MARK(2, t, 3 + w);
                 }
                 mma_commit(&bars[C::kBarVEmpty + s]);
                 return true;
@@ -293,248 +391,219 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             bool ok = mbar_wait(&bars[C::kBarQ], 0, abort_flag, &g_attn_err, 5);
             tc_fence_after();
-            for (int t = 0; ok && t < n_tiles; ++t) {
-                const int s = t % C::kStages;
-                const uint32_t ph = (t / C::kStages) & 1;
+            if (ok) ok = issue_qk(0);
+            for (int t = 0; ok && t < n_max; ++t) {
                 SAGE_MARK(2, t, 0);
-                if (!(ok = mbar_wait(&bars[C::kBarKFull + s], ph, abort_flag, &g_attn_err, 6))) break;
-                SAGE_MARK(2, t, 1);
-                tc_fence_after();
-                const uint64_t kdesc = umma_desc_kmajor(sK + s * C::kKBytes, D);
-                for (int w = 0; w < QT && ok; ++w) {
-                    // S_w holds the 1.5 * 2^23 bias (written by the softmax warps
-                    // after their last read, phase t of s_empty); the MMA adds onto it
-                    ok = mbar_wait(&bars[C::kBarSEmpty + w], t & 1, abort_flag, &g_attn_err, 7);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t qdesc = umma_desc_kmajor(sQ + w * C::kQBytes, D);
-#pragma unroll
-                    for (int kk = 0; kk < D / 32; ++kk)
-                        mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, 1u);
-                    mma_commit(&bars[C::kBarSFull + w]);
-                    SAGE_MARK(2, t, 2 + w);
-                }
-                if (!ok) break;
-                mma_commit(&bars[C::kBarKEmpty + s]);
-                if (t > 0) ok = issue_pv(t - 1);
-                SAGE_MARK(2, t, 4);
+                if (t + 1 < n_max) ok = issue_qk(t + 1);
+                if (ok) ok = issue_pv(t);
             }
-            if (ok) issue_pv(n_tiles - 1);
             // drain every MMA this thread issued before TMEM is released
             mma_commit(&bars[C::kBarFinal]);
             mbar_wait(&bars[C::kBarFinal], 0, abort_flag, &g_attn_err, 8);
         }
+      }
     } else {
+        reg_alloc<kSoftRegs>();
         // ---------------------------------------------------------- softmax
-        // Two threads per query row: warp = tile (w) x column half (hf) x
-        // lane quarter (ww); the thread owns TMEM lane 32 ww + lane (its row)
-        // and key columns [64 hf, 64 hf + 64) of the score tile, and output
-        // columns [hf D/2, (hf + 1) D/2) of the accumulator. The two halves of
-        // a row exchange their maxima (and, at the end, their sums) through
-        // shared memory.
-        const int w = warp >> 3, hf = (warp >> 2) & 1, ww = warp & 3;
+        // warp = query tile (w) x lane quarter (ww); the thread owns TMEM
+        // lane 32 ww + lane: query row r of tile w, its 128 score columns and
+        // its D output columns
+        const int w = warp >> 2, ww = warp & 3;
         const int r = ww * 32 + lane;
         const int i = q_row0 + w * BM + r;
         const bool valid = i < p.Lq;
+        const int n_t = n_w[w];
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(ww * 32) << 16);
-        const uint32_t s_col = w * BN + hf * (BN / 2);
-        const uint32_t o_col = 256 + w * BM + hf * (D / 2);
+        const uint32_t s_col = w * BN;
+        const uint32_t o_col = 256 + w * BM;
         const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + (i >> p.lg_blk_q)]) : 0.0f;
         const float arow = qsc * p.logit_scale_log2;
-        int jlim = valid ? p.Lk - 1 : -1;
+        // last key this row sees (rows past Lq compute on zero padding and
+        // are never written)
+        int jlim = p.Lk - 1;
         if (CAUSAL && valid) jlim = min(jlim, i + (p.Lk - p.Lq));
-        uint8_t* sP = smem + C::kOffP + w * C::kPBytes;
+        uint8_t* sPw = smem + C::kOffP + w * C::kPBufs * C::kPBytes;   // this tile's P buffers
         const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
-        float* xmax = reinterpret_cast<float*>(smem + C::kOffXmax);   // [2][QT][2][BM]
-        float* xsum = reinterpret_cast<float*>(smem + C::kOffXsum);   // [QT][2][BM]
-        constexpr int kHalfChunks = BN / 64;                           // 32-key chunks per half
-
-        // S_w starts as the bias 1.5 * 2^23 in every column: int32 accumulation
-        // onto it leaves bits that read directly as the fp32 value 1.5 * 2^23 +
-        // acc (exact, |acc| < 2^21)
-#pragma unroll 1
-        for (int ch = 0; ch < kHalfChunks; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
-
-        float m = -INFINITY, dsum = 0.0f;
-        bool ok = true;
 #ifdef SAGE_ATTN_TRACE
-        const bool tr = trace_on && lane == 0 && ww == 0 && hf == 0;
+        const bool tr = trace_on && lane == 0 && ww == 0;
 #define SMARK(k) SAGE_MARK(w, t, k)
 #define trace_on tr
 #else
 #define SMARK(k)
 #endif
-        for (int t = 0; t < n_tiles; ++t) {
+
+        // S_w starts as the bias 1.5 * 2^23 in every column: int32 accumulation
+        // onto it leaves bits that read directly as the fp32 value 1.5 * 2^23 +
+        // acc (exact, |acc| < 2^21)
+        if (n_t > 0) {
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tmem_fill32(lane_addr + s_col + 32 * c, kMagicI);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
+        }
+
+        // tile 0 takes the first turn: tile 1 completes phase 0 of tok_0
+        if (w == 1 && lane == 0) mbar_arrive(&bars[C::kBarTok + 0]);
+
+        float m = -INFINITY, dsum = 0.0f;
+        bool ok = true;
+        for (int t = 0; t < n_t; ++t) {
             SMARK(0);
             ok = warp_all(mbar_wait(&bars[C::kBarSFull + w], t & 1, abort_flag, &g_attn_err, 9));
             if (!ok) break;
             tc_fence_after();
             SMARK(1);
-            const int j0 = t * BN;
-            const int jh = j0 + hf * (BN / 2);          // first key of this half
-            // halves that reach past this row's last visible key need masking
-            const bool need_mask = __any_sync(0xffffffffu, jh + BN / 2 - 1 > jlim);
+            // the whole score row into registers, then S goes back to the MMA
+            // warp with the bias rewritten for tile t + 1
+            uint32_t s[BN];
+            tmem_ld128(lane_addr + s_col, s);
+            tmem_wait_ld128(s);
+            SMARK(6);
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) tmem_fill32(lane_addr + s_col + 32 * c, kMagicI);
 
-            // QK and update_mdo (max part), on this half's columns. The biased
-            // accumulators are fp32 values 1.5 * 2^23 + acc (exact); y = acc * ksc
-            // is monotonic in acc (ksc >= 0), so each 32-key chunk's max is taken
-            // on the raw values (three-input max), then unbiased and scaled.
+            const int j0 = t * BN;
+            // a tile that reaches past some row's last visible key needs masking
+            const bool need_mask = __any_sync(0xffffffffu, j0 + BN - 1 > jlim);
+            float kc[NKB];
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
+                const int bi = min((j0 + kb * kKeysPerBlk) >> p.lg_blk_k, p.nbk - 1);
+                kc[kb] = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
+            }
+            // QK and update_mdo (max part). y = acc * kc is monotonic in acc
+            // (kc >= 0), so each K block's max is taken on the raw biased
+            // values (three-input max), then unbiased and scaled.
             float mt = -INFINITY;
-#pragma unroll 1
-            for (int ch = 0; ch < kHalfChunks; ++ch) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + s_col + 32 * ch, v);
-                tmem_wait_ld(v);
-                const float cm = need_mask ? chunk_max<true>(v, jh + 32 * ch, jlim)
-                                           : chunk_max<false>(v, jh + 32 * ch, jlim);
-                const int bi = min((jh + 32 * ch) >> p.lg_blk_k, p.nbk - 1);
-                const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
-                if (cm != -INFINITY) mt = fmaxf(mt, (cm - kMagicF) * kc);
+#pragma unroll
+            for (int kb = 0; kb < NKB; ++kb) {
+                const float cm = need_mask
+                    ? block_max<kKeysPerBlk, true>(s + kb * kKeysPerBlk, j0 + kb * kKeysPerBlk, jlim)
+                    : block_max<kKeysPerBlk, false>(s + kb * kKeysPerBlk, j0 + kb * kKeysPerBlk, jlim);
+                if (cm != -INFINITY) mt = fmaxf(mt, (cm - kMagicF) * kc[kb]);
             }
-            // combine with the other half of the row
-            float* xm = xmax + ((t & 1) * QT + w) * 2 * BM;
-            xm[hf * BM + r] = mt;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[C::kBarMax + w]);
-            ok = warp_all(mbar_wait(&bars[C::kBarMax + w], t & 1, abort_flag, &g_attn_err, 13));
-            if (!ok) break;
-            mt = fmaxf(mt, xm[(hf ^ 1) * BM + r]);
-            const float m_new = fmaxf(m, mt);
-            const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
-            const float alpha = ex2_approx(m - msub);
-            SMARK(3);
-            if (t > 0) {
-                // PV(t-1) must be complete before P is overwritten and O rescaled
-                ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (t - 1) & 1, abort_flag,
-                                        &g_attn_err, 10));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            SMARK(4);
-            // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m') =
-            // 2^(acc * ksc + log2(448) - m'), one FMA per key (f32x2); the
-            // exponential runs on the MUFU unit, except for every kPolyEvery-th
-            // key pair (FMA-pipe polynomial). Each 32-key chunk of P8 goes to
-            // shared memory in the 128B-swizzled K-major layout (16-byte chunk c
-            // of row r at c ^ (r & 7)).
-            const float cofs = kLog2_448 - msub;
-            const uint64_t cofs2 = f2_pack(cofs, cofs);
-            uint64_t acc2 = 0;
-#pragma unroll 1
-            for (int ch = 0; ch < kHalfChunks; ++ch) {
-                uint32_t v[32];
-                tmem_ld32(lane_addr + s_col + 32 * ch, v);
-                const int cg = hf * kHalfChunks + ch;      // 32-key chunk of the tile
-                const int bi = min((j0 + 32 * cg) >> p.lg_blk_k, p.nbk - 1);
-                const float kc = (bi < kKsSmem ? ks_s[bi] : __ldg(&ksrow[bi])) * arow;
-                const uint64_t kc2 = f2_pack(kc, kc);
-                tmem_wait_ld(v);
-                uint32_t pk[8];
-                if (need_mask) chunk_exp<true>(v, kc2, cofs2, j0 + 32 * cg, jlim, acc2, pk);
-                else chunk_exp<false>(v, kc2, cofs2, j0 + 32 * cg, jlim, acc2, pk);
-                uint8_t* prow = sP + r * 128;
-                *reinterpret_cast<uint4*>(prow + (((2 * cg) ^ (r & 7)) << 4)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(prow + (((2 * cg + 1) ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            }
-            // this half of the score tile has been read for the last time: put
-            // the bias back for the next tile's accumulation and release it
-#pragma unroll 1
-            for (int ch = 0; ch < kHalfChunks; ++ch) tmem_fill32(lane_addr + s_col + 32 * ch, kMagicI);
+            SMARK(7);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[C::kBarSEmpty + w]);
-            {
-                float r0, r1;
-                f2_unpack(acc2, r0, r1);
-                dsum = dsum * alpha + (r0 + r1);       // this half's share of d
-            }
-            SMARK(5);
+            const float m_new = fmaxf(m, mt);
+            const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
+            const float alpha = ex2_approx(m - msub);
+            SMARK(2);
+            // the exponentials of the two query tiles take turns (token tok_w,
+            // passed on below), so one tile's max and rescale overlap the
+            // other's MUFU work instead of both tiles contending for it
+            ok = warp_all(mbar_wait(&bars[C::kBarTok + w], t & 1, abort_flag, &g_attn_err, 12));
+            if (!ok) break;
+            SMARK(8);
+
+            // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m') =
+            // 2^(acc * kc + log2(448) - m'), one FMA per key (f32x2). Each
+            // 32-key chunk of P8 goes to shared memory in the 128B-swizzled
+            // K-major layout (16-byte chunk c of row r at c ^ (r & 7)). Buffer
+            // t & 1 was last read by PV(t - 2), awaited before tile t - 1's
+            // rescale.
+            uint8_t* prow = sPw + (t & 1) * C::kPBytes + r * 128;
+            const float tsum = need_mask ? row_exp<NKB, true>(s, kc, kLog2_448 - msub, j0, jlim, prow, r)
+                                         : row_exp<NKB, false>(s, kc, kLog2_448 - msub, j0, jlim, prow, r);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarTok + (w ^ 1)]);
+            dsum = dsum * alpha + tsum;
+            SMARK(3);
             if (t > 0) {
-                // update_mdo (rescale part): O *= alpha on this half's output
-                // columns, skipped when no row of the warp changed its max
+                // update_mdo (rescale part): PV(t-1) must have landed in O first;
+                // then O *= alpha, skipped when no row of the warp changed its max
+                ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (t - 1) & 1, abort_flag,
+                                        &g_attn_err, 10));
+                if (!ok) break;
+                tc_fence_after();
+                SMARK(4);
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll 1
-                    for (int c4 = 0; c4 < D / 64; ++c4) {
-                        uint32_t o[32];
-                        tmem_ld32(lane_addr + o_col + 32 * c4, o);
-                        tmem_wait_ld(o);
+                    const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(lane_addr + o_col + 32 * c4, o);
+                    for (int c2 = 0; c2 < D / 64; ++c2) {
+                        uint32_t o[64];
+                        tmem_ld32(lane_addr + o_col + 64 * c2, slice32(o));
+                        tmem_ld32(lane_addr + o_col + 64 * c2 + 32, slice32(o + 32));
+                        tmem_wait_ld(slice32(o));
+                        tmem_wait_ld(slice32(o + 32));
+#pragma unroll
+                        for (int e = 0; e < 64; e += 2) {
+                            float a0, a1;
+                            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), al2),
+                                      a0, a1);
+                            o[e] = __float_as_uint(a0);
+                            o[e + 1] = __float_as_uint(a1);
+                        }
+                        tmem_st32(lane_addr + o_col + 64 * c2, slice32(o));
+                        tmem_st32(lane_addr + o_col + 64 * c2 + 32, slice32(o + 32));
                     }
                     tmem_wait_st();
                 }
             }
-            SMARK(6);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[C::kBarPFull + w]);
-            SMARK(7);
+            SMARK(5);
             m = m_new;
         }
 #ifdef SAGE_ATTN_TRACE
 #undef trace_on
 #endif
-
-        // epilogue: out = O * v_scale / (448 d) -> bf16 (d = both halves' sums;
-        // 448 is inside the exponent), this half's columns, caller's strides
-        const float* vsrow = p.v_scale + (int64_t)bhk * D + hf * (D / 2);
-        __nv_bfloat16* orow = p.out + b * p.os0 + h * p.os1 + (int64_t)i * p.os2 +
-                              (int64_t)(hf * (D / 2)) * p.os3;
-        if (ok && n_tiles > 0) {
-            float* xs = xsum + w * 2 * BM;
-            xs[hf * BM + r] = dsum;
+        // the other tile may visit more key tiles (causal, or this tile lies
+        // past Lq): keep passing the turn until it is done
+        for (int t = n_t; ok && t < n_w[w ^ 1]; ++t) {
+            ok = warp_all(mbar_wait(&bars[C::kBarTok + w], t & 1, abort_flag, &g_attn_err, 13));
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[C::kBarSum + w]);
-            ok = warp_all(mbar_wait(&bars[C::kBarSum + w], 0, abort_flag, &g_attn_err, 14));
+            if (ok && lane == 0) mbar_arrive(&bars[C::kBarTok + (w ^ 1)]);
+        }
+
+        // epilogue: out = O * v_scale / (448 d) -> bf16 (448 is inside the
+        // exponent), caller's strides
+        __nv_bfloat16* orow = p.out + b * p.os0 + h * p.os1 + (int64_t)i * p.os2;
+        if (ok && n_t > 0) {
+            ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (n_t - 1) & 1, abort_flag,
+                                    &g_attn_err, 11));
             if (ok) {
-                const float dtot = dsum + xs[(hf ^ 1) * BM + r];
-                ok = warp_all(mbar_wait(&bars[C::kBarODone + w], (n_tiles - 1) & 1, abort_flag,
-                                        &g_attn_err, 11));
-                if (ok) {
-                    tc_fence_after();
-                    const float inv = dtot > 0.0f ? 1.0f / dtot : 0.0f;
+                tc_fence_after();
+                const float inv = dsum > 0.0f ? 1.0f / dsum : 0.0f;
 #pragma unroll 1
-                    for (int c4 = 0; c4 < D / 64; ++c4) {
-                        uint32_t o[32];
-                        tmem_ld32(lane_addr + o_col + 32 * c4, o);
-                        tmem_wait_ld(o);
-                        if (valid) {
-                            uint32_t packed[16];
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_addr + o_col + 32 * c, o);
+                    tmem_wait_ld(o);
+                    if (valid) {
+                        uint32_t packed[16];
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                const float v0 = __uint_as_float(o[e]) * (__ldg(&vsrow[32 * c4 + e]) * inv);
-                                const float v1 = __uint_as_float(o[e + 1]) * (__ldg(&vsrow[32 * c4 + e + 1]) * inv);
-                                const __nv_bfloat162 pr = __floats2bfloat162_rn(v0, v1);
-                                packed[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
-                            }
-                            if (p.out_vec) {
-                                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c4);
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 vs2 = *reinterpret_cast<const float2*>(vs_s + 32 * c + e);
+                            const float v0 = __uint_as_float(o[e]) * (vs2.x * inv);
+                            const float v1 = __uint_as_float(o[e + 1]) * (vs2.y * inv);
+                            const __nv_bfloat162 pr = __floats2bfloat162_rn(v0, v1);
+                            packed[e / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+                        }
+                        if (p.out_vec) {
+                            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-                                for (int q4 = 0; q4 < 4; ++q4)
-                                    dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1],
-                                                         packed[4 * q4 + 2], packed[4 * q4 + 3]);
-                            } else {
+                            for (int q4 = 0; q4 < 4; ++q4)
+                                dst[q4] = make_uint4(packed[4 * q4], packed[4 * q4 + 1],
+                                                     packed[4 * q4 + 2], packed[4 * q4 + 3]);
+                        } else {
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) {
-                                    const uint16_t bits16 = (e & 1) ? (packed[e / 2] >> 16) : (packed[e / 2] & 0xFFFFu);
-                                    *reinterpret_cast<uint16_t*>(orow + (int64_t)(32 * c4 + e) * p.os3) = bits16;
-                                }
+                            for (int e = 0; e < 32; ++e) {
+                                const uint16_t bits16 = (e & 1) ? (packed[e / 2] >> 16) : (packed[e / 2] & 0xFFFFu);
+                                *reinterpret_cast<uint16_t*>(orow + (int64_t)(32 * c + e) * p.os3) = bits16;
                             }
                         }
                     }
                 }
             }
-        } else if (n_tiles == 0 && valid) {
-            for (int d = 0; d < D / 2; ++d) orow[(int64_t)d * p.os3] = __float2bfloat16_rn(0.0f);
+        } else if (n_t == 0 && valid) {
+            for (int d = 0; d < D; ++d) orow[(int64_t)d * p.os3] = __float2bfloat16_rn(0.0f);
         }
     }
 
@@ -546,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_dealloc(tmem, 512);
     }
 }
-
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,

@@ -242,6 +242,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+// 128 consecutive 32-bit TMEM columns of this thread's lane in one load
+// (shape 32x32b, x128). Valid after tmem_wait_ld128(r).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, "
+        "%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, "
+        "%34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, "
+        "%50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64, %65, "
+        "%66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, "
+        "%82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, %96, %97, "
+        "%98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, "
+        "%111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, "
+        "%124, %125, %126, %127"
+        "}, [%128];"
+        : SAGE_R32(r), SAGE_R32((r + 32)), SAGE_R32((r + 64)), SAGE_R32((r + 96))
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld128(uint32_t (&r)[128]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : SAGE_RW32(r), SAGE_RW32((r + 32)), SAGE_RW32((r + 64)), SAGE_RW32((r + 96))
+                 :
+                 : "memory");
+}
+
 // Wait for this thread's outstanding tcgen05.ld; ties `r` to the wait so no
 // use of r can be scheduled before it.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
@@ -269,6 +295,18 @@ __device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t value) {
 
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Per-thread register budget of the calling warpgroup (every warp of the
+// warpgroup executes the same one): dealloc hands registers back to the
+// CTA's pool, alloc waits until the pool can grant the new budget.
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------ numerics
