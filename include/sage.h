@@ -117,8 +117,8 @@ sage_status sage_hadamard_destroy(sage_hadamard h);
  * and/or report D through `head_dim` (either may be NULL). */
 sage_status sage_hadamard_matrix(sage_hadamard h, int8_t* host_out, int* head_dim);
 
-/* Bytes of device workspace sage_quant_qk needs: the fp32 mean of K per
- * (b, kv head, d), B * Hk * D * 4. */
+/* Bytes of device workspace sage_quant_qk needs: fp64 partial column sums
+ * of K, up to 8 per (b, kv head, d): B * Hk * 8 * D * 8. */
 size_t sage_quant_qk_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
 
 /* Smooth, rotate and INT8-quantise Q and K.
@@ -150,7 +150,7 @@ sage_status sage_quant_qk(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf1
  * 8 MiB array built into the library; every GPU that loads the library holds
  * it until the process exits. Calls whose sage_quant_qk_workspace(...) exceeds
  * 8 MiB are rejected with SAGE_ERR_WORKSPACE before anything is launched
- * (8 MiB covers B * Hk * D <= 2 Mi).
+ * (8 MiB covers B * Hk * D <= 128 Ki, e.g. 1024 kv heads of D = 128).
  * The first call on a device looks the array's device address up
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture. Every call on a device shares the one array and leaves
@@ -162,8 +162,8 @@ sage_status sage_quant_qk_noalloc(sage_hadamard h, sage_cview4 q_bf16, sage_cvie
                                   int blk_q, int blk_k, int8_t* q8, float* q_scale, int8_t* k8,
                                   float* k_scale, float* k_mean, void* stream);
 
-/* Bytes of device workspace sage_quant_v needs: the fp32 multiplier 448 / a
- * per (b, h, d), B * Hk * D * 4. */
+/* Bytes of device workspace sage_quant_v needs: fp32 partial channel
+ * maxima, up to 8 per (b, h, d): B * Hk * 8 * D * 4. */
 size_t sage_quant_v_workspace(int B, int Hk, int L, int D);
 
 /* FP8 e4m3 (OCP e4m3fn, max 448) per-channel quantisation of V.

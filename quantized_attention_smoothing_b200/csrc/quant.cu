@@ -4,8 +4,8 @@
 // Numerics are a fixed operation graph so that results are bit-identical
 // to a plain sequential evaluation (this TU is compiled with -fmad=false,
 // and every rounding step uses an explicit _rn intrinsic):
-//   mean_K = fp32(fp64 sum / L)           (fp64 partial sums per CTA, then
-//                                          CTAs of the cluster in order)
+//   mean_K = fp32(fp64 sum / L)           (fp64 partial sums per CTA, per
+//                                          cluster, then clusters in order)
 //   x_s    = x - mean_K                   (fp32, K only)
 //   x_hat  = butterfly(x_s)               (fp32, stages h = 1, 2, ..., D/2)
 //   a      = max |x_hat| over the block;  s = a / 127;  r = 127 / a
@@ -17,17 +17,23 @@
 // "Sage2 SM89 Temporal Pair Experiment", Candidate (per-channel V scale);
 // "[FlyDSL] [Misc] pa_decode: ...", Changes (FP8_MAX of e4m3 = 448).
 //
-// Kernels (each a single pass over its tensor):
-//   column_stats_kernel  one cluster of 8 CTAs per (b, h) streams the head's
-//                        tokens and reduces the column statistic across the
-//                        cluster through distributed shared memory; the
-//                        leader CTA writes the finished per-channel values.
-//   qk_quant_kernel      one CTA per 128-token tile; the tile's rows arrive in
-//                        shared memory by bulk copies, then one thread owns
-//                        one token row, so all log2(D) butterfly stages stay
-//                        inside a thread.
-//   v_quant_kernel       one CTA per 128-token tile, staged the same way,
-//                        written out transposed [b, h, d, token].
+// Kernels:
+//   column_stats_kernel  clusters of 8 CTAs, `parts` clusters per (b, h),
+//                        each streaming a contiguous token range; a
+//                        cluster's CTAs reduce through distributed shared
+//                        memory and its leader writes the partial column
+//                        statistic (fp64 sums for K, fp32 maxima for V).
+//   qk_quant_kernel      persistent CTAs over 128-token tiles (Q tiles, then
+//                        K tiles). Each CTA keeps two tiles in flight: the
+//                        next tile arrives in shared memory by coalesced
+//                        16-byte cp.async copies while the current one is
+//                        converted, one
+//                        thread per token row, all log2(D) butterfly stages
+//                        inside the thread (f32x2 pairs), codes stored
+//                        straight from registers.
+//   v_quant_kernel       the same ring; output written transposed
+//                        [b, h, d, token].
+#include <algorithm>
 #include <type_traits>
 
 #include <cooperative_groups.h>
@@ -44,9 +50,11 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int kStatCluster = 8;      // CTAs per (b, h) in the statistics kernel
-constexpr int kStatThreads = 512;
+constexpr int kStatCluster = 8;      // CTAs per cluster in the statistics kernel
+constexpr int kStatThreads = 256;
 constexpr int kStatUnroll = 8;       // 16-byte loads in flight per thread
+constexpr int kMaxParts = 8;         // clusters per (b, h), at most
+constexpr int kQuantCtasPerSm = 3;   // resident quantisation CTAs per SM
 constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
@@ -78,30 +86,30 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* x) {
 }
 
 // ---------------------------------------------------------------- stats
-// grid (8 * B*Hh), 512 threads, clusters of 8 along x: CTA `rank` of the
-// cluster of head bh covers tokens [rank * span, (rank + 1) * span).
-// MODE 0 (K): fp64 column sums -> mean (fp32) into `ws`, and into `user`
-//             (the optional k_mean output) when given.
-// MODE 1 (V): fp32 column absmax a -> scale a / 448 into `user` (v_scale)
-//             and the multiplier 448 / a into `ws`.
+// grid (8 * parts * B*Hh), 256 threads, clusters of 8 along x. Cluster c =
+// blockIdx.x / 8 covers head bh = c / parts, part c % parts; CTA `rank` of
+// it covers tokens [(part * 8 + rank) * span, + span).
+// MODE 0 (K): fp64 column sums -> ws[(bh * parts + part) * D + d] (double).
+// MODE 1 (V): fp32 column absmax -> ws[(bh * parts + part) * D + d] (float).
 template <int D, int MODE>
 __global__ void __cluster_dims__(kStatCluster, 1, 1) __launch_bounds__(kStatThreads)
-    column_stats_kernel(View4 x, float* __restrict__ ws, float* __restrict__ user, int vec) {
+    column_stats_kernel(View4 x, int parts, void* __restrict__ ws, int vec) {
     constexpr int TPR = D / 8;                    // threads per token row
     constexpr int RPI = kStatThreads / TPR;       // token rows per load round
     using Acc = typename std::conditional<MODE == 0, double, float>::type;
     __shared__ Acc red[RPI][D];
-    __shared__ Acc part[D];
+    __shared__ Acc part_s[D];
 
     const int L = static_cast<int>(x.size[2]);
     const int Hh = static_cast<int>(x.size[1]);
     const int rank = blockIdx.x % kStatCluster;
-    const int bh = blockIdx.x / kStatCluster;
+    const int cid = blockIdx.x / kStatCluster;
+    const int bh = cid / parts, part = cid % parts;
     const int b = bh / Hh, h = bh % Hh;
     const int tid = threadIdx.x;
     const int cg8 = tid % TPR, rg = tid / TPR;
-    const int span = static_cast<int>(ceil_div(L, kStatCluster));
-    const int l0 = rank * span;
+    const int span = static_cast<int>(ceil_div(L, kStatCluster * parts));
+    const int l0 = (part * kStatCluster + rank) * span;
     const int l1 = min(L, l0 + span);
     const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
     const int64_t row0 = b * x.stride[0] + h * x.stride[1] + (int64_t)(cg8 * 8) * x.stride[3];
@@ -137,91 +145,71 @@ __global__ void __cluster_dims__(kStatCluster, 1, 1) __launch_bounds__(kStatThre
             if (MODE == 0) s = __dadd_rn(s, red[r][tid]);
             else s = fmaxf(s, red[r][tid]);
         }
-        part[tid] = s;
+        part_s[tid] = s;
     }
     cg::cluster_group cl = cg::this_cluster();
     cl.sync();
     if (rank == 0 && tid < D) {
-        Acc s = part[tid];
+        Acc s = part_s[tid];
         for (int r = 1; r < kStatCluster; ++r) {
-            const Acc o = cl.map_shared_rank(part, r)[tid];
+            const Acc o = cl.map_shared_rank(part_s, r)[tid];
             if (MODE == 0) s = __dadd_rn(s, o);
             else s = fmaxf(s, o);
         }
-        const int64_t o = (int64_t)bh * D + tid;
-        if (MODE == 0) {
-            const float m = __double2float_rn(__ddiv_rn(s, (double)L));
-            ws[o] = m;
-            if (user != nullptr) user[o] = m;
-        } else {
-            float sc = 0.0f, r = 0.0f;
-            if (s != 0.0f) {
-                sc = __fdiv_rn(s, 448.0f);
-                r = __fdiv_rn(448.0f, s);
-            }
-            user[o] = sc;
-            ws[o] = r;
-        }
+        static_cast<Acc*>(ws)[((int64_t)bh * parts + part) * D + tid] = s;
     }
     cl.sync();                  // the leader has read every CTA's partials
 }
 
 // ---------------------------------------------------------------- staging
-// The rows [0, nrows) of a 128-token tile of head (b, h), D bf16 each, into
-// shared memory at a pitch of D + 8 elements (rows land 16 bytes apart in
-// the bank space, so a thread reading its own row conflicts with nobody).
-// VEC views: one bulk copy per row, completion on `bar`; other views: a
-// strided element gather by the whole CTA. Returns false (and records a
-// timeout) if the copies never arrive.
+// Shared-memory image of one 128-token tile: row r at r * (D + 8) elements
+// (rows land 16 bytes apart in the bank space, so a thread reading its own
+// row conflicts with nobody).
 template <int D>
-__device__ __forceinline__ bool stage_tile(const View4& x, int b, int h, int l0, int nrows,
-                                           bool vec, uint16_t* tile, uint64_t* bar,
-                                           volatile int* abort_flag, unsigned site) {
-    constexpr int PITCH = D + 8;
-    const int tid = threadIdx.x;
+struct Tile {
+    static constexpr int kPitch = D + 8;
+    static constexpr int kElems = kTile * kPitch;
+};
+
+// Start bringing rows [0, nrows) of a 128-token tile of head (b, h) into
+// `tile`: the CTA's 128 threads issue 16-byte asynchronous copies
+// (cp.async, consecutive threads on consecutive 16 bytes of a row) and
+// commit them as one group. Only for views whose rows are contiguous and
+// 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int D>
+__device__ __forceinline__ void issue_tile(const View4& x, int b, int h, int l0, int nrows,
+                                           uint16_t* tile) {
+    constexpr int CPR = D / 8;                     // 16-byte chunks per row
     const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
     const int64_t hoff = b * x.stride[0] + h * x.stride[1];
-    if (vec) {
-        if (tid < 32) {
-            if (tid == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nrows * D * 2));
-            __syncwarp();
-            for (int r = tid; r < nrows; r += 32)
-                bulk_load(tile + r * PITCH, base + hoff + (int64_t)(l0 + r) * x.stride[2], D * 2, bar);
-        }
-        return mbar_wait(bar, 0, abort_flag, &g_quant_err, site);
+    for (int i = threadIdx.x; i < nrows * CPR; i += kTile) {
+        const int r = i / CPR, c = i % CPR;
+        cp_async16(tile + r * Tile<D>::kPitch + 8 * c, base + hoff + (int64_t)(l0 + r) * x.stride[2] + 8 * c);
     }
-    for (int i = tid; i < nrows * D; i += kTile) {
-        const int r = i / D, d = i % D;
-        tile[r * PITCH + d] = __ldg(base + hoff + (int64_t)(l0 + r) * x.stride[2] + (int64_t)d * x.stride[3]);
-    }
-    __syncthreads();
-    return true;
 }
 
+// Strided element gather of the same rows by the whole CTA (any view).
 template <int D>
-__device__ __forceinline__ void butterfly(float (&x)[D]) {
-    // stage h pairs (j, j + h) for j = (k / h) * 2h + k % h, k = 0 .. D/2 - 1
-#pragma unroll
-    for (int lg = 0; (1 << lg) < D; ++lg) {
-        const int h = 1 << lg;
-#pragma unroll
-        for (int k = 0; k < D / 2; ++k) {
-            const int j = ((k >> lg) << (lg + 1)) + (k & (h - 1));
-            const float a = x[j], c = x[j + h];
-            x[j] = __fadd_rn(a, c);
-            x[j + h] = __fsub_rn(a, c);
-        }
+__device__ __forceinline__ void gather_tile(const View4& x, int b, int h, int l0, int nrows,
+                                            uint16_t* tile) {
+    const uint16_t* base = static_cast<const uint16_t*>(x.ptr);
+    const int64_t hoff = b * x.stride[0] + h * x.stride[1];
+    for (int i = threadIdx.x; i < nrows * D; i += kTile) {
+        const int r = i / D, d = i % D;
+        tile[r * Tile<D>::kPitch + d] =
+            __ldg(base + hoff + (int64_t)(l0 + r) * x.stride[2] + (int64_t)d * x.stride[3]);
     }
-}
-
-// Low byte of the fp32 bit pattern of (y + 1.5 * 2^23) is rne(y) as a two's
-// complement byte for |y| < 2^22; four of them into one word.
-__device__ __forceinline__ uint32_t pack_round4(float y0, float y1, float y2, float y3) {
-    const uint32_t t0 = __float_as_uint(__fadd_rn(y0, kRoundMagic));
-    const uint32_t t1 = __float_as_uint(__fadd_rn(y1, kRoundMagic));
-    const uint32_t t2 = __float_as_uint(__fadd_rn(y2, kRoundMagic));
-    const uint32_t t3 = __float_as_uint(__fadd_rn(y3, kRoundMagic));
-    return __byte_perm(__byte_perm(t0, t1, 0x0040), __byte_perm(t2, t3, 0x0040), 0x5410);
 }
 
 __device__ __forceinline__ uint32_t pack_clamp4(float y0, float y1, float y2, float y3) {
@@ -236,253 +224,399 @@ __device__ __forceinline__ uint32_t pack_clamp4(float y0, float y1, float y2, fl
     return word;
 }
 
-// ---------------------------------------------------------------- Q/K int8
-// One CTA of 128 threads per (tensor, b, h, 128-token tile); thread r owns
-// token row r of the tile. Q tiles come first in the grid, then K tiles.
-template <int D>
-__global__ void __launch_bounds__(kTile) qk_quant_kernel(
-    View4 q, View4 k, int blk_q, int blk_k, int n_qtiles, const float* __restrict__ kmean,
-    int8_t* __restrict__ q8, float* __restrict__ q_scale, int8_t* __restrict__ k8,
-    float* __restrict__ k_scale, int qvec, int kvec) {
-    constexpr int PITCH = D + 8;                  // staged input row pitch (elements)
-    constexpr int OPITCH = D + 16;                // staged output row pitch (bytes)
-    static_assert(kTile * OPITCH <= kTile * PITCH * 2, "output staging reuses the tile");
-    __shared__ __align__(128) uint16_t tile[kTile * PITCH];
-    __shared__ __align__(16) float mean_s[D];
-    __shared__ float wmax[kTile / 32];
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ int abort_flag;
+// fp32 pairs (sm_100 f32x2 arithmetic): each lane is one IEEE RN operation,
+// so results equal the scalar ones bit for bit. A product feeding an add must
+// not be written as mul.rn.f32x2 + add.rn.f32x2: ptxas contracts that pair
+// into one FMA (a single rounding) despite the explicit rounding modifiers.
+__device__ __forceinline__ uint64_t p2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float p2lo(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float p2hi(uint64_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+__device__ __forceinline__ uint64_t p2add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t p2sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t p2fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t p2mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 
-    const bool isK = blockIdx.x >= (unsigned)n_qtiles;
-    const View4& x = isK ? k : q;
-    const int tile_lin = isK ? blockIdx.x - n_qtiles : blockIdx.x;
+// The butterfly of `butterfly` on a row held as D/2 pairs x2[i] = (x[2i],
+// x[2i+1]): stage h = 1 inside each pair, stages h = 2 .. D/2 as pair
+// operations between pairs i and i + h/2. Same operations, same order per
+// element, so the same bits.
+template <int D>
+__device__ __forceinline__ void butterfly_pairs(uint64_t (&x2)[D / 2]) {
+#pragma unroll
+    for (int i = 0; i < D / 2; ++i) {
+        const float a = p2lo(x2[i]), c = p2hi(x2[i]);
+        x2[i] = p2(__fadd_rn(a, c), __fsub_rn(a, c));
+    }
+#pragma unroll
+    for (int lg = 0; (2 << lg) < D; ++lg) {
+        const int hp = 1 << lg;                  // pair distance = h / 2
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) {
+            const int i = ((k >> lg) << (lg + 1)) + (k & (hp - 1));
+            const uint64_t a = x2[i], c = x2[i + hp];
+            x2[i] = p2add(a, c);
+            x2[i + hp] = p2sub(a, c);
+        }
+    }
+}
+
+// One 128-token tile of the Q-then-K tile list: tiles [0, n_qtiles) walk Q
+// head by head, the rest walk K.
+struct QkTile {
+    bool isK;
+    int bh, b, h, tl, l0, nrows, ntiles;
+};
+
+__device__ __forceinline__ QkTile qk_tile(int t, int n_qtiles, const View4& q, const View4& k) {
+    QkTile r;
+    r.isK = t >= n_qtiles;
+    const View4& x = r.isK ? k : q;
+    const int lin = r.isK ? t - n_qtiles : t;
     const int L = static_cast<int>(x.size[2]);
     const int Hh = static_cast<int>(x.size[1]);
-    const int ntiles = static_cast<int>(ceil_div(L, kTile));
-    const int bh = tile_lin / ntiles, tl = tile_lin % ntiles;
-    const int b = bh / Hh, h = bh % Hh;
-    const int blk = isK ? blk_k : blk_q;
-    const int nb = static_cast<int>(ceil_div(L, blk));
-    const bool vec = (isK ? kvec : qvec) != 0;
+    r.ntiles = static_cast<int>(ceil_div(L, kTile));
+    r.bh = lin / r.ntiles;
+    r.tl = lin % r.ntiles;
+    r.b = r.bh / Hh;
+    r.h = r.bh % Hh;
+    r.l0 = r.tl * kTile;
+    r.nrows = min(kTile, L - r.l0);
+    return r;
+}
+
+// ---------------------------------------------------------------- Q/K int8
+// Persistent CTAs of 128 threads; CTA c takes tiles c, c + G, c + 2G, ...
+// (G = gridDim.x) and thread r owns token row r of the current tile. Two
+// shared-memory tile buffers alternate: while tile i is converted, tile
+// i + 1 is in flight. The K mean of a head is finished here from the
+// statistics kernel's per-cluster fp64 sums (in cluster order).
+template <int D>
+__global__ void __launch_bounds__(kTile) qk_quant_kernel(
+    View4 q, View4 k, int blk_q, int blk_k, int n_qtiles, int n_tiles,
+    const double* __restrict__ ksum, int parts, int8_t* __restrict__ q8,
+    float* __restrict__ q_scale, int8_t* __restrict__ k8, float* __restrict__ k_scale,
+    float* __restrict__ k_mean, int qvec, int kvec) {
+    constexpr int PITCH = Tile<D>::kPitch;        // staged input row pitch (elements)
+    extern __shared__ __align__(128) uint16_t qk_smem[];
+    uint16_t* tiles = qk_smem;                    // [2][Tile<D>::kElems]
+    __shared__ __align__(16) float mean_s[D];
+    __shared__ float wmax[kTile / 32];
+
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int l0 = tl * kTile;
-    const int nrows = min(kTile, L - l0);
 
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (isK && tid < D) mean_s[tid] = kmean[(int64_t)bh * D + tid];
-    __syncthreads();
-    if (!stage_tile<D>(x, b, h, l0, nrows, vec, tile, &bar, &abort_flag, 1)) return;
-
-    const bool valid = tid < nrows;
-    float v[D];
-    {
-        const uint16_t* row = tile + tid * PITCH;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            const uint4 u = valid ? *reinterpret_cast<const uint4*>(row + 8 * c) : make_uint4(0, 0, 0, 0);
-            unpack8(u, v + 8 * c);
+    auto is_vec = [&](const QkTile& tr) { return (tr.isK ? kvec : qvec) != 0; };
+    // every thread commits one copy group per tile slot (empty for gathered
+    // tiles), so "at most one group pending" always means "the current tile
+    // has landed"
+    auto start = [&](int t, int buf) {
+        if (t < n_tiles) {
+            const QkTile tr = qk_tile(t, n_qtiles, q, k);
+            if (is_vec(tr))
+                issue_tile<D>(tr.isK ? k : q, tr.b, tr.h, tr.l0, tr.nrows, tiles + buf * Tile<D>::kElems);
         }
-    }
-    if (isK && valid) {
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c) {
-            const float4 m = *reinterpret_cast<const float4*>(mean_s + 4 * c);
-            v[4 * c] = __fsub_rn(v[4 * c], m.x);
-            v[4 * c + 1] = __fsub_rn(v[4 * c + 1], m.y);
-            v[4 * c + 2] = __fsub_rn(v[4 * c + 2], m.z);
-            v[4 * c + 3] = __fsub_rn(v[4 * c + 3], m.w);
+        cp_async_commit();
+    };
+    const int G = gridDim.x;
+    start(blockIdx.x, 0);
+    start(blockIdx.x + G, 1);
+
+    for (int it = 0, t = blockIdx.x; t < n_tiles; ++it, t += G) {
+        const int buf = it & 1;
+        uint16_t* tile = tiles + buf * Tile<D>::kElems;
+        const QkTile tr = qk_tile(t, n_qtiles, q, k);
+        const View4& x = tr.isK ? k : q;
+        if (tr.isK && tid < D) {
+            double sum = 0.0;
+            for (int pp = 0; pp < parts; ++pp) sum = __dadd_rn(sum, ksum[((int64_t)tr.bh * parts + pp) * D + tid]);
+            const float mn = __double2float_rn(__ddiv_rn(sum, (double)x.size[2]));
+            mean_s[tid] = mn;
+            if (k_mean != nullptr && tr.tl == 0) k_mean[(int64_t)tr.bh * D + tid] = mn;
         }
-    }
-    butterfly<D>(v);
+        cp_async_wait<1>();                      // this thread's copies of tile t are in
+        if (!is_vec(tr)) gather_tile<D>(x, tr.b, tr.h, tr.l0, tr.nrows, tile);
+        __syncthreads();                         // everyone's copies (and mean_s) are in
 
-    float a = 0.0f;
+        const bool valid = tid < tr.nrows;
+        uint64_t x2[D / 2];
+        {
+            const uint16_t* row = tile + tid * PITCH;
 #pragma unroll
-    for (int j = 0; j < D; ++j) a = fmaxf(a, fabsf(v[j]));
-    // a >= +0, so the bit patterns order like the values
-    const unsigned am = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
-    if (lane == 0) wmax[warp] = __uint_as_float(am);
-    __syncthreads();              // every row has left the tile; block maxima are in
-    const int wpb = blk / 32;     // warps per quantisation block (blk in {32, 64, 128})
-    const int w0 = (warp / wpb) * wpb;
-    float amax = 0.0f;
-    for (int w = w0; w < w0 + wpb; ++w) amax = fmaxf(amax, wmax[w]);
-    float s = 0.0f, rr = 0.0f;
-    if (amax != 0.0f) {
-        s = __fdiv_rn(amax, 127.0f);
-        rr = __fdiv_rn(127.0f, amax);
-    }
-    const int l = l0 + tid;
-    if (valid && (l & (blk - 1)) == 0) {
-        float* scales = isK ? k_scale : q_scale;
-        scales[(int64_t)bh * nb + l / blk] = s;
-    }
-
-    // |x_hat * r| <= a * fl(127 / a) rounds to at most 127 whenever r is
-    // finite, so the magic-number rounding needs no clamp; a block whose
-    // amax is so small that 127 / a overflows takes the clamped conversion.
-    uint8_t* ost = reinterpret_cast<uint8_t*>(tile);
-    uint8_t* orow = ost + tid * OPITCH;
-    if (isfinite(rr)) {
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 u = valid ? *reinterpret_cast<const uint4*>(row + 8 * c) : make_uint4(0, 0, 0, 0);
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float* p = v + 16 * c + 4 * i;
-                w4[i] = pack_round4(__fmul_rn(p[0], rr), __fmul_rn(p[1], rr), __fmul_rn(p[2], rr),
-                                    __fmul_rn(p[3], rr));
+                for (int e = 0; e < 4; ++e)
+                    x2[4 * c + e] = p2(bf16_bits_to_f32(w[e] & 0xFFFFu), __uint_as_float(w[e] & 0xFFFF0000u));
             }
-            *reinterpret_cast<uint4*>(orow + 16 * c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-    } else {
+        if (tr.isK && valid) {
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
-            uint32_t w4[4];
+            for (int c = 0; c < D / 2; ++c) x2[c] = p2sub(x2[c], *reinterpret_cast<const uint64_t*>(mean_s + 2 * c));
+        }
+        butterfly_pairs<D>(x2);
+
+        float a = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float* p = v + 16 * c + 4 * i;
-                w4[i] = pack_clamp4(__fmul_rn(p[0], rr), __fmul_rn(p[1], rr), __fmul_rn(p[2], rr),
-                                    __fmul_rn(p[3], rr));
+        for (int j = 0; j < D / 2; ++j) a = fmax3(a, fabsf(p2lo(x2[j])), fabsf(p2hi(x2[j])));
+        // a >= +0, so the bit patterns order like the values
+        const unsigned am = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+        if (lane == 0) wmax[warp] = __uint_as_float(am);
+        __syncthreads();              // every row has left the buffer; block maxima are in
+        start(t + 2 * G, buf);
+        const int blk = tr.isK ? blk_k : blk_q;
+        const int nb = static_cast<int>(ceil_div(x.size[2], blk));
+        const int wpb = blk / 32;     // warps per quantisation block (blk in {32, 64, 128})
+        const int w0 = (warp / wpb) * wpb;
+        float amax = 0.0f;
+        for (int w = w0; w < w0 + wpb; ++w) amax = fmaxf(amax, wmax[w]);
+        float s = 0.0f, rr = 0.0f;
+        if (amax != 0.0f) {
+            s = __fdiv_rn(amax, 127.0f);
+            rr = __fdiv_rn(127.0f, amax);
+        }
+        const int l = tr.l0 + tid;
+        if (valid && (l & (blk - 1)) == 0) {
+            float* scales = tr.isK ? k_scale : q_scale;
+            scales[(int64_t)tr.bh * nb + l / blk] = s;
+        }
+
+        // |x_hat * r| <= a * fl(127 / a) rounds to at most 127 whenever r is
+        // finite, so the magic-number rounding needs no clamp; a block whose
+        // amax is so small that 127 / a overflows takes the clamped conversion.
+        // Each thread stores its own code row (rows past L are the zero
+        // padding).
+        uint4* dst = reinterpret_cast<uint4*>((tr.isK ? k8 : q8) +
+                                              ((int64_t)tr.bh * tr.ntiles * kTile + tr.l0 + tid) * D);
+        if (isfinite(rr)) {
+            const uint64_t rr2 = p2(rr, rr), mg2 = p2(kRoundMagic, kRoundMagic);
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    // the product is rounded on its own (an FMA with +0), so the
+                    // magic add that follows cannot be contracted into it
+                    const uint64_t t01 = p2add(p2fma(x2[8 * c + 2 * i], rr2, 0ull), mg2);
+                    const uint64_t t23 = p2add(p2fma(x2[8 * c + 2 * i + 1], rr2, 0ull), mg2);
+                    w4[i] = __byte_perm(__byte_perm(__float_as_uint(p2lo(t01)), __float_as_uint(p2hi(t01)), 0x0040),
+                                        __byte_perm(__float_as_uint(p2lo(t23)), __float_as_uint(p2hi(t23)), 0x0040),
+                                        0x5410);
+                }
+                dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            *reinterpret_cast<uint4*>(orow + 16 * c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-    }
-    __syncthreads();
-    // the tile's 128 output rows are one contiguous run of 128 * D bytes
-    int8_t* dst = (isK ? k8 : q8) + ((int64_t)bh * ntiles * kTile + l0) * D;
+        } else {
 #pragma unroll
-    for (int i = tid; i < kTile * (D / 16); i += kTile) {
-        const int r = i / (D / 16), c = i % (D / 16);
-        reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(ost + r * OPITCH + 16 * c);
+            for (int c = 0; c < D / 16; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint64_t* pv = x2 + 8 * c + 2 * i;
+                    w4[i] = pack_clamp4(__fmul_rn(p2lo(pv[0]), rr), __fmul_rn(p2hi(pv[0]), rr),
+                                        __fmul_rn(p2lo(pv[1]), rr), __fmul_rn(p2hi(pv[1]), rr));
+                }
+                dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+        }
     }
 }
 
 // ---------------------------------------------------------------- V e4m3
-// One CTA of 128 threads per (b, h, 128-token tile). Thread t covers the
-// channel pair (2p, 2p + 1), p = t % (D/2), over the token group t / (D/2).
-// Writes V transposed: v8t[b, h, d, token].
+// Persistent CTAs of 128 threads over 128-token tiles of V, the same
+// two-buffer ring as qk_quant_kernel. Thread t covers the channel pair
+// (2p, 2p + 1), p = t % (D/2), over the token group t / (D/2), and stores its
+// codes straight to the transposed output v8t[b, h, d, token]. The channel
+// maxima are finished here from the statistics kernel's per-cluster maxima;
+// the first tile of each head also writes its v_scale.
 template <int D>
-__global__ void __launch_bounds__(kTile) v_quant_kernel(View4 x, const float* __restrict__ vmul,
+__global__ void __launch_bounds__(kTile) v_quant_kernel(View4 x, int n_tiles,
+                                                        const float* __restrict__ vmax, int parts,
+                                                        float* __restrict__ v_scale,
                                                         uint8_t* __restrict__ v8t, int vec) {
-    constexpr int PITCH = D + 8;
+    constexpr int PITCH = Tile<D>::kPitch;
     constexpr int P = D / 2;                     // channel pairs
     constexpr int G = kTile / P;                 // token groups
     constexpr int TT = kTile / G;                // tokens per thread
-    constexpr int OPITCH = kTile + 16;           // staged output row pitch (bytes)
-    static_assert(D * OPITCH <= kTile * PITCH * 2, "output staging reuses the tile");
-    __shared__ __align__(128) uint16_t tile[kTile * PITCH];
+    extern __shared__ __align__(128) uint16_t v_smem[];
+    uint16_t* tiles = v_smem;                    // [2][Tile<D>::kElems]
     __shared__ float rmul[D];
-    __shared__ __align__(8) uint64_t bar;
-    __shared__ int abort_flag;
 
     const int L = static_cast<int>(x.size[2]);
     const int Hh = static_cast<int>(x.size[1]);
     const int ntiles = static_cast<int>(ceil_div(L, kTile));
-    const int bh = blockIdx.x / ntiles, tl = blockIdx.x % ntiles;
-    const int b = bh / Hh, h = bh % Hh;
     const int tid = threadIdx.x;
-    const int l0 = tl * kTile;
-    const int nrows = min(kTile, L - l0);
 
-    if (tid == 0) {
-        mbar_init(&bar, 1);
-        abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (tid < D) rmul[tid] = vmul[(int64_t)bh * D + tid];
-    __syncthreads();
-    if (!stage_tile<D>(x, b, h, l0, nrows, vec != 0, tile, &bar, &abort_flag, 2)) return;
+    // one copy group per tile slot and thread (empty for gathered views)
+    auto start = [&](int t, int buf) {
+        if (t < n_tiles && vec) {
+            const int bh = t / ntiles, tl = t % ntiles;
+            issue_tile<D>(x, bh / Hh, bh % Hh, tl * kTile, min(kTile, L - tl * kTile),
+                          tiles + buf * Tile<D>::kElems);
+        }
+        cp_async_commit();
+    };
+    const int GS = gridDim.x;
+    start(blockIdx.x, 0);
+    start(blockIdx.x + GS, 1);
 
     const int p = tid % P, g = tid / P;
-    const float r0 = rmul[2 * p], r1 = rmul[2 * p + 1];
-    uint32_t w0[TT / 4], w1[TT / 4];
-#pragma unroll
-    for (int t4 = 0; t4 < TT / 4; ++t4) {
-        float y0[4], y1[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int tok = g * TT + 4 * t4 + i;
-            const uint32_t u =
-                tok < nrows ? *reinterpret_cast<const uint32_t*>(tile + tok * PITCH + 2 * p) : 0u;
-            y0[i] = __fmul_rn(bf16_bits_to_f32(u & 0xFFFFu), r0);
-            y1[i] = __fmul_rn(__uint_as_float(u & 0xFFFF0000u), r1);
+    for (int it = 0, t = blockIdx.x; t < n_tiles; ++it, t += GS) {
+        const int buf = it & 1;
+        uint16_t* tile = tiles + buf * Tile<D>::kElems;
+        const int bh = t / ntiles, tl = t % ntiles;
+        const int l0 = tl * kTile;
+        const int nrows = min(kTile, L - l0);
+        if (tid < D) {
+            float a = 0.0f;
+            for (int pp = 0; pp < parts; ++pp) a = fmaxf(a, vmax[((int64_t)bh * parts + pp) * D + tid]);
+            float sc = 0.0f, r = 0.0f;
+            if (a != 0.0f) {
+                sc = __fdiv_rn(a, 448.0f);
+                r = __fdiv_rn(448.0f, a);
+            }
+            rmul[tid] = r;
+            if (tl == 0) v_scale[(int64_t)bh * D + tid] = sc;
         }
-        w0[t4] = e4m3x2_rn_satfinite(y0[0], y0[1]) | (uint32_t(e4m3x2_rn_satfinite(y0[2], y0[3])) << 16);
-        w1[t4] = e4m3x2_rn_satfinite(y1[0], y1[1]) | (uint32_t(e4m3x2_rn_satfinite(y1[2], y1[3])) << 16);
-    }
-    __syncthreads();              // every read of the tile is done
-    uint8_t* ost = reinterpret_cast<uint8_t*>(tile);
+        cp_async_wait<1>();                      // this thread's copies of tile t are in
+        if (!vec) gather_tile<D>(x, bh / Hh, bh % Hh, l0, nrows, tile);
+        __syncthreads();                         // everyone's copies (and rmul) are in
+
+        const uint64_t r2 = p2(rmul[2 * p], rmul[2 * p + 1]);
+        uint32_t w0[TT / 4], w1[TT / 4];
 #pragma unroll
-    for (int c = 0; c < TT / 16; ++c) {
-        *reinterpret_cast<uint4*>(ost + (2 * p) * OPITCH + g * TT + 16 * c) =
-            make_uint4(w0[4 * c], w0[4 * c + 1], w0[4 * c + 2], w0[4 * c + 3]);
-        *reinterpret_cast<uint4*>(ost + (2 * p + 1) * OPITCH + g * TT + 16 * c) =
-            make_uint4(w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
-    }
-    __syncthreads();
-    const int64_t Lpad = (int64_t)ntiles * kTile;
-    uint8_t* dst = v8t + (int64_t)bh * D * Lpad + l0;
+        for (int t4 = 0; t4 < TT / 4; ++t4) {
+            float y0[4], y1[4];
 #pragma unroll
-    for (int i = tid; i < D * (kTile / 16); i += kTile) {
-        const int d = i / (kTile / 16), c = i % (kTile / 16);
-        *reinterpret_cast<uint4*>(dst + (int64_t)d * Lpad + 16 * c) =
-            *reinterpret_cast<const uint4*>(ost + d * OPITCH + 16 * c);
+            for (int i = 0; i < 4; ++i) {
+                const int tok = g * TT + 4 * t4 + i;
+                const uint32_t u =
+                    tok < nrows ? *reinterpret_cast<const uint32_t*>(tile + tok * PITCH + 2 * p) : 0u;
+                const uint64_t y = p2mul(p2(bf16_bits_to_f32(u & 0xFFFFu), __uint_as_float(u & 0xFFFF0000u)), r2);
+                y0[i] = p2lo(y);
+                y1[i] = p2hi(y);
+            }
+            w0[t4] = e4m3x2_rn_satfinite(y0[0], y0[1]) | (uint32_t(e4m3x2_rn_satfinite(y0[2], y0[3])) << 16);
+            w1[t4] = e4m3x2_rn_satfinite(y1[0], y1[1]) | (uint32_t(e4m3x2_rn_satfinite(y1[2], y1[3])) << 16);
+        }
+        __syncthreads();              // every read of the buffer is done
+        start(t + 2 * GS, buf);
+        // channels 2p and 2p + 1, tokens [g TT, g TT + TT) of the tile: two
+        // contiguous runs of TT bytes in the transposed output
+        const int64_t Lpad = (int64_t)ntiles * kTile;
+        uint8_t* dst = v8t + ((int64_t)bh * D + 2 * p) * Lpad + l0 + g * TT;
+#pragma unroll
+        for (int c = 0; c < TT / 16; ++c) {
+            reinterpret_cast<uint4*>(dst)[c] = make_uint4(w0[4 * c], w0[4 * c + 1], w0[4 * c + 2], w0[4 * c + 3]);
+            reinterpret_cast<uint4*>(dst + Lpad)[c] =
+                make_uint4(w1[4 * c], w1[4 * c + 1], w1[4 * c + 2], w1[4 * c + 3]);
+        }
     }
+}
+
+// Clusters per (b, h) for the statistics kernels: about three 256-thread
+// CTAs per SM over the whole grid, between 1 and kMaxParts.
+int stat_parts(int BH) {
+    const int want = num_sms() * 3;
+    const int per_part = BH * kStatCluster;
+    return std::max(1, std::min(kMaxParts, (want + per_part / 2) / per_part));
+}
+
+template <int D>
+size_t quant_smem_bytes() {
+    return 2 * Tile<D>::kElems * sizeof(uint16_t);
+}
+
+template <int D>
+cudaError_t launch_qk_d(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
+                        float* q_scale, int8_t* k8, float* k_scale, float* k_mean, void* ws,
+                        cudaStream_t s) {
+    const int B = (int)q.size[0], H = (int)q.size[1], Lq = (int)q.size[2];
+    const int Hk = (int)k.size[1], Lk = (int)k.size[2];
+    const int parts = stat_parts(B * Hk);
+    column_stats_kernel<D, 0><<<kStatCluster * parts * B * Hk, kStatThreads, 0, s>>>(
+        k, parts, ws, view_vec8(k));
+    const int n_qtiles = B * H * (int)ceil_div(Lq, kTile);
+    const int n_tiles = n_qtiles + B * Hk * (int)ceil_div(Lk, kTile);
+    const int grid = std::min(n_tiles, num_sms() * kQuantCtasPerSm);
+    auto kern = qk_quant_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)quant_smem_bytes<D>());
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kTile, quant_smem_bytes<D>(), s>>>(q, k, blk_q, blk_k, n_qtiles, n_tiles,
+                                                    static_cast<const double*>(ws), parts, q8,
+                                                    q_scale, k8, k_scale, k_mean, view_vec8(q),
+                                                    view_vec8(k));
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_v_d(const View4& v, uint8_t* v8t, float* v_scale, void* ws, cudaStream_t s) {
+    const int B = (int)v.size[0], Hk = (int)v.size[1], L = (int)v.size[2];
+    const int parts = stat_parts(B * Hk);
+    column_stats_kernel<D, 1><<<kStatCluster * parts * B * Hk, kStatThreads, 0, s>>>(
+        v, parts, ws, view_vec8(v));
+    const int n_tiles = B * Hk * (int)ceil_div(L, kTile);
+    const int grid = std::min(n_tiles, num_sms() * kQuantCtasPerSm);
+    auto kern = v_quant_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)quant_smem_bytes<D>());
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kTile, quant_smem_bytes<D>(), s>>>(v, n_tiles, static_cast<const float*>(ws), parts,
+                                                    v_scale, v8t, view_vec8(v));
+    return cudaGetLastError();
 }
 
 }  // namespace
 
 size_t quant_qk_ws_bytes(int B, int Hk, int Lk, int D) {
     (void)Lk;
-    return (size_t)B * Hk * D * sizeof(float);
+    return (size_t)B * Hk * kMaxParts * D * sizeof(double);
 }
 
 size_t quant_v_ws_bytes(int B, int Hk, int L, int D) {
     (void)L;
-    return (size_t)B * Hk * D * sizeof(float);
+    return (size_t)B * Hk * kMaxParts * D * sizeof(float);
 }
 
 cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
                             float* q_scale, int8_t* k8, float* k_scale, float* k_mean, void* ws,
                             cudaStream_t s) {
-    const int B = (int)q.size[0], H = (int)q.size[1], Lq = (int)q.size[2], D = (int)q.size[3];
-    const int Hk = (int)k.size[1], Lk = (int)k.size[2];
-    const int kvec = view_vec8(k), qvec = view_vec8(q);
-    float* mean = static_cast<float*>(ws);
-    const int sgrid = kStatCluster * B * Hk;
-    const int n_qtiles = B * H * (int)ceil_div(Lq, kTile);
-    const int n_ktiles = B * Hk * (int)ceil_div(Lk, kTile);
-    if (D == 128) {
-        column_stats_kernel<128, 0><<<sgrid, kStatThreads, 0, s>>>(k, mean, k_mean, kvec);
-        qk_quant_kernel<128><<<n_qtiles + n_ktiles, kTile, 0, s>>>(
-            q, k, blk_q, blk_k, n_qtiles, mean, q8, q_scale, k8, k_scale, qvec, kvec);
-    } else {
-        column_stats_kernel<64, 0><<<sgrid, kStatThreads, 0, s>>>(k, mean, k_mean, kvec);
-        qk_quant_kernel<64><<<n_qtiles + n_ktiles, kTile, 0, s>>>(
-            q, k, blk_q, blk_k, n_qtiles, mean, q8, q_scale, k8, k_scale, qvec, kvec);
-    }
-    return cudaGetLastError();
+    return q.size[3] == 128
+               ? launch_qk_d<128>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s)
+               : launch_qk_d<64>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s);
 }
 
 cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,
                            cudaStream_t s) {
-    const int B = (int)v.size[0], Hk = (int)v.size[1], L = (int)v.size[2], D = (int)v.size[3];
-    const int vec = view_vec8(v);
-    float* vmul = static_cast<float*>(ws);
-    const int sgrid = kStatCluster * B * Hk;
-    const int ntiles = B * Hk * (int)ceil_div(L, kTile);
-    if (D == 128) {
-        column_stats_kernel<128, 1><<<sgrid, kStatThreads, 0, s>>>(v, vmul, v_scale, vec);
-        v_quant_kernel<128><<<ntiles, kTile, 0, s>>>(v, vmul, v8t, vec);
-    } else {
-        column_stats_kernel<64, 1><<<sgrid, kStatThreads, 0, s>>>(v, vmul, v_scale, vec);
-        v_quant_kernel<64><<<ntiles, kTile, 0, s>>>(v, vmul, v8t, vec);
-    }
-    return cudaGetLastError();
+    return v.size[3] == 128 ? launch_v_d<128>(v, v8t, v_scale, ws, s)
+                            : launch_v_d<64>(v, v8t, v_scale, ws, s);
 }
 
 unsigned read_clear_quant_error() {
@@ -493,16 +627,15 @@ unsigned read_clear_quant_error() {
 }
 
 }  // namespace sage
-
 // ---------------------------------------------------------------- no-allocation variant
 // sage_quant_qk_noalloc: the same Q/K smoothing + rotation + INT8 quantisation
 // as sage_quant_qk, for callers that cannot allocate device memory at the
 // point of the call -- for instance a serving loop whose device memory is
 // budgeted once at start-up, or code that must not risk the implicit device
-// synchronisation that cudaMalloc / cudaFree can cause. Its scratch (the fp32
-// per-channel mean of K, written by the statistics kernel before the
-// quantisation kernel reads it) lives in the fixed array below instead of a
-// caller workspace.
+// synchronisation that cudaMalloc / cudaFree can cause. Its scratch (the fp64
+// per-cluster column sums of K, written by the statistics kernel before the
+// quantisation kernel reads them) lives in the fixed array below instead of
+// a caller workspace.
 #include <mutex>
 
 #include "../../include/sage.h"

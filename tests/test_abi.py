@@ -53,9 +53,9 @@ def test_status_strings(L):
 
 
 def test_workspace_sizes_are_host_only(L):
-    # K: the fp32 mean per (b, kv head, d); V: the fp32 multiplier 448 / a per (b, h, d)
-    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 128 * 4
-    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 128 * 4
+    # up to 8 partial statistics per (b, kv head, d): fp64 sums of K, fp32 maxima of V
+    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 8 * 128 * 8
+    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 8 * 128 * 4
     assert L.sage_attn_fwd_workspace(1, 24, 24, 4096, 4096, 128) == 0
     assert L.sage_quant_qk_workspace(0, 1, 1, 1, 1, 64) == 0
 
