@@ -85,12 +85,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;   // log2(FP8_MAX of e4m3)
 constexpr int kMagicI = 0x4B400000;               // bit pattern of 1.5 * 2^23
 constexpr float kMagicF = 12582912.0f;            // 1.5 * 2^23
-// every kPolyEvery-th key pair takes its exponential from exp2_poly_x2
-// instead of the MUFU unit (0 = never)
+// every kPolyEvery-th key pair takes its exponential from exp2_poly_x2 (FMA
+// pipe) instead of the MUFU unit, which relieves the MUFU queue of the warp
+// converting its row (0 = never)
 #ifndef SAGE_POLY_EVERY
-#define SAGE_POLY_EVERY 0
+#define SAGE_POLY_EVERY 8
 #endif
 constexpr int kPolyEvery = SAGE_POLY_EVERY;
+
 
 // K block scales of one head staged in shared memory (larger heads read the
 // rest from global memory)
