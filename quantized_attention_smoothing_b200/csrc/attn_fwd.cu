@@ -296,6 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float* ks_s = reinterpret_cast<float*>(smem + C::kOffKs);
     float* vs_s = reinterpret_cast<float*>(smem + C::kOffVs);
+    // launched as a programmatic dependent of the V quantisation: everything
+    // above overlapped its tail; the quantised operands are read only below
+    pdl_wait();
     {
         const float* ksrc = p.k_scale + (int64_t)bhk * p.nbk;
         const int nks = min(p.nbk, kKsSmem);
@@ -646,8 +649,8 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, Cfg<D>::kSmemBytes, s>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    e = launch_pdl(kern, grid, dim3(kThreads), Cfg<D>::kSmemBytes, s, tq, tk, tv, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, int NKB>

@@ -24,7 +24,9 @@
 //                        memory and its leader writes the partial column
 //                        statistic (fp64 sums for K, fp32 maxima for V).
 //   qk_quant_kernel      persistent CTAs over 128-token tiles (Q tiles, then
-//                        K tiles). Each CTA keeps two tiles in flight: the
+//                        K tiles), launched as a programmatic dependent of
+//                        the K statistics kernel: Q tiles run while the
+//                        statistics are computed, K tiles wait for them. Each CTA keeps two tiles in flight: the
 //                        next tile arrives in shared memory by coalesced
 //                        16-byte cp.async copies while the current one is
 //                        converted, one
@@ -94,6 +96,7 @@ __device__ __forceinline__ void unpack8(const uint4& u, float* x) {
 template <int D, int MODE>
 __global__ void __cluster_dims__(kStatCluster, 1, 1) __launch_bounds__(kStatThreads)
     column_stats_kernel(View4 x, int parts, void* __restrict__ ws, int vec) {
+    pdl_launch_dependents();                      // the quantisation kernel may start now
     constexpr int TPR = D / 8;                    // threads per token row
     constexpr int RPI = kStatThreads / TPR;       // token rows per load round
     using Acc = typename std::conditional<MODE == 0, double, float>::type;
@@ -348,11 +351,17 @@ __global__ void __launch_bounds__(kTile) qk_quant_kernel(
     start(blockIdx.x, 0);
     start(blockIdx.x + G, 1);
 
+    bool stats_ready = false;
     for (int it = 0, t = blockIdx.x; t < n_tiles; ++it, t += G) {
         const int buf = it & 1;
         uint16_t* tile = tiles + buf * Tile<D>::kElems;
         const QkTile tr = qk_tile(t, n_qtiles, q, k);
         const View4& x = tr.isK ? k : q;
+        if (tr.isK && !stats_ready) {
+            // Q tiles ran alongside the statistics kernel; K tiles need its sums
+            pdl_wait();
+            stats_ready = true;
+        }
         if (tr.isK && tid < D) {
             double sum = 0.0;
             for (int pp = 0; pp < parts; ++pp) sum = __dadd_rn(sum, ksum[((int64_t)tr.bh * parts + pp) * D + tid]);
@@ -485,6 +494,8 @@ __global__ void __launch_bounds__(kTile) v_quant_kernel(View4 x, int n_tiles,
     const int GS = gridDim.x;
     start(blockIdx.x, 0);
     start(blockIdx.x + GS, 1);
+    pdl_wait();                                  // the channel maxima are complete
+    pdl_launch_dependents();                     // the attention kernel may start its prologue
 
     const int p = tid % P, g = tid / P;
     for (int it = 0, t = blockIdx.x; t < n_tiles; ++it, t += GS) {
@@ -569,11 +580,11 @@ cudaError_t launch_qk_d(const View4& q, const View4& k, int blk_q, int blk_k, in
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)quant_smem_bytes<D>());
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTile, quant_smem_bytes<D>(), s>>>(q, k, blk_q, blk_k, n_qtiles, n_tiles,
-                                                    static_cast<const double*>(ws), parts, q8,
-                                                    q_scale, k8, k_scale, k_mean, view_vec8(q),
-                                                    view_vec8(k));
-    return cudaGetLastError();
+    // programmatic launch: the Q tiles overlap the statistics kernel
+    e = launch_pdl(kern, dim3(grid), dim3(kTile), quant_smem_bytes<D>(), s, q, k, blk_q, blk_k,
+                   n_qtiles, n_tiles, static_cast<const double*>(ws), parts, q8, q_scale, k8,
+                   k_scale, k_mean, view_vec8(q), view_vec8(k));
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D>
@@ -588,9 +599,9 @@ cudaError_t launch_v_d(const View4& v, uint8_t* v8t, float* v_scale, void* ws, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)quant_smem_bytes<D>());
     if (e != cudaSuccess) return e;
-    kern<<<grid, kTile, quant_smem_bytes<D>(), s>>>(v, n_tiles, static_cast<const float*>(ws), parts,
-                                                    v_scale, v8t, view_vec8(v));
-    return cudaGetLastError();
+    e = launch_pdl(kern, dim3(grid), dim3(kTile), quant_smem_bytes<D>(), s, v, n_tiles,
+                   static_cast<const float*>(ws), parts, v_scale, v8t, view_vec8(v));
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

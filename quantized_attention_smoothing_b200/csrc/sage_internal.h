@@ -29,6 +29,25 @@ constexpr unsigned kErrTimeoutCode = 1u;    // low byte of a device error word
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
+// Launch `kern` with programmatic stream serialisation: it may start while
+// the preceding kernel of the stream is still running, and must call
+// griddepcontrol.wait before touching that kernel's outputs.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+}
+
 // Number of SMs of the current device (looked up once per device).
 inline int num_sms() {
     static int cache[64] = {};

@@ -102,6 +102,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// ------------------------------------------------------------ programmatic dependent launch
+
+// Let the next kernel in the stream (launched with programmatic stream
+// serialisation) start scheduling its CTAs.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the preceding kernel in the stream has completed and its memory
+// operations are visible (no-op when this kernel was not launched as a
+// dependent).
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------ TMA
 
 // Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
