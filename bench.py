@@ -80,6 +80,25 @@ def attn_traffic():
     return int(m_b.group(1))
 
 
+def rank_max(x, world, device):
+    """Max of a per-rank scalar over all ranks of the default process group
+    (identity for a single rank): every multi-rank time in the JSON line is
+    the slowest rank's."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(ops_per_step, steps, world, elapsed_ms):
+    """Whole-job TOPS: each of `world` ranks runs its own replica of the
+    workload (`ops_per_step` per step), timed as the slowest rank."""
+    return world * ops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 def work_ops(cfg):
     ops = 4.0 * cfg["B"] * cfg["H"] * cfg["L"] * cfg["L"] * cfg["D"]
     return ops / 2 if cfg["causal"] else ops
@@ -284,11 +303,7 @@ def run_sage(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(x, world, "cuda")
 
     cfg = dict(workloads.PREFILL[args.workload], key=args.workload)
     B, H, Hk, L, D = cfg["B"], cfg["H"], cfg["Hk"], cfg["L"], cfg["D"]
@@ -342,7 +357,7 @@ def run_sage(args):
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1))
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     ops = work_ops(cfg)
-    value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_value(ops, args.steps, world, elapsed_ms)
 
     pk, pk_src = peaks()
     peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
@@ -386,7 +401,7 @@ def run_sage(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e = {"value": world * ops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+    e2e = {"value": job_value(ops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
            "d2h_bytes_per_step": oh.numel() * oh.element_size(),
            "ms_per_step": e2e_ms / args.e2e_steps}
