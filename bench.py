@@ -369,42 +369,67 @@ def run_sage(args):
                 "attn_ms": attn_ms}
 
     # end to end through the public API: pinned host inputs -> device ->
-    # quantise + attention -> result back to pinned host memory, every step
+    # quantise + attention -> result back to pinned host memory, every step.
+    # Steps are pipelined over two device buffer pairs and three streams
+    # (host->device copies, compute, device->host copies): the inputs of step
+    # i + 1 travel while step i computes and step i - 1's result comes back.
     qh = q.permute(0, 2, 1, 3).contiguous().pin_memory()      # [B, L, H, D] host buffers
     kh = k.permute(0, 2, 1, 3).contiguous().pin_memory()
     vh = v.permute(0, 2, 1, 3).contiguous().pin_memory()
-    oh = torch.empty((B, L, H, D), dtype=torch.bfloat16).pin_memory()
-    qd, kd, vd = (torch.empty_like(x, device="cuda") for x in (qh, kh, vh))
-    od = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda")
+    oh = [torch.empty((B, L, H, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dev_in = [[torch.empty_like(x, device="cuda") for x in (qh, kh, vh)] for _ in range(2)]
+    dev_out = [torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     ebufs = sets[0][3]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    n_e2e = args.e2e_steps + 2
+    ev_in = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_comp = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_out = [torch.cuda.Event() for _ in range(n_e2e)]
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        qd, kd, vd = dev_in[j]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[i - 2])        # step i - 2 has read these inputs
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            ev_in[i].record(s_in)
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_out[i - 2])           # step i - 2's result has left dev_out[j]
         sage.sage_attention(h, qd.permute(0, 2, 1, 3), kd.permute(0, 2, 1, 3),
                             vd.permute(0, 2, 1, 3), blk_q, blk_k, scale, causal,
-                            out=od.permute(0, 2, 1, 3), bufs=ebufs, stream=stream)
-        oh.copy_(od, non_blocking=True)
+                            out=dev_out[j].permute(0, 2, 1, 3), bufs=ebufs, stream=stream)
+        ev_comp[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[i])
+            oh[j].copy_(dev_out[j], non_blocking=True)
+            ev_out[i].record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(args.e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[args.e2e_steps - 1])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     e2e = {"value": job_value(ops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
-           "d2h_bytes_per_step": oh.numel() * oh.element_size(),
-           "ms_per_step": e2e_ms / args.e2e_steps}
+           "d2h_bytes_per_step": oh[0].numel() * oh[0].element_size(),
+           "ms_per_step": e2e_ms / args.e2e_steps,
+           "pipeline": "h2d, compute and d2h on three streams over two buffer pairs"}
 
     dec = None if args.no_decode else bench_decode(sage, torch, stream)
 
