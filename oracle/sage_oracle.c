@@ -411,7 +411,9 @@ void or_attn_exact_head(const uint16_t* q, const uint16_t* k, const uint16_t* v,
  *   large enough; the T tokens are causal among themselves).
  *   S_j = (sum_e dec(q8_e) dec(k8_je)) * s * ksc_j * softmax_scale / D
  *   (the cached keys are taken as already rotated, so the same 1/D holds).
- *   Exact fp64 softmax over the window; out = sum_j p_j vsc_j dec(v8_j).
+ *   fp64 softmax over the window (m = max_j S_j, p_j = exp(S_j - m));
+ *   PV on bf16 operands ([PA], Changes: PV_BF16): w_j = bf16(fp32(p_j) *
+ *   vsc_j), exact bf16 of dec(v8_j); out = sum_j w_j dec(v8_j) / sum_j p_j.
  * out[T][H][D] bf16. */
 void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
                    const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
@@ -458,7 +460,10 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
                 const int64_t tok = (phys * Hk + hk) * page + (j % page);
                 double pj = exp(sv[u] - mx);
                 den += pj;
-                double w = pj * (double)vsc[tok];
+                /* PV on bf16 operands: the weight p_j * v_scale_j is formed
+                   in fp32 and rounded to bf16 (nearest even) */
+                const float wf = (float)pj * vsc[tok];
+                double w = (double)or_bf16_to_f32(or_f64_to_bf16((double)wf));
                 for (int e = 0; e < D; ++e) o[e] += w * or_e4m3_decode(vc[tok * D + e]);
             }
             for (int e = 0; e < D; ++e) {

@@ -5,29 +5,42 @@
 // to the FP8 format of the cache (Q here), PV on bf16 operands because a
 // per-token V scale cannot be factored out of the sum).
 //
-// Split-KV. decode_split_kernel: CTA (split, b * Hk + hk), 8 warps, handles
-// up to 512 consecutive keys of the union of the T query tokens' windows for
-// all R = T * (H / Hk) query rows of kv head hk. Two warpgroups take
-// alternate 64-key chunks (16 rows per warp) with their own running softmax
-// state, merged at the end:
-//   0. the keys' cache rows are looked up through the page table (page ids
-//      bounds-checked) and every K row, V row and per-token scale of the
-//      split is requested at once with cp.async, one commit group per
-//      64-key chunk;
-//   1. while those land, the Q rows are rotated and quantised: bf16 -> fp32
-//      butterfly (two threads per row, the last stage across the pair by
-//      shuffles) -> e4m3 with scale max|q_hat| / 448 (the fp32 operations
-//      of the quantisation kernels);
-//   2. per 64-key chunk, once its copies have landed: V decoded exactly to
-//      bf16; S = Q8 K8^T with e4m3 mma.sync (fp32 accumulate), scaled by
-//      s_q * s_k * softmax_scale / D, masked to each row's own window (no
-//      per-key test for chunks inside every row's window);
-//      online softmax in base 2; P' = p * s_v rounded to bf16; O += P' V with
-//      bf16 mma.sync;
-//   3. the second warpgroup's (m, l, O) merged into the first's, then to the
-//      workspace.
-// decode_combine_kernel merges the splits (log-sum-exp) and writes bf16
-// through the caller's strides.
+// One kernel. The keys of sequence b (the union of its T query tokens'
+// windows, [lo, ctx)) are cut into 128-key tiles aligned to absolute key
+// positions, so a tile is one page (page 128) or 128 / page whole pages.
+// The tiles of (b, kv head hk) are shared out among up to 8 CTAs that form
+// one thread-block cluster; CTA = 16 warps:
+//   warps 0-7  softmax: warps w and w + 4 own query rows 16w .. 16w + 15
+//              (R = T * H/Hk rows, row r = t * G + g, padded to 64) -- M = 64
+//              MMAs keep those rows in TMEM lanes 32w .. 32w + 15 -- warp w
+//              the tile's columns 0-63, warp w + 4 columns 64-127;
+//   warps 8-11 V converters: e4m3 V tile -> exact bf16, in the key order of
+//              the P operand;
+//   warp 12    producer: page-table lookups, one TMA box per page for K and
+//              for V, per-token scales by cp.async, all on one mbarrier;
+//   warp 13    TMEM owner and MMA issuer (warps 14, 15 only join the merge).
+// Per tile: S = Q8 K8^T (e4m3 tcgen05 MMAs, M=64 N=128, fp32 in TMEM,
+// double-buffered) -> logits S * s_q * k_scale_j * softmax_scale / D in
+// base 2, masked to each row's own window -> running max m -> p = 2^(x - m)
+// -> P' = bf16(p * v_scale_j) -> O[i & 1] += P' V (bf16 tcgen05 MMAs, fp32
+// in TMEM). Even and odd tiles accumulate into two O's, so the rescale of
+// the one tile i adds to (by 2^(m_old - m) for rows whose max rose) waits
+// for PV(i - 2), not for PV(i - 1); the epilogue adds the two at the final
+// max. The query rows are rotated and quantised to e4m3 in the prologue
+// (fp32 butterfly, scale max|q_hat| / 448, the operations of the quantisation
+// kernels). At the end every CTA leaves (m, l, O) of its tiles in shared
+// memory and the CTAs of the cluster merge them (log-sum-exp) through
+// distributed shared memory and write bf16 through the caller's strides.
+//
+// Every mbarrier wait is bounded; on timeout the CTA records an error word,
+// raises its abort flag, drains its own copies and MMAs and still takes part
+// in both cluster barriers.
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -38,151 +51,126 @@ namespace sage {
 namespace {
 
 __device__ unsigned g_decode_err;
-constexpr unsigned kErrDecodeRange = 2u;     // ctx or page id out of range (clamped)
+constexpr unsigned kErrDecodeRange = 2u;     // ctx or page id out of range (clamped / masked)
 
 constexpr int kD = 128;
-constexpr int kSplit = 512;                  // keys per CTA
-constexpr int kChunk = 64;                   // keys per inner step
-constexpr int kNChunk = kSplit / kChunk;     // 64-key chunks per CTA
-constexpr int kDecThreads = 256;             // two warpgroups of 4 warps
-constexpr int kMaxRows = 64;                 // T * (H / Hk)
-constexpr int kKPitch = kD + 16;             // bytes per K row in smem
-constexpr int kVPitch = kD + 8;              // bf16 elements per V row in smem
+constexpr int kKeys = 128;                   // keys per tile
+constexpr int kRows = 64;                    // query rows per CTA (M of every MMA)
+constexpr int kStages = 3;                   // K / V / scale ring
+constexpr int kMaxSplit = 8;                 // CTAs per (sequence, kv head) = cluster size
+constexpr int kSoftWarps = 8;                // warps 0..7
+constexpr int kConvWarp0 = 8;                // warps 8..11
+constexpr int kTmaWarp = 12;
+constexpr int kMmaWarp = 13;                 // warps 14, 15 idle until the merge
+constexpr int kThreads = 512;
+// registers per thread of each warpgroup (setmaxnreg; 256 x 192 + 128 x 64 +
+// 128 x 56 <= 512 x 128, the launch's registers). Only the softmax warps ever
+// grow their share, after the others have shrunk theirs, and no warp grows
+// it again later: a warp that did could take registers another one waits for.
+constexpr int kRegsSoft = 192, kRegsConv = 64, kRegsProd = 56;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kOcPitch = kD + 4;             // fp32 row pitch of the merge area
 
-// dynamic shared memory of decode_split_kernel
-struct DecSmem {
-    static constexpr int kOffK = 0;                                   // [kSplit][kKPitch] e4m3
-    static constexpr int kOffV = kOffK + kSplit * kKPitch;            // [kSplit][kD] e4m3
-    static constexpr int kOffVbf = kOffV + kSplit * kD;               // [2][kChunk][kVPitch] bf16
-    static constexpr int kOffQ = kOffVbf + 2 * kChunk * kVPitch * 2;  // [kMaxRows][kD] e4m3
-    static constexpr int kOffKs = kOffQ + kMaxRows * kD;              // [kSplit] fp32
-    static constexpr int kOffVs = kOffKs + kSplit * 4;                // [kSplit] fp32
-    static constexpr int kOffTok = kOffVs + kSplit * 4;               // [kSplit] int64 (-1: none)
-    static constexpr int kOffSq = kOffTok + kSplit * 8;               // [kMaxRows] fp32
-    static constexpr int kOffBad = kOffSq + kMaxRows * 4;             // [kNChunk] int
-    static constexpr int kBytes = kOffBad + kNChunk * 4;
-    // merge area of the second warpgroup's state, over the K rows (read by then)
-    static constexpr int kMergeBytes = 4 * 32 * (64 + 4) * 4;
-    static_assert(kMergeBytes <= kSplit * kKPitch, "merge area");
-    static_assert(kBytes <= 227 * 1024, "shared memory");
+// dynamic shared memory (offsets from a 1024-byte aligned base)
+struct Sm {
+    static constexpr int kQ = 0;                                   // [64][128] e4m3, 128B swizzle
+    static constexpr int kKStage = kKeys * kD;                     // 16 KB
+    static constexpr int kK = kQ + kRows * kD;                     // [stage][128][128] e4m3, 128B swizzle
+    static constexpr int kV = kK + kStages * kKStage;              // [stage][128][128] e4m3, 128B swizzle
+    static constexpr int kPBuf = 2 * kRows * 128;                  // two 64-key atoms [64][128 B] bf16
+    static constexpr int kP = kV + kStages * kKStage;              // [2 bufs] P' (A of PV)
+    static constexpr int kVbBuf = 2 * kKeys * 128;                 // two 64-channel halves [128][128 B] bf16
+    static constexpr int kVb = kP + 2 * kPBuf;                     // [2 bufs] bf16 V (B of PV)
+    static constexpr int kScale = kVb + 2 * kVbBuf;                // [stage] ks[128] | vs[128] fp32
+    static constexpr int kSq = kScale + kStages * 2 * kKeys * 4;   // [64] fp32 query scales
+    static constexpr int kMeta = kSq + kRows * 4;                  // [stage] int: pages with a bad id
+    static constexpr int kRmax = kMeta + 16;                       // [tile parity][half][64] fp32 row maxima
+    static constexpr int kLsum = kRmax + 2 * 2 * kRows * 4;        // [half][64] fp32 row sums
+    static constexpr int kBar = kLsum + 2 * kRows * 4;
+    // barriers
+    static constexpr int kKvFull = 0, kKvEmpty = 3, kSFull = 6, kSFree = 8, kPReady = 10,
+                         kPvDone = 12, kFinal = 14, kQReady = 15, kRmaxBar = 16, kNumBars = 20;
+    static constexpr int kMisc = kBar + kNumBars * 8;              // TMEM base, abort flag
+    static constexpr int kBytes = kMisc + 16;
+    // merge area, over the K stages (free once the last tile is consumed)
+    static constexpr int kOc = kK;                                 // [64][kOcPitch] fp32
+    static constexpr int kStat = kOc + kRows * kOcPitch * 4;       // [64] (m, l)
+    static_assert(kOcPitch % 4 == 0, "merge rows are 16-byte aligned");
+    static_assert(kStat + kRows * 8 <= kV, "merge area fits in the K stages");
+    static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0 && kVb % 1024 == 0,
+                  "swizzled tiles are 1024-byte aligned");
+    static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
 };
 
 struct DecParams {
     const uint16_t* q;
     int64_t qs0, qs1, qs2, qs3;              // q strides [B, T, H, D] (elements)
-    const uint8_t* kc;
-    const uint8_t* vc;
     const float* ksc;
     const float* vsc;
     const int32_t* ptab;
     const int32_t* ctx;
-    int T, H, Hk, G, R, Rpad, page, max_pages, num_pages, window, nsplit;
+    int T, H, Hk, G, R, page, lg_page, max_pages, num_pages, window, nsplit;
     int q_vec;                               // q rows contiguous and 16-byte aligned
     float logit_scale_log2;                  // softmax_scale / D * log2(e)
-    float* part;                             // [B*Hk][nsplit][Rpad][D + 2]
     __nv_bfloat16* out;
     int64_t os0, os1, os2, os3;
 };
 
-__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+// The A operand (P') of the PV MMA holds a row's 128 keys in this order:
+// position 16i + 8c + m <-> key 16i + c + 2m (c = 0, 1; m = 0..7), which
+// is what a softmax thread holds (its columns have one parity c), so it
+// writes 16 contiguous bytes per 16 keys. V rows are stored in the same
+// order.
+__device__ __forceinline__ int pv_position(int key) {
+    return (key & ~15) + 8 * (key & 1) + ((key & 15) >> 1);
+}
+
+// Two e4m3 codes (byte 0 -> low half) -> bf16x2 with exactly the same
+// values: e4m3 -> f16 is exact; an f16 of an e4m3 value has its three low
+// mantissa bits zero and a normal exponent, so its bits shifted right by 3
+// read as a bf16 of value x * 2^-112, and the bf16 product by 2^112 is exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(pair)));
+    const uint32_t bits = ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
     uint32_t r;
-    const uint16_t in = static_cast<uint16_t>(code);
-    asm("{\n\t.reg .b32 h2;\n\tcvt.rn.f16x2.e4m3x2 h2, %1;\n\tmov.b32 %0, h2;\n\t}" : "=r"(r) : "h"(in));
-    return __half2float(__ushort_as_half(static_cast<uint16_t>(r & 0xFFFFu)));
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x77807780u));   // 2^112
+    return r;
 }
 
-// four e4m3 bytes -> two packed bf16 pairs (exact: e4m3 values are bf16 values)
-__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    uint32_t h01, h23;
-    const uint16_t w01 = static_cast<uint16_t>(w & 0xFFFFu), w23 = static_cast<uint16_t>(w >> 16);
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(w01));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(w23));
-    const __half2 a = *reinterpret_cast<const __half2*>(&h01);
-    const __half2 b = *reinterpret_cast<const __half2*>(&h23);
-    const __nv_bfloat162 ab = __floats2bfloat162_rn(__low2float(a), __high2float(a));
-    const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(b), __high2float(b));
-    lo = *reinterpret_cast<const uint32_t*>(&ab);
-    hi = *reinterpret_cast<const uint32_t*>(&bb);
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// Barrier `id` (1..15) of `count` threads (whole warps).
+__device__ __forceinline__ void named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-    const uint32_t d = smem_u32(dst);
-    const int n = valid ? 16 : 0;                 // 0 bytes read -> zero fill
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
+// CTA-wide and cluster-wide barriers in their non-aligned forms: the threads
+// may reach them from different code (each thread arrives exactly once).
+__device__ __forceinline__ void bar_sync_all(int count) {
+    asm volatile("bar.sync 0, %0;" ::"r"(count) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_wait() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool valid) {
-    const uint32_t d = smem_u32(dst);
-    const int n = valid ? 4 : 0;
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
-}
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const DecParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Sm::kBar);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Sm::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Sm::kMisc + 4);
+    float* sq = reinterpret_cast<float*>(sm + Sm::kSq);
+    int* meta = reinterpret_cast<int*>(sm + Sm::kMeta);
+    float* scl = reinterpret_cast<float*>(sm + Sm::kScale);
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-
-// Wait until at most `pending` (0 .. 3) of this thread's commit groups are
-// outstanding.
-__device__ __forceinline__ void cp_async_wait_pending(int pending) {
-    switch (pending) {
-        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
-        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
-        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
-        default: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
-    }
-}
-static_assert(kNChunk == 8, "each warpgroup commits 4 chunk groups");
-
-// Barrier of one warpgroup (named barrier 1 + grp, 128 threads).
-__device__ __forceinline__ void group_sync(int grp) {
-    asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
-}
-
-__device__ __forceinline__ void mma_e4m3_16832(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* row_addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(smem_u32(row_addr)));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecParams p) {
-    extern __shared__ __align__(128) uint8_t dsm[];
-    uint8_t (*ks8)[kKPitch] = reinterpret_cast<uint8_t (*)[kKPitch]>(dsm + DecSmem::kOffK);
-    uint8_t (*vs8)[kD] = reinterpret_cast<uint8_t (*)[kD]>(dsm + DecSmem::kOffV);
-    __nv_bfloat16 (*vbf)[kVPitch] = reinterpret_cast<__nv_bfloat16 (*)[kVPitch]>(dsm + DecSmem::kOffVbf);
-    uint8_t (*q8s)[kD] = reinterpret_cast<uint8_t (*)[kD]>(dsm + DecSmem::kOffQ);
-    float* kscl = reinterpret_cast<float*>(dsm + DecSmem::kOffKs);
-    float* vscl = reinterpret_cast<float*>(dsm + DecSmem::kOffVs);
-    int64_t* tokr = reinterpret_cast<int64_t*>(dsm + DecSmem::kOffTok);
-    float* sq = reinterpret_cast<float*>(dsm + DecSmem::kOffSq);
-    int* chunk_bad = reinterpret_cast<int*>(dsm + DecSmem::kOffBad);
-
-    const int split = blockIdx.x, bhk = blockIdx.y;
+    const int split = blockIdx.x;                 // == rank in the cluster
+    const int bhk = blockIdx.y;
     const int b = bhk / p.Hk, hk = bhk % p.Hk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, tg = lane & 3;
-    const int grp = warp >> 2, gtid = tid & 127;     // warpgroup, thread within it
 
     int ctx = p.ctx[b];
     const int cap = p.max_pages * p.page;
@@ -190,371 +178,614 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecPara
         if (tid == 0 && split == 0) atomicCAS(&g_decode_err, 0u, kErrDecodeRange);
         ctx = max(0, min(ctx, cap));
     }
+    // keys [lo, ctx) as 128-key tiles [t0, t1) at absolute positions; this
+    // CTA's share is [tb, tb + nt)
     const int lo = max(0, ctx - p.T - p.window + 1);
-    const int k_begin = lo + split * kSplit;
-    const int k_end = min(ctx, k_begin + kSplit);      // exclusive
-    const int nk = max(0, k_end - k_begin);
+    const int t0 = lo / kKeys, t1 = (ctx + kKeys - 1) / kKeys;
+    const int n_all = max(0, t1 - t0);
+    const int tb = t0 + (split * n_all) / p.nsplit;
+    const int nt = t0 + ((split + 1) * n_all) / p.nsplit - tb;
 
-    // ---- 0. cache rows of this split's keys, then every K / V row and
-    // per-token scale requested at once; warpgroup grp requests the chunks it
-    // will process (c = grp, grp + 2, ...), one commit group per chunk
-    if (tid < kNChunk) chunk_bad[tid] = 0;
+    if (tid == 0) {
+        for (int i = 0; i < Sm::kNumBars; ++i) {
+            uint32_t cnt = 1;
+            if (i >= Sm::kKvFull && i < Sm::kKvFull + kStages) cnt = 1 + 32;      // expect_tx + scale copies
+            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + kSoftWarps + 4;  // QK commit + warps
+            if (i >= Sm::kSFree && i < Sm::kSFree + 2) cnt = kSoftWarps;
+            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = kSoftWarps + 4;
+            if (i == Sm::kQReady) cnt = kSoftWarps;
+            if (i >= Sm::kRmaxBar && i < Sm::kRmaxBar + 4) cnt = 2;                     // the warp pair
+            mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    // the producer's first page-table entries, requested before the barrier
+    const int ppt = kKeys / p.page;                  // pages per tile (divides 32)
+    int pg_first = 0;
+    if (warp == kTmaWarp) {
+        const int lp = tb * ppt + lane;
+        if (lp < (tb + nt) * ppt && lp * p.page < ctx && lp * p.page + p.page > lo)
+            pg_first = __ldg(&p.ptab[(int64_t)b * p.max_pages + lp]);
+    }
+
+    tc_fence_before();
     __syncthreads();
-    for (int kr = tid; kr < kSplit; kr += kDecThreads) {
-        int64_t tok = -1;
-        if (kr < nk) {
-            const int j = k_begin + kr;
-            const int pg = __ldg(&p.ptab[(int64_t)b * p.max_pages + j / p.page]);
-            if (pg < 0 || pg >= p.num_pages) {
-                atomicCAS(&g_decode_err, 0u, kErrDecodeRange);
-                atomicOr(&chunk_bad[kr / kChunk], 1);
-            } else {
-                tok = ((int64_t)pg * p.Hk + hk) * p.page + (j % p.page);
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    // TMEM columns: S double buffer [0, 256); O of even tiles [256, 384), of
+    // odd tiles [384, 512)
+    constexpr uint32_t kOCol = 256;
+
+
+    if (warp >= kTmaWarp) {
+      reg_dealloc<kRegsProd>();
+      if (warp == kTmaWarp) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+        }
+        // physical pages of the CTA's logical pages tb * ppt + 32 c + lane,
+        // fetched 32 at a time; pages holding no key of [lo, ctx) are not
+        // looked up (page 0 stands in; their keys are masked)
+        int chunk = -1, phys_l = 0;
+        bool bad_l = false;
+        int issued = 0;
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kStages;
+            if (!warp_all(mbar_wait(&bars[Sm::kKvEmpty + s], ((i / kStages) & 1) ^ 1, abort_flag,
+                                    &g_decode_err, 1)))
+                break;
+            if ((i * ppt) / 32 != chunk) {
+                chunk = (i * ppt) / 32;
+                const int lp = tb * ppt + 32 * chunk + lane;
+                const int k0 = lp * p.page;
+                phys_l = 0;
+                bad_l = false;
+                if (lp < (tb + nt) * ppt && k0 < ctx && k0 + p.page > lo) {
+                    const int pg = chunk == 0 ? pg_first : __ldg(&p.ptab[(int64_t)b * p.max_pages + lp]);
+                    if (pg < 0 || pg >= p.num_pages) {
+                        bad_l = true;
+                        atomicCAS(&g_decode_err, 0u, kErrDecodeRange);
+                    } else {
+                        phys_l = pg;
+                    }
+                }
             }
-        }
-        tokr[kr] = tok;
-    }
-    __syncthreads();
-    for (int c = grp; c < kNChunk; c += 2) {
-        // 64 keys x (8 K pieces + 8 V pieces) of 16 bytes; two scales per key
-        for (int i = gtid; i < kChunk * 16; i += 128) {
-            const int kr = c * kChunk + i / 16, piece = i % 16;
-            const int64_t tok = tokr[kr];
-            const bool ok = tok >= 0;
-            const int64_t off = ok ? tok * kD + (piece & 7) * 16 : 0;
-            if (piece < 8) cp_async16(&ks8[kr][piece * 16], p.kc + off, ok);
-            else cp_async16(&vs8[kr][(piece - 8) * 16], p.vc + off, ok);
-        }
-        {
-            const int kr = c * kChunk + (gtid & (kChunk - 1));
-            const int64_t tok = tokr[kr];
-            if (gtid < kChunk) cp_async4(&kscl[kr], p.ksc + (tok >= 0 ? tok : 0), tok >= 0);
-            else cp_async4(&vscl[kr], p.vsc + (tok >= 0 ? tok : 0), tok >= 0);
-        }
-        cp_async_commit();
-    }
-
-    // ---- 1. query rows: rotate and quantise to e4m3, two threads per row
-    // (thread half hq holds elements [64 hq, 64 hq + 64)). Every thread runs
-    // the whole sequence, shuffles included; rows past R load zeros, which
-    // gives them zero codes and a zero scale.
-    if (grp == 0) {
-        const int r = tid >> 1, hq = tid & 1;
-        const bool rv = r < p.R;
-        const int t = rv ? r / p.G : 0, h = rv ? hk * p.G + r % p.G : 0;
-        const uint16_t* src = p.q + b * p.qs0 + t * p.qs1 + h * p.qs2 + (int64_t)(hq * 64) * p.qs3;
-        float x[64];
-        if (p.q_vec) {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 u = rv ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            const int slot0 = (i * ppt) % 32;             // this tile's pages: lanes slot0 ..
+            const int phys = __shfl_sync(0xffffffffu, phys_l, slot0 + (lane < ppt ? lane : 0));
+            const bool bad = __shfl_sync(0xffffffffu, bad_l ? 1 : 0, slot0 + (lane < ppt ? lane : 0)) != 0 && lane < ppt;
+            const unsigned badm = __ballot_sync(0xffffffffu, bad);
+            if (lane == 0) {
+                meta[s] = static_cast<int>(badm);
+                mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * Sm::kKStage);
+            }
+            for (int q = 0; q < ppt; ++q) {
+                const int pq = __shfl_sync(0xffffffffu, phys, q);
+                if (lane == 0) {
+                    const int z = pq * p.Hk + hk;
+                    tma_load_3d(sm + Sm::kK + s * Sm::kKStage + q * p.page * kD, &tmK,
+                                &bars[Sm::kKvFull + s], 0, 0, z);
+                    tma_load_3d(sm + Sm::kV + s * Sm::kKStage + q * p.page * kD, &tmV,
+                                &bars[Sm::kKvFull + s], 0, 0, z);
+                }
+            }
+            // per-token scales of keys 4 lane .. 4 lane + 3, stored by key
+            // parity (index (key & 1) * 64 + key / 2) for the softmax threads
+            {
+                const int kq = 4 * lane;
+                const int pq = __shfl_sync(0xffffffffu, phys, kq / p.page);
+                const int64_t src = ((int64_t)pq * p.Hk + hk) * p.page + (kq % p.page);
+                float* dst = scl + s * 2 * kKeys;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    x[8 * c + 2 * e] = __uint_as_float(w[e] << 16);
-                    x[8 * c + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+                    const int key = kq + e, at = (key & 1) * 64 + (key >> 1);
+                    cp_async_4(dst + at, p.ksc + src + e);
+                    cp_async_4(dst + kKeys + at, p.vsc + src + e);
+                }
+                cp_async_mbar_arrive(&bars[Sm::kKvFull + s]);
+            }
+            issued = i + 1;
+        }
+        // no copy of this CTA may land after it exits
+        for (int i = max(0, issued - kStages); i < issued; ++i)
+            mbar_wait_drain(&bars[Sm::kKvFull + i % kStages], (i / kStages) & 1);
+      } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nt > 0) {
+            constexpr uint32_t kIdescQK = umma_idesc(1, 0, kRows, kKeys);              // e4m3 -> f32
+            constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, 64) | (1u << 16);    // bf16, B MN-major
+            const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), 128);
+            bool ok = mbar_wait(&bars[Sm::kQReady], 0, abort_flag, &g_decode_err, 12);
+            for (int i = 0; ok && i <= nt; ++i) {
+                if (i < nt) {
+                    // S(i) = Q8 K8(i)^T into S buffer i & 1
+                    const int s = i % kStages;
+                    ok = mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2);
+                    if (ok && i >= 2)
+                        ok = mbar_wait(&bars[Sm::kSFree + (i & 1)], ((i - 2) >> 1) & 1, abort_flag,
+                                       &g_decode_err, 3);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), 128);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 32; ++kk)
+                        mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK,
+                                  kk > 0 ? 1u : 0u);
+                    mma_commit(&bars[Sm::kSFull + (i & 1)]);
+                    mma_commit(&bars[Sm::kKvEmpty + s]);
+                }
+                if (i >= 1) {
+                    // O[j & 1] += P'(j) V(j): two 64-channel halves x 8 steps of 16 keys
+                    const int j = i - 1;
+                    ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
+                    const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                        for (int st = 0; st < kKeys / 16; ++st)
+                            mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
+                                        umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
+                                        umma_desc_kmajor(vb + hf * (kKeys * 128), 128) + 128 * st,
+                                        kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
+                    mma_commit(&bars[Sm::kPvDone + (j & 1)]);
                 }
             }
+            // drain every MMA this thread issued before TMEM is released
+            mma_commit(&bars[Sm::kFinal]);
+            mbar_wait_drain(&bars[Sm::kFinal], 0);
+        }
+      }
+        tc_fence_before();
+        bar_sync_all(kThreads);
+        if (warp == kMmaWarp) {                     // TMEM is read by nobody any more
+            __syncwarp();
+            tc_fence_after();
+            tmem_dealloc(tmem, 512);
+        }
+        cluster_arrive_wait();
+        cluster_arrive_wait();
+    } else if (warp < kSoftWarps) {
+      reg_alloc<kRegsSoft>();
+        // ------------------------------------------------------------ softmax
+        // ---- query rows: rotate and quantise to e4m3, four threads per row
+        // (thread qq holds elements [32 qq, 32 qq + 32)), written as the
+        // K-major 128B-swizzled A operand of QK. Every thread of warps 0-7
+        // runs the whole sequence, shuffles included; rows past R load zeros,
+        // which gives them zero codes and a zero scale.
+        {
+            const int r = tid >> 2, qq = tid & 3;
+            const bool rv = r < p.R;
+            const int t = rv ? r / p.G : 0, h = rv ? hk * p.G + r % p.G : 0;
+            const uint16_t* src = p.q + b * p.qs0 + t * p.qs1 + h * p.qs2 + (int64_t)(qq * 32) * p.qs3;
+            float x[32];
+            if (p.q_vec) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 u = rv ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+                    const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[8 * c + 2 * e] = __uint_as_float(wd[e] << 16);
+                        x[8 * c + 2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int d = 0; d < 32; ++d)
+                    x[d] = rv ? __uint_as_float(static_cast<uint32_t>(__ldg(src + d * p.qs3)) << 16) : 0.0f;
+            }
+            // stages h = 1 .. 16 inside the quarter
+#pragma unroll
+            for (int lg = 0; lg < 5; ++lg) {
+                const int hh = 1 << lg;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const int j = ((kk >> lg) << (lg + 1)) + (kk & (hh - 1));
+                    const float a = x[j], c = x[j + hh];
+                    x[j] = __fadd_rn(a, c);
+                    x[j + hh] = __fsub_rn(a, c);
+                }
+            }
+            // stages h = 32 and 64 across the row's threads: x[j] +- x[j + h]
+#pragma unroll
+            for (int st = 1; st <= 2; st <<= 1) {
+                const bool upper = (qq & st) != 0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float y = __shfl_xor_sync(0xffffffffu, x[j], st);
+                    x[j] = upper ? __fsub_rn(y, x[j]) : __fadd_rn(x[j], y);
+                }
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int d = 0; d < 32; ++d) amax = fmaxf(amax, fabsf(x[d]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+            float s = 0.0f, rr = 0.0f;
+            if (amax != 0.0f) {
+                s = __fdiv_rn(amax, 448.0f);
+                rr = __fdiv_rn(448.0f, amax);
+            }
+            if (qq == 0) sq[r] = s;
+            uint8_t* qrow = sm + Sm::kQ + r * 128;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {            // 16-byte chunk 2 qq + c of the row
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int d = 16 * c + 4 * e;
+                    const uint32_t lo16 = e4m3x2_rn_satfinite(__fmul_rn(x[d], rr), __fmul_rn(x[d + 1], rr));
+                    const uint32_t hi16 = e4m3x2_rn_satfinite(__fmul_rn(x[d + 2], rr), __fmul_rn(x[d + 3], rr));
+                    w4[e] = lo16 | (hi16 << 16);
+                }
+                const int chunk = 2 * qq + c;
+                *reinterpret_cast<uint4*>(qrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();                // the QK MMAs read these rows
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Sm::kQReady]);
+        named_sync(1, kSoftWarps * 32);              // every row's s_q is in shared memory
+
+        // thread: query row r (TMEM lane 32 qw + lr) and the columns
+        // 64 hh + 2k + cpar (k = 0..31) of every tile; warps qw and qw + 4
+        // share their rows and exchange row maxima through shared memory
+        const int qw = warp & 3, hh = warp >> 2;
+        const int lr = (lane >> 2) + 8 * (lane & 1);
+        const int cpar = (lane >> 1) & 1;
+        const int r = 16 * qw + lr;
+        const bool rv = r < p.R;
+        const int pq = rv ? ctx - p.T + r / p.G : -1;     // the row's query position
+        const float cq = rv ? sq[r] * p.logit_scale_log2 : 0.0f;
+        const uint64_t cq2 = f2_pack(cq, cq);
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * qw) << 16) + 64 * hh;
+        float* rmax = reinterpret_cast<float*>(sm + Sm::kRmax);
+        float o_fin[32];                              // end-of-split state, merged below
+        float m_fin = -INFINITY;
+        // m_run: running max; m_acc[a]: the max O[a] is expressed against
+        float m_run = -INFINITY, lsum = 0.0f;
+        float m_acc[2] = {-INFINITY, -INFINITY};
+        bool ok = true;
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kStages, bf = i & 1;
+            ok = warp_all(mbar_wait(&bars[Sm::kSFull + bf], (i >> 1) & 1, abort_flag, &g_decode_err, 5));
+            if (ok)
+                ok = warp_all(mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag,
+                                        &g_decode_err, 6));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[32];
+            tmem_ld16x32(taddr + 128 * bf, sv);
+            tmem_wait_ld(sv);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[Sm::kSFree + bf]);
+
+            const float* ksP = scl + s * 2 * kKeys + cpar * 64 + 32 * hh;   // k_scale of column 64hh + 2k + cpar
+            const float* vsP = ksP + kKeys;
+            const int key0 = (tb + i) * kKeys;
+            const int badm = meta[s];
+            // base-2 logits
+            float x[32];
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+                const float4 kq = *reinterpret_cast<const float4*>(ksP + 4 * k4);
+                const uint64_t a01 = f2_mul(f2_mul(f2_pack(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
+                                                   f2_pack(kq.x, kq.y)), cq2);
+                const uint64_t a23 = f2_mul(f2_mul(f2_pack(__uint_as_float(sv[4 * k4 + 2]), __uint_as_float(sv[4 * k4 + 3])),
+                                                   f2_pack(kq.z, kq.w)), cq2);
+                f2_unpack(a01, x[4 * k4], x[4 * k4 + 1]);
+                f2_unpack(a23, x[4 * k4 + 2], x[4 * k4 + 3]);
+            }
+            // masks: rows past R; keys outside the row's window; bad pages.
+            // A tile inside every row's window with no bad page needs none.
+            const bool full = badm == 0 && key0 >= ctx - p.window && key0 + kKeys - 1 <= ctx - p.T;
+            if (!rv) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) x[k] = -INFINITY;
+            } else if (!full) {
+                // the row sees columns [clo, chi] of the tile; register k is
+                // column 64 hh + 2k + cpar
+                const int base = key0 + 64 * hh + cpar;
+                const int clo = pq - p.window + 1 - base, chi = pq - base;
+#pragma unroll
+                for (int k = 0; k < 32; ++k) x[k] = (2 * k >= clo && 2 * k <= chi) ? x[k] : -INFINITY;
+                if (badm != 0) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        if ((badm >> ((64 * hh + 2 * k + cpar) >> p.lg_page)) & 1) x[k] = -INFINITY;
+                }
+            }
+            // row max: four chains, a tree, the column partner, the other half
+            float m4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) m4[c] = fmax3(x[c], x[c + 4], x[c + 8]);
+#pragma unroll
+            for (int k = 12; k < 28; k += 8)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) m4[c] = fmax3(m4[c], x[k + c], x[k + c + 4]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) m4[c] = fmaxf(m4[c], x[28 + c]);
+            float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            float* rm = rmax + (i & 1) * (2 * kRows);
+            if (cpar == 0) rm[hh * kRows + r] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[Sm::kRmaxBar + qw]);
+            ok = warp_all(mbar_wait(&bars[Sm::kRmaxBar + qw], i & 1, abort_flag, &g_decode_err, 13));
+            if (!ok) break;
+            mx = fmaxf(mx, rm[(hh ^ 1) * kRows + r]);
+            const float m_new = fmaxf(m_run, mx);
+            if (m_run != -INFINITY && m_new != m_run) lsum *= ex2_approx(m_run - m_new);
+            m_run = m_new;
+            const float sub = m_new == -INFINITY ? 0.0f : m_new;
+            // O[bf] (tiles i - 2, i - 4, ...) is brought to m_new before PV(i)
+            const float m_o = m_acc[bf];
+            const bool resc = m_o != -INFINITY && m_o != m_new;
+            const float alpha = resc ? ex2_approx(m_o - m_new) : 1.0f;
+            m_acc[bf] = m_new;
+
+            // P' buffer bf is free once PV(i - 2) is done
+            if (i >= 2) {
+                ok = warp_all(mbar_wait(&bars[Sm::kPvDone + bf], ((i - 2) >> 1) & 1, abort_flag,
+                                        &g_decode_err, 7));
+                if (!ok) break;
+            }
+            uint8_t* prow = sm + Sm::kP + bf * Sm::kPBuf + hh * (kRows * 128) + r * 128;
+#pragma unroll
+            for (int i8 = 0; i8 < 4; ++i8) {      // keys 64hh + 16 i8 + cpar + 2m = registers 8 i8 + m
+                const float4 va = *reinterpret_cast<const float4*>(vsP + 8 * i8);
+                const float4 vb = *reinterpret_cast<const float4*>(vsP + 8 * i8 + 4);
+                const float vsv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+                uint32_t wd[4];
+#pragma unroll
+                for (int m = 0; m < 8; m += 2) {
+                    const float p0 = ex2_approx(x[8 * i8 + m] - sub);
+                    const float p1 = ex2_approx(x[8 * i8 + m + 1] - sub);
+                    lsum += p0 + p1;
+                    const __nv_bfloat162 pr = __floats2bfloat162_rn(p0 * vsv[m], p1 * vsv[m + 1]);
+                    wd[m / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+                }
+                const int chunk = 2 * i8 + cpar;
+                *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+            // O[bf] *= alpha for the rows whose max rose since tile i - 2 (PV(i - 2),
+            // its last writer, is done: waited for above); this warp's 64
+            // output channels
+            if (__any_sync(0xffffffffu, resc)) {
+                tc_fence_after();
+                uint32_t o[32];
+                tmem_ld16x32(taddr + kOCol + 128 * bf, o);
+                tmem_wait_ld(o);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                tmem_st16x32(taddr + kOCol + 128 * bf, o);
+                tmem_wait_st();
+            }
+            fence_proxy_async_smem();               // P' is read by the PV MMAs
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[Sm::kPReady + bf]);
+                mbar_arrive(&bars[Sm::kKvEmpty + s]);
+            }
+        }
+        bool have = ok && nt > 0;
+        if (have)
+            have = warp_all(mbar_wait(&bars[Sm::kPvDone + ((nt - 1) & 1)], ((nt - 1) >> 1) & 1,
+                                      abort_flag, &g_decode_err, 9));
+        if (have) {
+            // O = O[0] 2^(m_acc0 - m) + O[1] 2^(m_acc1 - m), m = m_run
+            tc_fence_after();
+            uint32_t o0[32], o1[32];
+            tmem_ld16x32(taddr + kOCol, o0);
+            tmem_wait_ld(o0);
+            const float w0 = m_acc[0] == -INFINITY ? 0.0f : ex2_approx(m_acc[0] - m_run);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o_fin[k] = __uint_as_float(o0[k]) * w0;
+            if (nt > 1) {
+                tmem_ld16x32(taddr + kOCol + 128, o1);
+                tmem_wait_ld(o1);
+                const float w1 = m_acc[1] == -INFINITY ? 0.0f : ex2_approx(m_acc[1] - m_run);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o_fin[k] = fmaf(__uint_as_float(o1[k]), w1, o_fin[k]);
+            }
+            m_fin = m_run;
         } else {
 #pragma unroll
-            for (int d = 0; d < 64; ++d)
-                x[d] = rv ? __uint_as_float(static_cast<uint32_t>(__ldg(src + d * p.qs3)) << 16) : 0.0f;
+            for (int k = 0; k < 32; ++k) o_fin[k] = 0.0f;
+            lsum = 0.0f;
         }
-        // stages h = 1 .. 32 inside the half
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        if (cpar == 0) reinterpret_cast<float*>(sm + Sm::kLsum)[hh * kRows + r] = lsum;
+        // ---- merge the splits of (b, hk) across the cluster (only the
+        // softmax warps hold registers enough for it). Every role ends with
+        // the same three barriers, reached from its own code: the CTA
+        // barrier (all roles done, the K stages free), then two cluster
+        // barriers around the exchange.
+        tc_fence_before();
+        bar_sync_all(kThreads);
+        {
+            float* oc = reinterpret_cast<float*>(sm + Sm::kOc);
+            float2* stat = reinterpret_cast<float2*>(sm + Sm::kStat);
 #pragma unroll
-        for (int lg = 0; lg < 6; ++lg) {
-            const int hh = 1 << lg;
-#pragma unroll
-            for (int kk = 0; kk < 32; ++kk) {
-                const int j = ((kk >> lg) << (lg + 1)) + (kk & (hh - 1));
-                const float a = x[j], c = x[j + hh];
-                x[j] = __fadd_rn(a, c);
-                x[j + hh] = __fsub_rn(a, c);
+            for (int k = 0; k < 32; ++k) oc[r * kOcPitch + 64 * hh + 2 * k + cpar] = o_fin[k];
+            if (hh == 0 && cpar == 0) {
+                const float* ls = reinterpret_cast<const float*>(sm + Sm::kLsum);
+                stat[r] = make_float2(m_fin, ls[r] + ls[kRows + r]);
             }
-        }
-        // stage h = 64 across the pair: x[j] +- x[j + 64]
+            __syncwarp();
+            cluster_arrive_wait();
+            // CTA `split` writes rows split, split + nsplit, ...; thread: one
+            // row and four channels; all remote loads issued before any use
+            for (int idx = tid;; idx += kSoftWarps * 32) {
+                const int rr = split + p.nsplit * (idx >> 5), d4 = 4 * (idx & 31);
+                if (rr >= p.R) break;
+                float2 st[kMaxSplit];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            const float y = __shfl_xor_sync(0xffffffffu, x[j], 1);
-            x[j] = hq == 0 ? __fadd_rn(x[j], y) : __fsub_rn(y, x[j]);
-        }
-        float amax = 0.0f;
+                for (int sp = 0; sp < kMaxSplit; ++sp)
+                    st[sp] = sp < p.nsplit ? dsmem_ld_f32x2(dsmem_addr(&stat[rr], sp)) : make_float2(-INFINITY, 0.0f);
+                float4 ov[kMaxSplit];
 #pragma unroll
-        for (int d = 0; d < 64; ++d) amax = fmaxf(amax, fabsf(x[d]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        float s = 0.0f, rr = 0.0f;
-        if (amax != 0.0f) {
-            s = __fdiv_rn(amax, 448.0f);
-            rr = __fdiv_rn(448.0f, amax);
-        }
-        if (hq == 0) sq[r] = s;
+                for (int sp = 0; sp < kMaxSplit; ++sp)
+                    ov[sp] = sp < p.nsplit ? dsmem_ld_f32x4(dsmem_addr(&oc[rr * kOcPitch + d4], sp))
+                                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                float M = -INFINITY;
 #pragma unroll
-        for (int d = 0; d < 64; d += 16) {
-            uint32_t w4[4];
+                for (int sp = 0; sp < kMaxSplit; ++sp) M = fmaxf(M, st[sp].x);
+                float den = 0.0f;
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (M != -INFINITY) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const uint32_t lo16 = e4m3x2_rn_satfinite(__fmul_rn(x[d + 4 * e], rr), __fmul_rn(x[d + 4 * e + 1], rr));
-                const uint32_t hi16 = e4m3x2_rn_satfinite(__fmul_rn(x[d + 4 * e + 2], rr), __fmul_rn(x[d + 4 * e + 3], rr));
-                w4[e] = lo16 | (hi16 << 16);
-            }
-            *reinterpret_cast<uint4*>(&q8s[r][hq * 64 + d]) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-    }
-    __syncthreads();
-
-    // A fragments of this warp's 16 rows (4 k-steps of 32 channels), kept in registers
-    const int row0 = (warp & 3) * 16;
-    uint32_t qa[4][4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        qa[kk][0] = *reinterpret_cast<const uint32_t*>(&q8s[row0 + g][kk * 32 + tg * 4]);
-        qa[kk][1] = *reinterpret_cast<const uint32_t*>(&q8s[row0 + g + 8][kk * 32 + tg * 4]);
-        qa[kk][2] = *reinterpret_cast<const uint32_t*>(&q8s[row0 + g][kk * 32 + 16 + tg * 4]);
-        qa[kk][3] = *reinterpret_cast<const uint32_t*>(&q8s[row0 + g + 8][kk * 32 + 16 + tg * 4]);
-    }
-    // per-thread rows: ra = row0 + g, rb = row0 + g + 8
-    const int ra = row0 + g, rb = ra + 8;
-    const bool va = ra < p.R, vb_ = rb < p.R;
-    const int pa = va ? ctx - p.T + ra / p.G : -1;      // query position of each row
-    const int pb = vb_ ? ctx - p.T + rb / p.G : -1;
-    const float ca = va ? sq[ra] * p.logit_scale_log2 : 0.0f;
-    const float cb = vb_ ? sq[rb] * p.logit_scale_log2 : 0.0f;
-
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
-
-    const int nchunks = (nk + kChunk - 1) / kChunk;
-    __nv_bfloat16 (*vb)[kVPitch] = vbf + grp * kChunk;   // this warpgroup's bf16 V chunk
-    for (int ci = 0; grp + 2 * ci < nchunks; ++ci) {
-        const int c = grp + 2 * ci;
-        const int c0 = c * kChunk;                      // chunk's first key, split-relative
-        cp_async_wait_pending(kNChunk / 2 - 1 - ci);   // this thread's copies of chunk c are in
-        group_sync(grp);                                // the group's; its previous vb reads done
-        // V e4m3 -> bf16 (exact)
-        for (int i = gtid; i < kChunk * (kD / 4); i += 128) {
-            const int kr = i / (kD / 4), c4 = (i % (kD / 4)) * 4;
-            uint32_t lo2, hi2;
-            e4m3x4_to_bf16x4(*reinterpret_cast<const uint32_t*>(&vs8[c0 + kr][c4]), lo2, hi2);
-            *reinterpret_cast<uint2*>(&vb[kr][c4]) = make_uint2(lo2, hi2);
-        }
-        group_sync(grp);
-        // keys [jf, jf + 64) inside every row's window and all present: no
-        // per-key tests
-        const int jf = k_begin + c0;
-        const bool full = c0 + kChunk <= nk && !chunk_bad[c] && jf + kChunk - 1 <= ctx - p.T &&
-                          jf > ctx - 1 - p.window;
-
-        // ---- 2b. S = Q8 K8^T for 64 keys (8 n-tiles of 8 keys)
-        float sacc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.0f;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&ks8[c0 + nt * 8 + g][kk * 32 + tg * 4]);
-                const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&ks8[c0 + nt * 8 + g][kk * 32 + 16 + tg * 4]);
-                mma_e4m3_16832(sacc[nt], qa[kk], b0, b1);
-            }
-        }
-        // scale, mask to each row's window, base-2 logits
-        float mx_a = -INFINITY, mx_b = -INFINITY;
-        if (full) {
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float ksv = kscl[c0 + nt * 8 + tg * 2 + e];
-                    sacc[nt][e] = sacc[nt][e] * ca * ksv;
-                    sacc[nt][2 + e] = sacc[nt][2 + e] * cb * ksv;
-                    mx_a = fmaxf(mx_a, sacc[nt][e]);
-                    mx_b = fmaxf(mx_b, sacc[nt][2 + e]);
+                    for (int sp = 0; sp < kMaxSplit; ++sp) {
+                        const float wgt = st[sp].x == -INFINITY ? 0.0f : ex2_approx(st[sp].x - M);
+                        den = fmaf(wgt, st[sp].y, den);
+                        acc.x = fmaf(wgt, ov[sp].x, acc.x);
+                        acc.y = fmaf(wgt, ov[sp].y, acc.y);
+                        acc.z = fmaf(wgt, ov[sp].z, acc.z);
+                        acc.w = fmaf(wgt, ov[sp].w, acc.w);
+                    }
                 }
-            // rows past R: logits are 0 * ..., masked here as before
-            if (!va) mx_a = -INFINITY;
-            if (!vb_) mx_b = -INFINITY;
-            if (!va || !vb_) {
+                const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+                const int t = rr / p.G, h = hk * p.G + rr % p.G;
+                __nv_bfloat16* dst = p.out + b * p.os0 + t * p.os1 + h * p.os2 + (int64_t)d4 * p.os3;
+                const float y[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt) {
-                    if (!va) sacc[nt][0] = sacc[nt][1] = -INFINITY;
-                    if (!vb_) sacc[nt][2] = sacc[nt][3] = -INFINITY;
-                }
+                for (int e = 0; e < 4; ++e) dst[(int64_t)e * p.os3] = __float2bfloat16_rn(y[e]);
             }
-        } else {
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int kr = c0 + nt * 8 + tg * 2 + e;
-                    const int j = k_begin + kr;
-                    const float ksv = kscl[kr];
-                    const bool okk = kr < nk && tokr[kr] >= 0;
-                    const bool vis_a = okk && j <= pa && j > pa - p.window;
-                    const bool vis_b = okk && j <= pb && j > pb - p.window;
-                    sacc[nt][e] = vis_a ? sacc[nt][e] * ca * ksv : -INFINITY;
-                    sacc[nt][2 + e] = vis_b ? sacc[nt][2 + e] * cb * ksv : -INFINITY;
-                    mx_a = fmaxf(mx_a, sacc[nt][e]);
-                    mx_b = fmaxf(mx_b, sacc[nt][2 + e]);
-                }
+            __syncwarp();
+            cluster_arrive_wait();                  // no CTA leaves while others read it
         }
+    } else {
+      reg_dealloc<kRegsConv>();
+        // ------------------------------------------------------------ V converters
+        // lane -> V row kap of the tile (warp cw: rows 32 cw .. 32 cw + 31),
+        // chosen so that the eight lanes of a quarter-warp read eight
+        // different 16-byte bank groups and write eight different ones
+        const int cw = warp - kConvWarp0;
+        const int q8 = lane >> 3, e8 = lane & 7;
+        const int kap = 32 * cw + 16 * (q8 >> 1) + 2 * e8 + ((e8 >> 2) ^ (q8 & 1));
+        const int pos = pv_position(kap);
+        bool ok = true;
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kStages, bf = i & 1;
+            ok = warp_all(mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 10));
+            if (ok && i >= 2)
+                ok = warp_all(mbar_wait(&bars[Sm::kPvDone + bf], ((i - 2) >> 1) & 1, abort_flag,
+                                        &g_decode_err, 11));
+            if (!ok) break;
+            const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + kap * 128;
+            uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + pos * 128;
 #pragma unroll
-        for (int o2 = 1; o2 <= 2; o2 <<= 1) {
-            mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, o2));
-            mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, o2));
-        }
-        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float sub_a = mn_a == -INFINITY ? 0.0f : mn_a;
-        const float sub_b = mn_b == -INFINITY ? 0.0f : mn_b;
-        const float al_a = ex2_approx(m_a - sub_a), al_b = ex2_approx(m_b - sub_b);
-        // P' = p * s_v (bf16) as A fragments of the PV mma (two n-tiles = 16 keys)
-        uint32_t pa_frag[4][4];
-        float ls_a = 0.0f, ls_b = 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            float pv[4];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int kr = c0 + nt * 8 + tg * 2 + e;
-                const float pa_ = ex2_approx(sacc[nt][e] - sub_a);
-                const float pb_ = ex2_approx(sacc[nt][2 + e] - sub_b);
-                ls_a += pa_;
-                ls_b += pb_;
-                pv[e] = pa_ * vscl[kr];
-                pv[2 + e] = pb_ * vscl[kr];
+            for (int c = 0; c < 8; ++c) {           // channels 16c .. 16c + 15
+                const uint4 u = *reinterpret_cast<const uint4*>(vrow + ((c ^ (kap & 7)) << 4));
+                const uint32_t o0 = e4m3x2_to_bf16x2(u.x), o1 = e4m3x2_to_bf16x2(u.x >> 16);
+                const uint32_t o2 = e4m3x2_to_bf16x2(u.y), o3 = e4m3x2_to_bf16x2(u.y >> 16);
+                const uint32_t o4 = e4m3x2_to_bf16x2(u.z), o5 = e4m3x2_to_bf16x2(u.z >> 16);
+                const uint32_t o6 = e4m3x2_to_bf16x2(u.w), o7 = e4m3x2_to_bf16x2(u.w >> 16);
+                uint8_t* half = dst + (c >> 2) * (kKeys * 128);
+                const int ch = 2 * (c & 3);
+                *reinterpret_cast<uint4*>(half + ((ch ^ (pos & 7)) << 4)) = make_uint4(o0, o1, o2, o3);
+                *reinterpret_cast<uint4*>(half + (((ch + 1) ^ (pos & 7)) << 4)) = make_uint4(o4, o5, o6, o7);
             }
-            const int ks = nt >> 1, half = nt & 1;
-            pa_frag[ks][half * 2 + 0] = pack_bf16(pv[0], pv[1]);     // row g
-            pa_frag[ks][half * 2 + 1] = pack_bf16(pv[2], pv[3]);     // row g + 8
-        }
-#pragma unroll
-        for (int o2 = 1; o2 <= 2; o2 <<= 1) {
-            ls_a += __shfl_xor_sync(0xffffffffu, ls_a, o2);
-            ls_b += __shfl_xor_sync(0xffffffffu, ls_b, o2);
-        }
-        l_a = l_a * al_a + ls_a;
-        l_b = l_b * al_b + ls_b;
-        m_a = mn_a;
-        m_b = mn_b;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            o[n][0] *= al_a;
-            o[n][1] *= al_a;
-            o[n][2] *= al_b;
-            o[n][3] *= al_b;
-        }
-        // ---- 2c. O += P' V (4 k-steps of 16 keys x 16 n-tiles of 8 channels)
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            // A fragment layout of m16n8k16: {row g: k 0-7 pair, row g+8: k 0-7 pair,
-            // row g: k 8-15 pair, row g+8: k 8-15 pair}
-            const uint32_t afr[4] = {pa_frag[ks][0], pa_frag[ks][1], pa_frag[ks][2], pa_frag[ks][3]};
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {        // pairs of n-tiles
-                // lanes 0-15 address keys ks*16 + (lane & 15) of n-tile 2np,
-                // lanes 16-31 the same keys of n-tile 2np + 1
-                const int krow = ks * 16 + (lane & 15);
-                const int col = (2 * np + (lane >> 4)) * 8;
-                uint32_t bfr[4];
-                ldmatrix_x4_trans(bfr, &vb[krow][col]);
-                mma_bf16_16816(o[2 * np], afr, bfr[0], bfr[1]);
-                mma_bf16_16816(o[2 * np + 1], afr, bfr[2], bfr[3]);
+            fence_proxy_async_smem();               // read by the PV MMAs
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[Sm::kPReady + bf]);
+                mbar_arrive(&bars[Sm::kKvEmpty + s]);
             }
         }
-    }
-    cp_async_wait_pending(0);       // no copy may outlive the CTA
-
-    // ---- 3. merge the second warpgroup's state into the first's, over the
-    // K rows (every read of them is done after this barrier)
-    __syncthreads();
-    float* mg = reinterpret_cast<float*>(dsm + DecSmem::kOffK) + ((warp & 3) * 32 + lane) * (64 + 4);
-    if (grp == 1) {
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-            *reinterpret_cast<float4*>(mg + 4 * n) = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
-        *reinterpret_cast<float4*>(mg + 64) = make_float4(m_a, m_b, l_a, l_b);
-    }
-    __syncthreads();
-    if (grp == 1) return;
-    {
-        const float4 st = *reinterpret_cast<const float4*>(mg + 64);
-        const float Ma = fmaxf(m_a, st.x), Mb = fmaxf(m_b, st.y);
-        const float w0a = m_a == -INFINITY ? 0.0f : ex2_approx(m_a - Ma);
-        const float w1a = st.x == -INFINITY ? 0.0f : ex2_approx(st.x - Ma);
-        const float w0b = m_b == -INFINITY ? 0.0f : ex2_approx(m_b - Mb);
-        const float w1b = st.y == -INFINITY ? 0.0f : ex2_approx(st.y - Mb);
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            const float4 o1 = *reinterpret_cast<const float4*>(mg + 4 * n);
-            o[n][0] = o[n][0] * w0a + o1.x * w1a;
-            o[n][1] = o[n][1] * w0a + o1.y * w1a;
-            o[n][2] = o[n][2] * w0b + o1.z * w1b;
-            o[n][3] = o[n][3] * w0b + o1.w * w1b;
-        }
-        l_a = l_a * w0a + st.z * w1a;
-        l_b = l_b * w0b + st.w * w1b;
-        m_a = Ma;
-        m_b = Mb;
-    }
-
-    // partial results of this split
-    // (rows beyond Rpad exist only as padding of the 4 x 16 row grid)
-    if (row0 < p.Rpad) {
-        const int64_t base = ((int64_t)bhk * p.nsplit + split) * p.Rpad;
-        float* rowa = p.part + (base + ra) * (kD + 2);
-        float* rowb = p.part + (base + rb) * (kD + 2);
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            *reinterpret_cast<float2*>(rowa + n * 8 + tg * 2) = make_float2(o[n][0], o[n][1]);
-            *reinterpret_cast<float2*>(rowb + n * 8 + tg * 2) = make_float2(o[n][2], o[n][3]);
-        }
-        if (tg == 0) {
-            rowa[kD] = m_a;
-            rowa[kD + 1] = l_a;
-            rowb[kD] = m_b;
-            rowb[kD + 1] = l_b;
-        }
+        tc_fence_before();
+        bar_sync_all(kThreads);
+        cluster_arrive_wait();
+        cluster_arrive_wait();
     }
 }
 
-// One CTA per (row, b * hk), one thread per channel: merges the splits of
-// the row (log-sum-exp rescaling) and writes bf16.
-__global__ void __launch_bounds__(kD) decode_combine_kernel(const DecParams p) {
-    const int r = blockIdx.x, bhk = blockIdx.y;
-    const int b = bhk / p.Hk, hk = bhk % p.Hk;
-    const int d = threadIdx.x;
-    const int t = r / p.G, h = hk * p.G + r % p.G;
-    const int64_t stride = (int64_t)p.Rpad * (kD + 2);
-    const float* row0 = p.part + ((int64_t)bhk * p.nsplit * p.Rpad + r) * (kD + 2);
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, __ldg(row0 + s * stride + kD));
-    float acc = 0.0f, den = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int s = 0; s < p.nsplit; ++s) {
-            const float* row = row0 + s * stride;
-            const float ms = __ldg(row + kD);
-            const float w = (ms == -INFINITY) ? 0.0f : ex2_approx(ms - M);
-            acc = fmaf(w, __ldg(row + d), acc);
-            den = fmaf(w, __ldg(row + kD + 1), den);
-        }
-    }
-    const float y = den > 0.0f ? acc / den : 0.0f;
-    p.out[b * p.os0 + t * p.os1 + h * p.os2 + (int64_t)d * p.os3] = __float2bfloat16_rn(y);
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The cache [num_pages, Hk, page, 128] e4m3 as a 3-D map {128 bytes, page
+// rows, num_pages * Hk}; one box = one page of one kv head, 128B swizzle.
+bool encode_cache(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int page) {
+    auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(page),
+                                static_cast<cuuint64_t>(num_pages) * Hk};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(page) * kD};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(page), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int nsplit_for(int T, int window) {
-    return static_cast<int>(ceil_div(window + T - 1, kSplit));
+constexpr int kSmemBytes = Sm::kBytes + 1024;
+
+// How many clusters of `size` CTAs of decode_kernel fit on the current
+// device at once (queried once per device and size).
+int max_active_clusters(int size) {
+    static std::mutex mu;
+    static int cache[64][kMaxSplit + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+    std::lock_guard<std::mutex> lock(mu);
+    int& c = cache[dev][size];
+    if (c == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(size, 1);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = size;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, decode_kernel, &cfg) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        c = n;
+    }
+    return c;
+}
+
+// CTAs per (sequence, kv head) = cluster size: the one (up to 8) that
+// minimises waves x tiles per CTA for the most 128-key tiles a sequence can
+// span; of equal choices the largest.
+int pick_nsplit(int n_clusters, int T, int window, int page, int max_pages) {
+    const int64_t span = std::min<int64_t>((int64_t)window + T - 1, (int64_t)max_pages * page);
+    const int64_t tiles = std::max<int64_t>(1, ceil_div(span, kKeys) + 1);
+    int best = 1;
+    int64_t best_cost = INT64_MAX;
+    for (int sz = static_cast<int>(std::min<int64_t>(kMaxSplit, tiles)); sz >= 1; --sz) {
+        const int64_t waves = ceil_div(n_clusters, max_active_clusters(sz));
+        const int64_t cost = waves * ceil_div(tiles, sz);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = sz;
+        }
+    }
+    return best;
 }
 
 }  // namespace
 
-size_t decode_ws_bytes(int B, int T, int H, int Hk, int D, int window) {
-    const int R = T * (H / Hk);
-    const int Rpad = static_cast<int>(round_up(R, 16));
-    return (size_t)B * Hk * nsplit_for(T, window) * Rpad * (D + 2) * sizeof(float);
-}
+size_t decode_ws_bytes(int, int, int, int, int, int) { return 0; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     DecParams p;
@@ -563,8 +794,6 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     p.qs1 = a.q.stride[1];
     p.qs2 = a.q.stride[2];
     p.qs3 = a.q.stride[3];
-    p.kc = a.k_cache;
-    p.vc = a.v_cache;
     p.ksc = a.k_scale;
     p.vsc = a.v_scale;
     p.ptab = a.page_table;
@@ -574,14 +803,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     p.Hk = a.Hk;
     p.G = a.H / a.Hk;
     p.R = a.T * p.G;
-    p.Rpad = static_cast<int>(round_up(p.R, 16));
     p.page = a.page_size;
+    p.lg_page = 31 - __builtin_clz(static_cast<unsigned>(a.page_size));
     p.max_pages = a.max_pages;
     p.num_pages = a.num_pages;
     p.window = a.window;
-    p.nsplit = nsplit_for(a.T, a.window);
     p.logit_scale_log2 = a.softmax_scale / static_cast<float>(a.D) * kLog2e;
-    p.part = static_cast<float*>(a.ws);
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.os0 = a.out_stride[0];
     p.os1 = a.out_stride[1];
@@ -591,12 +818,26 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
                a.q.stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.q.ptr) % 16 == 0)
                   ? 1
                   : 0;
-    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, DecSmem::kBytes);
+    CUtensorMap tk, tv;
+    if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size) ||
+        !encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    decode_split_kernel<<<dim3(p.nsplit, a.B * a.Hk), kDecThreads, DecSmem::kBytes, s>>>(p);
-    decode_combine_kernel<<<dim3(p.R, a.B * a.Hk), kD, 0, s>>>(p);
-    return cudaGetLastError();
+    p.nsplit = pick_nsplit(a.B * a.Hk, a.T, a.window, a.page_size, a.max_pages);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.nsplit, a.B * a.Hk);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = p.nsplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel, tk, tv, p);
 }
 
 unsigned read_clear_decode_error() {

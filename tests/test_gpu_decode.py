@@ -12,7 +12,7 @@ import torch
 import oracle
 import quantized_attention_smoothing_b200 as sage
 import workloads
-from gpu_helpers import bits, compare_output
+from gpu_helpers import COS_ORACLE, MAX_ABS, bf16_ulp, bits, compare_output, cosine, workloads_f32
 
 pytestmark = pytest.mark.gpu
 
@@ -79,3 +79,35 @@ def test_decode_strided_views(h128):
     b, _ = _run(h128, d, 512, 0.08, q_layout="strided", out_layout="strided")
     assert np.array_equal(a, b)
     compare_output(a, ref, None, label="strided")
+
+
+def test_decode_dominant_keys(h128):
+    """Keys whose k_scale is multiplied by 40, spread over the window, give
+    logits far above the running maximum in later tiles of a split (O is
+    rescaled in TMEM there) and rows dominated by one key. Both sides round
+    every PV weight w_j = p_j * v_scale_j to bf16 but evaluate p_j in
+    different precisions (fp32 exp2 of fp32 logits against fp64 exp), so a
+    weight near a rounding boundary can land one bf16 ulp (2^-8 relative)
+    apart: the bound adds 2^-8 * sum_j w_j |v_j| / l, which the oracle gives
+    when run on the V codes with their sign bits cleared."""
+    d = workloads.make_decode(B=4, T=4, H=16, Hk=1, D=128, page=128, ctx_lo=3000, ctx_hi=5000,
+                              seed=4242)
+    ksc = d["k_scale"].clone()
+    rng = np.random.default_rng(5)
+    for b in range(4):
+        ctx = int(d["ctx_lens"][b])
+        lo = max(0, ctx - 4 - 4096 + 1)
+        for j in rng.integers(lo, ctx, size=24):
+            pg = int(d["page_table"][b, j // 128])
+            ksc[pg, 0, j % 128] *= 40.0
+    d["k_scale"] = ksc
+    scale = 1.0 / math.sqrt(128)
+    gpu, ref = _run(h128, d, 4096, scale)
+    _, vabs = oracle.decode(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), d["v_cache"].numpy() & 0x7F,
+                            d["k_scale"].numpy(), d["v_scale"].numpy(), d["page_table"].numpy(),
+                            d["ctx_lens"].numpy(), 4096, scale, want_f64=True)
+    g = workloads_f32(gpu).astype(np.float64)
+    ulp = bf16_ulp(np.maximum(np.abs(g), np.abs(ref)))
+    excess = np.abs(g - ref) - ulp / 2 - 2.0 ** -8 * vabs
+    assert float(excess.max()) <= MAX_ABS, float(excess.max())
+    assert cosine(g, ref) >= COS_ORACLE

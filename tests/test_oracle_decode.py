@@ -5,7 +5,8 @@
   the FlyDSL pa_decode page prints (tests/golden/window_tiles.txt).
 * The oracle's paged, GQA, per-token-scaled decode equals a brute-force
   computation over the un-paged cache that uses torch's float8 conversion for
-  the query quantisation and scipy's Hadamard matrix for the rotation.
+  the query quantisation, scipy's Hadamard matrix for the rotation and
+  torch's bfloat16 conversion for the PV weights p_j * v_scale_j.
 """
 import math
 import os
@@ -81,8 +82,10 @@ def _brute_decode(oracle_mod, d, window, scale):
                 sl = slice(lo, p + 1)
                 logits = (K[sl] @ q8) * float(s) * ks[sl] * (scale / D)
                 w = np.exp(logits - logits.max())
-                w /= w.sum()
-                out[b, t, h] = (w * vs[sl]) @ V[sl]
+                # bf16 PV operand: fp32 product rounded by torch's bf16 cast
+                wv = w.astype(np.float32) * vs[sl].astype(np.float32)
+                wv = torch.from_numpy(wv).to(torch.bfloat16).to(torch.float64).numpy()
+                out[b, t, h] = (wv @ V[sl]) / w.sum()
     return out
 
 
