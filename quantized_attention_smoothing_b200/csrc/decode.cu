@@ -125,16 +125,16 @@ __device__ __forceinline__ int pv_position(int key) {
     return (key & ~15) + 8 * (key & 1) + ((key & 15) >> 1);
 }
 
-// Two e4m3 codes (byte 0 -> low half) -> bf16x2 with exactly the same
-// values: e4m3 -> f16 is exact; an f16 of an e4m3 value has its three low
-// mantissa bits zero and a normal exponent, so its bits shifted right by 3
-// read as a bf16 of value x * 2^-112, and the bf16 product by 2^112 is exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t pair) {
-    uint32_t h;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(pair)));
-    const uint32_t bits = ((h >> 3) & 0x0FFF0FFFu) | (h & 0x80008000u);
+// e4m3 codes -> bf16 with exactly the same values, integer operations only.
+// A code's 7 magnitude bits placed at bf16 bits 4..10 and its sign at bit 15
+// read as a bf16 of value x * 2^-120 (exponent field e of a normal code kept,
+// a subnormal code a bf16 subnormal), and the bf16 product by 2^120 is exact.
+// `sel` picks the two code bytes of `w` (0x1404: bytes 0, 1; 0x3424: 2, 3).
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
+    const uint32_t t = __byte_perm(w, 0u, sel);          // code bytes at bits 8..15 and 24..31
+    const uint32_t bits = ((t >> 4) & 0x07F007F0u) | (t & 0x80008000u);
     uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x77807780u));   // 2^112
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7B807B80u));   // 2^120
     return r;
 }
 
@@ -534,12 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float alpha = resc ? ex2_approx(m_o - m_new) : 1.0f;
             m_acc[bf] = m_new;
 
-            // P' buffer bf is free once PV(i - 2) is done
-            if (i >= 2) {
-                ok = warp_all(mbar_wait(&bars[Sm::kPvDone + bf], ((i - 2) >> 1) & 1, abort_flag,
-                                        &g_decode_err, 7));
-                if (!ok) break;
-            }
+            // P' buffer bf is free: PV(i - 2), its reader, is done -- the MMA
+            // thread issues it before QK(i), and the commit that completed
+            // S(i) covers every MMA that thread started earlier
             uint8_t* prow = sm + Sm::kP + bf * Sm::kPBuf + hh * (kRows * 128) + r * 128;
 #pragma unroll
             for (int i8 = 0; i8 < 4; ++i8) {      // keys 64hh + 16 i8 + cpar + 2m = registers 8 i8 + m
@@ -559,8 +556,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
             // O[bf] *= alpha for the rows whose max rose since tile i - 2 (PV(i - 2),
-            // its last writer, is done: waited for above); this warp's 64
-            // output channels
+            // its last writer, is done, as above); this warp's 64 output
+            // channels
             if (__any_sync(0xffffffffu, resc)) {
                 tc_fence_after();
                 uint32_t o[32];
@@ -688,10 +685,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 8; ++c) {           // channels 16c .. 16c + 15
                 const uint4 u = *reinterpret_cast<const uint4*>(vrow + ((c ^ (kap & 7)) << 4));
-                const uint32_t o0 = e4m3x2_to_bf16x2(u.x), o1 = e4m3x2_to_bf16x2(u.x >> 16);
-                const uint32_t o2 = e4m3x2_to_bf16x2(u.y), o3 = e4m3x2_to_bf16x2(u.y >> 16);
-                const uint32_t o4 = e4m3x2_to_bf16x2(u.z), o5 = e4m3x2_to_bf16x2(u.z >> 16);
-                const uint32_t o6 = e4m3x2_to_bf16x2(u.w), o7 = e4m3x2_to_bf16x2(u.w >> 16);
+                const uint32_t o0 = e4m3x2_to_bf16x2(u.x, 0x1404u), o1 = e4m3x2_to_bf16x2(u.x, 0x3424u);
+                const uint32_t o2 = e4m3x2_to_bf16x2(u.y, 0x1404u), o3 = e4m3x2_to_bf16x2(u.y, 0x3424u);
+                const uint32_t o4 = e4m3x2_to_bf16x2(u.z, 0x1404u), o5 = e4m3x2_to_bf16x2(u.z, 0x3424u);
+                const uint32_t o6 = e4m3x2_to_bf16x2(u.w, 0x1404u), o7 = e4m3x2_to_bf16x2(u.w, 0x3424u);
                 uint8_t* half = dst + (c >> 2) * (kKeys * 128);
                 const int ch = 2 * (c & 3);
                 *reinterpret_cast<uint4*>(half + ((ch ^ (pos & 7)) << 4)) = make_uint4(o0, o1, o2, o3);

@@ -111,3 +111,18 @@ def test_decode_dominant_keys(h128):
     excess = np.abs(g - ref) - ulp / 2 - 2.0 ** -8 * vabs
     assert float(excess.max()) <= MAX_ABS, float(excess.max())
     assert cosine(g, ref) >= COS_ORACLE
+
+
+def test_decode_subnormal_v_codes(h128):
+    """A V cache of e4m3 subnormal codes only (exponent field 0, values
+    m * 2^-9, m = 0..7, either sign) with a large v_scale: the exact e4m3 ->
+    bf16 conversion of V must keep them (flushing them would zero the
+    output)."""
+    d = workloads.make_decode(B=2, T=4, H=16, Hk=1, D=128, page=128, ctx_lo=500, ctx_hi=900, seed=99)
+    g = torch.Generator().manual_seed(3)
+    codes = torch.randint(0, 16, d["v_cache"].shape, generator=g, dtype=torch.int32)
+    d["v_cache"] = ((codes & 7) | ((codes & 8) << 4)).to(torch.uint8)
+    d["v_scale"] = torch.full_like(d["v_scale"], 64.0)
+    gpu, ref = _run(h128, d, 4096, 1.0 / math.sqrt(128))
+    assert np.abs(ref).max() > 0.05
+    compare_output(gpu, ref, None, label="subnormal V")
