@@ -248,9 +248,13 @@ class QuantBuffers:
         self.k_mean = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
         self.v8_t = torch.empty((B, Hk, D, round_up(Lk, 128)), dtype=torch.uint8, device=dev)
         self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
-        ws = max(sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D), sage_quant_v_workspace(B, Hk, Lk, D),
-                 sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D), 16)
+        ws = max(sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D), sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D), 16)
         self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev)
+        # the V quantisation has its own workspace so it can run on a second
+        # stream beside the Q/K quantisation
+        self.ws_v = torch.empty((max(sage_quant_v_workspace(B, Hk, Lk, D), 16),), dtype=torch.uint8,
+                                device=dev)
+        self.side = torch.cuda.Stream(device=dev)
 
 
 def sage_attention(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, out=None, bufs=None,
@@ -264,9 +268,23 @@ def sage_attention(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, out=No
         bufs = QuantBuffers(B, H, Hk, Lq, Lk, D, blk_q, blk_k, q.device.index)
     if out is None:
         out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=q.device).permute(0, 2, 1, 3)
-    sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
-                  bufs.k_mean, bufs.ws, stream)
-    sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws, stream)
+    quantise(h, q, k, v, blk_q, blk_k, bufs, stream)
     sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale, B, H, Hk,
                   Lq, Lk, D, blk_q, blk_k, softmax_scale, causal, out, None, stream)
     return out, bufs
+
+
+def quantise(h, q, k, v, blk_q, blk_k, bufs, stream=None):
+    """sage_quant_qk on `stream` and, beside it, sage_quant_v on the
+    buffers' second stream (the two read and write disjoint buffers); work
+    issued to `stream` afterwards waits for both."""
+    s = torch.cuda.current_stream() if stream is None else stream
+    fork = torch.cuda.Event()
+    fork.record(s)
+    bufs.side.wait_event(fork)
+    sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                  bufs.k_mean, bufs.ws, s)
+    sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v, bufs.side)
+    join = torch.cuda.Event()
+    join.record(bufs.side)
+    s.wait_event(join)

@@ -36,7 +36,7 @@ def gpu_quant(h, q, k, v, blk_q, blk_k):
     bufs = sage.QuantBuffers(B, H, Hk, Lq, Lk, D, blk_q, blk_k)
     sage.sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
                        bufs.k_mean, bufs.ws)
-    sage.sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws)
+    sage.sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v)
     torch.cuda.synchronize()
     assert sage.sage_device_error() == sage.SAGE_OK
     return bufs
