@@ -226,7 +226,10 @@ const char* sage_status_string(sage_status s);
 /* Synchronise `stream`, then read and clear the library's device error
  * words on the current device: SAGE_ERR_TIMEOUT if a bounded wait expired
  * since the last call, SAGE_ERR_CUDA if the stream reports a CUDA error,
- * SAGE_OK otherwise. */
+ * SAGE_ERR_INVALID_ARG if sage_attn_decode met device-side arguments out of
+ * range (a context length above max_pages * page_size, clamped; or a page id
+ * outside [0, num_pages) for a page holding keys of a window, whose keys were
+ * then left out), SAGE_OK otherwise. */
 sage_status sage_device_error(void* stream);
 
 #ifdef __cplusplus

@@ -51,7 +51,7 @@ namespace sage {
 namespace {
 
 __device__ unsigned g_decode_err;
-constexpr unsigned kErrDecodeRange = 2u;     // ctx or page id out of range (clamped / masked)
+constexpr unsigned kErrDecodeRange = kErrRangeCode;   // ctx or page id out of range (clamped / masked)
 
 constexpr int kD = 128;
 constexpr int kKeys = 128;                   // keys per tile

@@ -352,6 +352,7 @@ sage_status sage_device_error(void* stream) {
     if ((a & 0xFFu) == sage::kErrTimeoutCode || (d & 0xFFu) == sage::kErrTimeoutCode ||
         (q & 0xFFu) == sage::kErrTimeoutCode)
         return SAGE_ERR_TIMEOUT;
+    if ((d & 0xFFu) == sage::kErrRangeCode) return SAGE_ERR_INVALID_ARG;
     return SAGE_OK;
 }
 

@@ -26,6 +26,7 @@ inline bool view_vec8(const View4& v) {
 
 constexpr int kTile = 128;                  // token tile of every kernel
 constexpr unsigned kErrTimeoutCode = 1u;    // low byte of a device error word
+constexpr unsigned kErrRangeCode = 2u;      // decode: a page id or context length out of range
 
 __host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 

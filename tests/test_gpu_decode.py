@@ -126,3 +126,21 @@ def test_decode_subnormal_v_codes(h128):
     gpu, ref = _run(h128, d, 4096, 1.0 / math.sqrt(128))
     assert np.abs(ref).max() > 0.05
     compare_output(gpu, ref, None, label="subnormal V")
+
+
+def test_decode_reports_bad_page_ids(h128):
+    """A page-table entry outside [0, num_pages) for a page inside the window
+    is not dereferenced: its keys are left out, the output stays finite and
+    sage_device_error reports SAGE_ERR_INVALID_ARG (then clears it)."""
+    d = workloads.make_decode(B=2, T=4, H=16, Hk=1, D=128, page=128, ctx_lo=600, ctx_hi=900, seed=5)
+    ptab = d["page_table"].clone()
+    ptab[1, 2] = d["num_pages"] + 7
+    q = d["q"].cuda()
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    sage.sage_attn_decode(h128, q, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(),
+                          d["v_scale"].cuda(), ptab.cuda(), d["ctx_lens"].cuda(), 128, d["num_pages"],
+                          4096, 1.0 / math.sqrt(128), out, ws)
+    assert sage.sage_device_error() == sage.SAGE_ERR_INVALID_ARG
+    assert sage.sage_device_error() == sage.SAGE_OK
+    assert torch.isfinite(out.float()).all()
