@@ -36,6 +36,7 @@
 // raises its abort flag, drains its own copies and MMAs and still takes part
 // in both cluster barriers.
 #include <algorithm>
+#include <cfloat>
 #include <climits>
 #include <cstdint>
 #include <mutex>
@@ -445,14 +446,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = 16 * qw + lr;
         const bool rv = r < p.R;
         const int pq = rv ? ctx - p.T + r / p.G : -1;     // the row's query position
-        const float cq = rv ? sq[r] * p.logit_scale_log2 : 0.0f;
+        // base-2 logit of a key = (acc * k_scale) * cq; cq kept >= FLT_MIN so
+        // that a masked key (-inf) times cq stays -inf (a zero query row has
+        // acc = 0, so its logits are 0 either way)
+        const float cq = fmaxf(rv ? sq[r] * p.logit_scale_log2 : 0.0f, FLT_MIN);
         const uint64_t cq2 = f2_pack(cq, cq);
         const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * qw) << 16) + 64 * hh;
         float* rmax = reinterpret_cast<float*>(sm + Sm::kRmax);
         float o_fin[32];                              // end-of-split state, merged below
         float m_fin = -INFINITY;
         // m_run: running max; m_acc[a]: the max O[a] is expressed against
-        float m_run = -INFINITY, lsum = 0.0f;
+        float m_run = -INFINITY;
+        uint64_t lsum2 = f2_pack(0.0f, 0.0f);         // running sum as an f32x2 pair
         float m_acc[2] = {-INFINITY, -INFINITY};
         bool ok = true;
         for (int i = 0; i < nt; ++i) {
@@ -474,15 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float* vsP = ksP + kKeys;
             const int key0 = (tb + i) * kKeys;
             const int badm = meta[s];
-            // base-2 logits
+            // y = acc * k_scale; the logit is y * cq, and cq > 0 keeps the
+            // order, so the row max is taken on y
             float x[32];
 #pragma unroll
             for (int k4 = 0; k4 < 8; ++k4) {
                 const float4 kq = *reinterpret_cast<const float4*>(ksP + 4 * k4);
-                const uint64_t a01 = f2_mul(f2_mul(f2_pack(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
-                                                   f2_pack(kq.x, kq.y)), cq2);
-                const uint64_t a23 = f2_mul(f2_mul(f2_pack(__uint_as_float(sv[4 * k4 + 2]), __uint_as_float(sv[4 * k4 + 3])),
-                                                   f2_pack(kq.z, kq.w)), cq2);
+                const uint64_t a01 = f2_mul(f2_pack(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
+                                            f2_pack(kq.x, kq.y));
+                const uint64_t a23 = f2_mul(f2_pack(__uint_as_float(sv[4 * k4 + 2]), __uint_as_float(sv[4 * k4 + 3])),
+                                            f2_pack(kq.z, kq.w));
                 f2_unpack(a01, x[4 * k4], x[4 * k4 + 1]);
                 f2_unpack(a23, x[4 * k4 + 2], x[4 * k4 + 3]);
             }
@@ -524,10 +530,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = warp_all(mbar_wait(&bars[Sm::kRmaxBar + qw], i & 1, abort_flag, &g_decode_err, 13));
             if (!ok) break;
             mx = fmaxf(mx, rm[(hh ^ 1) * kRows + r]);
+            mx = mx == -INFINITY ? -INFINITY : mx * cq;   // the max of the logits y * cq
             const float m_new = fmaxf(m_run, mx);
-            if (m_run != -INFINITY && m_new != m_run) lsum *= ex2_approx(m_run - m_new);
+            if (m_run != -INFINITY && m_new != m_run) {
+                const float a = ex2_approx(m_run - m_new);
+                lsum2 = f2_mul(lsum2, f2_pack(a, a));
+            }
             m_run = m_new;
             const float sub = m_new == -INFINITY ? 0.0f : m_new;
+            const uint64_t nsub2 = f2_pack(-sub, -sub);
             // O[bf] (tiles i - 2, i - 4, ...) is brought to m_new before PV(i)
             const float m_o = m_acc[bf];
             const bool resc = m_o != -INFINITY && m_o != m_new;
@@ -546,10 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t wd[4];
 #pragma unroll
                 for (int m = 0; m < 8; m += 2) {
-                    const float p0 = ex2_approx(x[8 * i8 + m] - sub);
-                    const float p1 = ex2_approx(x[8 * i8 + m + 1] - sub);
-                    lsum += p0 + p1;
-                    const __nv_bfloat162 pr = __floats2bfloat162_rn(p0 * vsv[m], p1 * vsv[m + 1]);
+                    float e0, e1;
+                    f2_unpack(f2_fma(f2_pack(x[8 * i8 + m], x[8 * i8 + m + 1]), cq2, nsub2), e0, e1);
+                    const float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
+                    const uint64_t p2 = f2_pack(p0, p1);
+                    lsum2 = f2_add(lsum2, p2);
+                    float w0, w1;
+                    f2_unpack(f2_mul(p2, f2_pack(vsv[m], vsv[m + 1])), w0, w1);
+                    const __nv_bfloat162 pr = __floats2bfloat162_rn(w0, w1);
                     wd[m / 2] = *reinterpret_cast<const uint32_t*>(&pr);
                 }
                 const int chunk = 2 * i8 + cpar;
@@ -600,8 +615,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
             for (int k = 0; k < 32; ++k) o_fin[k] = 0.0f;
-            lsum = 0.0f;
+            lsum2 = f2_pack(0.0f, 0.0f);
         }
+        float l0, l1;
+        f2_unpack(lsum2, l0, l1);
+        float lsum = l0 + l1;
         lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
         if (cpar == 0) reinterpret_cast<float*>(sm + Sm::kLsum)[hh * kRows + r] = lsum;
         // ---- merge the splits of (b, hk) across the cluster (only the
