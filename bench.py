@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--fused-q", action="store_true",
+                    help="rotate and quantise Q inside the attention kernel (sage_attn_fwd_q16)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the paged-decode measurement and print its object")
     return ap.parse_args()
@@ -338,13 +340,17 @@ def run_sage(args):
 
     def step(i, timed):
         qs, ks, vs_, bufs, out = sets[i % len(sets)]
-        # Q/K quantisation on `stream`, V quantisation beside it on a second
-        # stream, attention after both
-        sage.quantise(h, qs, ks, vs_, blk_q, blk_k, bufs, stream)
+        # Q/K (or K) quantisation on `stream`, V quantisation beside it on a
+        # second stream, attention after both
+        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
         if timed:
             ev[i][0].record(stream)
-        sage.sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
-                           B, H, Hk, L, L, D, blk_q, blk_k, scale, causal, out, None, stream)
+        if args.fused_q:
+            sage.sage_attn_fwd_q16(h, qs, blk_q, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
+                                   Hk, L, blk_k, scale, causal, out, None, stream)
+        else:
+            sage.sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
+                               B, H, Hk, L, L, D, blk_q, blk_k, scale, causal, out, None, stream)
         if timed:
             ev[i][1].record(stream)
 

@@ -162,6 +162,13 @@ sage_status sage_quant_qk_noalloc(sage_hadamard h, sage_cview4 q_bf16, sage_cvie
                                   int blk_q, int blk_k, int8_t* q8, float* q_scale, int8_t* k8,
                                   float* k_scale, float* k_mean, void* stream);
 
+/* sage_quant_qk for K alone (K mean, smoothing, rotation, INT8 codes and
+ * scales, the same bits as sage_quant_qk's K outputs), for callers whose Q is
+ * quantised inside sage_attn_fwd_q16. k_bf16: [B, Hk, Lk, D]; ws: at least
+ * sage_quant_qk_workspace(B, Hk, Hk, Lk, Lk, D) bytes. */
+sage_status sage_quant_k(sage_hadamard h, sage_cview4 k_bf16, int blk_k, int8_t* k8,
+                         float* k_scale, float* k_mean, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace sage_quant_v needs: fp32 partial channel
  * maxima, up to 8 per (b, h, d): B * Hk * 8 * D * 4. */
 size_t sage_quant_v_workspace(int B, int Hk, int L, int D);
@@ -195,6 +202,23 @@ sage_status sage_attn_fwd(const int8_t* q8, const float* q_scale, const int8_t* 
                           int H, int Hk, int Lq, int Lk, int D, int blk_q, int blk_k,
                           float softmax_scale, int causal, sage_view4 out_bf16, void* ws,
                           size_t ws_bytes, void* stream);
+
+/* Q rotated and quantised inside the attention kernel: the per-token
+ * rotate + absmax + INT8 step of the pypto DSV4 page ("qr_hadamard_quant")
+ * fused into the attention CTA, on-chip, so the Q operand never round-trips
+ * through HBM (that page fused it through global memory and lost). Each query row is read once as bf16, rotated with the butterfly and
+ * quantised to INT8 with the block scale a / 127 of its blk_q-row block --
+ * the arithmetic of sage_quant_qk, so the codes, scales and output are the
+ * bits that sage_quant_qk + sage_attn_fwd produce -- and its codes go straight
+ * into the shared-memory operand of QK. q8 / q_scale are never written.
+ *   q_bf16: [B, H, Lq, D] bf16 view of any strides (D == the handle's D);
+ *   k8, k_scale: from sage_quant_k (or sage_quant_qk) with the same blk_k;
+ *   v8_t, v_scale: from sage_quant_v; out_bf16: [B, H, Lq, D] bf16 view.
+ * Supported as for sage_attn_fwd. ws may be NULL. */
+sage_status sage_attn_fwd_q16(sage_hadamard h, sage_cview4 q_bf16, int blk_q, const int8_t* k8,
+                              const float* k_scale, const uint8_t* v8_t, const float* v_scale,
+                              int Hk, int Lk, int blk_k, float softmax_scale, int causal,
+                              sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace sage_attn_decode needs (split-KV partials). */
 size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window);

@@ -28,8 +28,8 @@ SAGE_ERR_TIMEOUT = 6
 EXPORTS = (
     "sage_hadamard_init", "sage_hadamard_destroy", "sage_hadamard_matrix",
     "sage_quant_qk_workspace", "sage_quant_qk", "sage_quant_qk_noalloc",
-    "sage_quant_v_workspace", "sage_quant_v",
-    "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_decode_workspace",
+    "sage_quant_v_workspace", "sage_quant_v", "sage_quant_k",
+    "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_fwd_q16", "sage_attn_decode_workspace",
     "sage_attn_decode", "sage_status_string", "sage_device_error",
 )
 
@@ -80,10 +80,15 @@ def lib():
     L.sage_quant_v_workspace.argtypes = [i32] * 4
     L.sage_quant_v.restype = i32
     L.sage_quant_v.argtypes = [CView4, vp, vp, vp, sz, vp]
+    L.sage_quant_k.restype = i32
+    L.sage_quant_k.argtypes = [vp, CView4, i32, vp, vp, vp, vp, sz, vp]
     L.sage_attn_fwd_workspace.restype = sz
     L.sage_attn_fwd_workspace.argtypes = [i32] * 6
     L.sage_attn_fwd.restype = i32
     L.sage_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp] + [i32] * 8 + [f32, i32, View4, vp, sz, vp]
+    L.sage_attn_fwd_q16.restype = i32
+    L.sage_attn_fwd_q16.argtypes = [vp, CView4, i32, vp, vp, vp, vp, i32, i32, i32, f32, i32, View4,
+                                    vp, sz, vp]
     L.sage_attn_decode_workspace.restype = sz
     L.sage_attn_decode_workspace.argtypes = [i32] * 6
     L.sage_attn_decode.restype = i32
@@ -197,6 +202,21 @@ def sage_quant_qk_noalloc(h, q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mea
            "sage_quant_qk_noalloc")
 
 
+def sage_quant_k(h, k, blk_k, k8, k_scale, k_mean=None, ws=None, stream=None):
+    _check(lib().sage_quant_k(h.handle, _view(k, CView4), int(blk_k), _ptr(k8), _ptr(k_scale),
+                              _ptr(k_mean), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                              _stream(stream)), "sage_quant_k")
+
+
+def sage_attn_fwd_q16(h, q, blk_q, k8, k_scale, v8_t, v_scale, Hk, Lk, blk_k, softmax_scale,
+                      causal, out, ws=None, stream=None):
+    _check(lib().sage_attn_fwd_q16(h.handle, _view(q, CView4), int(blk_q), _ptr(k8), _ptr(k_scale),
+                                   _ptr(v8_t), _ptr(v_scale), int(Hk), int(Lk), int(blk_k),
+                                   float(softmax_scale), 1 if causal else 0, _view(out, View4),
+                                   _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                   _stream(stream)), "sage_attn_fwd_q16")
+
+
 def sage_quant_v(v, v8_t, v_scale, ws=None, stream=None):
     _check(lib().sage_quant_v(_view(v, CView4), _ptr(v8_t), _ptr(v_scale), _ptr(ws),
                               0 if ws is None else ws.numel() * ws.element_size(),
@@ -274,16 +294,36 @@ def sage_attention(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, out=No
     return out, bufs
 
 
+def sage_attention_q16(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, out=None, bufs=None,
+                       stream=None):
+    """sage_attention with Q rotated and quantised inside the attention
+    kernel (sage_quant_k + sage_quant_v beside it + sage_attn_fwd_q16): the
+    same output bits, no q8 / q_scale round trip."""
+    B, H, Lq, D = q.shape
+    Hk, Lk = k.shape[1], k.shape[2]
+    if bufs is None:
+        bufs = QuantBuffers(B, H, Hk, Lq, Lk, D, blk_q, blk_k, q.device.index)
+    if out is None:
+        out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=q.device).permute(0, 2, 1, 3)
+    quantise(h, None, k, v, blk_q, blk_k, bufs, stream)
+    sage_attn_fwd_q16(h, q, blk_q, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale, Hk, Lk, blk_k,
+                      softmax_scale, causal, out, None, stream)
+    return out, bufs
+
+
 def quantise(h, q, k, v, blk_q, blk_k, bufs, stream=None):
-    """sage_quant_qk on `stream` and, beside it, sage_quant_v on the
-    buffers' second stream (the two read and write disjoint buffers); work
-    issued to `stream` afterwards waits for both."""
+    """sage_quant_qk (sage_quant_k when q is None) on `stream` and, beside
+    it, sage_quant_v on the buffers' second stream (the two read and write
+    disjoint buffers); work issued to `stream` afterwards waits for both."""
     s = torch.cuda.current_stream() if stream is None else stream
     fork = torch.cuda.Event()
     fork.record(s)
     bufs.side.wait_event(fork)
-    sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
-                  bufs.k_mean, bufs.ws, s)
+    if q is None:
+        sage_quant_k(h, k, blk_k, bufs.k8, bufs.k_scale, bufs.k_mean, bufs.ws, s)
+    else:
+        sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                      bufs.k_mean, bufs.ws, s)
     sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v, bufs.side)
     join = torch.cuda.Event()
     join.record(bufs.side)

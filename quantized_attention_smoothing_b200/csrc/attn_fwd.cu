@@ -42,12 +42,14 @@
 // an error word, raises a CTA-wide abort flag, drains its own MMAs and
 // returns.
 #include <climits>
+#include <cstring>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
+#include "quant_rows.cuh"
 
 namespace sage {
 namespace {
@@ -126,7 +128,8 @@ struct Cfg {
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kOffKs = kOffMisc + 16;             // K block scales of the head
     static constexpr int kOffVs = kOffKs + kKsSmem * 4;      // V channel scales of the head
-    static constexpr int kSmemBytes = kOffVs + D * 4 + 1024; // + runtime alignment
+    static constexpr int kOffQmax = kOffVs + D * 4;          // [8] row-block maxima (in-CTA Q)
+    static constexpr int kSmemBytes = kOffQmax + 8 * 4 + 1024; // + runtime alignment
     static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -142,6 +145,15 @@ struct Params {
     float logit_scale_log2;        // softmax_scale / D * log2(e)
     int heavy_first;
     int out_vec;
+};
+
+// The in-CTA Q path: Q rows read as bf16 [B, H, Lq, D] and rotated and
+// quantised by the softmax threads (q8 / q_scale unused). A separate,
+// trailing kernel parameter, so the separate-Q kernel's code is unchanged.
+struct QParams {
+    const uint16_t* qbf;
+    int64_t qs0, qs1, qs2, qs3;
+    int q_vec;                     // 16-byte row loads possible
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
@@ -238,10 +250,10 @@ __device__ __forceinline__ float row_exp(uint32_t (&s)[BN], const float (&kc)[NK
     return r0 + r1;
 }
 
-template <int D, int NKB, bool CAUSAL>
+template <int D, int NKB, bool CAUSAL, bool QF>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                    const __grid_constant__ CUtensorMap tmV, const Params p) {
+                    const __grid_constant__ CUtensorMap tmV, const Params p, const QParams qp) {
     using C = Cfg<D>;
     constexpr int kKeysPerBlk = BN / NKB;
     extern __shared__ uint8_t smem_raw[];
@@ -285,7 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool four = (i >= C::kBarSEmpty && i < C::kBarSEmpty + QT) ||
                               (i >= C::kBarPFull && i < C::kBarPFull + QT) ||
                               (i >= C::kBarTok && i < C::kBarTok + QT);
-            mbar_init(&bars[i], four ? 4u : 1u);
+            uint32_t cnt = four ? 4u : 1u;
+            if (i == C::kBarQ && QF) cnt = 4u * QT;         // the softmax warps write Q
+            mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -315,13 +329,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (warp == kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0 && n_max > 0) {
-            tma_prefetch_desc(&tmQ);
+            if (!QF) tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(&bars[C::kBarQ], QT * C::kQBytes);
-            for (int w = 0; w < QT; ++w)
-                tma_load_2d(smem + C::kOffQ + w * C::kQBytes, &tmQ, &bars[C::kBarQ], 0,
-                            bh * p.LpadQ + q_row0 + w * BM);
+            if (!QF) {
+                mbar_arrive_expect_tx(&bars[C::kBarQ], QT * C::kQBytes);
+                for (int w = 0; w < QT; ++w)
+                    tma_load_2d(smem + C::kOffQ + w * C::kQBytes, &tmQ, &bars[C::kBarQ], 0,
+                                bh * p.LpadQ + q_row0 + w * BM);
+            }
             for (int t = 0; t < n_max; ++t) {
                 const int s = t % C::kStages;
                 const uint32_t ph = (t / C::kStages) & 1;
@@ -421,7 +437,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(ww * 32) << 16);
         const uint32_t s_col = w * BN;
         const uint32_t o_col = 256 + w * BM;
-        const float qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + (i >> p.lg_blk_q)]) : 0.0f;
+        float qsc;
+        if constexpr (QF) {
+            // in-CTA Q: this thread's row is rotated and quantised with the
+            // arithmetic of the Q/K quantisation kernel (same tile rows, same
+            // block maxima), so the codes and scales are the same bits; the
+            // codes go straight into the swizzled A operand of QK
+            uint64_t x2[D / 2];
+            {
+                const uint16_t* src = qp.qbf + (bh / p.H) * qp.qs0 + (bh % p.H) * qp.qs1 + (int64_t)i * qp.qs2;
+                if (qp.q_vec) {
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) {
+                        const uint4 u = valid ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
+                        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            x2[4 * c + e] = qrow::p2(qrow::bf16_bits_to_f32(wd[e] & 0xFFFFu), __uint_as_float(wd[e] & 0xFFFF0000u));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < D / 2; ++e) {
+                        const uint32_t lo = valid ? __ldg(src + (int64_t)(2 * e) * qp.qs3) : 0u;
+                        const uint32_t hi = valid ? __ldg(src + (int64_t)(2 * e + 1) * qp.qs3) : 0u;
+                        x2[e] = qrow::p2(qrow::bf16_bits_to_f32(lo), qrow::bf16_bits_to_f32(hi));
+                    }
+                }
+            }
+            qrow::butterfly_pairs<D>(x2);
+            float a = 0.0f;
+#pragma unroll
+            for (int j = 0; j < D / 2; ++j) a = fmax3(a, fabsf(qrow::p2lo(x2[j])), fabsf(qrow::p2hi(x2[j])));
+            // a >= +0, so the bit patterns order like the values
+            const unsigned am = __reduce_max_sync(0xffffffffu, __float_as_uint(a));
+            float* qmax = reinterpret_cast<float*>(smem + C::kOffQmax);
+            if (lane == 0) qmax[warp] = __uint_as_float(am);
+            asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");   // this tile's four warps
+            const int wpb = p.blk_q >> 5, w0 = (ww / wpb) * wpb;        // warps of the row's block
+            float amax = 0.0f;
+            for (int k = w0; k < w0 + wpb; ++k) amax = fmaxf(amax, qmax[4 * w + k]);
+            float sq = 0.0f, rr = 0.0f;
+            if (amax != 0.0f) {
+                sq = __fdiv_rn(amax, 127.0f);
+                rr = __fdiv_rn(127.0f, amax);
+            }
+            uint8_t* qdst = smem + C::kOffQ + w * C::kQBytes + r * D;
+#pragma unroll
+            for (int c = 0; c < D / 16; ++c) {
+                // 16-byte chunk c of the row at its 128B (D = 128) or 64B
+                // (D = 64) swizzled position, as the TMA path would place it
+                const int sc = D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+                *reinterpret_cast<uint4*>(qdst + (sc << 4)) = qrow::row_codes16<D>(x2, rr, c);
+            }
+            fence_proxy_async_smem();              // read by the QK MMAs
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[C::kBarQ]);
+            qsc = valid ? sq : 0.0f;
+        } else {
+            qsc = valid ? __ldg(&p.q_scale[(int64_t)bh * p.nbq + (i >> p.lg_blk_q)]) : 0.0f;
+        }
         const float arow = qsc * p.logit_scale_log2;
         // last key this row sees (rows past Lq compute on zero padding and
         // are never written)
@@ -644,29 +718,31 @@ bool encode_u8_2d(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t row
 
 template <int D, int NKB, bool CAUSAL>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     const Params& p, dim3 grid, cudaStream_t s) {
-    auto kern = attn_fwd_kernel<D, NKB, CAUSAL>;
+                     const Params& p, const QParams& qp, bool qfused, dim3 grid, cudaStream_t s) {
+    auto kern = qfused ? attn_fwd_kernel<D, NKB, CAUSAL, true> : attn_fwd_kernel<D, NKB, CAUSAL, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg<D>::kSmemBytes);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, grid, dim3(kThreads), Cfg<D>::kSmemBytes, s, tq, tk, tv, p);
+    e = launch_pdl(kern, grid, dim3(kThreads), Cfg<D>::kSmemBytes, s, tq, tk, tv, p, qp);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int D, int NKB>
 cudaError_t launch_c(bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
-                     const CUtensorMap& tv, const Params& p, dim3 grid, cudaStream_t s) {
-    return causal ? launch_t<D, NKB, true>(tq, tk, tv, p, grid, s)
-                  : launch_t<D, NKB, false>(tq, tk, tv, p, grid, s);
+                     const CUtensorMap& tv, const Params& p, const QParams& qp, bool qfused,
+                     dim3 grid, cudaStream_t s) {
+    return causal ? launch_t<D, NKB, true>(tq, tk, tv, p, qp, qfused, grid, s)
+                  : launch_t<D, NKB, false>(tq, tk, tv, p, qp, qfused, grid, s);
 }
 
 template <int D>
 cudaError_t launch_d(int nkb, bool causal, const CUtensorMap& tq, const CUtensorMap& tk,
-                     const CUtensorMap& tv, const Params& p, dim3 grid, cudaStream_t s) {
+                     const CUtensorMap& tv, const Params& p, const QParams& qp, bool qfused,
+                     dim3 grid, cudaStream_t s) {
     switch (nkb) {
-        case 1: return launch_c<D, 1>(causal, tq, tk, tv, p, grid, s);
-        case 2: return launch_c<D, 2>(causal, tq, tk, tv, p, grid, s);
-        default: return launch_c<D, 4>(causal, tq, tk, tv, p, grid, s);
+        case 1: return launch_c<D, 1>(causal, tq, tk, tv, p, qp, qfused, grid, s);
+        case 2: return launch_c<D, 2>(causal, tq, tk, tv, p, qp, qfused, grid, s);
+        default: return launch_c<D, 4>(causal, tq, tk, tv, p, qp, qfused, grid, s);
     }
 }
 
@@ -676,7 +752,8 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
     const int LpadQ = static_cast<int>(round_up(a.Lq, kTile));
     const int LpadK = static_cast<int>(round_up(a.Lk, kTile));
     CUtensorMap tq, tk, tv;
-    if (!encode_u8_2d(&tq, a.q8, a.D, (uint64_t)a.B * a.H * LpadQ, a.D, BM) ||
+    memset(&tq, 0, sizeof tq);                     // not read by the in-CTA Q path
+    if ((!a.qfused && !encode_u8_2d(&tq, a.q8, a.D, (uint64_t)a.B * a.H * LpadQ, a.D, BM)) ||
         !encode_u8_2d(&tk, a.k8, a.D, (uint64_t)a.B * a.Hk * LpadK, a.D, BN) ||
         !encode_u8_2d(&tv, a.v8t, LpadK, (uint64_t)a.B * a.Hk * a.D, BN, a.D))
         return cudaErrorInvalidValue;
@@ -707,11 +784,21 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
                  a.out_stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.out) % 16 == 0)
                     ? 1
                     : 0;
+    QParams qp;
+    qp.qbf = static_cast<const uint16_t*>(a.q16.ptr);
+    qp.qs0 = a.q16.stride[0];
+    qp.qs1 = a.q16.stride[1];
+    qp.qs2 = a.q16.stride[2];
+    qp.qs3 = a.q16.stride[3];
+    qp.q_vec = (a.qfused && a.q16.stride[3] == 1 && a.q16.stride[0] % 8 == 0 && a.q16.stride[1] % 8 == 0 &&
+               a.q16.stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.q16.ptr) % 16 == 0)
+                  ? 1
+                  : 0;
     const int nqt = static_cast<int>(ceil_div(a.Lq, QT * BM));
     const dim3 grid = a.causal ? dim3(a.B * a.H, nqt) : dim3(nqt, a.B * a.H);
     const int nkb = BN / a.blk_k;
-    return a.D == 128 ? launch_d<128>(nkb, a.causal != 0, tq, tk, tv, p, grid, s)
-                      : launch_d<64>(nkb, a.causal != 0, tq, tk, tv, p, grid, s);
+    return a.D == 128 ? launch_d<128>(nkb, a.causal != 0, tq, tk, tv, p, qp, a.qfused != 0, grid, s)
+                      : launch_d<64>(nkb, a.causal != 0, tq, tk, tv, p, qp, a.qfused != 0, grid, s);
 }
 
 #ifdef SAGE_ATTN_TRACE

@@ -43,6 +43,7 @@
 
 #include "sage_internal.h"
 #include "sage_ptx.cuh"
+#include "quant_rows.cuh"
 
 namespace sage {
 
@@ -50,6 +51,7 @@ __device__ unsigned g_quant_err;
 
 namespace {
 
+using namespace qrow;
 namespace cg = cooperative_groups;
 
 constexpr int kStatCluster = 8;      // CTAs per cluster in the statistics kernel
@@ -57,11 +59,6 @@ constexpr int kStatThreads = 256;
 constexpr int kStatUnroll = 8;       // 16-byte loads in flight per thread
 constexpr int kMaxParts = 8;         // clusters per (b, h), at most
 constexpr int kQuantCtasPerSm = 3;   // resident quantisation CTAs per SM
-constexpr float kRoundMagic = 12582912.0f;   // 1.5 * 2^23
-
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
-    return __uint_as_float(bits16 << 16);
-}
 
 // Load 8 consecutive (along D) bf16 values of one token row as raw bits.
 // VEC: one 16-byte load (caller guarantees alignment); else 8 scalar loads.
@@ -215,82 +212,6 @@ __device__ __forceinline__ void gather_tile(const View4& x, int b, int h, int l0
     }
 }
 
-__device__ __forceinline__ uint32_t pack_clamp4(float y0, float y1, float y2, float y3) {
-    const float y[4] = {y0, y1, y2, y3};
-    uint32_t word = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        int code = __float2int_rn(y[i]);
-        code = max(-127, min(127, code));
-        word |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * i);
-    }
-    return word;
-}
-
-// fp32 pairs (sm_100 f32x2 arithmetic): each lane is one IEEE RN operation,
-// so results equal the scalar ones bit for bit. A product feeding an add must
-// not be written as mul.rn.f32x2 + add.rn.f32x2: ptxas contracts that pair
-// into one FMA (a single rounding) despite the explicit rounding modifiers.
-__device__ __forceinline__ uint64_t p2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float p2lo(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo;
-}
-__device__ __forceinline__ float p2hi(uint64_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return hi;
-}
-__device__ __forceinline__ uint64_t p2add(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t p2sub(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t p2fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-__device__ __forceinline__ uint64_t p2mul(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-
-// The butterfly of `butterfly` on a row held as D/2 pairs x2[i] = (x[2i],
-// x[2i+1]): stage h = 1 inside each pair, stages h = 2 .. D/2 as pair
-// operations between pairs i and i + h/2. Same operations, same order per
-// element, so the same bits.
-template <int D>
-__device__ __forceinline__ void butterfly_pairs(uint64_t (&x2)[D / 2]) {
-#pragma unroll
-    for (int i = 0; i < D / 2; ++i) {
-        const float a = p2lo(x2[i]), c = p2hi(x2[i]);
-        x2[i] = p2(__fadd_rn(a, c), __fsub_rn(a, c));
-    }
-#pragma unroll
-    for (int lg = 0; (2 << lg) < D; ++lg) {
-        const int hp = 1 << lg;                  // pair distance = h / 2
-#pragma unroll
-        for (int k = 0; k < D / 4; ++k) {
-            const int i = ((k >> lg) << (lg + 1)) + (k & (hp - 1));
-            const uint64_t a = x2[i], c = x2[i + hp];
-            x2[i] = p2add(a, c);
-            x2[i + hp] = p2sub(a, c);
-        }
-    }
-}
-
 // One 128-token tile of the Q-then-K tile list: tiles [0, n_qtiles) walk Q
 // head by head, the rest walk K.
 struct QkTile {
@@ -417,43 +338,12 @@ __global__ void __launch_bounds__(kTile) qk_quant_kernel(
             scales[(int64_t)tr.bh * nb + l / blk] = s;
         }
 
-        // |x_hat * r| <= a * fl(127 / a) rounds to at most 127 whenever r is
-        // finite, so the magic-number rounding needs no clamp; a block whose
-        // amax is so small that 127 / a overflows takes the clamped conversion.
         // Each thread stores its own code row (rows past L are the zero
         // padding).
         uint4* dst = reinterpret_cast<uint4*>((tr.isK ? k8 : q8) +
                                               ((int64_t)tr.bh * tr.ntiles * kTile + tr.l0 + tid) * D);
-        if (isfinite(rr)) {
-            const uint64_t rr2 = p2(rr, rr), mg2 = p2(kRoundMagic, kRoundMagic);
 #pragma unroll
-            for (int c = 0; c < D / 16; ++c) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    // the product is rounded on its own (an FMA with +0), so the
-                    // magic add that follows cannot be contracted into it
-                    const uint64_t t01 = p2add(p2fma(x2[8 * c + 2 * i], rr2, 0ull), mg2);
-                    const uint64_t t23 = p2add(p2fma(x2[8 * c + 2 * i + 1], rr2, 0ull), mg2);
-                    w4[i] = __byte_perm(__byte_perm(__float_as_uint(p2lo(t01)), __float_as_uint(p2hi(t01)), 0x0040),
-                                        __byte_perm(__float_as_uint(p2lo(t23)), __float_as_uint(p2hi(t23)), 0x0040),
-                                        0x5410);
-                }
-                dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < D / 16; ++c) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint64_t* pv = x2 + 8 * c + 2 * i;
-                    w4[i] = pack_clamp4(__fmul_rn(p2lo(pv[0]), rr), __fmul_rn(p2hi(pv[0]), rr),
-                                        __fmul_rn(p2lo(pv[1]), rr), __fmul_rn(p2hi(pv[1]), rr));
-                }
-                dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
-        }
+        for (int c = 0; c < D / 16; ++c) dst[c] = row_codes16<D>(x2, rr, c);
     }
 }
 
@@ -567,13 +457,13 @@ size_t quant_smem_bytes() {
 template <int D>
 cudaError_t launch_qk_d(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
                         float* q_scale, int8_t* k8, float* k_scale, float* k_mean, void* ws,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool with_q) {
     const int B = (int)q.size[0], H = (int)q.size[1], Lq = (int)q.size[2];
     const int Hk = (int)k.size[1], Lk = (int)k.size[2];
     const int parts = stat_parts(B * Hk);
     column_stats_kernel<D, 0><<<kStatCluster * parts * B * Hk, kStatThreads, 0, s>>>(
         k, parts, ws, view_vec8(k));
-    const int n_qtiles = B * H * (int)ceil_div(Lq, kTile);
+    const int n_qtiles = with_q ? B * H * (int)ceil_div(Lq, kTile) : 0;
     const int n_tiles = n_qtiles + B * Hk * (int)ceil_div(Lk, kTile);
     const int grid = std::min(n_tiles, num_sms() * kQuantCtasPerSm);
     auto kern = qk_quant_kernel<D>;
@@ -618,10 +508,10 @@ size_t quant_v_ws_bytes(int B, int Hk, int L, int D) {
 
 cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
                             float* q_scale, int8_t* k8, float* k_scale, float* k_mean, void* ws,
-                            cudaStream_t s) {
-    return q.size[3] == 128
-               ? launch_qk_d<128>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s)
-               : launch_qk_d<64>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s);
+                            cudaStream_t s, bool with_q) {
+    return k.size[3] == 128
+               ? launch_qk_d<128>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s, with_q)
+               : launch_qk_d<64>(q, k, blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, ws, s, with_q);
 }
 
 cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,

@@ -197,6 +197,27 @@ sage_status sage_quant_qk(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf1
                                                static_cast<cudaStream_t>(stream)));
 }
 
+sage_status sage_quant_k(sage_hadamard h, sage_cview4 k_bf16, int blk_k, int8_t* k8,
+                         float* k_scale, float* k_mean, void* ws, size_t ws_bytes, void* stream) {
+    if (!h || !k_bf16.ptr || !k8 || !k_scale) return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(k_bf16.size, k_bf16.stride)) return SAGE_ERR_INVALID_ARG;
+    const int64_t B = k_bf16.size[0], Hk = k_bf16.size[1], Lk = k_bf16.size[2], D = k_bf16.size[3];
+    if (D != h->D) return SAGE_ERR_INVALID_ARG;
+    if (!blk_ok(blk_k)) return SAGE_ERR_UNSUPPORTED;
+    if (B * Hk * sage::round_up(Lk, 128) >= (int64_t(1) << 31)) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(k8, 16) || !aligned(k_scale, 4) || !aligned(k_mean, 4) || !aligned(k_bf16.ptr, 2))
+        return SAGE_ERR_ALIGNMENT;
+    const size_t need = sage::quant_qk_ws_bytes((int)B, (int)Hk, (int)Lk, (int)D);
+    if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return SAGE_ERR_ALIGNMENT;
+    int dev = -1;
+    if (!current_device(&dev)) return SAGE_ERR_CUDA;
+    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
+    const sage::View4 kv = to_view(k_bf16);
+    return launch_status(sage::launch_quant_qk(kv, kv, blk_k, blk_k, nullptr, nullptr, k8, k_scale,
+                                               k_mean, ws, static_cast<cudaStream_t>(stream), false));
+}
+
 size_t sage_quant_v_workspace(int B, int Hk, int L, int D) {
     if (B < 1 || Hk < 1 || L < 1 || D < 1) return 0;
     return sage::quant_v_ws_bytes(B, Hk, L, D);
@@ -277,6 +298,62 @@ sage_status sage_attn_fwd(const int8_t* q8, const float* q_scale, const int8_t* 
         a.out_size[i] = out_bf16.size[i];
         a.out_stride[i] = out_bf16.stride[i];
     }
+    if (!sage::tensor_map_encoder()) return SAGE_ERR_CUDA;
+    return launch_status(sage::launch_attn_fwd(a, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_attn_fwd_q16(sage_hadamard h, sage_cview4 q_bf16, int blk_q, const int8_t* k8,
+                              const float* k_scale, const uint8_t* v8_t, const float* v_scale,
+                              int Hk, int Lk, int blk_k, float softmax_scale, int causal,
+                              sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!h || !q_bf16.ptr || !k8 || !k_scale || !v8_t || !v_scale || !out_bf16.ptr)
+        return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(q_bf16.size, q_bf16.stride) || !sizes_ok(out_bf16.size, out_bf16.stride))
+        return SAGE_ERR_INVALID_ARG;
+    const int64_t B = q_bf16.size[0], H = q_bf16.size[1], Lq = q_bf16.size[2], D = q_bf16.size[3];
+    if (Hk < 1 || Lk < 1 || !std::isfinite(softmax_scale)) return SAGE_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+        if (out_bf16.size[i] != q_bf16.size[i]) return SAGE_ERR_INVALID_ARG;
+    if (D != h->D) return SAGE_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+    if (H % Hk != 0 || !blk_ok(blk_q) || !blk_ok(blk_k)) return SAGE_ERR_UNSUPPORTED;
+    const int64_t nqt = sage::ceil_div(Lq, 256);
+    if (B * H > 65535 || nqt > 65535) return SAGE_ERR_UNSUPPORTED;
+    if (B * H * sage::round_up(Lq, 128) >= (int64_t(1) << 31) ||
+        B * Hk * sage::round_up(Lk, 128) >= (int64_t(1) << 31) || B * Hk * D >= (int64_t(1) << 31))
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(k8, 16) || !aligned(v8_t, 16) || !aligned(k_scale, 4) || !aligned(v_scale, 4) ||
+        !aligned(q_bf16.ptr, 2) || !aligned(out_bf16.ptr, 2))
+        return SAGE_ERR_ALIGNMENT;
+    int dev = -1;
+    if (!current_device(&dev)) return SAGE_ERR_CUDA;
+    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
+    sage::AttnArgs a;
+    a.q8 = nullptr;
+    a.q_scale = nullptr;
+    a.k8 = k8;
+    a.k_scale = k_scale;
+    a.v8t = v8_t;
+    a.v_scale = v_scale;
+    a.B = (int)B;
+    a.H = (int)H;
+    a.Hk = Hk;
+    a.Lq = (int)Lq;
+    a.Lk = Lk;
+    a.D = (int)D;
+    a.blk_q = blk_q;
+    a.blk_k = blk_k;
+    a.softmax_scale = softmax_scale;
+    a.causal = causal ? 1 : 0;
+    a.out = out_bf16.ptr;
+    for (int i = 0; i < 4; ++i) {
+        a.out_size[i] = out_bf16.size[i];
+        a.out_stride[i] = out_bf16.stride[i];
+    }
+    a.qfused = 1;
+    a.q16 = to_view(q_bf16);
     if (!sage::tensor_map_encoder()) return SAGE_ERR_CUDA;
     return launch_status(sage::launch_attn_fwd(a, static_cast<cudaStream_t>(stream)));
 }

@@ -67,9 +67,10 @@ __host__ __device__ inline int64_t ceil_div(int64_t x, int64_t m) { return (x + 
 // ---- quantisation (quant.cu)
 size_t quant_qk_ws_bytes(int B, int Hk, int Lk, int D);
 size_t quant_v_ws_bytes(int B, int Hk, int L, int D);
+// with_q = false: K alone (q, q8, q_scale unused)
 cudaError_t launch_quant_qk(const View4& q, const View4& k, int blk_q, int blk_k, int8_t* q8,
                             float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
-                            void* ws, cudaStream_t s);
+                            void* ws, cudaStream_t s, bool with_q = true);
 cudaError_t launch_quant_v(const View4& v, uint8_t* v8t, float* v_scale, void* ws,
                            cudaStream_t s);
 unsigned read_clear_quant_error();
@@ -88,6 +89,10 @@ struct AttnArgs {
     void* out;
     int64_t out_size[4];
     int64_t out_stride[4];
+    // in-CTA Q path: q8 / q_scale unused, Q rotated and quantised from this
+    // bf16 [B, H, Lq, D] view inside the attention kernel
+    int qfused = 0;
+    View4 q16 = {};
 };
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s);
 unsigned read_clear_attn_error();

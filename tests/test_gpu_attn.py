@@ -107,3 +107,37 @@ def test_attn_full_size_sampled_rows(handles, key, nrows):
     gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
                         cfg["causal"], rows=rows, exact=True)
     compare_output(gpu, ref, ex, label=key)
+
+
+@pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,blk_q,blk_k,causal", SHAPES)
+def test_attn_q16_same_bits(handles, B, H, Hk, Lq, Lk, D, blk_q, blk_k, causal):
+    """Q rotated and quantised inside the attention kernel (sage_quant_k +
+    sage_attn_fwd_q16) gives the same output bits as sage_quant_qk +
+    sage_attn_fwd: same codes, same block scales, same kernel after them."""
+    g = torch.Generator().manual_seed(Lq * 17 + Lk + D)
+    q = torch.randn((B, Lq, H, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    k = (torch.randn((B, Lk, Hk, D), generator=g) + torch.randn((B, 1, Hk, D), generator=g) * 2)
+    k = k.to(torch.bfloat16).permute(0, 2, 1, 3)
+    v = torch.randn((B, Lk, Hk, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    qg, kg, vg = to_gpu(q), to_gpu(k), to_gpu(v)
+    a, _ = sage.sage_attention(handles[D], qg, kg, vg, blk_q, blk_k, 0.1, causal)
+    b, _ = sage.sage_attention_q16(handles[D], qg, kg, vg, blk_q, blk_k, 0.1, causal)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    assert torch.equal(a, b)
+
+
+def test_attn_q16_strided_query(handles):
+    """The in-CTA Q path on a row-strided view (vector loads) and on a view
+    whose channels are not contiguous (scalar loads)."""
+    q, k, v = workloads.make_prefill(B=1, H=2, Hk=2, L=300, D=128, seed=21, kbias_std=2.0)
+    kg, vg = to_gpu(k), to_gpu(v)
+    ref, _ = sage.sage_attention(handles[128], to_gpu(q), kg, vg, 128, 64, 0.1, False)
+    wide = torch.zeros((1, 2, 300, 136), dtype=torch.bfloat16, device="cuda")
+    wide[..., :128] = to_gpu(q)
+    inter = torch.zeros((1, 2, 300, 128, 2), dtype=torch.bfloat16, device="cuda")
+    inter[..., 0] = to_gpu(q)
+    for qv in (wide[..., :128], inter[..., 0]):
+        o, _ = sage.sage_attention_q16(handles[128], qv, kg, vg, 128, 64, 0.1, False)
+        torch.cuda.synchronize()
+        assert torch.equal(o, ref)
