@@ -9,28 +9,32 @@
 // windows, [lo, ctx)) are cut into 128-key tiles aligned to absolute key
 // positions, so a tile is one page (page 128) or 128 / page whole pages.
 // The tiles of (b, kv head hk) are shared out among up to 8 CTAs that form
-// one thread-block cluster; CTA = 16 warps:
-//   warps 0-7  softmax: warps w and w + 4 own query rows 16w .. 16w + 15
-//              (R = T * H/Hk rows, row r = t * G + g, padded to 64) -- M = 64
-//              MMAs keep those rows in TMEM lanes 32w .. 32w + 15 -- warp w
-//              the tile's columns 0-63, warp w + 4 columns 64-127;
-//   warps 8-11 V converters: e4m3 V tile -> exact bf16, in the key order of
-//              the P operand;
+// one thread-block cluster (the size is picked at launch so that the grid
+// runs in one wave); CTA = 16 warps:
+//   warps 0-7  softmax: warps w and w + 4 (w < 4) own query rows 16w ..
+//              16w + 15 (R = T * H/Hk rows, row r = t * G + g, padded to 64)
+//              -- M = 64 MMAs keep those rows in TMEM lanes 32w .. 32w + 15
+//              -- warp w the tile's columns 0-63, warp w + 4 columns 64-127;
+//   warps 8-11 V converters: e4m3 V tile -> exact bf16 (integer bit
+//              placement and one bf16 multiply), in the key order of the P
+//              operand;
 //   warp 12    producer: page-table lookups, one TMA box per page for K and
 //              for V, per-token scales by cp.async, all on one mbarrier;
-//   warp 13    TMEM owner and MMA issuer (warps 14, 15 only join the merge).
+//   warp 13    TMEM owner and MMA issuer (warps 14, 15 only complete the
+//              producer's warpgroup).
 // Per tile: S = Q8 K8^T (e4m3 tcgen05 MMAs, M=64 N=128, fp32 in TMEM,
-// double-buffered) -> logits S * s_q * k_scale_j * softmax_scale / D in
-// base 2, masked to each row's own window -> running max m -> p = 2^(x - m)
-// -> P' = bf16(p * v_scale_j) -> O[i & 1] += P' V (bf16 tcgen05 MMAs, fp32
-// in TMEM). Even and odd tiles accumulate into two O's, so the rescale of
-// the one tile i adds to (by 2^(m_old - m) for rows whose max rose) waits
-// for PV(i - 2), not for PV(i - 1); the epilogue adds the two at the final
-// max. The query rows are rotated and quantised to e4m3 in the prologue
-// (fp32 butterfly, scale max|q_hat| / 448, the operations of the quantisation
-// kernels). At the end every CTA leaves (m, l, O) of its tiles in shared
-// memory and the CTAs of the cluster merge them (log-sum-exp) through
-// distributed shared memory and write bf16 through the caller's strides.
+// double-buffered) -> base-2 logits (S * k_scale_j) * s_q * softmax_scale /
+// D, masked to each row's own window -> running max m -> p = 2^(x - m) ->
+// P' = bf16(p * v_scale_j) -> O[i & 1] += P' V (bf16 tcgen05 MMAs, fp32 in
+// TMEM). Even and odd tiles accumulate into two O's: before PV(i), the rows
+// of O[i & 1] whose max rose since tile i - 2 are rescaled by 2^(m_old - m),
+// which needs PV(i - 2) done rather than PV(i - 1); the epilogue adds the two
+// O's at the final max. The query rows are rotated and quantised to e4m3 in
+// the prologue (fp32 butterfly, four threads per row, scale max|q_hat| / 448,
+// the operations of the quantisation kernels). At the end every CTA leaves
+// (m, l, O) of its tiles in shared memory and the CTAs of the cluster merge
+// them (log-sum-exp) through distributed shared memory and write bf16
+// through the caller's strides.
 //
 // Every mbarrier wait is bounded; on timeout the CTA records an error word,
 // raises its abort flag, drains its own copies and MMAs and still takes part
