@@ -64,6 +64,8 @@ def test_decode_window_family_workload(h128):
     (2, 2, 16, 2, 64, 257, 700, 256),    # page 64, R = 16
     (4, 4, 16, 1, 32, 4, 30, 4096),      # tiny contexts
     (1, 3, 12, 3, 128, 1000, 1000, 300), # T = 3, G = 4
+    (2, 4, 16, 2, 16, 5000, 6000, 8192), # page 16, long window: page ids refetched 32 at a time
+    (40, 2, 8, 1, 128, 1500, 2500, 4096),# 40 clusters: more than one wave of them
 ])
 def test_decode_shapes(h128, B, T, H, Hk, page, lo, hi, window):
     d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=128, page=page, ctx_lo=lo, ctx_hi=hi,
