@@ -2,8 +2,8 @@
 """Throughput of the quantised attention path on B200.
 
 One step = the whole hot path on one batch of seeded synthetic inputs that
-already sit in HBM: sage_quant_qk (K mean, smoothing, Hadamard rotation, INT8
-Q/K) + sage_quant_v (e4m3 V) + sage_attn_fwd (INT8 QK^T, online softmax, e4m3
+already sit in HBM: sage_quant_qkv (K mean, smoothing, Hadamard rotation, INT8
+Q/K, e4m3 V; two launches) + sage_attn_fwd (INT8 QK^T, online softmax, e4m3
 PV, bf16 out). Workload: non-causal video-DiT prefill B=1 H=24 L=4096 D=128
 (Q blocks 128 tokens, K blocks 64). Metric: TOPS = 4 B H L^2 D / step time.
 
@@ -340,8 +340,8 @@ def run_sage(args):
 
     def step(i, timed):
         qs, ks, vs_, bufs, out = sets[i % len(sets)]
-        # Q/K (or K) quantisation on `stream`, V quantisation beside it on a
-        # second stream, attention after both
+        # sage_quant_qkv on `stream` (with --fused-q: K on `stream`, V beside
+        # it on a second stream), then the attention
         sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
         if timed:
             ev[i][0].record(stream)
@@ -452,6 +452,35 @@ def run_sage(args):
            "ms_per_step": e2e_ms / args.e2e_steps,
            "pipeline": "h2d, compute and d2h on three streams over two buffer pairs"}
 
+    # the quantisation alone (both launches of sage_quant_qkv, or sage_quant_k
+    # + sage_quant_v with --fused-q), over the same rotating input sets
+    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.warmup):
+        qs, ks, vs_, bufs, _ = sets[i % len(sets)]
+        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        qs, ks, vs_, bufs, _ = sets[i % len(sets)]
+        qev[i][0].record(stream)
+        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
+        qev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if sage.sage_device_error(stream) != sage.SAGE_OK:
+        raise RuntimeError("device error while timing the quantisation")
+    q_times = sorted(a.elapsed_time(b) * 1e3 for a, b in qev)
+    q_us = statistics.median(q_times)
+    q_bytes = 3 * ((0 if args.fused_q else q.numel()) + k.numel() + v.numel())
+    quant = {"us_per_call": q_us,
+             "us_p10_p50_p90": [pct(q_times, 10), pct(q_times, 50), pct(q_times, 90)],
+             "algorithmic_bytes": q_bytes,
+             "achieved": q_bytes / (q_us * 1e-6) / 1e9, "unit": "GB/s",
+             "peak": pk["hbm_gbs"], "frac": q_bytes / (q_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+             "peak_source": pk_src + " copy bandwidth",
+             "bytes_rule": "2 B read + 1 B written per element of each quantised tensor; the "
+                           "statistics pass re-reads K and V (not counted)",
+             "launches_per_call": 4 if args.fused_q else 2}
+
     dec = None if args.no_decode else bench_decode(sage, torch, stream)
 
     cb = None
@@ -472,8 +501,9 @@ def run_sage(args):
             "roofline": roofline,
             "cpu_baseline": cb,
             "e2e": e2e,
+            "quant": quant,
             "decode": dec,
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": (5 if args.fused_q else 3) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line))

@@ -117,8 +117,9 @@ sage_status sage_hadamard_destroy(sage_hadamard h);
  * and/or report D through `head_dim` (either may be NULL). */
 sage_status sage_hadamard_matrix(sage_hadamard h, int8_t* host_out, int* head_dim);
 
-/* Bytes of device workspace sage_quant_qk needs: fp64 partial column sums
- * of K, up to 8 per (b, kv head, d): B * Hk * 8 * D * 8. */
+/* Bytes of device workspace sage_quant_qk needs: the fp32 K mean of every
+ * (b, kv head, d), passed from the statistics pass to the quantisation
+ * pass: B * Hk * D * 4. */
 size_t sage_quant_qk_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
 
 /* Smooth, rotate and INT8-quantise Q and K.
@@ -150,7 +151,7 @@ sage_status sage_quant_qk(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf1
  * 8 MiB array built into the library; every GPU that loads the library holds
  * it until the process exits. Calls whose sage_quant_qk_workspace(...) exceeds
  * 8 MiB are rejected with SAGE_ERR_WORKSPACE before anything is launched
- * (8 MiB covers B * Hk * D <= 128 Ki, e.g. 1024 kv heads of D = 128).
+ * (8 MiB covers B * Hk * D <= 2 Mi, e.g. 16384 kv heads of D = 128).
  * The first call on a device looks the array's device address up
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture. Every call on a device shares the one array and leaves
@@ -169,8 +170,8 @@ sage_status sage_quant_qk_noalloc(sage_hadamard h, sage_cview4 q_bf16, sage_cvie
 sage_status sage_quant_k(sage_hadamard h, sage_cview4 k_bf16, int blk_k, int8_t* k8,
                          float* k_scale, float* k_mean, void* ws, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace sage_quant_v needs: fp32 partial channel
- * maxima, up to 8 per (b, h, d): B * Hk * 8 * D * 4. */
+/* Bytes of device workspace sage_quant_v needs: the fp32 multiplier 448 / a
+ * of every (b, h, d): B * Hk * D * 4. */
 size_t sage_quant_v_workspace(int B, int Hk, int L, int D);
 
 /* FP8 e4m3 (OCP e4m3fn, max 448) per-channel quantisation of V.
@@ -178,9 +179,26 @@ size_t sage_quant_v_workspace(int B, int Hk, int L, int D);
  * Per (b, h, d): a = max over the L tokens of |v|, scale = a / 448,
  * code = e4m3_round_nearest_even_saturating(v * (448 / a)) (a = 0 gives
  * scale 0 and zero codes). Writes v8_t [B, Hk, D, Lpad(L)] (transposed) and
- * v_scale [B, Hk, D]. ws as for sage_quant_qk. */
+ * v_scale [B, Hk, D]. ws: at least sage_quant_v_workspace(...) bytes,
+ * 16-byte aligned, contents on entry irrelevant. */
 sage_status sage_quant_v(sage_cview4 v_bf16, uint8_t* v8_t, float* v_scale, void* ws,
                          size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace sage_quant_qkv needs:
+ * sage_quant_qk_workspace(...) + sage_quant_v_workspace(B, Hk, Lk, D). */
+size_t sage_quant_qkv_workspace(int B, int H, int Hk, int Lq, int Lk, int D);
+
+/* sage_quant_qk and sage_quant_v in one call, with the same outputs bit for
+ * bit: v_bf16 has k_bf16's sizes [B, Hk, Lk, D] (any strides). The K and V
+ * statistics run as one launch and the Q, K and V quantisation as a second,
+ * so the copy-bound V work shares the SMs with the Q/K rotation. ws: at
+ * least sage_quant_qkv_workspace(...) bytes, 16-byte aligned, contents on
+ * entry irrelevant. Errors as for sage_quant_qk, and INVALID_ARG when V's
+ * sizes differ from K's. */
+sage_status sage_quant_qkv(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16,
+                           sage_cview4 v_bf16, int blk_q, int blk_k, int8_t* q8, float* q_scale,
+                           int8_t* k8, float* k_scale, float* k_mean, uint8_t* v8_t,
+                           float* v_scale, void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace sage_attn_fwd needs (0 in this version). */
 size_t sage_attn_fwd_workspace(int B, int H, int Hk, int Lq, int Lk, int D);

@@ -28,7 +28,8 @@ SAGE_ERR_TIMEOUT = 6
 EXPORTS = (
     "sage_hadamard_init", "sage_hadamard_destroy", "sage_hadamard_matrix",
     "sage_quant_qk_workspace", "sage_quant_qk", "sage_quant_qk_noalloc",
-    "sage_quant_v_workspace", "sage_quant_v", "sage_quant_k",
+    "sage_quant_v_workspace", "sage_quant_v", "sage_quant_k", "sage_quant_qkv_workspace",
+    "sage_quant_qkv",
     "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_fwd_q16", "sage_attn_decode_workspace",
     "sage_attn_decode", "sage_status_string", "sage_device_error",
 )
@@ -82,6 +83,10 @@ def lib():
     L.sage_quant_v.argtypes = [CView4, vp, vp, vp, sz, vp]
     L.sage_quant_k.restype = i32
     L.sage_quant_k.argtypes = [vp, CView4, i32, vp, vp, vp, vp, sz, vp]
+    L.sage_quant_qkv_workspace.restype = sz
+    L.sage_quant_qkv_workspace.argtypes = [i32] * 6
+    L.sage_quant_qkv.restype = i32
+    L.sage_quant_qkv.argtypes = [vp, CView4, CView4, CView4, i32, i32] + [vp] * 8 + [sz, vp]
     L.sage_attn_fwd_workspace.restype = sz
     L.sage_attn_fwd_workspace.argtypes = [i32] * 6
     L.sage_attn_fwd.restype = i32
@@ -217,6 +222,19 @@ def sage_attn_fwd_q16(h, q, blk_q, k8, k_scale, v8_t, v_scale, Hk, Lk, blk_k, so
                                    _stream(stream)), "sage_attn_fwd_q16")
 
 
+def sage_quant_qkv_workspace(B, H, Hk, Lq, Lk, D):
+    return int(lib().sage_quant_qkv_workspace(B, H, Hk, Lq, Lk, D))
+
+
+def sage_quant_qkv(h, q, k, v, blk_q, blk_k, q8, q_scale, k8, k_scale, v8_t, v_scale, k_mean=None,
+                   ws=None, stream=None):
+    _check(lib().sage_quant_qkv(h.handle, _view(q, CView4), _view(k, CView4), _view(v, CView4),
+                                int(blk_q), int(blk_k), _ptr(q8), _ptr(q_scale), _ptr(k8),
+                                _ptr(k_scale), _ptr(k_mean), _ptr(v8_t), _ptr(v_scale), _ptr(ws),
+                                0 if ws is None else ws.numel() * ws.element_size(),
+                                _stream(stream)), "sage_quant_qkv")
+
+
 def sage_quant_v(v, v8_t, v_scale, ws=None, stream=None):
     _check(lib().sage_quant_v(_view(v, CView4), _ptr(v8_t), _ptr(v_scale), _ptr(ws),
                               0 if ws is None else ws.numel() * ws.element_size(),
@@ -268,10 +286,11 @@ class QuantBuffers:
         self.k_mean = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
         self.v8_t = torch.empty((B, Hk, D, round_up(Lk, 128)), dtype=torch.uint8, device=dev)
         self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
-        ws = max(sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D), sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D), 16)
+        ws = max(sage_quant_qkv_workspace(B, H, Hk, Lq, Lk, D), sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D),
+                 sage_attn_fwd_workspace(B, H, Hk, Lq, Lk, D), 16)
         self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev)
-        # the V quantisation has its own workspace so it can run on a second
-        # stream beside the Q/K quantisation
+        # for K and V without Q: the V quantisation has its own workspace so
+        # it can run on a second stream beside the K quantisation
         self.ws_v = torch.empty((max(sage_quant_v_workspace(B, Hk, Lk, D), 16),), dtype=torch.uint8,
                                 device=dev)
         self.side = torch.cuda.Stream(device=dev)
@@ -312,18 +331,19 @@ def sage_attention_q16(h, q, k, v, blk_q, blk_k, softmax_scale, causal=False, ou
 
 
 def quantise(h, q, k, v, blk_q, blk_k, bufs, stream=None):
-    """sage_quant_qk (sage_quant_k when q is None) on `stream` and, beside
-    it, sage_quant_v on the buffers' second stream (the two read and write
-    disjoint buffers); work issued to `stream` afterwards waits for both."""
+    """sage_quant_qkv on `stream`; when q is None, sage_quant_k on `stream`
+    and, beside it, sage_quant_v on the buffers' second stream (the two read
+    and write disjoint buffers), work issued to `stream` afterwards waiting
+    for both."""
     s = torch.cuda.current_stream() if stream is None else stream
+    if q is not None:
+        sage_quant_qkv(h, q, k, v, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                       bufs.v8_t, bufs.v_scale, bufs.k_mean, bufs.ws, s)
+        return
     fork = torch.cuda.Event()
     fork.record(s)
     bufs.side.wait_event(fork)
-    if q is None:
-        sage_quant_k(h, k, blk_k, bufs.k8, bufs.k_scale, bufs.k_mean, bufs.ws, s)
-    else:
-        sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
-                      bufs.k_mean, bufs.ws, s)
+    sage_quant_k(h, k, blk_k, bufs.k8, bufs.k_scale, bufs.k_mean, bufs.ws, s)
     sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v, bufs.side)
     join = torch.cuda.Event()
     join.record(bufs.side)

@@ -240,6 +240,49 @@ sage_status sage_quant_v(sage_cview4 v_bf16, uint8_t* v8_t, float* v_scale, void
                                               static_cast<cudaStream_t>(stream)));
 }
 
+size_t sage_quant_qkv_workspace(int B, int H, int Hk, int Lq, int Lk, int D) {
+    (void)H;
+    (void)Lq;
+    if (B < 1 || Hk < 1 || Lk < 1 || D < 1) return 0;
+    return sage::quant_qkv_ws_bytes(B, Hk, Lk, D);
+}
+
+sage_status sage_quant_qkv(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16,
+                           sage_cview4 v_bf16, int blk_q, int blk_k, int8_t* q8, float* q_scale,
+                           int8_t* k8, float* k_scale, float* k_mean, uint8_t* v8_t,
+                           float* v_scale, void* ws, size_t ws_bytes, void* stream) {
+    if (!h || !q_bf16.ptr || !k_bf16.ptr || !v_bf16.ptr || !q8 || !q_scale || !k8 || !k_scale ||
+        !v8_t || !v_scale)
+        return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(q_bf16.size, q_bf16.stride) || !sizes_ok(k_bf16.size, k_bf16.stride) ||
+        !sizes_ok(v_bf16.size, v_bf16.stride))
+        return SAGE_ERR_INVALID_ARG;
+    const int64_t B = q_bf16.size[0], H = q_bf16.size[1], Lq = q_bf16.size[2], D = q_bf16.size[3];
+    const int64_t Hk = k_bf16.size[1], Lk = k_bf16.size[2];
+    if (k_bf16.size[0] != B || k_bf16.size[3] != D) return SAGE_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i)
+        if (v_bf16.size[i] != k_bf16.size[i]) return SAGE_ERR_INVALID_ARG;
+    if (D != h->D) return SAGE_ERR_INVALID_ARG;
+    if (H % Hk != 0) return SAGE_ERR_UNSUPPORTED;
+    if (!blk_ok(blk_q) || !blk_ok(blk_k)) return SAGE_ERR_UNSUPPORTED;
+    if (B * H * sage::round_up(Lq, 128) >= (int64_t(1) << 31) ||
+        B * Hk * sage::round_up(Lk, 128) >= (int64_t(1) << 31))
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8_t, 16) || !aligned(q_scale, 4) ||
+        !aligned(k_scale, 4) || !aligned(k_mean, 4) || !aligned(v_scale, 4) ||
+        !aligned(q_bf16.ptr, 2) || !aligned(k_bf16.ptr, 2) || !aligned(v_bf16.ptr, 2))
+        return SAGE_ERR_ALIGNMENT;
+    const size_t need = sage::quant_qkv_ws_bytes((int)B, (int)Hk, (int)Lk, (int)D);
+    if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return SAGE_ERR_ALIGNMENT;
+    int dev = -1;
+    if (!current_device(&dev)) return SAGE_ERR_CUDA;
+    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
+    return launch_status(sage::launch_quant_qkv(to_view(q_bf16), to_view(k_bf16), to_view(v_bf16),
+                                                blk_q, blk_k, q8, q_scale, k8, k_scale, k_mean, v8_t,
+                                                v_scale, ws, static_cast<cudaStream_t>(stream)));
+}
+
 size_t sage_attn_fwd_workspace(int B, int H, int Hk, int Lq, int Lk, int D) {
     (void)B;
     (void)H;

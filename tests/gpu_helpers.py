@@ -30,13 +30,18 @@ def to_gpu(t):
     return t.to("cuda")
 
 
-def gpu_quant(h, q, k, v, blk_q, blk_k):
+def gpu_quant(h, q, k, v, blk_q, blk_k, fused=False):
+    """sage_quant_qk + sage_quant_v, or (fused) sage_quant_qkv."""
     B, H, Lq, D = q.shape
     Hk, Lk = k.shape[1], k.shape[2]
     bufs = sage.QuantBuffers(B, H, Hk, Lq, Lk, D, blk_q, blk_k)
-    sage.sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
-                       bufs.k_mean, bufs.ws)
-    sage.sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v)
+    if fused:
+        sage.sage_quant_qkv(h, q, k, v, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                            bufs.v8_t, bufs.v_scale, bufs.k_mean, bufs.ws)
+    else:
+        sage.sage_quant_qk(h, q, k, blk_q, blk_k, bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale,
+                           bufs.k_mean, bufs.ws)
+        sage.sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v)
     torch.cuda.synchronize()
     assert sage.sage_device_error() == sage.SAGE_OK
     return bufs

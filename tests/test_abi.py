@@ -53,9 +53,11 @@ def test_status_strings(L):
 
 
 def test_workspace_sizes_are_host_only(L):
-    # up to 8 partial statistics per (b, kv head, d): fp64 sums of K, fp32 maxima of V
-    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 8 * 128 * 8
-    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 8 * 128 * 4
+    # one fp32 statistic per (b, kv head, d): the K mean, the V multiplier 448 / a
+    assert L.sage_quant_qk_workspace(1, 24, 24, 4096, 4096, 128) == 1 * 24 * 128 * 4
+    assert L.sage_quant_v_workspace(1, 40, 32760, 128) == 1 * 40 * 128 * 4
+    assert L.sage_quant_qkv_workspace(2, 32, 8, 4096, 4096, 64) == 2 * (2 * 8 * 64 * 4)
+    assert L.sage_quant_qkv_workspace(1, 1, 0, 1, 1, 64) == 0
     assert L.sage_attn_fwd_workspace(1, 24, 24, 4096, 4096, 128) == 0
     assert L.sage_quant_qk_workspace(0, 1, 1, 1, 1, 64) == 0
 
@@ -123,6 +125,11 @@ def test_quant_validation_without_gpu(L):
     assert L.sage_quant_v(_cview(), p, p, p, 16, None) == sage.SAGE_ERR_WORKSPACE
     assert L.sage_quant_v(_cview(), ctypes.c_void_p(0x10001), p, p, 1 << 20, None) == \
         sage.SAGE_ERR_ALIGNMENT
+    # Q, K and V in one call: null handle, null V
+    assert L.sage_quant_qkv(None, _cview(), _cview(), _cview(), 64, 64, p, p, p, p, None, p, p, p,
+                            1 << 20, None) == sage.SAGE_ERR_INVALID_ARG
+    assert L.sage_quant_qkv(p, _cview(), _cview(), _cview(ptr=0), 64, 64, p, p, p, p, None, p, p,
+                            p, 1 << 20, None) == sage.SAGE_ERR_INVALID_ARG
 
 
 def test_hadamard_init_argument_checks(L):

@@ -28,10 +28,14 @@ def H64():
 
 
 def _check(h, q, k, v, blk_q, blk_k):
+    """Both entry paths -- sage_quant_qk + sage_quant_v, and sage_quant_qkv --
+    against the oracle."""
     ref = oracle.quant_qk(bits(q), bits(k), blk_q, blk_k)
     ref_v8t, ref_vs = oracle.quant_v(bits(v))
-    bufs = gpu_quant(h, to_gpu(q), to_gpu(k), to_gpu(v), blk_q, blk_k)
-    assert_quant_bitexact(bufs, ref, ref_v8t, ref_vs, q.shape[2], k.shape[2])
+    qg, kg, vg = to_gpu(q), to_gpu(k), to_gpu(v)
+    for fused in (False, True):
+        bufs = gpu_quant(h, qg, kg, vg, blk_q, blk_k, fused=fused)
+        assert_quant_bitexact(bufs, ref, ref_v8t, ref_vs, q.shape[2], k.shape[2])
 
 
 def test_hadamard_handle_matrix(H128, H64):
@@ -91,8 +95,30 @@ def test_quant_deterministic(H128):
     h = sage.Hadamard(64)
     a = gpu_quant(h, to_gpu(q), to_gpu(k), to_gpu(v), 64, 64)
     b = gpu_quant(h, to_gpu(q), to_gpu(k), to_gpu(v), 64, 64)
+    c = gpu_quant(h, to_gpu(q), to_gpu(k), to_gpu(v), 64, 64, fused=True)
     for name in ("q8", "q_scale", "k8", "k_scale", "k_mean", "v8_t", "v_scale"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
+        assert torch.equal(getattr(a, name), getattr(c, name)), name
+
+
+def test_quant_qkv_gqa_grid_parity():
+    """sage_quant_qkv over many heads and odd tile counts: the K/V tiles
+    alternate in the tile list and the persistent grid is made odd, so every
+    CTA sees both kinds; GQA gives Q more heads than K and V."""
+    h = sage.Hadamard(128)
+    q, k, v = workloads.make_prefill(B=2, H=12, Hk=3, L=1000, D=128, seed=4242, kbias_std=2.0,
+                                     outlier_channels=3, heavy_frac=0.02)
+    _check(h, q, k, v, 128, 64)
+
+
+def test_quant_qkv_rejects_mismatched_v(H128):
+    q, k, v = workloads.make_prefill(B=1, H=2, Hk=2, L=256, D=128, seed=3)
+    bufs = sage.QuantBuffers(1, 2, 2, 256, 256, 128, 64, 64)
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_quant_qkv(H128, to_gpu(q), to_gpu(k), to_gpu(v[:, :, :200]), 64, 64, bufs.q8,
+                            bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
+                            bufs.k_mean, bufs.ws)
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("key", ["c3", "c4"])

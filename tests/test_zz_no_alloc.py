@@ -66,7 +66,7 @@ def test_no_alloc_matches_workspace_entry_point_twice():
 
 def test_no_alloc_rejects_sizes_beyond_its_scratch():
     h = sage.Hadamard(128)
-    # 32768 kv heads of D = 128 need 32768 * 8 * 128 * 8 B = 256 MiB of K partial sums
+    # 32768 kv heads of D = 128 need 32768 * 128 * 4 B = 16 MiB of K means
     big = sage.CView4()
     big.ptr = 0x10000
     sizes = (1, 32768, 1, 128)
