@@ -1,9 +1,11 @@
 // quant_rows.cuh -- the per-row arithmetic of the INT8 quantisation of
-// Q and K, shared by the quantisation kernels and the attention kernel's
-// in-CTA Q path so that both produce the same bits: bf16 -> fp32, the
-// Sylvester butterfly on fp32 pairs, and the codes rne(x_hat * (127 / a))
+// Q and K: bf16 -> fp32, f32x2 operations, the Sylvester butterfly on fp32
+// pairs of a row held by one thread, and the codes rne(x_hat * (127 / a))
 // ("Sage v2 in AITER" / "qr_hadamard_quant": rotate, block absmax, scale,
-// INT8). Internal to libsage.
+// INT8). The attention kernel's in-CTA Q path uses the row helpers; the
+// quantisation kernels (a row spread over four threads) use the same
+// primitives in the same order, so both produce the same bits. Internal to
+// libsage.
 #pragma once
 
 #include <cstdint>
