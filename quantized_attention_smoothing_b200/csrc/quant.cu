@@ -55,8 +55,6 @@
 
 namespace sage {
 
-__device__ unsigned g_quant_err;
-
 namespace {
 
 using namespace qrow;
@@ -768,13 +766,6 @@ cudaError_t launch_quant_qkv(const View4& q, const View4& k, const View4& v, int
         return launch_quant_d<decltype(d)::value>(&q, &k, &v, blk_q, blk_k, q8, q_scale, k8, k_scale,
                                                   k_mean, v8t, v_scale, ws, s);
     });
-}
-
-unsigned read_clear_quant_error() {
-    unsigned v = 0, zero = 0;
-    if (cudaMemcpyFromSymbol(&v, g_quant_err, sizeof v) != cudaSuccess) return 0;
-    cudaMemcpyToSymbol(g_quant_err, &zero, sizeof zero);
-    return v;
 }
 
 }  // namespace sage

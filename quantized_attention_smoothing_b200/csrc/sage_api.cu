@@ -467,10 +467,8 @@ sage_status sage_device_error(void* stream) {
     const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     const unsigned a = sage::read_clear_attn_error();
     const unsigned d = sage::read_clear_decode_error();
-    const unsigned q = sage::read_clear_quant_error();
     if (e != cudaSuccess) return SAGE_ERR_CUDA;
-    if ((a & 0xFFu) == sage::kErrTimeoutCode || (d & 0xFFu) == sage::kErrTimeoutCode ||
-        (q & 0xFFu) == sage::kErrTimeoutCode)
+    if ((a & 0xFFu) == sage::kErrTimeoutCode || (d & 0xFFu) == sage::kErrTimeoutCode)
         return SAGE_ERR_TIMEOUT;
     if ((d & 0xFFu) == sage::kErrRangeCode) return SAGE_ERR_INVALID_ARG;
     return SAGE_OK;

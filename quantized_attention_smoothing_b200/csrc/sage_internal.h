@@ -78,7 +78,6 @@ size_t quant_qkv_ws_bytes(int B, int Hk, int Lk, int D);
 cudaError_t launch_quant_qkv(const View4& q, const View4& k, const View4& v, int blk_q, int blk_k,
                              int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
                              uint8_t* v8t, float* v_scale, void* ws, cudaStream_t s);
-unsigned read_clear_quant_error();
 
 // ---- attention forward (attn_fwd.cu)
 struct AttnArgs {
