@@ -16,6 +16,9 @@
  *   sage_quant_v         FP8 e4m3 quantisation of V with one scale per
  *                        channel ("Sage2 SM89 Temporal Pair Experiment",
  *                        Candidate: the kernel fuses a per-channel V scale).
+ *   sage_quant_qkv       both of the above in one call (two launches: the K
+ *                        and V statistics, then every Q, K and V tile), the
+ *                        same outputs bit for bit.
  *   sage_attn_fwd        S = Q8 K8^T in INT8, dequantised, online softmax in
  *                        128-key tiles with the per-tile order QK ->
  *                        update_mdo -> accumulate_d -> RS_32_to_8 -> PV
