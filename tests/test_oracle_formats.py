@@ -80,3 +80,40 @@ def test_bf16_rounding_matches_torch(oracle_mod):
     assert np.array_equal(ours, ref)
     back = oracle_mod.bf16_to_f32(ref)
     assert np.array_equal(back.view(np.uint32) >> 16, ref.astype(np.uint32))
+
+
+def test_e4m3_encode_every_rounding_boundary(oracle_mod):
+    """The encoder is a search over the sorted code values, so it is monotonic
+    and every fp32 input is pinned once each rounding boundary is: for every
+    pair of neighbouring finite codes, the midpoint (exact in fp32) and the
+    fp32 values just below and above it, both signs, against torch's cast."""
+    vals = np.sort(np.unique(np.abs(oracle_mod.e4m3_decode(np.arange(256))[
+        np.isfinite(oracle_mod.e4m3_decode(np.arange(256)))])))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    pts = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(np.inf)),
+                          vals.astype(np.float32)])
+    pts = np.concatenate([pts, -pts]).astype(np.float32)
+    ours = oracle_mod.e4m3_encode(pts.astype(np.float64))
+    ref = torch.from_numpy(pts).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert len(mids) == 126 and np.array_equal(ours, ref)
+
+
+def test_int8_magic_rounding_is_round_half_even():
+    """The quantisation kernels round x_hat * r to an integer by adding
+    1.5 * 2^23 in fp32 and keeping the low byte of the sum. For every fp32
+    value of magnitude in [2^-2, 128) (all smaller ones round to 0 both ways)
+    that equals round-half-even, as the oracle's rint does."""
+    magic = np.float32(12582912.0)
+    for e in range(-2, 7):
+        mant = np.arange(1 << 23, dtype=np.uint32)
+        bits = ((np.uint32(127 + e) << np.uint32(23)) | mant).view(np.float32)
+        for x in (bits, -bits):
+            s = (x + magic).astype(np.float32)
+            low = (s.view(np.uint32) & np.uint32(0xFF)).astype(np.uint8).view(np.int8)
+            ref = np.rint(x.astype(np.float64))
+            ok = np.abs(ref) <= 127
+            assert np.array_equal(low[ok].astype(np.int64), ref[ok].astype(np.int64)), e
+    small = np.array([0.25, -0.25, 0.5, -0.5, 1e-30, -1e-30, 0.0, -0.0], dtype=np.float32)
+    s = (small + magic).astype(np.float32)
+    assert np.array_equal((s.view(np.uint32) & np.uint32(0xFF)).astype(np.uint8).view(np.int8),
+                          np.rint(small).astype(np.int8))
