@@ -8,7 +8,9 @@ oracle by the GPU tests):
   127 * 128 (D = 128 products of two codes in [-127, 127]);
 * decode: an e4m3 code moved into the top byte of a bf16 lane and shifted
   right by 4 (sign kept) is a bf16 whose value times 2^120 is the code's
-  value, subnormal codes included."""
+  value, subnormal codes included;
+* attention: the FMA-pipe exp2 that takes every 8th key pair keeps its
+  stated relative error bound."""
 import numpy as np
 import torch
 
@@ -33,3 +35,53 @@ def test_e4m3_code_to_bf16_by_shift_and_scale():
     # the scaled values are bf16-representable and the subnormal codes (exponent field 0)
     # land on bf16 subnormals, which the multiply keeps
     assert (np.abs(as_f32[np.abs(ref) > 0]) < 2.0 ** -126).any()
+
+
+def _poly_coefficients():
+    """The degree-5 coefficients of the attention kernel's FMA-pipe exp2, read
+    from the CUDA source (highest degree first)."""
+    import os
+    import re
+    src = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "quantized_attention_smoothing_b200", "csrc", "sage_ptx.cuh")).read()
+    body = src[src.index("void exp2_poly_x2"):]
+    body = body[:body.index("\n}\n")]
+    hexes = re.findall(r"f2_pack\((0x[0-9a-fA-F.]+p[-+]?\d+)f,", body)
+    return [np.float32(float.fromhex(h)) for h in hexes]
+
+
+def _fma32(a, b, c):
+    # fp32 a*b + c: the product of two fp32 values is exact in fp64; the fp64
+    # sum then rounds far below fp32 precision, so this differs from the
+    # kernel's single rounding at most at exact fp32 halfway points (one fp32
+    # ulp), which the bound below does not depend on
+    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
+
+
+def test_exp2_polynomial_error_bound():
+    """The kernel's exp2 on the FMA pipe (a = n + f, n = rint(a) by the
+    1.5 * 2^23 bias, 2^f by a degree-5 polynomial in fp32 Horner form, 2^n
+    added into the exponent field) stays within its stated relative error
+    of 2.2e-7 over a in [-125, 9], evaluated step by step as the kernel does."""
+    coef = _poly_coefficients()
+    assert len(coef) == 6
+    g = np.random.default_rng(5)
+    a = np.concatenate([
+        g.uniform(-125.0, 9.0, 3_000_000),
+        g.uniform(-1.0, 1.0, 1_000_000),
+        np.arange(-125, 10, dtype=np.float64) + 0.5,      # f = +-0.5 ties
+        np.arange(-125, 10, dtype=np.float64),
+    ]).astype(np.float32)
+    a = np.maximum(a, np.float32(-125.0))
+    bias = np.float32(12582912.0)
+    t = (a + bias).astype(np.float32)
+    n = (t - bias).astype(np.float32)
+    f = _fma32(n, np.full_like(n, -1.0), a)
+    p = np.full_like(f, coef[0])
+    for c in coef[1:]:
+        p = _fma32(p, f, np.full_like(f, c))
+    e = (p.view(np.int32).astype(np.int64) + (t.view(np.int32).astype(np.int64) << 23)) & 0xFFFFFFFF
+    e = e.astype(np.uint32).view(np.float32).astype(np.float64)
+    exact = np.exp2(a.astype(np.float64))
+    rel = np.abs(e - exact) / exact
+    assert rel.max() <= 2.2e-7, rel.max()
