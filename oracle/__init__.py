@@ -65,6 +65,8 @@ def lib():
         L.or_attn_exact_head.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_double, ctypes.c_int, _i32p,
                                          ctypes.c_int, _f64p]
+        L.or_decode_quant_q_row.restype = None
+        L.or_decode_quant_q_row.argtypes = [_u16p, ctypes.c_int, _u8p, _f32p]
         L.or_decode_seq.restype = None
         L.or_decode_seq.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -309,3 +311,18 @@ def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, 
 
     _pool_map(one, list(range(B)), threads)
     return (out, o64) if want_f64 else out
+
+
+def decode_quant_q(q):
+    """The decode's query quantisation: every (b, t, h) row rotated and cast
+    to e4m3 with scale max|q_hat| / 448. q: uint16 [B, T, H, D] ->
+    (codes uint8 [B, T, H, D], scales float32 [B, T, H])."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    B, T, H, D = q.shape
+    rows = q.reshape(-1, D)
+    codes = np.zeros(rows.shape, dtype=np.uint8)
+    scales = np.zeros((rows.shape[0],), dtype=np.float32)
+    f = lib().or_decode_quant_q_row
+    for i in range(rows.shape[0]):
+        f(_p(rows[i], _u16p), D, _p(codes[i], _u8p), _p(scales[i:i + 1], _f32p))
+    return codes.reshape(B, T, H, D), scales.reshape(B, T, H)

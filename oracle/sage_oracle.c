@@ -415,11 +415,32 @@ void or_attn_exact_head(const uint16_t* q, const uint16_t* k, const uint16_t* v,
  *   PV on bf16 operands ([PA], Changes: PV_BF16): w_j = bf16(fp32(p_j) *
  *   vsc_j), exact bf16 of dec(v8_j); out = sum_j w_j dec(v8_j) / sum_j p_j.
  * out[T][H][D] bf16. */
+/* The query side of the decode, one (token, head) row: q_hat = fwht(q)
+ * (fp32); a = max |q_hat|; s = a/448, r = 448/a (IEEE fp32 divides);
+ * codes[e] = e4m3(fp32(q_hat[e] * r)) ([PA] Changes: Q quantised to the FP8
+ * format of the cache, FP8_MAX 448); a == 0 -> s = 0 and codes 0. */
+void or_decode_quant_q_row(const uint16_t* q, int D, uint8_t* codes, float* scale)
+{
+    float* qh = (float*)malloc(sizeof(float) * (size_t)D);
+    for (int e = 0; e < D; ++e) qh[e] = or_bf16_to_f32(q[e]);
+    or_fwht_f32(qh, D);
+    float a = 0.0f;
+    for (int e = 0; e < D; ++e) if (fabsf(qh[e]) > a) a = fabsf(qh[e]);
+    float s = 0.0f, r = 0.0f;
+    if (a != 0.0f) { s = a / 448.0f; r = 448.0f / a; }
+    for (int e = 0; e < D; ++e) {
+        float y = qh[e] * r;
+        codes[e] = (a != 0.0f) ? or_e4m3_encode((double)y) : 0;
+    }
+    *scale = s;
+    free(qh);
+}
+
 void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
                    const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
                    int page, int window, double softmax_scale, uint16_t* out, double* out_f64)
 {
-    float* qh = (float*)malloc(sizeof(float) * (size_t)D);
+    uint8_t* qc = (uint8_t*)malloc((size_t)D);
     double* q8 = (double*)malloc(sizeof(double) * (size_t)D);
     double* o = (double*)malloc(sizeof(double) * (size_t)D);
     double* sv = (double*)malloc(sizeof(double) * (size_t)(window > 0 ? window : 1));
@@ -428,16 +449,9 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
         for (int h = 0; h < H; ++h) {
             const int hk = h / group;
             const uint16_t* qr = q + ((int64_t)t * H + h) * D;
-            for (int e = 0; e < D; ++e) qh[e] = or_bf16_to_f32(qr[e]);
-            or_fwht_f32(qh, D);
-            float a = 0.0f;
-            for (int e = 0; e < D; ++e) if (fabsf(qh[e]) > a) a = fabsf(qh[e]);
-            float s = 0.0f, r = 0.0f;
-            if (a != 0.0f) { s = a / 448.0f; r = 448.0f / a; }
-            for (int e = 0; e < D; ++e) {
-                float y = qh[e] * r;
-                q8[e] = (a != 0.0f) ? or_e4m3_decode(or_e4m3_encode((double)y)) : 0.0;
-            }
+            float s = 0.0f;
+            or_decode_quant_q_row(qr, D, qc, &s);
+            for (int e = 0; e < D; ++e) q8[e] = or_e4m3_decode(qc[e]);
             const int p = ctx - T + t;
             int lo = p - window + 1;
             if (lo < 0) lo = 0;
@@ -475,5 +489,5 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
     free(sv);
     free(o);
     free(q8);
-    free(qh);
+    free(qc);
 }

@@ -156,3 +156,56 @@ def test_method_accuracy_gate_outliers_and_planted_mistake(oracle_mod):
                               False, rows=rows)
     bad = _cosine(oracle_mod.bf16_to_f32(bad_out), exact)
     assert bad < good and bad < 0.998
+
+
+def _numpy_softmax_attention(q, k, v, scale, causal, rows):
+    """Plain fp64 softmax(q k^T * scale) v with numpy, written independently
+    of the oracle: the reference every accuracy gate is taken against. The
+    causal mask is the bottom-right aligned one (key j visible to query i iff
+    j <= i + Lk - Lq); a row that sees no key is zero."""
+    B, H, Lq, D = q.shape
+    Hk, Lk = k.shape[1], k.shape[2]
+    qf = q.astype(np.float64)
+    kf = k.astype(np.float64)
+    vf = v.astype(np.float64)
+    out = np.zeros((B, H, len(rows), D))
+    for b in range(B):
+        for h in range(H):
+            hk = h // (H // Hk)
+            s = qf[b, h, rows] @ kf[b, hk].T * scale          # [n, Lk]
+            if causal:
+                vis = np.arange(Lk)[None, :] <= rows[:, None] + (Lk - Lq)
+                s = np.where(vis, s, -np.inf)
+            for n in range(len(rows)):
+                if not np.isfinite(s[n]).any():
+                    continue
+                w = np.exp(s[n] - s[n].max())
+                out[b, h, n] = (w / w.sum()) @ vf[b, hk]
+    return out
+
+
+@pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,causal,rows", [
+    (1, 2, 2, 37, 37, 64, False, None),          # non-causal
+    (1, 2, 2, 45, 45, 64, True, None),           # causal, Lq == Lk
+    (2, 2, 1, 19, 60, 128, True, None),          # causal, Lq < Lk (bottom-right), GQA
+    (1, 4, 2, 70, 23, 64, True, None),           # causal, Lq > Lk: leading rows see nothing
+    (1, 6, 2, 50, 50, 64, False, None),          # GQA, group 3
+    (1, 2, 2, 200, 180, 64, True, [0, 1, 19, 20, 21, 150, 199]),   # rows= subset
+])
+def test_exact_reference_equals_numpy_softmax(oracle_mod, B, H, Hk, Lq, Lk, D, causal, rows):
+    """or_attn_exact_head (the unquantised fp64 reference behind every
+    cosine >= 0.998 gate) against numpy: a wrong mask offset, a scale applied
+    twice or a wrong GQA head map would each fail here."""
+    g = torch.Generator().manual_seed(B * 1000 + Lq * 7 + Lk + H)
+    q = (torch.randn((B, H, Lq, D), generator=g) * 1.5).to(torch.bfloat16)
+    k = (torch.randn((B, Hk, Lk, D), generator=g) + 0.5).to(torch.bfloat16)
+    v = torch.randn((B, Hk, Lk, D), generator=g).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(D)
+    r = np.arange(Lq, dtype=np.int32) if rows is None else np.array(rows, dtype=np.int32)
+    got = oracle_mod.attn_exact(_bits(q), _bits(k), _bits(v), scale, causal, rows=r)
+    ref = _numpy_softmax_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                   scale, causal, r)
+    assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    if causal and Lq > Lk:
+        n_dark = Lq - Lk
+        assert (got[:, :, r < n_dark] == 0).all()

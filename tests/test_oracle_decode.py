@@ -105,3 +105,29 @@ def test_decode_matches_brute_force(oracle_mod, B, T, H, Hk, D, page, lo, hi, wi
     ref = _brute_decode(oracle_mod, d, window, scale)
     assert np.abs(o64 - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
     assert np.array_equal(out, oracle_mod.f64_to_bf16(o64))
+
+
+def test_decode_query_codes_match_torch_float8(oracle_mod):
+    """The decode's query quantisation (rotation by the butterfly, scale
+    max|q_hat| / 448, e4m3 codes) against scipy's Hadamard matrix and torch's
+    float8 cast, code for code; an all-zero row gives scale 0 and +0 codes."""
+    g = torch.Generator().manual_seed(11)
+    for D in (64, 128):
+        q = torch.randn((2, 3, 5, D), generator=g).to(torch.bfloat16)
+        q[1, 2, 4] = 0.0
+        codes, scales = oracle_mod.decode_quant_q(workloads.bits_u16(q))
+        Hmat = scipy.linalg.hadamard(D).astype(np.float64)
+        qf = q.float().numpy()
+        for idx in np.ndindex(q.shape[:3]):
+            qh = oracle_mod.fwht_f32(qf[idx][None, :])[0]
+            assert np.abs(qh - qf[idx] @ Hmat).max() <= 1e-4 * max(1e-30, np.abs(qf[idx]).sum())
+            a = np.float32(np.abs(qh).max())
+            if a == 0:
+                assert scales[idx] == 0 and (codes[idx] == 0).all()
+                continue
+            assert scales[idx] == np.float32(a / np.float32(448.0))
+            r = np.float32(448.0) / a
+            ref = torch.from_numpy((qh * r).astype(np.float32)).to(torch.float8_e4m3fn)
+            assert np.array_equal(codes[idx], ref.view(torch.uint8).numpy())
+            # the largest magnitude lands on 448 (code 0x7E, either sign)
+            assert ((codes[idx] & 0x7F) == 0x7E).any()
