@@ -4,15 +4,22 @@
 One step = the whole hot path on one batch of seeded synthetic inputs that
 already sit in HBM: sage_quant_qkv (K mean, smoothing, Hadamard rotation, INT8
 Q/K, e4m3 V; two launches) + sage_attn_fwd (INT8 QK^T, online softmax, e4m3
-PV, bf16 out). Workload: non-causal video-DiT prefill B=1 H=24 L=4096 D=128
-(Q blocks 128 tokens, K blocks 64). Metric: TOPS = 4 B H L^2 D / step time.
+PV, bf16 out). Default workload: the long non-causal video-DiT attention
+B=1 H=40 L=32760 D=128 (Q blocks 128 tokens, K blocks 64), the largest of the
+single-GPU workloads. Metric: TOPS = 4 B H L^2 D / step time (halved for
+causal). The line also carries the B1 H24 L4096 and the causal B2 H32 L8192
+workloads under "configs", each with its attention roofline and its
+quantisation bandwidth, and the paged FP8 decode under "decode".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sage|reference]
+                    [--workload c2|c3|c4]
 
-N > 1 runs under torchrun: every rank runs its own replica of the workload
-(the path has no exchange step), timing is the max over ranks, and `value`
-counts the work of all ranks. `--impl reference` times the CPU oracle on the
-host cores on a bounded sample of the same workload (rank 0 only).
+N > 1 runs under torchrun: the workload's kv heads (with their query heads)
+are split into N contiguous ranges, one per rank (the heads are independent,
+so no data crosses ranks); timing is the max over ranks and `value` counts
+the whole workload ("scaling": "strong"). `--impl reference` times the CPU
+oracle on the host cores on a bounded sample of the same workload (rank 0
+only).
 """
 import argparse
 import json
@@ -31,21 +38,22 @@ METRIC = "quantized-attn TOPS (4*B*H*L^2*D/t) and % of B200 INT8/FP8 tensor peak
 UNIT = "TOPS"
 INT8_OVER_BF16 = 2.0        # nominal dense INT8/FP8 : BF16 tensor ratio (4.5 : 2.25 PFLOP/s)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126e6
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sage", choices=["sage", "reference"])
-    ap.add_argument("--workload", default="c2", choices=["c1", "c2", "c3", "c4"])
-    ap.add_argument("--sets", type=int, default=4, help="rotating input sets (L2 defeat)")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--workload", default="c4", choices=["c1", "c2", "c3", "c4"])
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other prefill workloads")
     ap.add_argument("--fused-q", action="store_true",
                     help="rotate and quantise Q inside the attention kernel (sage_attn_fwd_q16)")
     ap.add_argument("--decode-only", action="store_true",
@@ -62,12 +70,12 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def attn_traffic():
-    """DRAM bytes per attn_fwd launch from the committed ncu summary, if the
-    kernel source is unchanged since the capture (else None)."""
+def attn_traffic(workload):
+    """DRAM bytes per attn_fwd launch on `workload` from the committed ncu
+    summary, if the kernel source is unchanged since the capture (else None)."""
     import hashlib
     import re
-    prof = os.path.join(ROOT, "profiles", "attn_fwd_dit_prefill_b1_h24_l4096_d128.md")
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_%s.md" % workload)
     if not os.path.exists(prof):
         return None
     text = open(prof).read()
@@ -101,10 +109,30 @@ def rank_max(x, world, device):
     return float(t.item())
 
 
-def job_value(ops_per_step, steps, world, elapsed_ms):
-    """Whole-job TOPS: each of `world` ranks runs its own replica of the
-    workload (`ops_per_step` per step), timed as the slowest rank."""
-    return world * ops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+def job_value(ops_per_step, steps, elapsed_ms):
+    """Whole-job TOPS: `ops_per_step` (the work of all ranks together) per
+    step, `steps` steps in `elapsed_ms` (the slowest rank's time)."""
+    return ops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
+def kv_head_range(Hk, world, rank):
+    """The contiguous kv heads [lo, hi) of `rank` when the Hk kv heads are
+    split over `world` ranks as evenly as possible (each rank also takes the
+    query heads that share those kv heads)."""
+    if world > Hk:
+        raise ValueError("cannot split %d kv heads over %d ranks" % (Hk, world))
+    return Hk * rank // world, Hk * (rank + 1) // world
+
+
+def shard_heads(cfg, q, k, v, world, rank):
+    """This rank's part of a prefill workload: its kv-head range and their
+    query heads (views, no copy)."""
+    if world == 1:
+        return cfg, q, k, v
+    group = cfg["H"] // cfg["Hk"]
+    lo, hi = kv_head_range(cfg["Hk"], world, rank)
+    return (dict(cfg, H=(hi - lo) * group, Hk=hi - lo), q[:, lo * group:hi * group], k[:, lo:hi],
+            v[:, lo:hi])
 
 
 def work_ops(cfg):
@@ -173,41 +201,64 @@ class ClockSampler:
 
 
 def cpu_baseline(cfg, seconds):
-    """The oracle as it stands, on the host cores (one head per thread), on
-    whole heads of the same workload, sized to about `seconds` of wall time."""
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    workload: the quantisation of every token of a set of heads (one head per
+    thread) and the attention of a seeded set of query rows of each, the
+    number of rows sized to about `seconds` of wall time. The two parts are
+    timed apart and scaled to the whole workload (quantisation by heads,
+    attention by heads and by the keys the sampled rows see), and the value
+    is the workload's ops over that whole-workload time."""
+    import numpy as np
+
     import oracle
     import workloads
 
     cores = os.cpu_count() or 1
     _, q, k, v = workloads.make_prefill_config(cfg["key"])
     b = workloads.bits_u16
-    qb, kb, vb = b(q), b(k), b(v)
-    L = cfg["L"]
-
-    def run(heads):
-        t = time.perf_counter()
-        qk = oracle.quant_qk(qb[:, :heads], kb[:, :heads], cfg["blk_q"], cfg["blk_k"], threads=cores)
-        v8t, vs = oracle.quant_v(vb[:, :heads], threads=cores)
-        oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, L, L, cfg["blk_q"],
-                    cfg["blk_k"], cfg["softmax_scale"], cfg["causal"], threads=cores)
-        return time.perf_counter() - t
-
     heads = min(cfg["H"], cores)
-    t1 = run(heads)                     # one wave: every core busy with one head
-    waves = max(1, int(seconds / max(t1, 1e-3)))
-    if waves > 1 and heads < cfg["H"]:
-        heads = min(cfg["H"], heads * waves)
-        t1 = run(heads)
-    ops = work_ops(dict(cfg, H=heads, B=1))
-    return {"value": ops / t1 / 1e12, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
-            "sample": "B=1, %d of %d heads, all %d query rows (quantise Q/K/V + attention), "
-                      "%.1f s on %d threads" % (heads, cfg["H"], L, t1, min(cores, heads))}
+    qb, kb, vb = b(q)[:1, :heads], b(k)[:1, :heads], b(v)[:1, :heads]
+    L = cfg["L"]
+    rng = np.random.default_rng(cfg["H"] * 7 + L)
+
+    t = time.perf_counter()
+    qk = oracle.quant_qk(qb, kb, cfg["blk_q"], cfg["blk_k"], threads=cores)
+    v8t, vs = oracle.quant_v(vb, threads=cores)
+    t_quant = time.perf_counter() - t
+
+    def keys_seen(rows):
+        return float(np.sum(np.minimum(rows + 1, L))) if cfg["causal"] else float(len(rows)) * L
+
+    def run(nrows):
+        rows = np.sort(rng.choice(L, size=nrows, replace=False)).astype(np.int32)
+        t = time.perf_counter()
+        oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, L, L, cfg["blk_q"],
+                    cfg["blk_k"], cfg["softmax_scale"], cfg["causal"], rows=rows, threads=cores)
+        return time.perf_counter() - t, rows
+
+    nrows = min(L, 16)
+    t_attn, rows = run(nrows)
+    budget = max(0.0, seconds - t_quant)
+    if nrows < L and t_attn < budget / 4:
+        nrows = int(min(L, max(nrows, nrows * budget / max(t_attn, 1e-3))))
+        t_attn, rows = run(nrows)
+    all_keys = float(L) * (L + 1) / 2 if cfg["causal"] else float(L) * L
+    # whole workload on the same threads: the heads in waves of `heads`, each
+    # wave's quantisation as measured, its attention scaled by keys
+    waves = cfg["B"] * cfg["H"] / float(heads)
+    t_whole = waves * (t_quant + t_attn * all_keys / keys_seen(rows))
+    value = work_ops(cfg) / t_whole / 1e12
+    return {"value": value, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": "B=1, %d of %d heads, one per thread: quantise every token of Q/K/V "
+                      "(%.1f s), attention of %d seeded query rows of %d (%.1f s); scaled to the "
+                      "whole workload (%d x %d heads): %.0f s"
+                      % (heads, cfg["H"], t_quant, nrows, L, t_attn, cfg["B"], cfg["H"], t_whole)}
 
 
 def bench_decode(sage, torch, stream, copies=8, reps=50):
     """Paged FP8 decode on the MTP4 / GQA16 / window-4096 workload: one call
-    = split kernel + merge kernel; `copies` cache copies rotate so the
-    working set exceeds L2; calls are captured in a CUDA graph and replayed."""
+    = one kernel launch; `copies` cache copies rotate so the working set
+    exceeds L2; calls are captured in a CUDA graph and replayed."""
     import workloads
     cfg, d = workloads.make_decode_config("c5")
     B, T, H, D = d["q"].shape
@@ -218,7 +269,7 @@ def bench_decode(sage, torch, stream, copies=8, reps=50):
     caches = [[d[x].cuda() for x in ("k_cache", "v_cache", "k_scale", "v_scale")]
               for _ in range(copies)]
     out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"]),),
+    ws = torch.empty((max(16, sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"])),),
                      dtype=torch.uint8, device="cuda")
 
     def call(i):
@@ -264,9 +315,132 @@ def bench_decode(sage, torch, stream, copies=8, reps=50):
             "us_per_call_p10_p50_p90": [pct(times, 10) * 1e3, pct(times, 50) * 1e3, pct(times, 90) * 1e3],
             "algorithmic_bytes": algo,
             "achieved": gbs, "unit": "GB/s", "peak": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
-            "peak_source": pk_src + " copy bandwidth", "launches_per_call": 1,
+            "peak_source": pk_src + " copy bandwidth (burst)", "launches_per_call": 1,
             "timing": "median of 5 replays of a CUDA graph of %d calls over %d rotating cache copies"
                       % (reps, copies)}
+
+
+class Prefill:
+    """Device-resident input sets of one prefill workload (this rank's heads)
+    and the timed loops over them."""
+
+    def __init__(self, sage, torch, cfg, q, k, v, fused_q=False):
+        self.sage, self.torch, self.cfg, self.fused_q = sage, torch, cfg, fused_q
+        B, H, Hk, L, D = cfg["B"], cfg["H"], cfg["Hk"], cfg["L"], cfg["D"]
+        self.h = sage.Hadamard(D)
+        self.q_cpu, self.k_cpu, self.v_cpu = q, k, v
+        in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+        self.set_bytes = in_bytes + 2 * q.numel() * 2
+        # rotate enough input sets that consecutive steps never find their
+        # inputs in the 126 MB L2
+        n_sets = max(2, int(math.ceil(2 * L2_BYTES / max(self.set_bytes, 1))))
+        self.sets = []
+        for _ in range(n_sets):
+            qs, ks, vs_ = q.cuda(), k.cuda(), v.cuda()          # [B,H,L,D] views of [B,L,H,D]
+            bufs = sage.QuantBuffers(B, H, Hk, L, L, D, cfg["blk_q"], cfg["blk_k"])
+            out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
+            self.sets.append((qs, ks, vs_, bufs, out))
+
+    def quantise(self, i, stream):
+        qs, ks, vs_, bufs, _ = self.sets[i % len(self.sets)]
+        c = self.cfg
+        self.sage.quantise(self.h, None if self.fused_q else qs, ks, vs_, c["blk_q"], c["blk_k"],
+                           bufs, stream)
+
+    def attention(self, i, stream):
+        qs, _, _, bufs, out = self.sets[i % len(self.sets)]
+        c = self.cfg
+        if self.fused_q:
+            self.sage.sage_attn_fwd_q16(self.h, qs, c["blk_q"], bufs.k8, bufs.k_scale, bufs.v8_t,
+                                        bufs.v_scale, c["Hk"], c["L"], c["blk_k"], c["softmax_scale"],
+                                        c["causal"], out, None, stream)
+        else:
+            self.sage.sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t,
+                                    bufs.v_scale, c["B"], c["H"], c["Hk"], c["L"], c["L"], c["D"],
+                                    c["blk_q"], c["blk_k"], c["softmax_scale"], c["causal"], out,
+                                    None, stream)
+
+    def timed_steps(self, steps, warmup, stream, barrier, clocks=None):
+        """Whole steps (quantise + attention): total elapsed ms and the
+        per-step attention launch times (ms), CUDA events on `stream`."""
+        torch = self.torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(warmup):
+            self.quantise(i, stream)
+            self.attention(i, stream)
+        torch.cuda.synchronize()
+        if self.sage.sage_device_error(stream) != self.sage.SAGE_OK:
+            raise RuntimeError("device error during warm-up")
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        cm = clocks if clocks is not None else _NullCtx()
+        with cm:
+            barrier()
+            torch.cuda.synchronize()
+            t0.record(stream)
+            for i in range(steps):
+                self.quantise(i, stream)
+                ev[i][0].record(stream)
+                self.attention(i, stream)
+                ev[i][1].record(stream)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        if self.sage.sage_device_error(stream) != self.sage.SAGE_OK:
+            raise RuntimeError("device error during the timed steps")
+        return t0.elapsed_time(t1), sorted(a.elapsed_time(b) for a, b in ev)
+
+    def timed_quant(self, steps, warmup, stream):
+        """The quantisation call alone (its launches), microseconds per call."""
+        torch = self.torch
+        qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for i in range(warmup):
+            self.quantise(i, stream)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            qev[i][0].record(stream)
+            self.quantise(i, stream)
+            qev[i][1].record(stream)
+        torch.cuda.synchronize()
+        if self.sage.sage_device_error(stream) != self.sage.SAGE_OK:
+            raise RuntimeError("device error while timing the quantisation")
+        return sorted(a.elapsed_time(b) * 1e3 for a, b in qev)
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def quant_object(pf, q_times, pk, pk_src):
+    q_us = statistics.median(q_times)
+    q_bytes = 3 * ((0 if pf.fused_q else pf.q_cpu.numel()) + pf.k_cpu.numel() + pf.v_cpu.numel())
+    gbs = q_bytes / (q_us * 1e-6) / 1e9
+    return {"us_per_call": q_us,
+            "us_p10_p50_p90": [pct(q_times, 10), pct(q_times, 50), pct(q_times, 90)],
+            "algorithmic_bytes": q_bytes, "achieved": gbs, "unit": "GB/s",
+            "peak": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
+            "peak_source": pk_src + " copy bandwidth (burst)",
+            "bytes_rule": "2 B read + 1 B written per element of each quantised tensor; the "
+                          "statistics pass re-reads K and V (not counted)",
+            "launches_per_call": 4 if pf.fused_q else 2}
+
+
+def roofline_object(ops, attn_times, pk, pk_src, traffic):
+    peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
+    attn_ms = statistics.mean(attn_times)
+    achieved = ops / (attn_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved, "peak": peak_tops,
+            "unit": "TFLOP/s", "frac": achieved / peak_tops, "traffic": traffic,
+            "peak_source": "%s bf16 burst x %.0f (INT8/FP8 : BF16 nominal)" % (pk_src, INT8_OVER_BF16),
+            "frac_of_sustained": achieved / (pk["bf16_tflops_sustained"] * INT8_OVER_BF16),
+            "attn_ms": attn_ms,
+            "attn_ms_p10_p50_p90": [pct(attn_times, 10), pct(attn_times, 50), pct(attn_times, 90)]}
 
 
 def run_reference(args):
@@ -288,13 +462,84 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": len(vals), "warmup": 0,
         "ms_per_step": work_ops(dict(cfg)) / (value * 1e12) * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "int8+e4m3",
         "data": "synthetic", "config": {"workload": cfg["name"], "B": cfg["B"], "H": cfg["H"],
                                         "L": cfg["L"], "D": cfg["D"]},
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+
+
+def measure_e2e(sage, torch, pf, steps, stream, barrier, max_over_ranks, ops_all):
+    """End to end through the public API: pinned host inputs -> device ->
+    quantise + attention -> result back to pinned host memory, every step.
+    Steps are pipelined over two device buffer pairs and three streams
+    (host->device copies, compute, device->host copies): the inputs of step
+    i + 1 travel while step i computes and step i - 1's result comes back."""
+    c = pf.cfg
+    B, H, L, D = c["B"], c["H"], c["L"], c["D"]
+    q, k, v = pf.q_cpu, pf.k_cpu, pf.v_cpu
+    qh = q.permute(0, 2, 1, 3).contiguous().pin_memory()      # [B, L, H, D] host buffers
+    kh = k.permute(0, 2, 1, 3).contiguous().pin_memory()
+    vh = v.permute(0, 2, 1, 3).contiguous().pin_memory()
+    oh = [torch.empty((B, L, H, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dev_in = [[torch.empty_like(x, device="cuda") for x in (qh, kh, vh)] for _ in range(2)]
+    dev_out = [torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    ebufs = pf.sets[0][3]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    n_e2e = steps + 2
+    ev_in = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_comp = [torch.cuda.Event() for _ in range(n_e2e)]
+    ev_out = [torch.cuda.Event() for _ in range(n_e2e)]
+
+    def e2e_step(i):
+        j = i % 2
+        qd, kd, vd = dev_in[j]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[i - 2])        # step i - 2 has read these inputs
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            ev_in[i].record(s_in)
+        stream.wait_event(ev_in[i])
+        if i >= 2:
+            stream.wait_event(ev_out[i - 2])           # step i - 2's result has left dev_out[j]
+        sage.sage_attention(pf.h, qd.permute(0, 2, 1, 3), kd.permute(0, 2, 1, 3),
+                            vd.permute(0, 2, 1, 3), c["blk_q"], c["blk_k"], c["softmax_scale"],
+                            c["causal"], out=dev_out[j].permute(0, 2, 1, 3), bufs=ebufs,
+                            stream=stream)
+        ev_comp[i].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[i])
+            oh[j].copy_(dev_out[j], non_blocking=True)
+            ev_out[i].record(s_out)
+
+    for i in range(2):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(steps):
+        e2e_step(i)
+    stream.wait_event(ev_out[steps - 1])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    if sage.sage_device_error(stream) != sage.SAGE_OK:
+        raise RuntimeError("device error during the end-to-end steps")
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    return {"value": job_value(ops_all, steps, e2e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
+            "d2h_bytes_per_step": oh[0].numel() * oh[0].element_size(),
+            "ms_per_step": e2e_ms / steps,
+            "pipeline": "h2d, compute and d2h on three streams over two buffer pairs"}
 
 
 def run_sage(args):
@@ -320,188 +565,72 @@ def run_sage(args):
     def max_over_ranks(x):
         return rank_max(x, world, "cuda")
 
-    cfg = dict(workloads.PREFILL[args.workload], key=args.workload)
-    B, H, Hk, L, D = cfg["B"], cfg["H"], cfg["Hk"], cfg["L"], cfg["D"]
-    blk_q, blk_k, scale, causal = cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"], cfg["causal"]
-    _, q, k, v = workloads.make_prefill_config(args.workload)
-
-    h = sage.Hadamard(D)
-    stream = torch.cuda.current_stream()
-    sets = []
-    for _ in range(args.sets):
-        qs, ks, vs_ = q.cuda(), k.cuda(), v.cuda()          # [B,H,L,D] views of [B,L,H,D]
-        bufs = sage.QuantBuffers(B, H, Hk, L, L, D, blk_q, blk_k)
-        out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
-        sets.append((qs, ks, vs_, bufs, out))
-    set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + 2 * q.numel() * 2
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-
-    def step(i, timed):
-        qs, ks, vs_, bufs, out = sets[i % len(sets)]
-        # sage_quant_qkv on `stream` (with --fused-q: K on `stream`, V beside
-        # it on a second stream), then the attention
-        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
-        if timed:
-            ev[i][0].record(stream)
-        if args.fused_q:
-            sage.sage_attn_fwd_q16(h, qs, blk_q, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
-                                   Hk, L, blk_k, scale, causal, out, None, stream)
-        else:
-            sage.sage_attn_fwd(bufs.q8, bufs.q_scale, bufs.k8, bufs.k_scale, bufs.v8_t, bufs.v_scale,
-                               B, H, Hk, L, L, D, blk_q, blk_k, scale, causal, out, None, stream)
-        if timed:
-            ev[i][1].record(stream)
-
-    for i in range(args.warmup):
-        step(i, False)
-    torch.cuda.synchronize()
-    if sage.sage_device_error(stream) != sage.SAGE_OK:
-        raise RuntimeError("device error during warm-up")
-
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local, enabled=not args.no_clocks) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i, True)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    if sage.sage_device_error(stream) != sage.SAGE_OK:
-        raise RuntimeError("device error during the timed steps")
-    elapsed_ms = max_over_ranks(t0.elapsed_time(t1))
-    attn_times = sorted(a.elapsed_time(b) for a, b in ev)
-    attn_ms = statistics.mean(attn_times)
-    ops = work_ops(cfg)
-    value = job_value(ops, args.steps, world, elapsed_ms)
-
     pk, pk_src = peaks()
-    peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
-    achieved = ops / (attn_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "attn_fwd", "achieved": achieved, "peak": peak_tops,
-                "unit": "TFLOP/s", "frac": achieved / peak_tops, "traffic": attn_traffic(),
-                "peak_source": "%s bf16 burst x %.0f (INT8/FP8 : BF16 nominal)" % (pk_src, INT8_OVER_BF16),
-                "frac_of_sustained": achieved / (pk["bf16_tflops_sustained"] * INT8_OVER_BF16),
-                "attn_ms": attn_ms,
-                "attn_ms_p10_p50_p90": [pct(attn_times, 10), pct(attn_times, 50), pct(attn_times, 90)]}
+    stream = torch.cuda.current_stream()
+    full_cfg = dict(workloads.PREFILL[args.workload], key=args.workload)
+    _, q, k, v = workloads.make_prefill_config(args.workload)
+    cfg, q, k, v = shard_heads(full_cfg, q, k, v, world, rank)
+    ops_all = work_ops(full_cfg)                 # the whole workload, all ranks together
+    pf = Prefill(sage, torch, cfg, q, k, v, fused_q=args.fused_q)
 
-    # end to end through the public API: pinned host inputs -> device ->
-    # quantise + attention -> result back to pinned host memory, every step.
-    # Steps are pipelined over two device buffer pairs and three streams
-    # (host->device copies, compute, device->host copies): the inputs of step
-    # i + 1 travel while step i computes and step i - 1's result comes back.
-    qh = q.permute(0, 2, 1, 3).contiguous().pin_memory()      # [B, L, H, D] host buffers
-    kh = k.permute(0, 2, 1, 3).contiguous().pin_memory()
-    vh = v.permute(0, 2, 1, 3).contiguous().pin_memory()
-    oh = [torch.empty((B, L, H, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    dev_in = [[torch.empty_like(x, device="cuda") for x in (qh, kh, vh)] for _ in range(2)]
-    dev_out = [torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    ebufs = sets[0][3]
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    n_e2e = args.e2e_steps + 2
-    ev_in = [torch.cuda.Event() for _ in range(n_e2e)]
-    ev_comp = [torch.cuda.Event() for _ in range(n_e2e)]
-    ev_out = [torch.cuda.Event() for _ in range(n_e2e)]
+    clk = ClockSampler(local, enabled=not args.no_clocks)
+    elapsed_local, attn_times = pf.timed_steps(args.steps, args.warmup, stream, barrier, clocks=clk)
+    elapsed_ms = max_over_ranks(elapsed_local)
+    value = job_value(ops_all, args.steps, elapsed_ms)
+    roofline = roofline_object(work_ops(cfg), attn_times, pk, pk_src,
+                               attn_traffic(cfg["name"]) if world == 1 else None)
+    e2e = measure_e2e(sage, torch, pf, args.e2e_steps, stream, barrier, max_over_ranks, ops_all)
+    quant = quant_object(pf, pf.timed_quant(args.steps, args.warmup, stream), pk, pk_src)
+    set_desc = "%d rotating input sets of %.0f MB (> 126 MB L2 between uses)" % (len(pf.sets),
+                                                                                  pf.set_bytes / 1e6)
+    del pf
+    torch.cuda.empty_cache()
 
-    def e2e_step(i):
-        j = i % 2
-        qd, kd, vd = dev_in[j]
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(ev_comp[i - 2])        # step i - 2 has read these inputs
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            ev_in[i].record(s_in)
-        stream.wait_event(ev_in[i])
-        if i >= 2:
-            stream.wait_event(ev_out[i - 2])           # step i - 2's result has left dev_out[j]
-        sage.sage_attention(h, qd.permute(0, 2, 1, 3), kd.permute(0, 2, 1, 3),
-                            vd.permute(0, 2, 1, 3), blk_q, blk_k, scale, causal,
-                            out=dev_out[j].permute(0, 2, 1, 3), bufs=ebufs, stream=stream)
-        ev_comp[i].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_comp[i])
-            oh[j].copy_(dev_out[j], non_blocking=True)
-            ev_out[i].record(s_out)
-
-    for i in range(2):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
-    for i in range(args.e2e_steps):
-        e2e_step(i)
-    stream.wait_event(ev_out[args.e2e_steps - 1])
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e = {"value": job_value(ops, args.e2e_steps, world, e2e_ms), "unit": UNIT,
-           "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in (qh, kh, vh)),
-           "d2h_bytes_per_step": oh[0].numel() * oh[0].element_size(),
-           "ms_per_step": e2e_ms / args.e2e_steps,
-           "pipeline": "h2d, compute and d2h on three streams over two buffer pairs"}
-
-    # the quantisation alone (both launches of sage_quant_qkv, or sage_quant_k
-    # + sage_quant_v with --fused-q), over the same rotating input sets
-    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.warmup):
-        qs, ks, vs_, bufs, _ = sets[i % len(sets)]
-        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        qs, ks, vs_, bufs, _ = sets[i % len(sets)]
-        qev[i][0].record(stream)
-        sage.quantise(h, None if args.fused_q else qs, ks, vs_, blk_q, blk_k, bufs, stream)
-        qev[i][1].record(stream)
-    torch.cuda.synchronize()
-    if sage.sage_device_error(stream) != sage.SAGE_OK:
-        raise RuntimeError("device error while timing the quantisation")
-    q_times = sorted(a.elapsed_time(b) * 1e3 for a, b in qev)
-    q_us = statistics.median(q_times)
-    q_bytes = 3 * ((0 if args.fused_q else q.numel()) + k.numel() + v.numel())
-    quant = {"us_per_call": q_us,
-             "us_p10_p50_p90": [pct(q_times, 10), pct(q_times, 50), pct(q_times, 90)],
-             "algorithmic_bytes": q_bytes,
-             "achieved": q_bytes / (q_us * 1e-6) / 1e9, "unit": "GB/s",
-             "peak": pk["hbm_gbs"], "frac": q_bytes / (q_us * 1e-6) / 1e9 / pk["hbm_gbs"],
-             "peak_source": pk_src + " copy bandwidth",
-             "bytes_rule": "2 B read + 1 B written per element of each quantised tensor; the "
-                           "statistics pass re-reads K and V (not counted)",
-             "launches_per_call": 4 if args.fused_q else 2}
+    # the other prefill workloads (one GPU only): each with its own step
+    # throughput, attention roofline and quantisation bandwidth
+    extra = {}
+    if world == 1 and not args.no_extra:
+        for key in ("c2", "c3", "c4"):
+            if key == args.workload:
+                continue
+            ecfg = dict(workloads.PREFILL[key], key=key)
+            _, eq, ek, ev_ = workloads.make_prefill_config(key)
+            epf = Prefill(sage, torch, ecfg, eq, ek, ev_, fused_q=args.fused_q)
+            esteps = max(args.steps, 20)
+            el, at = epf.timed_steps(esteps, max(args.warmup, 3), stream, barrier)
+            eops = work_ops(ecfg)
+            extra[key] = {
+                "workload": ecfg["name"], "causal": ecfg["causal"],
+                "value": job_value(eops, esteps, el), "unit": UNIT, "ms_per_step": el / esteps,
+                "steps": esteps,
+                "roofline": roofline_object(eops, at, pk, pk_src, attn_traffic(ecfg["name"])),
+                "quant": quant_object(epf, epf.timed_quant(esteps, 3, stream), pk, pk_src),
+                "l2": "%d rotating input sets of %.0f MB" % (len(epf.sets), epf.set_bytes / 1e6)}
+            del epf
+            torch.cuda.empty_cache()
 
     dec = None if args.no_decode else bench_decode(sage, torch, stream)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(cfg, args.cpu_seconds)
+        cb = cpu_baseline(full_cfg, args.cpu_seconds)
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "int8+e4m3", "data": "synthetic",
-            "config": {"workload": cfg["name"], "B": B, "H": H, "L": L, "D": D,
-                       "blk_q": blk_q, "blk_k": blk_k, "causal": causal,
-                       "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "%d rotating input sets of %.0f MB (> 126 MB L2)"
-                             % (len(sets), set_bytes / 1e6)},
+            "config": {"workload": full_cfg["name"], "B": full_cfg["B"], "H": full_cfg["H"],
+                       "L": full_cfg["L"], "D": full_cfg["D"], "blk_q": full_cfg["blk_q"],
+                       "blk_k": full_cfg["blk_k"], "causal": full_cfg["causal"],
+                       "parallelism": ("kv-head shards over %d ranks" % world) if world > 1 else "single",
+                       "l2": set_desc},
             "roofline": roofline,
             "cpu_baseline": cb,
             "e2e": e2e,
             "quant": quant,
+            "configs": extra,
             "decode": dec,
             "gpu_launches": (5 if args.fused_q else 3) * args.steps,
             "clocks": clk.summary(),

@@ -104,13 +104,15 @@ typedef struct sage_view4 {
 typedef struct sage_hadamard_s* sage_hadamard;
 
 /* Build the Sylvester Hadamard rotation H_D (entries +-1, H H^T = D I) for
- * head_dim D in {64, 128} once, on host and on `device` ("Sage v2
+ * head_dim D in {64, 128} once, for use with `device` ("Sage v2
  * improvements": created once, reused by every call). The kernels apply it
  * as the fp32 butterfly x -> x H (stages h = 1, 2, ..., D/2, each output one
  * IEEE add or subtract), unnormalised; the 1/D that Q H (K H)^T carries is
- * folded into the logit scale by sage_attn_fwd. *out receives the handle.
- * Errors: INVALID_ARG (out NULL, device < 0), UNSUPPORTED (other D),
- * CUDA (device not usable). */
+ * folded into the logit scale by sage_attn_fwd. The butterfly's pattern is
+ * H, so the handle holds the matrix on the host only (sage_hadamard_matrix)
+ * and no device memory. *out receives the handle.
+ * Errors: INVALID_ARG (out NULL, device < 0 or past the device count),
+ * UNSUPPORTED (other D), CUDA (device count unavailable). */
 sage_status sage_hadamard_init(int head_dim, int device, sage_hadamard* out);
 
 /* Free a handle from sage_hadamard_init (NULL is accepted). */
@@ -255,15 +257,20 @@ size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window
  * (fp32), per-(t, h) e4m3 quantisation with scale max|q_hat| / 448; keys j in
  * [max(0, p - window + 1), p]; S_j = (q8 . k8_j) * s_q * k_scale_j *
  * softmax_scale / D; softmax; out = sum_j p_j v_scale_j v8_j -> bf16.
- * out_bf16: [B, T, H, D] bf16 view. Supported: D == 128, page_size in
- * {16, 32, 64, 128}, H % Hk == 0, H / Hk <= 16, T * (H / Hk) <= 64,
- * window >= 1. ws: at least sage_attn_decode_workspace(...) bytes. */
+ * out_bf16: [B, T, H, D] bf16 view. q8_out (nullable, 16-byte aligned):
+ * receives the e4m3 codes of the rotated queries, contiguous [B, T, H, D];
+ * q_scale_out (nullable): their scales s_q, contiguous fp32 [B, T, H] (the
+ * codes the QK product used, for callers that reuse them or check them).
+ * Supported: D == 128, page_size in {16, 32, 64, 128}, H % Hk == 0,
+ * H / Hk <= 16, T * (H / Hk) <= 64, window >= 1. ws: at least
+ * sage_attn_decode_workspace(...) bytes. */
 sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
                              const uint8_t* v_cache, const float* k_scale, const float* v_scale,
                              const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
                              int H, int Hk, int D, int page_size, int max_pages, int num_pages,
-                             int window, float softmax_scale, sage_view4 out_bf16, void* ws,
-                             size_t ws_bytes, void* stream);
+                             int window, float softmax_scale, sage_view4 out_bf16,
+                             uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
+                             void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* sage_status_string(sage_status s);
@@ -276,6 +283,29 @@ const char* sage_status_string(sage_status s);
  * outside [0, num_pages) for a page holding keys of a window, whose keys were
  * then left out), SAGE_OK otherwise. */
 sage_status sage_device_error(void* stream);
+
+/* Kernel ids reported by sage_device_error_where. */
+#define SAGE_KERNEL_ATTN 1
+#define SAGE_KERNEL_DECODE 2
+#define SAGE_KERNEL_PROBE 3
+
+/* sage_device_error, also saying where the reported error was recorded:
+ * *kernel receives a SAGE_KERNEL_* id (0 with SAGE_OK), *site the number of
+ * the wait (or check) inside that kernel that recorded it. Either pointer
+ * may be NULL. Reads and clears the same error words as sage_device_error. */
+sage_status sage_device_error_where(void* stream, int* kernel, int* site);
+
+/* Failure-path probe (diagnostic; no page counterpart): enqueue one small
+ * kernel whose bounded mbarrier wait is never satisfied. The wait gives up
+ * after limit_ns nanoseconds (1 us .. 10 s), records a timeout at site 1 of
+ * SAGE_KERNEL_PROBE and raises its CTA's abort flag; a second waiter of the
+ * CTA (the kernels' default 2 s limit) must then end early through that
+ * flag, and the TMEM the CTA holds is released -- the path every kernel of
+ * the library takes when one of its waits expires. The next
+ * sage_device_error_where on `stream` reports SAGE_ERR_TIMEOUT, kernel 3,
+ * site 1; the device stays usable. Errors: INVALID_ARG (limit out of range),
+ * CUDA (launch failed). */
+sage_status sage_wait_probe(uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

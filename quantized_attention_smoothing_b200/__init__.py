@@ -31,8 +31,13 @@ EXPORTS = (
     "sage_quant_v_workspace", "sage_quant_v", "sage_quant_k", "sage_quant_qkv_workspace",
     "sage_quant_qkv",
     "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_fwd_q16", "sage_attn_decode_workspace",
-    "sage_attn_decode", "sage_status_string", "sage_device_error",
+    "sage_attn_decode", "sage_status_string", "sage_device_error", "sage_device_error_where",
+    "sage_wait_probe",
 )
+
+SAGE_KERNEL_ATTN = 1
+SAGE_KERNEL_DECODE = 2
+SAGE_KERNEL_PROBE = 3
 
 
 class SageError(RuntimeError):
@@ -98,9 +103,13 @@ def lib():
     L.sage_attn_decode_workspace.argtypes = [i32] * 6
     L.sage_attn_decode.restype = i32
     L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 9 + \
-        [f32, View4, vp, sz, vp]
+        [f32, View4, vp, vp, vp, sz, vp]
     L.sage_device_error.restype = i32
     L.sage_device_error.argtypes = [vp]
+    L.sage_device_error_where.restype = i32
+    L.sage_device_error_where.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    L.sage_wait_probe.restype = i32
+    L.sage_wait_probe.argtypes = [ctypes.c_uint64, vp]
     _lib = L
     return L
 
@@ -251,20 +260,34 @@ def sage_attn_fwd(q8, q_scale, k8, k_scale, v8_t, v_scale, B, H, Hk, Lq, Lk, D, 
 
 
 def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_lens, page_size,
-                     num_pages, window, softmax_scale, out, ws=None, stream=None):
+                     num_pages, window, softmax_scale, out, ws=None, stream=None, q8_out=None,
+                     q_scale_out=None):
     B, T, H, D = q.shape
     Hk = k_cache.shape[1]
     max_pages = page_table.shape[1]
     _check(lib().sage_attn_decode(h.handle, _view(q, CView4), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(k_scale), _ptr(v_scale), _ptr(page_table), _ptr(ctx_lens),
                                   B, T, H, Hk, D, int(page_size), int(max_pages), int(num_pages),
-                                  int(window), float(softmax_scale), _view(out, View4), _ptr(ws),
+                                  int(window), float(softmax_scale), _view(out, View4),
+                                  _ptr(q8_out), _ptr(q_scale_out), _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "sage_attn_decode")
 
 
 def sage_device_error(stream=None):
     return int(lib().sage_device_error(_stream(stream)))
+
+
+def sage_device_error_where(stream=None):
+    """(status, kernel id, site) of the error words; reads and clears them."""
+    k = ctypes.c_int()
+    s = ctypes.c_int()
+    st = int(lib().sage_device_error_where(_stream(stream), ctypes.byref(k), ctypes.byref(s)))
+    return st, k.value, s.value
+
+
+def sage_wait_probe(limit_ns, stream=None):
+    _check(lib().sage_wait_probe(int(limit_ns), _stream(stream)), "sage_wait_probe")
 
 
 # ---------------------------------------------------------------- convenience

@@ -27,6 +27,7 @@ SOURCES = {
     "attn_fwd.cu": [],
     "decode.cu": [],
     "sage_api.cu": [],
+    "probe.cu": [],
 }
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ARCH + ["-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v",

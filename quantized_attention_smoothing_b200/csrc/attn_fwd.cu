@@ -56,20 +56,6 @@ namespace {
 
 __device__ unsigned g_attn_err;
 
-#ifdef SAGE_ATTN_TRACE
-// Development-only phase timestamps (clock64) of CTA (0, 0): rows 0/1 are
-// softmax warps 0 and 4 (lane 0), row 2 the MMA thread; 16 tiles x 12 marks.
-__device__ long long g_attn_trace[3][16][12];
-#define SAGE_MARK(row, t, k)                                                         \
-    do {                                                                             \
-        if (trace_on && (t) < 16) g_attn_trace[row][t][k] = clock64();               \
-    } while (0)
-#else
-#define SAGE_MARK(row, t, k) \
-    do {                     \
-    } while (0)
-#endif
-
 constexpr int BM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;          // keys per tile
 constexpr int QT = 2;            // query tiles per CTA
@@ -90,10 +76,7 @@ constexpr float kMagicF = 12582912.0f;            // 1.5 * 2^23
 // every kPolyEvery-th key pair takes its exponential from exp2_poly_x2 (FMA
 // pipe) instead of the MUFU unit, which relieves the MUFU queue of the warp
 // converting its row (0 = never)
-#ifndef SAGE_POLY_EVERY
-#define SAGE_POLY_EVERY 8
-#endif
-constexpr int kPolyEvery = SAGE_POLY_EVERY;
+constexpr int kPolyEvery = 8;
 
 
 // K block scales of one head staged in shared memory (larger heads read the
@@ -288,9 +271,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_w[w] = q_row0 + w * BM < p.Lq ? (kv_end + BN - 1) / BN : 0;
     }
     const int n_max = max(n_w[0], n_w[1]);
-#ifdef SAGE_ATTN_TRACE
-    const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0;
-#endif
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kNumBars; ++i) {
@@ -380,7 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < D / 32; ++kk)
                         mma_i8_ss(tmem + w * BN, qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, 1u);
                     mma_commit(&bars[C::kBarSFull + w]);
-                    SAGE_MARK(2, t, 1 + w);
                 }
                 mma_commit(&bars[C::kBarKEmpty + s]);
                 return true;
@@ -404,7 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_f8_ss(tmem + 256 + w * BM, pdesc + 2 * kk, vdesc + 2 * kk, kIdescPV,
                                   (t > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(&bars[C::kBarODone + w]);
-                    SAGE_MARK(2, t, 3 + w);
                 }
                 mma_commit(&bars[C::kBarVEmpty + s]);
                 return true;
@@ -414,7 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             if (ok) ok = issue_qk(0);
             for (int t = 0; ok && t < n_max; ++t) {
-                SAGE_MARK(2, t, 0);
                 if (t + 1 < n_max) ok = issue_qk(t + 1);
                 if (ok) ok = issue_pv(t);
             }
@@ -503,13 +480,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (CAUSAL && valid) jlim = min(jlim, i + (p.Lk - p.Lq));
         uint8_t* sPw = smem + C::kOffP + w * C::kPBufs * C::kPBytes;   // this tile's P buffers
         const float* ksrow = p.k_scale + (int64_t)bhk * p.nbk;
-#ifdef SAGE_ATTN_TRACE
-        const bool tr = trace_on && lane == 0 && ww == 0;
-#define SMARK(k) SAGE_MARK(w, t, k)
-#define trace_on tr
-#else
-#define SMARK(k)
-#endif
 
         // S_w starts as the bias 1.5 * 2^23 in every column: int32 accumulation
         // onto it leaves bits that read directly as the fp32 value 1.5 * 2^23 +
@@ -529,17 +499,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m = -INFINITY, dsum = 0.0f;
         bool ok = true;
         for (int t = 0; t < n_t; ++t) {
-            SMARK(0);
             ok = warp_all(mbar_wait(&bars[C::kBarSFull + w], t & 1, abort_flag, &g_attn_err, 9));
             if (!ok) break;
             tc_fence_after();
-            SMARK(1);
             // the whole score row into registers, then S goes back to the MMA
             // warp with the bias rewritten for tile t + 1
             uint32_t s[BN];
             tmem_ld128(lane_addr + s_col, s);
             tmem_wait_ld128(s);
-            SMARK(6);
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c) tmem_fill32(lane_addr + s_col + 32 * c, kMagicI);
 
@@ -563,7 +530,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     : block_max<kKeysPerBlk, false>(s + kb * kKeysPerBlk, j0 + kb * kKeysPerBlk, jlim);
                 if (cm != -INFINITY) mt = fmaxf(mt, (cm - kMagicF) * kc[kb]);
             }
-            SMARK(7);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -571,13 +537,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float m_new = fmaxf(m, mt);
             const float msub = (m_new == -INFINITY) ? 0.0f : m_new;
             const float alpha = ex2_approx(m - msub);
-            SMARK(2);
             // the exponentials of the two query tiles take turns (token tok_w,
             // passed on below), so one tile's max and rescale overlap the
             // other's MUFU work instead of both tiles contending for it
             ok = warp_all(mbar_wait(&bars[C::kBarTok + w], t & 1, abort_flag, &g_attn_err, 12));
             if (!ok) break;
-            SMARK(8);
 
             // accumulate_d and RS_32_to_8: p448 = 448 * 2^(y - m') =
             // 2^(acc * kc + log2(448) - m'), one FMA per key (f32x2). Each
@@ -591,7 +555,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[C::kBarTok + (w ^ 1)]);
             dsum = dsum * alpha + tsum;
-            SMARK(3);
             if (t > 0) {
                 // update_mdo (rescale part): PV(t-1) must have landed in O first;
                 // then O *= alpha, skipped when no row of the warp changed its max
@@ -599,7 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &g_attn_err, 10));
                 if (!ok) break;
                 tc_fence_after();
-                SMARK(4);
                 if (__any_sync(0xffffffffu, alpha != 1.0f)) {
                     const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll
@@ -627,12 +589,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[C::kBarPFull + w]);
-            SMARK(5);
             m = m_new;
         }
-#ifdef SAGE_ATTN_TRACE
-#undef trace_on
-#endif
         // the other tile may visit more key tiles (causal, or this tile lies
         // past Lq): keep passing the turn until it is done
         for (int t = n_t; ok && t < n_w[w ^ 1]; ++t) {
@@ -800,18 +758,6 @@ cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s) {
     return a.D == 128 ? launch_d<128>(nkb, a.causal != 0, tq, tk, tv, p, qp, a.qfused != 0, grid, s)
                       : launch_d<64>(nkb, a.causal != 0, tq, tk, tv, p, qp, a.qfused != 0, grid, s);
 }
-
-#ifdef SAGE_ATTN_TRACE
-extern "C" __attribute__((visibility("default"))) int sage_debug_attn_trace(long long* host) {
-    return cudaMemcpyFromSymbol(host, g_attn_trace, sizeof(g_attn_trace)) == cudaSuccess ? 0 : -1;
-}
-extern "C" __attribute__((visibility("default"))) unsigned long long sage_debug_wait_polls(int reset) {
-    unsigned long long v = 0, z = 0;
-    cudaMemcpyFromSymbol(&v, g_wait_polls, sizeof v);
-    if (reset) cudaMemcpyToSymbol(g_wait_polls, &z, sizeof z);
-    return v;
-}
-#endif
 
 unsigned read_clear_attn_error() {
     unsigned v = 0, zero = 0;

@@ -119,6 +119,8 @@ struct DecParams {
     float logit_scale_log2;                  // softmax_scale / D * log2(e)
     __nv_bfloat16* out;
     int64_t os0, os1, os2, os3;
+    uint8_t* q8_out;                         // optional: e4m3 query codes [B, T, H, D]
+    float* qs_out;                           // optional: query scales [B, T, H]
 };
 
 // The A operand (P') of the PV MMA holds a row's 128 keys in this order:
@@ -421,6 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 rr = __fdiv_rn(448.0f, amax);
             }
             if (qq == 0) sq[r] = s;
+            // the codes and scale also go to the caller's optional outputs
+            // (written once, by the first CTA of the cluster)
+            const bool qout = rv && split == 0 && p.q8_out != nullptr;
+            const int64_t qtok = ((int64_t)b * p.T + t) * p.H + h;
+            if (rv && split == 0 && qq == 0 && p.qs_out != nullptr) p.qs_out[qtok] = s;
             uint8_t* qrow = sm + Sm::kQ + r * 128;
 #pragma unroll
             for (int c = 0; c < 2; ++c) {            // 16-byte chunk 2 qq + c of the row
@@ -430,10 +437,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int d = 16 * c + 4 * e;
                     const uint32_t lo16 = e4m3x2_rn_satfinite(__fmul_rn(x[d], rr), __fmul_rn(x[d + 1], rr));
                     const uint32_t hi16 = e4m3x2_rn_satfinite(__fmul_rn(x[d + 2], rr), __fmul_rn(x[d + 3], rr));
-                    w4[e] = lo16 | (hi16 << 16);
+                    w4[e] = amax != 0.0f ? (lo16 | (hi16 << 16)) : 0u;   // a zero row: +0 codes
                 }
                 const int chunk = 2 * qq + c;
                 *reinterpret_cast<uint4*>(qrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                if (qout)
+                    *reinterpret_cast<uint4*>(p.q8_out + qtok * kD + 16 * chunk) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
             fence_proxy_async_smem();                // the QK MMAs read these rows
         }
@@ -833,6 +843,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     p.os1 = a.out_stride[1];
     p.os2 = a.out_stride[2];
     p.os3 = a.out_stride[3];
+    p.q8_out = a.q8_out;
+    p.qs_out = a.q_scale_out;
     p.q_vec = (a.q.stride[3] == 1 && a.q.stride[0] % 8 == 0 && a.q.stride[1] % 8 == 0 &&
                a.q.stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.q.ptr) % 16 == 0)
                   ? 1

@@ -774,10 +774,10 @@ cudaError_t launch_quant_qkv(const View4& q, const View4& k, const View4& v, int
 // as sage_quant_qk, for callers that cannot allocate device memory at the
 // point of the call -- for instance a serving loop whose device memory is
 // budgeted once at start-up, or code that must not risk the implicit device
-// synchronisation that cudaMalloc / cudaFree can cause. Its scratch (the fp64
-// per-cluster column sums of K, written by the statistics kernel before the
-// quantisation kernel reads them) lives in the fixed array below instead of
-// a caller workspace.
+// synchronisation that cudaMalloc / cudaFree can cause. Its scratch -- the
+// fp32 K mean of every (b, kv head), B * Hk * D * 4 bytes, written by the
+// statistics kernel and read by the tile kernel -- lives in the fixed array
+// below instead of a caller workspace.
 #include <mutex>
 
 #include "../../include/sage.h"

@@ -14,11 +14,14 @@
 #include "../../include/sage.h"
 #include "sage_internal.h"
 
+// The rotation is applied by the kernels as the butterfly x -> x H, whose
+// add / subtract pattern is H itself, so no kernel reads the matrix: the
+// handle keeps it on the host (for sage_hadamard_matrix) together with the
+// device it was built for, which every call checks.
 struct sage_hadamard_s {
     int D;
     int device;
     int8_t* host;      // D x D, +-1, row-major
-    int8_t* dev;       // device copy (built once, reused)
 };
 
 namespace sage {
@@ -98,7 +101,6 @@ sage_status sage_hadamard_init(int head_dim, int device, sage_hadamard* out) {
     if (!h) return SAGE_ERR_CUDA;
     h->D = D;
     h->device = device;
-    h->dev = nullptr;
     h->host = static_cast<int8_t*>(std::malloc((size_t)D * D));
     if (!h->host) {
         delete h;
@@ -125,29 +127,12 @@ sage_status sage_hadamard_init(int head_dim, int device, sage_hadamard* out) {
                 return SAGE_ERR_CUDA;
             }
         }
-    int prev = 0;
-    cudaGetDevice(&prev);
-    cudaError_t e = cudaSetDevice(device);
-    if (e == cudaSuccess) e = cudaMalloc(&h->dev, (size_t)D * D);
-    if (e == cudaSuccess) e = cudaMemcpy(h->dev, h->host, (size_t)D * D, cudaMemcpyHostToDevice);
-    cudaSetDevice(prev);
-    if (e != cudaSuccess) {
-        if (h->dev) cudaFree(h->dev);
-        std::free(h->host);
-        delete h;
-        return SAGE_ERR_CUDA;
-    }
     *out = h;
     return SAGE_OK;
 }
 
 sage_status sage_hadamard_destroy(sage_hadamard h) {
     if (!h) return SAGE_OK;
-    int prev = 0;
-    cudaGetDevice(&prev);
-    cudaSetDevice(h->device);
-    cudaFree(h->dev);
-    cudaSetDevice(prev);
     std::free(h->host);
     delete h;
     return SAGE_OK;
@@ -410,8 +395,9 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
                              const uint8_t* v_cache, const float* k_scale, const float* v_scale,
                              const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
                              int H, int Hk, int D, int page_size, int max_pages, int num_pages,
-                             int window, float softmax_scale, sage_view4 out_bf16, void* ws,
-                             size_t ws_bytes, void* stream) {
+                             int window, float softmax_scale, sage_view4 out_bf16,
+                             uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
+                             void* stream) {
     if (!h || !q_bf16.ptr || !k_cache || !v_cache || !k_scale || !v_scale || !page_table ||
         !ctx_lens || !out_bf16.ptr)
         return SAGE_ERR_INVALID_ARG;
@@ -431,7 +417,8 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
     if ((int64_t)num_pages * Hk * page_size * D >= (int64_t(1) << 40)) return SAGE_ERR_UNSUPPORTED;
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_scale, 4) ||
         !aligned(v_scale, 4) || !aligned(page_table, 4) || !aligned(ctx_lens, 4) ||
-        !aligned(q_bf16.ptr, 2) || !aligned(out_bf16.ptr, 2))
+        !aligned(q_bf16.ptr, 2) || !aligned(out_bf16.ptr, 2) || !aligned(q8_out, 16) ||
+        !aligned(q_scale_out, 4))
         return SAGE_ERR_ALIGNMENT;
     const size_t need = sage::decode_ws_bytes(B, T, H, Hk, D, window);
     if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
@@ -460,18 +447,42 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
     a.out = out_bf16.ptr;
     for (int i = 0; i < 4; ++i) a.out_stride[i] = out_bf16.stride[i];
     a.ws = ws;
+    a.q8_out = q8_out;
+    a.q_scale_out = q_scale_out;
     return launch_status(sage::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 
-sage_status sage_device_error(void* stream) {
+sage_status sage_device_error_where(void* stream, int* kernel, int* site) {
+    if (kernel) *kernel = 0;
+    if (site) *site = 0;
     const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-    const unsigned a = sage::read_clear_attn_error();
-    const unsigned d = sage::read_clear_decode_error();
+    // error words of the kernels, in the order of SAGE_KERNEL_* ids 1, 2, 3
+    const unsigned words[3] = {sage::read_clear_attn_error(), sage::read_clear_decode_error(),
+                               sage::read_clear_probe_error()};
     if (e != cudaSuccess) return SAGE_ERR_CUDA;
-    if ((a & 0xFFu) == sage::kErrTimeoutCode || (d & 0xFFu) == sage::kErrTimeoutCode)
-        return SAGE_ERR_TIMEOUT;
-    if ((d & 0xFFu) == sage::kErrRangeCode) return SAGE_ERR_INVALID_ARG;
-    return SAGE_OK;
+    sage_status st = SAGE_OK;
+    for (int i = 0; i < 3; ++i) {
+        const unsigned code = words[i] & 0xFFu;
+        sage_status si = SAGE_OK;
+        if (code == sage::kErrTimeoutCode) si = SAGE_ERR_TIMEOUT;
+        else if (code == sage::kErrRangeCode) si = SAGE_ERR_INVALID_ARG;
+        // a timeout outranks a range error; the first kernel in id order wins a tie
+        const bool take = si != SAGE_OK && (st == SAGE_OK || (si == SAGE_ERR_TIMEOUT && st != SAGE_ERR_TIMEOUT));
+        if (take) {
+            st = si;
+            if (kernel) *kernel = i + 1;
+            if (site) *site = static_cast<int>(words[i] >> 8);
+        }
+    }
+    return st;
+}
+
+sage_status sage_device_error(void* stream) { return sage_device_error_where(stream, nullptr, nullptr); }
+
+sage_status sage_wait_probe(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000ull || limit_ns > 10000000000ull) return SAGE_ERR_INVALID_ARG;
+    return launch_status(sage::launch_wait_probe(static_cast<unsigned long long>(limit_ns),
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -115,10 +115,16 @@ struct DecodeArgs {
     void* out;
     int64_t out_stride[4];
     void* ws;
+    uint8_t* q8_out;           // optional [B, T, H, D] e4m3 query codes
+    float* q_scale_out;        // optional [B, T, H] query scales
 };
 size_t decode_ws_bytes(int B, int T, int H, int Hk, int D, int window);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 unsigned read_clear_decode_error();
+
+// ---- bounded-wait timeout probe (probe.cu)
+cudaError_t launch_wait_probe(unsigned long long limit_ns, cudaStream_t s);
+unsigned read_clear_probe_error();
 
 // ---- driver entry point for tensor-map encoding (sage_api.cu)
 void* tensor_map_encoder();

@@ -26,10 +26,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 
 // ------------------------------------------------------------ mbarrier
 
-#ifdef SAGE_ATTN_TRACE
-__device__ unsigned long long g_wait_polls;   // development-only poll counter
-#endif
-
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                  : "memory");
@@ -79,22 +75,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t pari
 
 // Wait until the phase with the given parity of `bar` has completed.
 // Bounded: returns false (after recording `site` in *err and raising the
-// CTA's abort flag) when the wait exceeds kWaitTimeoutNs, or as soon as
+// CTA's abort flag) when the wait exceeds `limit_ns`, or as soon as
 // another role of the CTA has raised the abort flag (seen within one
 // suspend interval).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag, unsigned* err,
-                                          unsigned site) {
+                                          unsigned site,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-#ifdef SAGE_ATTN_TRACE
-        atomicAdd(&g_wait_polls, 1ull);
-#endif
         if (mbar_try_wait_sleep(a, parity, 200000u)) return true;
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        if (global_timer_ns() - t0 > limit_ns) {
             atomicCAS(err, 0u, kErrTimeout | (site << 8));
             *abort_flag = 1;
             return false;

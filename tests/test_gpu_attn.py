@@ -1,8 +1,11 @@
 """GPU parity of the quantised attention forward (tcgen05 kernel) against
 the CPU oracle. Element-wise on small shapes spanning several 128-key tiles
 with ragged tails, causal masks (bottom-right aligned), GQA, both head dims
-and all block sizes; on sampled rows at the full workload sizes. The oracle
-quantises the original inputs itself (nothing it uses comes from the GPU)."""
+and all block sizes, for both the separate-Q and the in-CTA-Q paths; at the
+full workload sizes every element of the B1 H24 L4096 workload, every element
+of a quarter of the causal B2 H32 L8192 workload's heads, and sampled rows of
+the B1 H40 L32760 workload. The oracle quantises the original inputs itself
+(nothing it uses comes from the GPU)."""
 import math
 
 import numpy as np
@@ -24,21 +27,43 @@ def handles():
     return {64: sage.Hadamard(64), 128: sage.Hadamard(128)}
 
 
-def _run(handles, q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True):
-    D = q.shape[3]
-    out, _ = sage.sage_attention(handles[D], to_gpu(q), to_gpu(k), to_gpu(v), blk_q, blk_k, scale,
-                                 causal)
-    torch.cuda.synchronize()
-    assert sage.sage_device_error() == sage.SAGE_OK
-    gpu = bits(out)                                     # [B, H, Lq, D]
+def _oracle(q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True):
+    """The oracle's quantised output (fp64 before its bf16 rounding) and the
+    unquantised fp64 reference, from the original bf16 inputs."""
     qk = oracle.quant_qk(bits(q), bits(k), blk_q, blk_k)
     v8t, vs = oracle.quant_v(bits(v))
     _, ref = oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, q.shape[2], k.shape[2],
                          blk_q, blk_k, scale, causal, rows=rows, want_f64=True)
     ex = oracle.attn_exact(bits(q), bits(k), bits(v), scale, causal, rows=rows) if exact else None
+    return ref, ex
+
+
+def _run(handles, q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True, fused_q=False,
+         heads=None):
+    """GPU output (bf16 bits) of the whole path, and the oracle's on the same
+    inputs. heads: compare only these head indices (the GPU runs them all)."""
+    D = q.shape[3]
+    run = sage.sage_attention_q16 if fused_q else sage.sage_attention
+    out, _ = run(handles[D], to_gpu(q), to_gpu(k), to_gpu(v), blk_q, blk_k, scale, causal)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    gpu = bits(out)                                     # [B, H, Lq, D]
+    if heads is not None:
+        gpu = gpu[:, heads]
+        q, k, v = q[:, heads], k[:, heads], v[:, heads]
+    ref, ex = _oracle(q, k, v, blk_q, blk_k, scale, causal, rows=rows, exact=exact)
     if rows is not None:
         gpu = gpu[:, :, rows]
     return gpu, ref, ex
+
+
+def _shape_inputs(B, H, Hk, Lq, Lk, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, Lq, H, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    k = (torch.randn((B, Lk, Hk, D), generator=g) + torch.randn((B, 1, Hk, D), generator=g) * 2)
+    k = k.to(torch.bfloat16).permute(0, 2, 1, 3)
+    v = torch.randn((B, Lk, Hk, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    return q, k, v
 
 
 SHAPES = [
@@ -56,11 +81,7 @@ SHAPES = [
 
 @pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,blk_q,blk_k,causal", SHAPES)
 def test_attn_matches_oracle_elementwise(handles, B, H, Hk, Lq, Lk, D, blk_q, blk_k, causal):
-    g = torch.Generator().manual_seed(Lq * 31 + Lk + D)
-    q = torch.randn((B, Lq, H, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
-    k = (torch.randn((B, Lk, Hk, D), generator=g) + torch.randn((B, 1, Hk, D), generator=g) * 2)
-    k = k.to(torch.bfloat16).permute(0, 2, 1, 3)
-    v = torch.randn((B, Lk, Hk, D), generator=g).to(torch.bfloat16).permute(0, 2, 1, 3)
+    q, k, v = _shape_inputs(B, H, Hk, Lq, Lk, D, Lq * 31 + Lk + D)
     scale = 1.0 / math.sqrt(D)
     gpu, ref, ex = _run(handles, q, k, v, blk_q, blk_k, scale, causal)
     compare_output(gpu, ref, ex, label=str((B, H, Hk, Lq, Lk, D, causal)))
@@ -100,13 +121,45 @@ def test_attn_deterministic(handles):
     assert torch.equal(a, b)
 
 
-@pytest.mark.parametrize("key,nrows", [("c2", 24), ("c3", 8), ("c4", 4)])
-def test_attn_full_size_sampled_rows(handles, key, nrows):
-    cfg, q, k, v = workloads.make_prefill_config(key)
-    rows = sample_rows(cfg["L"], nrows, seed=cfg["H"])
+def test_attn_full_size_c2_every_element(handles):
+    """The B1 H24 L4096 D128 video-DiT workload compared in full: every
+    output element of every head against the oracle."""
+    cfg, q, k, v = workloads.make_prefill_config("c2")
+    gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
+                        cfg["causal"], exact=True)
+    compare_output(gpu, ref, ex, label="c2 full")
+
+
+def test_attn_full_size_c3_quarter_of_heads(handles):
+    """The causal B2 H32 L8192 D128 workload: every output element of a
+    seeded quarter of its heads (8 of 32, in both batches) against the
+    oracle; the GPU computes all heads in one launch."""
+    cfg, q, k, v = workloads.make_prefill_config("c3")
+    heads = np.sort(np.random.default_rng(cfg["H"]).choice(cfg["H"], size=cfg["H"] // 4,
+                                                            replace=False))
+    gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
+                        cfg["causal"], exact=True, heads=heads)
+    compare_output(gpu, ref, ex, label="c3 heads %s" % heads.tolist())
+
+
+def test_attn_full_size_c4_sampled_rows(handles):
+    """The long B1 H40 L32760 D128 workload (a ragged last tile) on sampled
+    rows of every head, tile edges and the tail included."""
+    cfg, q, k, v = workloads.make_prefill_config("c4")
+    rows = sample_rows(cfg["L"], 4, seed=cfg["H"])
     gpu, ref, ex = _run(handles, q, k, v, cfg["blk_q"], cfg["blk_k"], cfg["softmax_scale"],
                         cfg["causal"], rows=rows, exact=True)
-    compare_output(gpu, ref, ex, label=key)
+    compare_output(gpu, ref, ex, label="c4")
+
+
+@pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,blk_q,blk_k,causal", SHAPES)
+def test_attn_q16_matches_oracle_elementwise(handles, B, H, Hk, Lq, Lk, D, blk_q, blk_k, causal):
+    """Q rotated and quantised inside the attention kernel, compared with the
+    oracle element by element (the oracle quantises Q itself)."""
+    q, k, v = _shape_inputs(B, H, Hk, Lq, Lk, D, Lq * 29 + Lk + D + 5)
+    scale = 1.0 / math.sqrt(D)
+    gpu, ref, ex = _run(handles, q, k, v, blk_q, blk_k, scale, causal, fused_q=True)
+    compare_output(gpu, ref, ex, label="q16 " + str((B, H, Hk, Lq, Lk, D, causal)))
 
 
 @pytest.mark.parametrize("B,H,Hk,Lq,Lk,D,blk_q,blk_k,causal", SHAPES)
@@ -141,3 +194,5 @@ def test_attn_q16_strided_query(handles):
         o, _ = sage.sage_attention_q16(handles[128], qv, kg, vg, 128, 64, 0.1, False)
         torch.cuda.synchronize()
         assert torch.equal(o, ref)
+    oref, ex = _oracle(q, k, v, 128, 64, 0.1, False)
+    compare_output(bits(ref), oref, ex, label="q16 strided")
