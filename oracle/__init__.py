@@ -60,7 +60,11 @@ def lib():
         L.or_attn_head.argtypes = [_i8p, _f32p, _i8p, _f32p, _u8p, ctypes.c_int64, _f32p,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int,
-                                   _i32p, ctypes.c_int, _u16p, _f64p]
+                                   _i32p, ctypes.c_int, _u16p, _f64p, _f64p]
+        L.or_p_fp32_delta.restype = ctypes.c_double
+        L.or_p_fp32_delta.argtypes = [ctypes.c_double, ctypes.c_double]
+        L.or_e4m3_flip_step.restype = ctypes.c_double
+        L.or_e4m3_flip_step.argtypes = [ctypes.c_double, ctypes.c_double]
         L.or_attn_exact_head.restype = None
         L.or_attn_exact_head.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_double, ctypes.c_int, _i32p,
@@ -209,18 +213,21 @@ def quant_v(v, threads=None):
 # ---------------------------------------------------------------- attention
 
 def attn(q8, qs, k8, ks, v8t, vs, Lq, Lk, blk_q, blk_k, softmax_scale, causal, rows=None,
-         quantize_p=True, threads=None, want_f64=False):
+         quantize_p=True, threads=None, want_f64=False, want_flip=False):
     """Quantised attention over the quantised operands.
-    Returns bf16 bits [B, H, nrows, D] (and the fp64 values if want_f64)."""
+    Returns bf16 bits [B, H, nrows, D] (and the fp64 values if want_f64, and
+    then also the per-element fp32 P-rounding margin if want_flip)."""
     B, H, _, D = q8.shape
     Hk = k8.shape[1]
     group = H // Hk
+    want_f64 = want_f64 or want_flip
     if rows is None:
         rows = np.arange(Lq, dtype=np.int32)
     rows = np.ascontiguousarray(rows, dtype=np.int32)
     n = rows.size
     out = np.zeros((B, H, n, D), dtype=np.uint16)
     o64 = np.zeros((B, H, n, D), dtype=np.float64) if want_f64 else None
+    flip = np.zeros((B, H, n, D), dtype=np.float64) if want_flip else None
 
     def one(bh):
         b, h = bh
@@ -233,16 +240,22 @@ def attn(q8, qs, k8, ks, v8t, vs, Lq, Lk, blk_q, blk_k, softmax_scale, causal, r
         a_vs = np.ascontiguousarray(vs[b, hk])
         oo = np.zeros((n, D), dtype=np.uint16)
         of = np.zeros((n, D), dtype=np.float64) if want_f64 else None
+        ff = np.zeros((n, D), dtype=np.float64) if want_flip else None
         lib().or_attn_head(_p(a_q8, _i8p), _p(a_qs, _f32p), _p(a_k8, _i8p), _p(a_ks, _f32p),
                            _p(a_v8, _u8p), a_v8.shape[1], _p(a_vs, _f32p), Lq, Lk, D, blk_q,
                            blk_k, float(softmax_scale), int(bool(causal)), int(bool(quantize_p)),
                            _p(rows, _i32p), n, _p(oo, _u16p),
-                           _p(of, _f64p) if want_f64 else None)
+                           _p(of, _f64p) if want_f64 else None,
+                           _p(ff, _f64p) if want_flip else None)
         out[b, h] = oo
         if want_f64:
             o64[b, h] = of
+        if want_flip:
+            flip[b, h] = ff
 
     _pool_map(one, [(b, h) for b in range(B) for h in range(H)], threads)
+    if want_flip:
+        return out, o64, flip
     return (out, o64) if want_f64 else out
 
 

@@ -281,6 +281,42 @@ void or_quant_v_head(const uint16_t* v, int L, int D, int Lpad, uint8_t* v8t, fl
 }
 
 /* ------------------------------------------------------------------ */
+/* The fp32 rounding margin of P ([S2TP] Candidate: RS_32_to_8)        */
+/* ------------------------------------------------------------------ */
+
+/* The scores are converted to FP8 from fp32 ("RS_32_to_8"), so an
+ * implementation's 448 p carries fp32 error before the e4m3 rounding, and a
+ * code whose exact value lies that close to a rounding midpoint may round
+ * the other way. Relative error bound of such an fp32 p = exp(x - m), x and
+ * m natural-log logits: the logit is formed with a few fp32 roundings
+ * relative to |x| and |m| (2^-24 each, in base-2 units), and the exponential
+ * adds a few fp32 ulps; delta = (log2(e) (|x| + |m|) + 16) * 2^-21 bounds
+ * both with a margin of about four. */
+double or_p_fp32_delta(double x, double m)
+{
+    return (1.4426950408889634 * (fabs(x) + fabs(m)) + 16.0) * 0x1p-21;   /* log2(e) */
+}
+
+/* If a value v >= 0 rounded to e4m3 with a relative perturbation up to
+ * delta could land on a neighbouring code of e4m3(v), the distance to that
+ * neighbour (the step the code can move by); else 0. */
+double or_e4m3_flip_step(double v, double delta)
+{
+    const uint8_t c = or_e4m3_encode(v);          /* 0 .. 0x7E, v >= 0 */
+    const double here = or_e4m3_decode(c);
+    double st = 0.0;
+    if (c < 0x7E) {                               /* the midpoint above */
+        const double up = or_e4m3_decode((uint8_t)(c + 1));
+        if (v * (1.0 + delta) >= 0.5 * (here + up)) st = up - here;
+    }
+    if (c > 0) {                                  /* the midpoint below */
+        const double dn = or_e4m3_decode((uint8_t)(c - 1));
+        if (v * (1.0 - delta) <= 0.5 * (here + dn) && here - dn > st) st = here - dn;
+    }
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Quantised attention, one (b,h), selected query rows ([S2TP] order)  */
 /* ------------------------------------------------------------------ */
 
@@ -300,14 +336,20 @@ void or_quant_v_head(const uint16_t* v, int L, int D, int Lpad, uint8_t* v8t, fl
  * a row with no visible key writes zeros. With quantize_p == 0 the e4m3
  * rounding of P is skipped (P8 = 448 * p exactly), which must then equal
  * exact softmax over the dequantised operands. out_f64 (optional) receives
- * the value before the bf16 rounding. */
+ * the value before the bf16 rounding. flip_f64 (optional) receives, per
+ * output element, how far an fp32 implementation of the same sequence may
+ * land from out_f64 through P codes that round the other way: the sum over
+ * the keys whose 448 p lies within or_p_fp32_delta of an e4m3 rounding
+ * midpoint of step * |V| * vs / (448 d), carried through the rescales like O. */
 void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const float* ks,
                   const uint8_t* v8t, int64_t ldv, const float* vs, int Lq, int Lk, int D,
                   int blk_q, int blk_k, double softmax_scale, int causal, int quantize_p,
-                  const int32_t* rows, int nrows, uint16_t* out, double* out_f64)
+                  const int32_t* rows, int nrows, uint16_t* out, double* out_f64,
+                  double* flip_f64)
 {
     const double c = softmax_scale / (double)D;
     double* O = (double*)malloc(sizeof(double) * (size_t)D);
+    double* F = (double*)malloc(sizeof(double) * (size_t)D);
     double* x = (double*)malloc(sizeof(double) * OR_KEY_TILE);
     double vdec[256];
     for (int t = 0; t < 256; ++t) vdec[t] = or_e4m3_decode((uint8_t)t);
@@ -317,7 +359,7 @@ void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const flo
         const int8_t* qi = q8 + (int64_t)i * D;
         const double qscale = (double)qs[i / blk_q];
         double m = -INFINITY, dsum = 0.0;
-        for (int e = 0; e < D; ++e) O[e] = 0.0;
+        for (int e = 0; e < D; ++e) O[e] = F[e] = 0.0;
 
         for (int t0 = 0; t0 < Lk; t0 += OR_KEY_TILE) {
             int t1 = t0 + OR_KEY_TILE < Lk ? t0 + OR_KEY_TILE : Lk;
@@ -338,6 +380,7 @@ void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const flo
             if (mnew == -INFINITY) continue;      /* nothing visible yet */
             double alpha = (m == -INFINITY) ? 0.0 : exp(m - mnew);
             for (int e = 0; e < D; ++e) O[e] *= alpha;
+            for (int e = 0; e < D; ++e) F[e] *= alpha;
             /* accumulate_d, RS_32_to_8, PV */
             dsum *= alpha;
             for (int j = t0; j < t1; ++j) {
@@ -346,6 +389,14 @@ void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const flo
                 dsum += p;
                 double p8 = quantize_p ? or_e4m3_decode(or_e4m3_encode(p * 448.0)) : p * 448.0;
                 for (int e = 0; e < D; ++e) O[e] += p8 * vdec[v8t[(int64_t)e * ldv + j]];
+                if (flip_f64 && quantize_p) {
+                    /* the step this P code moves by if an fp32 evaluation of
+                       448 p (relative error up to or_p_fp32_delta) rounds it
+                       the other way */
+                    const double st = or_e4m3_flip_step(p * 448.0, or_p_fp32_delta(x[j - t0], mnew));
+                    if (st > 0.0)
+                        for (int e = 0; e < D; ++e) F[e] += st * fabs(vdec[v8t[(int64_t)e * ldv + j]]);
+                }
             }
             m = mnew;
         }
@@ -353,10 +404,13 @@ void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const flo
             double y = dsum > 0.0 ? O[e] * (double)vs[e] / (448.0 * dsum) : 0.0;
             out[(int64_t)r * D + e] = or_f64_to_bf16(y);
             if (out_f64) out_f64[(int64_t)r * D + e] = y;
+            if (flip_f64)
+                flip_f64[(int64_t)r * D + e] = dsum > 0.0 ? F[e] * (double)vs[e] / (448.0 * dsum) : 0.0;
         }
     }
     free(x);
     free(O);
+    free(F);
 }
 
 /* Unquantised reference, one (b,h): fp64 softmax(q k^T * softmax_scale) v

@@ -209,3 +209,89 @@ def test_exact_reference_equals_numpy_softmax(oracle_mod, B, H, Hk, Lq, Lk, D, c
     if causal and Lq > Lk:
         n_dark = Lq - Lk
         assert (got[:, :, r < n_dark] == 0).all()
+
+
+def _e4m3_round(x):
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(
+        torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _fp32_p_attention(oracle_mod, qk, v8t, vs, h, L, D, blk, scale, rel_noise, rng):
+    """The method's per-tile sequence written with numpy, independently of the
+    oracle, with 448 p formed in fp32 the way a GPU kernel forms it (fp32
+    logit scales, fp32 base-2 logits, fp32 exp2), then multiplied by
+    (1 + u), |u| <= rel_noise, before the e4m3 cast; O and d in fp64."""
+    q8 = qk["q8"][0, h, :L].astype(np.int64)
+    k8 = qk["k8"][0, h, :L].astype(np.int64)
+    acc = q8 @ k8.T
+    qs = np.repeat(qk["qs"][0, h], blk)[:L]
+    ks = np.repeat(qk["ks"][0, h], blk)[:L]
+    vdec = oracle_mod.e4m3_decode(v8t[0, h, :, :L]).T
+    arow = (qs.astype(np.float32) * np.float32(scale / D * math.log2(math.e))).astype(np.float32)
+    kc = (ks[None, :].astype(np.float32) * arow[:, None]).astype(np.float32)
+    y = (acc.astype(np.float32) * kc).astype(np.float32)
+    m = np.full(L, -np.inf, dtype=np.float32)
+    d = np.zeros(L)
+    O = np.zeros((L, D))
+    for t0 in range(0, L, 128):
+        yt = y[:, t0:t0 + 128]
+        mn = np.maximum(m, yt.max(1))
+        alpha = np.where(np.isfinite(m), np.exp2((m - mn).astype(np.float32)).astype(np.float64), 0.0)
+        p448 = np.exp2((yt + np.float32(math.log2(448.0)) - mn[:, None]).astype(np.float32))
+        p448 = p448.astype(np.float64) * (1.0 + rel_noise * rng.uniform(-1.0, 1.0, p448.shape))
+        O *= alpha[:, None]
+        d = d * alpha + (p448 / 448.0).sum(1)
+        O += _e4m3_round(p448) @ vdec[t0:t0 + 128]
+        m = mn
+    return O * vs[0, h][None, :].astype(np.float64) / (448.0 * d[:, None])
+
+
+def test_p_rounding_margin_bounds_an_fp32_evaluation(oracle_mod):
+    """The oracle's per-element margin for P codes that an fp32 evaluation
+    may round the other way ("RS_32_to_8": scores are fp32 before the FP8
+    cast). An independent numpy evaluation with fp32 logits and exponentials
+    (plus noise of 1e-6 relative, inside the margin's error bound) lands
+    within that margin of the oracle everywhere, though it moves elements by
+    more than 1e-4 through flipped codes; with noise a hundred times larger
+    the margin no longer holds (it is not vacuous)."""
+    H, L, D, scale = 4, 1024, 64, 0.125
+    g = torch.Generator().manual_seed(5)
+    q = (torch.randn((1, H, L, D), generator=g) * 2).to(torch.bfloat16)
+    k = (torch.randn((1, H, L, D), generator=g) * 2 + 1).to(torch.bfloat16)
+    v = torch.randn((1, H, L, D), generator=g).to(torch.bfloat16)
+    qk = oracle_mod.quant_qk(_bits(q), _bits(k), 64, 64)
+    v8t, vs = oracle_mod.quant_v(_bits(v))
+    _, y, margin = oracle_mod.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, L, L, 64, 64,
+                                   scale, False, want_flip=True)
+    assert (margin >= 0).all() and (margin > 0).any()
+    rng = np.random.default_rng(0)
+    moved = 0
+    for h in range(H):
+        got = _fp32_p_attention(oracle_mod, qk, v8t, vs, h, L, D, 64, scale, 1e-6, rng)
+        dev = np.abs(got - y[0, h])
+        # 1e-5: the fp32 exponentials' own effect on d and on the codes that do not flip
+        assert (dev <= margin[0, h] + 1e-5).all(), float((dev - margin[0, h]).max())
+        moved += int((dev > 1e-4).sum())
+    assert moved > 0                       # flipped codes did move elements
+    worst = 0.0
+    for h in range(H):
+        got = _fp32_p_attention(oracle_mod, qk, v8t, vs, h, L, D, 64, scale, 1e-4, rng)
+        worst = max(worst, float((np.abs(got - y[0, h]) - margin[0, h]).max()))
+    assert worst > 1e-3
+
+
+def test_e4m3_flip_step_at_the_midpoints(oracle_mod):
+    """or_e4m3_flip_step: zero away from the rounding midpoints, the
+    neighbouring code's distance at them, with the e4m3 grid checked against
+    torch's float8 decode."""
+    L = oracle_mod.lib()
+    grid = torch.arange(0, 127, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(1, 126):
+        lo, here, hi = grid[c - 1], grid[c], grid[c + 1]
+        mid_up = 0.5 * (here + hi)
+        assert L.or_e4m3_flip_step(here, 1e-6) == 0.0
+        assert L.or_e4m3_flip_step(mid_up * (1 - 1e-7), 1e-6) == hi - here
+        assert L.or_e4m3_flip_step(mid_up * (1 + 1e-7), 1e-6) == hi - here
+        assert L.or_e4m3_flip_step(0.5 * (lo + here) * (1 + 1e-7), 1e-6) == here - lo
+    assert L.or_e4m3_flip_step(448.0, 1e-3) == 0.0                 # saturates: no code above
+    assert L.or_e4m3_flip_step(2.0 ** -10 * (1 - 1e-7), 1e-6) == 2.0 ** -9
