@@ -1,11 +1,16 @@
 """Shared helpers of the GPU parity tests: run the CUDA path through the
 C-ABI binding on seeded inputs, run the oracle on the same inputs, compare.
 
-Tolerance of the bf16 attention output (derived in the design doc): the GPU's
-fp32 result may differ from the oracle's fp64 value y by at most 2e-3 before
-its final bf16 rounding, so element-wise |gpu - y| <= 2e-3 + ulp_bf16(y)/2;
-the cosine against the oracle must be >= 0.9999 and against unquantised
-fp64 attention >= 0.998.
+Tolerance of the bf16 attention output: the GPU's fp32 result may differ
+from the oracle's fp64 value y by at most 2e-3 before its final bf16
+rounding, so element-wise |gpu - y| <= 2e-3 + ulp_bf16(y)/2, plus, where the
+oracle reports one, the margin of the P codes that an fp32 evaluation of
+448 p may round the other way (the scores are fp32 before the FP8 cast, and
+a code whose exact value lies within fp32 error of an e4m3 rounding midpoint
+can land on either side; the oracle gives the effect of moving each such
+code by one step). The cosine against the oracle must be >= 0.9999 and
+against unquantised fp64 attention >= 0.998. Every comparison reports how
+many elements needed the margin.
 """
 import math
 
@@ -78,15 +83,22 @@ def bf16_ulp(x):
     return 2.0 ** (e - 7)
 
 
-def compare_output(gpu_bf16_bits, oracle_f64, exact_f64=None, label=""):
+def compare_output(gpu_bf16_bits, oracle_f64, exact_f64=None, label="", margin=None):
     g = workloads_f32(gpu_bf16_bits).astype(np.float64)
     y = oracle_f64
+    if isinstance(y, tuple):                 # (oracle value, P-rounding margin)
+        y, margin = y
     ulp = bf16_ulp(np.maximum(np.abs(g), np.abs(y)))
-    excess = np.abs(g - y) - ulp / 2
+    plain = np.abs(g - y) - ulp / 2
+    excess = plain if margin is None else plain - margin
     worst = float(excess.max())
     cos = cosine(g, y)
-    stats = {"max_excess": worst, "max_abs": float(np.abs(g - y).max()), "cos_oracle": cos}
-    assert worst <= MAX_ABS, "%s: |gpu - oracle| exceeds 2e-3 + ulp/2 by %g" % (label, worst)
+    stats = {"max_excess": worst, "max_abs": float(np.abs(g - y).max()), "cos_oracle": cos,
+             "beyond_plain_bar": int((plain > MAX_ABS).sum()), "elements": int(plain.size)}
+    if stats["beyond_plain_bar"]:
+        print("%s: %d of %d elements beyond 2e-3 + ulp/2 (largest %.3g), each within the P-rounding "
+              "margin" % (label, stats["beyond_plain_bar"], plain.size, float(plain.max())))
+    assert worst <= MAX_ABS, "%s: |gpu - oracle| exceeds 2e-3 + ulp/2 (+ margin) by %g" % (label, worst)
     assert cos >= COS_ORACLE, "%s: cosine vs oracle %.6f" % (label, cos)
     if exact_f64 is not None:
         ce = cosine(g, exact_f64)

@@ -28,14 +28,15 @@ def handles():
 
 
 def _oracle(q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True):
-    """The oracle's quantised output (fp64 before its bf16 rounding) and the
-    unquantised fp64 reference, from the original bf16 inputs."""
+    """The oracle's quantised output (fp64 before its bf16 rounding) with its
+    P-rounding margin, and the unquantised fp64 reference, from the original
+    bf16 inputs."""
     qk = oracle.quant_qk(bits(q), bits(k), blk_q, blk_k)
     v8t, vs = oracle.quant_v(bits(v))
-    _, ref = oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, q.shape[2], k.shape[2],
-                         blk_q, blk_k, scale, causal, rows=rows, want_f64=True)
+    _, ref, margin = oracle.attn(qk["q8"], qk["qs"], qk["k8"], qk["ks"], v8t, vs, q.shape[2],
+                                 k.shape[2], blk_q, blk_k, scale, causal, rows=rows, want_flip=True)
     ex = oracle.attn_exact(bits(q), bits(k), bits(v), scale, causal, rows=rows) if exact else None
-    return ref, ex
+    return (ref, margin), ex
 
 
 def _run(handles, q, k, v, blk_q, blk_k, scale, causal, rows=None, exact=True, fused_q=False,
