@@ -69,6 +69,18 @@ def lib():
         L.or_attn_exact_head.argtypes = [_u16p, _u16p, _u16p, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_double, ctypes.c_int, _i32p,
                                          ctypes.c_int, _f64p]
+        L.or_e2m1_decode.restype = ctypes.c_double
+        L.or_e2m1_decode.argtypes = [ctypes.c_uint8]
+        L.or_e2m1_encode.restype = ctypes.c_uint8
+        L.or_e2m1_encode.argtypes = [ctypes.c_double]
+        L.or_quant_mxfp4_head.restype = None
+        L.or_quant_mxfp4_head.argtypes = [_u16p, _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          _u8p, _u8p]
+        L.or_attn_mxfp4_head.restype = None
+        L.or_attn_mxfp4_head.argtypes = [_u8p, _u8p, _u8p, _u8p, _u8p, ctypes.c_int64, _f32p,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                         ctypes.c_int, ctypes.c_int, _i32p, ctypes.c_int, _u16p,
+                                         _f64p, _f64p]
         L.or_decode_quant_q_row.restype = None
         L.or_decode_quant_q_row.argtypes = [_u16p, ctypes.c_int, _u8p, _f32p]
         L.or_decode_seq.restype = None
@@ -339,3 +351,95 @@ def decode_quant_q(q):
     for i in range(rows.shape[0]):
         f(_p(rows[i], _u16p), D, _p(codes[i], _u8p), _p(scales[i:i + 1], _f32p))
     return codes.reshape(B, T, H, D), scales.reshape(B, T, H)
+
+
+# ---------------------------------------------------------------- MXFP4 variant
+
+def e2m1_decode(codes):
+    L = lib()
+    table = np.array([L.or_e2m1_decode(c) for c in range(16)], dtype=np.float64)
+    return table[np.asarray(codes, dtype=np.uint8) & 15]
+
+
+def e2m1_encode(x):
+    x = np.asarray(x, dtype=np.float64)
+    f = lib().or_e2m1_encode
+    return np.array([f(float(v)) for v in x.ravel()], dtype=np.uint8).reshape(x.shape)
+
+
+def _quant_mxfp4(x, mean, threads):
+    B, H, L, D = x.shape
+    Lpad = round_up(L, 128)
+    codes = np.zeros((B, H, Lpad, D // 2), dtype=np.uint8)
+    sf = np.zeros((B, H, Lpad, D // 32), dtype=np.uint8)
+
+    def one(bh):
+        b, h = bh
+        xx = np.ascontiguousarray(x[b, h])
+        mp = None
+        if mean is not None:
+            mm = np.ascontiguousarray(mean[b, h], dtype=np.float32)
+            mp = _p(mm, _f32p)
+        cc = np.zeros((Lpad, D // 2), dtype=np.uint8)
+        ss = np.zeros((Lpad, D // 32), dtype=np.uint8)
+        lib().or_quant_mxfp4_head(_p(xx, _u16p), mp, L, D, Lpad, _p(cc, _u8p), _p(ss, _u8p))
+        codes[b, h] = cc
+        sf[b, h] = ss
+
+    _pool_map(one, [(b, h) for b in range(B) for h in range(H)], threads)
+    return codes, sf
+
+
+def quant_qk_mxfp4(q, k, threads=None):
+    """Smooth K, rotate Q and K, quantise both to MXFP4 (E2M1 codes, one e8m0
+    scale per 32 elements of a row). q: uint16 [B, H, Lq, D]; k: uint16
+    [B, Hk, Lk, D]. Codes [B, H, Lpad, D/2] (element 2i in the low nibble),
+    scales [B, H, Lpad, D/32] in plain row-major order."""
+    kmean = k_mean(k)
+    q4, qsf = _quant_mxfp4(q, None, threads)
+    k4, ksf = _quant_mxfp4(k, kmean, threads)
+    return {"q4": q4, "qsf": qsf, "k4": k4, "ksf": ksf, "kmean": kmean}
+
+
+def attn_mxfp4(q4, qsf, k4, ksf, v8t, vs, Lq, Lk, softmax_scale, causal, rows=None,
+               quantize_p=True, threads=None, want_f64=False, want_flip=False):
+    """Quantised attention with MXFP4 Q / K and FP8 P / V. Returns bf16 bits
+    [B, H, nrows, D] (and the fp64 values, and the P-rounding margin)."""
+    B, H, _, D2 = q4.shape
+    D = 2 * D2
+    Hk = k4.shape[1]
+    group = H // Hk
+    want_f64 = want_f64 or want_flip
+    if rows is None:
+        rows = np.arange(Lq, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    n = rows.size
+    out = np.zeros((B, H, n, D), dtype=np.uint16)
+    o64 = np.zeros((B, H, n, D), dtype=np.float64) if want_f64 else None
+    flip = np.zeros((B, H, n, D), dtype=np.float64) if want_flip else None
+
+    def one(bh):
+        b, h = bh
+        hk = h // group
+        a = [np.ascontiguousarray(t) for t in (q4[b, h], qsf[b, h], k4[b, hk], ksf[b, hk])]
+        a_v8 = np.ascontiguousarray(v8t[b, hk])
+        a_vs = np.ascontiguousarray(vs[b, hk])
+        oo = np.zeros((n, D), dtype=np.uint16)
+        of = np.zeros((n, D), dtype=np.float64) if want_f64 else None
+        ff = np.zeros((n, D), dtype=np.float64) if want_flip else None
+        lib().or_attn_mxfp4_head(_p(a[0], _u8p), _p(a[1], _u8p), _p(a[2], _u8p), _p(a[3], _u8p),
+                                 _p(a_v8, _u8p), a_v8.shape[1], _p(a_vs, _f32p), Lq, Lk, D,
+                                 float(softmax_scale), int(bool(causal)), int(bool(quantize_p)),
+                                 _p(rows, _i32p), n, _p(oo, _u16p),
+                                 _p(of, _f64p) if want_f64 else None,
+                                 _p(ff, _f64p) if want_flip else None)
+        out[b, h] = oo
+        if want_f64:
+            o64[b, h] = of
+        if want_flip:
+            flip[b, h] = ff
+
+    _pool_map(one, [(b, h) for b in range(B) for h in range(H)], threads)
+    if want_flip:
+        return out, o64, flip
+    return (out, o64) if want_f64 else out

@@ -41,6 +41,15 @@
  *     the unquantised probabilities; out = bf16_rne(O*vs/(448*d));
  *   - causal mask is bottom-right aligned: key j is visible to query i iff
  *     j <= i + (Lk - Lq); a row that sees no key outputs zeros.
+ *   - the MXFP4 variant ([SV2] changelog: fav3_sage_mxfp4 with a Hadamard
+ *     block BLOCK_R = 128, i.e. the whole head for D <= 128; [PA]: MXFP4 is
+ *     packed E2M1 with float8_e8m0fnu scales, and Q / P use E4M3 as their
+ *     FP8 format): Q and K (K smoothed as above) are rotated, then quantised
+ *     per row in blocks of 32 consecutive elements to E2M1 codes with one
+ *     power-of-two scale 2^E each, E = floor(log2(amax)) - 2 (the OCP MX
+ *     rule: the largest E2M1 value 6 has exponent 2), codes
+ *     e2m1_rne_satfinite(x * 2^-E); QK^T over the dequantised values, then
+ *     the same per-tile softmax, e4m3 P and FP8 V as above.
  */
 #include <math.h>
 #include <stdint.h>
@@ -177,6 +186,33 @@ void or_fwht_rows_f32(float* x, int64_t rows, int D)
     for (int64_t r = 0; r < rows; ++r) or_fwht_f32(x + r * D, D);
 }
 
+/* OCP MX FP4 E2M1: 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit,
+ * no infinities or NaN. Magnitudes of codes 0..7: 0, 0.5 (subnormal), 1,
+ * 1.5, 2, 3, 4, 6; bit 3 is the sign. */
+double or_e2m1_decode(uint8_t code)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    const double v = mag[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* Round to the nearest E2M1 value, ties to the even code, magnitudes at or
+ * beyond 6 saturate to 6 ("satfinite"); the sign is kept (-0 -> 0x8). */
+uint8_t or_e2m1_encode(double x)
+{
+    const uint8_t sign = signbit(x) ? 8 : 0;
+    const double ax = fabs(x);
+    if (ax >= 6.0) return (uint8_t)(sign | 7);
+    int c = 0;                                    /* largest code with value <= ax */
+    while (c < 7 && or_e2m1_decode((uint8_t)(c + 1)) <= ax) ++c;
+    if (c < 7) {
+        const double lo = or_e2m1_decode((uint8_t)c), hi = or_e2m1_decode((uint8_t)(c + 1));
+        const double mid = 0.5 * (lo + hi);
+        if (ax > mid || (ax == mid && (c & 1))) ++c;
+    }
+    return (uint8_t)(sign | c);
+}
+
 /* ------------------------------------------------------------------ */
 /* K smoothing statistic                                               */
 /* ------------------------------------------------------------------ */
@@ -245,6 +281,58 @@ void or_quant_i8_head(const uint16_t* x, const float* mean, int L, int D, int bl
     for (int l = L; l < Lpad; ++l)
         for (int d = 0; d < D; ++d) codes[(int64_t)l * D + d] = 0;
     free(rot);
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 quantisation of Q or K ([SV2] fav3_sage_mxfp4, [PA] MXFP4)    */
+/* ------------------------------------------------------------------ */
+
+/* One (b,h) slice x[L][D] (bf16). If mean is not NULL it is subtracted
+ * first (fp32); each row is rotated with or_fwht_f32. Per row and block of
+ * 32 consecutive elements:
+ *   a = max |x_hat| over the block (fp32);
+ *   E = floor(log2(a)) - 2, clamped to [-127, 127]; a == 0 gives E = -127;
+ *   code = e2m1(x_hat * 2^-E) (a scaling by a power of two: exact);
+ *   scale byte = E + 127 (e8m0: the value 2^E).
+ * Output codes[Lpad][D/2], element 2i in the low nibble of byte i (rows
+ * L..Lpad-1 zero), sf[Lpad][D/32] (rows L..Lpad-1 zero). */
+void or_quant_mxfp4_head(const uint16_t* x, const float* mean, int L, int D, int Lpad,
+                         uint8_t* codes, uint8_t* sf)
+{
+    float* row = (float*)malloc(sizeof(float) * (size_t)D);
+    const int nb = D / 32;
+    memset(codes, 0, (size_t)Lpad * (size_t)(D / 2));
+    memset(sf, 0, (size_t)Lpad * (size_t)nb);
+    for (int l = 0; l < L; ++l) {
+        for (int d = 0; d < D; ++d) {
+            float v = or_bf16_to_f32(x[(int64_t)l * D + d]);
+            if (mean) v = v - mean[d];
+            row[d] = v;
+        }
+        or_fwht_f32(row, D);
+        for (int b = 0; b < nb; ++b) {
+            float a = 0.0f;
+            for (int e = 0; e < 32; ++e) {
+                float v = fabsf(row[32 * b + e]);
+                if (v > a) a = v;
+            }
+            int E = -127;
+            if (a > 0.0f) {
+                int ex;
+                frexp((double)a, &ex);            /* a = f * 2^ex, f in [0.5, 1) */
+                E = (ex - 1) - 2;                 /* floor(log2(a)) - 2 */
+                if (E < -127) E = -127;
+                if (E > 127) E = 127;
+            }
+            sf[(int64_t)l * nb + b] = (uint8_t)(E + 127);
+            for (int e = 0; e < 32; ++e) {
+                const int d = 32 * b + e;
+                const uint8_t c = (a > 0.0f) ? or_e2m1_encode(ldexp((double)row[d], -E)) : 0;
+                codes[(int64_t)l * (D / 2) + d / 2] |= (uint8_t)((d & 1) ? (c << 4) : c);
+            }
+        }
+    }
+    free(row);
 }
 
 /* ------------------------------------------------------------------ */
@@ -411,6 +499,93 @@ void or_attn_head(const int8_t* q8, const float* qs, const int8_t* k8, const flo
     free(x);
     free(O);
     free(F);
+}
+
+/* Quantised attention with MXFP4 Q and K, one (b, h), selected query rows.
+ * q4[Lq_pad][D/2], qsf[Lq_pad][D/32], k4[Lk_pad][D/2], ksf[Lk_pad][D/32]
+ * (layouts of or_quant_mxfp4_head), v8t[D][ldv] and vs[D] as for
+ * or_attn_head. For each requested row i, with c = softmax_scale / D:
+ *   x_ij = c * sum_b 2^(Eq_ib + Ek_jb) * sum_{d in block b} e2m1(q_id) e2m1(k_jd)
+ * (exact in fp64), masked as in or_attn_head; then the same per-tile
+ * sequence QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV in 128-key
+ * tiles, e4m3 P scaled by 448, out = bf16(O * vs / (448 d)). out_f64 and
+ * flip_f64 (optional) as for or_attn_head. */
+void or_attn_mxfp4_head(const uint8_t* q4, const uint8_t* qsf, const uint8_t* k4, const uint8_t* ksf,
+                        const uint8_t* v8t, int64_t ldv, const float* vs, int Lq, int Lk, int D,
+                        double softmax_scale, int causal, int quantize_p, const int32_t* rows,
+                        int nrows, uint16_t* out, double* out_f64, double* flip_f64)
+{
+    const double c = softmax_scale / (double)D;
+    const int nb = D / 32;
+    double* O = (double*)malloc(sizeof(double) * (size_t)D);
+    double* F = (double*)malloc(sizeof(double) * (size_t)D);
+    double* x = (double*)malloc(sizeof(double) * OR_KEY_TILE);
+    double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+    double vdec[256];
+    for (int t = 0; t < 256; ++t) vdec[t] = or_e4m3_decode((uint8_t)t);
+
+    for (int r = 0; r < nrows; ++r) {
+        const int i = rows[r];
+        /* the query row's element values without their block scales */
+        for (int d = 0; d < D; ++d) {
+            const uint8_t byte = q4[(int64_t)i * (D / 2) + d / 2];
+            qd[d] = or_e2m1_decode((uint8_t)((d & 1) ? (byte >> 4) : (byte & 15)));
+        }
+        double m = -INFINITY, dsum = 0.0;
+        for (int e = 0; e < D; ++e) O[e] = F[e] = 0.0;
+
+        for (int t0 = 0; t0 < Lk; t0 += OR_KEY_TILE) {
+            int t1 = t0 + OR_KEY_TILE < Lk ? t0 + OR_KEY_TILE : Lk;
+            double mt = -INFINITY;
+            for (int j = t0; j < t1; ++j) {
+                int visible = !causal || (int64_t)j <= (int64_t)i + (Lk - Lq);
+                if (!visible) { x[j - t0] = -INFINITY; continue; }
+                double acc = 0.0;
+                for (int b = 0; b < nb; ++b) {
+                    double part = 0.0;
+                    for (int d = 32 * b; d < 32 * b + 32; ++d) {
+                        const uint8_t byte = k4[(int64_t)j * (D / 2) + d / 2];
+                        part += qd[d] * or_e2m1_decode((uint8_t)((d & 1) ? (byte >> 4) : (byte & 15)));
+                    }
+                    const int E = (int)qsf[(int64_t)i * nb + b] - 127 + (int)ksf[(int64_t)j * nb + b] - 127;
+                    acc += ldexp(part, E);
+                }
+                double v = acc * c;
+                x[j - t0] = v;
+                if (v > mt) mt = v;
+            }
+            double mnew = m > mt ? m : mt;
+            if (mnew == -INFINITY) continue;
+            double alpha = (m == -INFINITY) ? 0.0 : exp(m - mnew);
+            for (int e = 0; e < D; ++e) O[e] *= alpha;
+            for (int e = 0; e < D; ++e) F[e] *= alpha;
+            dsum *= alpha;
+            for (int j = t0; j < t1; ++j) {
+                if (x[j - t0] == -INFINITY) continue;
+                double p = exp(x[j - t0] - mnew);
+                dsum += p;
+                double p8 = quantize_p ? or_e4m3_decode(or_e4m3_encode(p * 448.0)) : p * 448.0;
+                for (int e = 0; e < D; ++e) O[e] += p8 * vdec[v8t[(int64_t)e * ldv + j]];
+                if (flip_f64 && quantize_p) {
+                    const double st = or_e4m3_flip_step(p * 448.0, or_p_fp32_delta(x[j - t0], mnew));
+                    if (st > 0.0)
+                        for (int e = 0; e < D; ++e) F[e] += st * fabs(vdec[v8t[(int64_t)e * ldv + j]]);
+                }
+            }
+            m = mnew;
+        }
+        for (int e = 0; e < D; ++e) {
+            double y = dsum > 0.0 ? O[e] * (double)vs[e] / (448.0 * dsum) : 0.0;
+            out[(int64_t)r * D + e] = or_f64_to_bf16(y);
+            if (out_f64) out_f64[(int64_t)r * D + e] = y;
+            if (flip_f64)
+                flip_f64[(int64_t)r * D + e] = dsum > 0.0 ? F[e] * (double)vs[e] / (448.0 * dsum) : 0.0;
+        }
+    }
+    free(qd);
+    free(x);
+    free(F);
+    free(O);
 }
 
 /* Unquantised reference, one (b,h): fp64 softmax(q k^T * softmax_scale) v
