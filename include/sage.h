@@ -243,6 +243,45 @@ sage_status sage_attn_fwd_q16(sage_hadamard h, sage_cview4 q_bf16, int blk_q, co
                               int Hk, int Lk, int blk_k, float softmax_scale, int causal,
                               sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream);
 
+/* MXFP4 variant: Q and K quantised to OCP MX FP4 ("Sage v2 improvements",
+ * Changelog: the fav3_sage_mxfp4 attention with a Hadamard block BLOCK_R =
+ * 128, i.e. the whole head for D <= 128; "[FlyDSL] [Misc] pa_decode ...",
+ * Changes: MXFP4 is packed E2M1 with float8_e8m0fnu scales, and Q / P use
+ * E4M3 as their FP8 format). K is smoothed (its per-(b,h) mean subtracted,
+ * as in sage_quant_qk) and Q and K rotated by the butterfly, then per row and
+ * block of 32 consecutive elements: a = max |x_hat|, E = floor(log2 a) - 2
+ * clamped to [-127, 125] (E = -127 for a = 0 or a subnormal a), codes
+ * E2M1(x_hat * 2^-E) rounded to nearest even and saturating at 6 (a zero
+ * block gets +0 codes), scale byte E + 127 (e8m0).
+ *   q_bf16: [B, H, Lq, D], k_bf16: [B, Hk, Lk, D] bf16 views, D in {64, 128}
+ *   (the handle's D), H % Hk == 0.
+ * Layouts (16-byte aligned):
+ *   q4 / k4    uint8 [B, H(k), Lpad, D/2]: element 2i of a row in the low
+ *              nibble of byte i; rows >= L zero
+ *   q_sf / k_sf uint8 [B, H(k), Lpad/128, 512]: per 128-row tile, the scale
+ *              of row r, block j at byte 16 (r mod 32) + 4 (r div 32) + j
+ *              (the order the block-scaled MMA reads); unused bytes zero
+ * k_mean (nullable) and ws as for sage_quant_qk (ws: at least
+ * sage_quant_qk_workspace(...) bytes). Errors as for sage_quant_qk. */
+sage_status sage_quant_qk_mx(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16, uint8_t* q4,
+                             uint8_t* q_sf, uint8_t* k4, uint8_t* k_sf, float* k_mean, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Quantised attention with MXFP4 Q and K (from sage_quant_qk_mx) and FP8 V
+ * (from sage_quant_v): for query row i of head h (kv head h / (H / Hk)) and
+ * key j, with c = softmax_scale / D,
+ *   x_ij = c * sum over 32-element blocks b of 2^(Eq_ib + Ek_jb) *
+ *          sum_{d in b} e2m1(q_id) e2m1(k_jd)
+ * (the block-scaled E2M1 MMA); then the per-tile sequence of sage_attn_fwd:
+ * 128-key tiles, running max and denominator, P8 = e4m3(448 exp(x - m)), FP8
+ * PV, out = bf16(O * v_scale / (448 d)); causal as for sage_attn_fwd.
+ * out_bf16: [B, H, Lq, D] bf16 view of any strides. Supported: D in {64, 128},
+ * softmax_scale > 0. ws may be NULL. */
+sage_status sage_attn_fwd_mx(const uint8_t* q4, const uint8_t* q_sf, const uint8_t* k4,
+                             const uint8_t* k_sf, const uint8_t* v8_t, const float* v_scale, int B,
+                             int H, int Hk, int Lq, int Lk, int D, float softmax_scale, int causal,
+                             sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace sage_attn_decode needs (split-KV partials). */
 size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window);
 
@@ -288,6 +327,7 @@ sage_status sage_device_error(void* stream);
 #define SAGE_KERNEL_ATTN 1
 #define SAGE_KERNEL_DECODE 2
 #define SAGE_KERNEL_PROBE 3
+#define SAGE_KERNEL_ATTN_MX 4
 
 /* sage_device_error, also saying where the reported error was recorded:
  * *kernel receives a SAGE_KERNEL_* id (0 with SAGE_OK), *site the number of

@@ -32,12 +32,13 @@ EXPORTS = (
     "sage_quant_qkv",
     "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_fwd_q16", "sage_attn_decode_workspace",
     "sage_attn_decode", "sage_status_string", "sage_device_error", "sage_device_error_where",
-    "sage_wait_probe",
+    "sage_wait_probe", "sage_quant_qk_mx", "sage_attn_fwd_mx",
 )
 
 SAGE_KERNEL_ATTN = 1
 SAGE_KERNEL_DECODE = 2
 SAGE_KERNEL_PROBE = 3
+SAGE_KERNEL_ATTN_MX = 4
 
 
 class SageError(RuntimeError):
@@ -108,6 +109,10 @@ def lib():
     L.sage_device_error.argtypes = [vp]
     L.sage_device_error_where.restype = i32
     L.sage_device_error_where.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    L.sage_quant_qk_mx.restype = i32
+    L.sage_quant_qk_mx.argtypes = [vp, CView4, CView4, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.sage_attn_fwd_mx.restype = i32
+    L.sage_attn_fwd_mx.argtypes = [vp] * 6 + [i32] * 6 + [f32, i32, View4, vp, sz, vp]
     L.sage_wait_probe.restype = i32
     L.sage_wait_probe.argtypes = [ctypes.c_uint64, vp]
     _lib = L
@@ -274,6 +279,22 @@ def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_l
                                   _stream(stream)), "sage_attn_decode")
 
 
+def sage_quant_qk_mx(h, q, k, q4, q_sf, k4, k_sf, k_mean=None, ws=None, stream=None):
+    _check(lib().sage_quant_qk_mx(h.handle, _view(q, CView4), _view(k, CView4), _ptr(q4), _ptr(q_sf),
+                                  _ptr(k4), _ptr(k_sf), _ptr(k_mean), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
+           "sage_quant_qk_mx")
+
+
+def sage_attn_fwd_mx(q4, q_sf, k4, k_sf, v8_t, v_scale, B, H, Hk, Lq, Lk, D, softmax_scale, causal,
+                     out, ws=None, stream=None):
+    _check(lib().sage_attn_fwd_mx(_ptr(q4), _ptr(q_sf), _ptr(k4), _ptr(k_sf), _ptr(v8_t), _ptr(v_scale),
+                                  B, H, Hk, Lq, Lk, D, float(softmax_scale), int(bool(causal)),
+                                  _view(out, View4), _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
+           "sage_attn_fwd_mx")
+
+
 def sage_device_error(stream=None):
     return int(lib().sage_device_error(_stream(stream)))
 
@@ -371,3 +392,39 @@ def quantise(h, q, k, v, blk_q, blk_k, bufs, stream=None):
     join = torch.cuda.Event()
     join.record(bufs.side)
     s.wait_event(join)
+
+
+class MxBuffers:
+    """Device buffers of the MXFP4 Q / K and FP8 V operands for one shape."""
+
+    def __init__(self, B, H, Hk, Lq, Lk, D, device=None):
+        dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+        LpQ, LpK = round_up(Lq, 128), round_up(Lk, 128)
+        self.q4 = torch.empty((B, H, LpQ, D // 2), dtype=torch.uint8, device=dev)
+        self.q_sf = torch.empty((B, H, LpQ // 128, 512), dtype=torch.uint8, device=dev)
+        self.k4 = torch.empty((B, Hk, LpK, D // 2), dtype=torch.uint8, device=dev)
+        self.k_sf = torch.empty((B, Hk, LpK // 128, 512), dtype=torch.uint8, device=dev)
+        self.k_mean = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
+        self.v8_t = torch.empty((B, Hk, D, LpK), dtype=torch.uint8, device=dev)
+        self.v_scale = torch.empty((B, Hk, D), dtype=torch.float32, device=dev)
+        self.ws = torch.empty((max(sage_quant_qk_workspace(B, H, Hk, Lq, Lk, D), 16),),
+                              dtype=torch.uint8, device=dev)
+        self.ws_v = torch.empty((max(sage_quant_v_workspace(B, Hk, Lk, D), 16),), dtype=torch.uint8,
+                                device=dev)
+
+
+def sage_attention_mx(h, q, k, v, softmax_scale, causal=False, out=None, bufs=None, stream=None):
+    """MXFP4 Q / K + FP8 V path: sage_quant_qk_mx + sage_quant_v +
+    sage_attn_fwd_mx on [B, H(k), L, D] bf16 views. Returns (out, bufs)."""
+    B, H, Lq, D = q.shape
+    Hk, Lk = k.shape[1], k.shape[2]
+    if bufs is None:
+        bufs = MxBuffers(B, H, Hk, Lq, Lk, D, q.device.index)
+    if out is None:
+        out = torch.empty((B, Lq, H, D), dtype=torch.bfloat16, device=q.device).permute(0, 2, 1, 3)
+    s = torch.cuda.current_stream() if stream is None else stream
+    sage_quant_qk_mx(h, q, k, bufs.q4, bufs.q_sf, bufs.k4, bufs.k_sf, bufs.k_mean, bufs.ws, s)
+    sage_quant_v(v, bufs.v8_t, bufs.v_scale, bufs.ws_v, s)
+    sage_attn_fwd_mx(bufs.q4, bufs.q_sf, bufs.k4, bufs.k_sf, bufs.v8_t, bufs.v_scale, B, H, Hk, Lq, Lk,
+                     D, softmax_scale, causal, out, None, s)
+    return out, bufs

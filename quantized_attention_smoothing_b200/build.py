@@ -25,6 +25,7 @@ HEADER = os.path.join(ROOT, "include", "sage.h")
 SOURCES = {
     "quant.cu": ["-fmad=false"],
     "attn_fwd.cu": [],
+    "attn_mx.cu": [],
     "decode.cu": [],
     "sage_api.cu": [],
     "probe.cu": [],

@@ -275,6 +275,11 @@ struct QuantJob {
     int8_t* k8;
     float* k_scale;
     uint8_t* v8t;
+    // MXFP4 outputs (quant_tiles_kernel<D, true>): E2M1 codes and e8m0 scales
+    uint8_t* q4;
+    uint8_t* q_sf;
+    uint8_t* k4;
+    uint8_t* k_sf;
 };
 
 enum : int { kKindQ = 0, kKindK = 1, kKindV = 2 };
@@ -338,13 +343,14 @@ struct TileDesc {
     const float* stat;     // K: the head's mean; V: its multipliers 448 / a; Q: null
     void* out;             // Q/K: codes of row l0; V: v8t[b, h, 0, l0]
     float* scale;          // Q/K: scale of the block holding row l0
+    uint8_t* sf;           // MXFP4 Q/K: the tile's 512-byte scale-factor block
     int64_t rstride;       // token-row stride of the view (elements)
     int64_t lpad;          // V: row pitch of the transposed output
     int kind, nrows, vec, blk;
     int b, h, l0, unused;
 };
 
-template <int D>
+template <int D, bool MX>
 __device__ TileDesc make_desc(int t, const QuantJob& j) {
     const TileRef r = tile_ref(t, j);
     const View4& x = view_of(j, r.kind);
@@ -360,11 +366,19 @@ __device__ TileDesc make_desc(int t, const QuantJob& j) {
             (int64_t)r.l0 * x.stride[2];
     d.rstride = x.stride[2];
     d.lpad = (int64_t)r.ntiles * kTile;
+    d.sf = nullptr;
     if (r.kind == kKindV) {
         d.blk = 0;
         d.stat = j.v_rmul_ws + (int64_t)r.bh * D;
         d.out = j.v8t + (int64_t)r.bh * D * d.lpad + r.l0;
         d.scale = nullptr;
+    } else if (MX) {
+        const bool isK = r.kind == kKindK;
+        d.blk = 0;
+        d.stat = isK ? j.k_mean_ws + (int64_t)r.bh * D : nullptr;
+        d.out = (isK ? j.k4 : j.q4) + ((int64_t)r.bh * d.lpad + r.l0) * (D / 2);
+        d.scale = nullptr;
+        d.sf = (isK ? j.k_sf : j.q_sf) + ((int64_t)r.bh * d.lpad + r.l0) / kTile * 512;
     } else {
         const bool isK = r.kind == kKindK;
         d.blk = isK ? j.blk_k : j.blk_q;
@@ -462,6 +476,22 @@ __device__ __forceinline__ uint2 codes8_clamp(const uint64_t (&x2)[N], int k0, f
     return make_uint2(w[0], w[1]);
 }
 
+// Eight E2M1 codes (round to nearest even, saturating) of the four value
+// pairs, element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1x8(uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(w)
+        : "f"(p2lo(a)), "f"(p2hi(a)), "f"(p2lo(b)), "f"(p2hi(b)), "f"(p2lo(c)), "f"(p2hi(c)),
+          "f"(p2lo(d)), "f"(p2hi(d)));
+    return w;
+}
+
 // ---------------------------------------------------------------- kernel
 // Persistent CTAs of 512 threads; CTA c takes tiles c, c + G, c + 2G, ...
 // (G = gridDim.x, odd when K and V alternate, so every CTA gets both
@@ -470,7 +500,16 @@ __device__ __forceinline__ uint2 codes8_clamp(const uint64_t (&x2)[N], int k0, f
 // descriptor of tile i + kQStages at the top of iteration i, while the
 // copies of tile i land. The first K or V tile a CTA issues waits for the
 // statistics kernel (griddepcontrol.wait).
-template <int D>
+// MX = true: Q and K tiles are written as MXFP4 instead of INT8: per row and
+// block of 32 consecutive elements (the four threads of the row's quad hold
+// 8 elements each), a = max |x_hat|, E = floor(log2 a) - 2 clamped to
+// [-127, 125] (-127 for a = 0 or a subnormal a), codes
+// e2m1_rn_satfinite(x_hat * 2^-E) (an exact power-of-two scaling), scale
+// byte E + 127; an all-zero block gets +0 codes. Codes are packed two per
+// byte, element 2i in the low nibble; scale bytes go to the tile's 512-byte
+// block in the layout the block-scaled MMA reads (row r, block b at
+// 16 (r mod 32) + 4 (r div 32) + b; unused blocks of a D = 64 row are 0).
+template <int D, bool MX>
 __global__ void __launch_bounds__(kQThreads, kQMinCtas) quant_tiles_kernel(QuantJob j) {
     constexpr int kTileElems = kTile * D;
     constexpr int NM = D / 32;                    // Q/K: 8-value chunks per thread
@@ -528,7 +567,7 @@ __global__ void __launch_bounds__(kQThreads, kQMinCtas) quant_tiles_kernel(Quant
     if (tid == 0) {
 #pragma unroll
         for (int s = 0; s < kQStages; ++s)
-            if (blockIdx.x + s * G < n_tiles) tdesc[s] = make_desc<D>(blockIdx.x + s * G, j);
+            if (blockIdx.x + s * G < n_tiles) tdesc[s] = make_desc<D, MX>(blockIdx.x + s * G, j);
     }
     __syncthreads();
 #pragma unroll
@@ -539,7 +578,7 @@ __global__ void __launch_bounds__(kQThreads, kQMinCtas) quant_tiles_kernel(Quant
         const int slot = it % NSLOT;
         const int nslot = (it + kQStages) % NSLOT;
         const int tn = t + kQStages * G;
-        if (tid == 0 && tn < n_tiles) tdesc[nslot] = make_desc<D>(tn, j);
+        if (tid == 0 && tn < n_tiles) tdesc[nslot] = make_desc<D, MX>(tn, j);
         uint16_t* tile = tiles + buf * kTileElems;
         const float* st = stat + buf * D;
         const TileDesc& d = tdesc[slot];
@@ -614,6 +653,36 @@ __global__ void __launch_bounds__(kQThreads, kQMinCtas) quant_tiles_kernel(Quant
             }
             quad_butterfly<D>(x2, sub);
 
+            if constexpr (MX) {
+                // every read of the buffer is done once all threads are here
+                __syncthreads();
+                start(tn, nslot, buf);
+                uint8_t* codes = static_cast<uint8_t*>(d.out) + r * (D / 2) + 4 * sub;
+#pragma unroll
+                for (int m = 0; m < NM; ++m) {
+                    float a = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) a = fmax3(a, fabsf(p2lo(x2[4 * m + e])), fabsf(p2hi(x2[4 * m + e])));
+                    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+                    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+                    const int ef = static_cast<int>(__float_as_uint(a) >> 23);      // a >= +0
+                    const int E = ef == 0 ? -127 : max(ef - 129, -127);
+                    const float sc = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);   // 2^-E
+                    const uint64_t sc2 = p2(sc, sc);
+                    uint32_t w = e2m1x8(p2mul(x2[4 * m], sc2), p2mul(x2[4 * m + 1], sc2),
+                                        p2mul(x2[4 * m + 2], sc2), p2mul(x2[4 * m + 3], sc2));
+                    if (a == 0.0f) w = 0u;
+                    if (valid) *reinterpret_cast<uint32_t*>(codes + 16 * m) = w;
+                    else *reinterpret_cast<uint32_t*>(codes + 16 * m) = 0u;
+                    if (sub == 0) d.sf[16 * (r & 31) + 4 * (r >> 5) + m] = valid ? static_cast<uint8_t>(E + 127) : 0;
+                }
+                if (D == 64 && sub == 0) {
+                    d.sf[16 * (r & 31) + 4 * (r >> 5) + 2] = 0;
+                    d.sf[16 * (r & 31) + 4 * (r >> 5) + 3] = 0;
+                }
+                continue;
+            }
+
             float a = 0.0f;
 #pragma unroll
             for (int k = 0; k < NP; ++k) a = fmax3(a, fabsf(p2lo(x2[k])), fabsf(p2hi(x2[k])));
@@ -657,10 +726,13 @@ size_t tiles_smem_bytes() {
 // The statistics of the given tensors, then the tiles of the given tensors;
 // null views are skipped. ws: [B * Hk][D] fp32 K means (when k), then
 // [B * Hk][D] fp32 V multipliers (when v).
-template <int D>
+// MX = true: Q and K as MXFP4 (q4 / q_sf / k4 / k_sf; no V, no INT8 outputs)
+template <int D, bool MX = false>
 cudaError_t launch_quant_d(const View4* q, const View4* k, const View4* v, int blk_q, int blk_k,
                            int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
-                           uint8_t* v8t, float* v_scale, void* ws, cudaStream_t s) {
+                           uint8_t* v8t, float* v_scale, void* ws, cudaStream_t s,
+                           uint8_t* q4 = nullptr, uint8_t* q_sf = nullptr, uint8_t* k4 = nullptr,
+                           uint8_t* k_sf = nullptr) {
     const View4 none = {};
     const int nkh = k ? (int)(k->size[0] * k->size[1]) : 0;
     const int nvh = v ? (int)(v->size[0] * v->size[1]) : 0;
@@ -705,10 +777,14 @@ cudaError_t launch_quant_d(const View4* q, const View4* k, const View4* v, int b
     j.k8 = k8;
     j.k_scale = k_scale;
     j.v8t = v8t;
+    j.q4 = q4;
+    j.q_sf = q_sf;
+    j.k4 = k4;
+    j.k_sf = k_sf;
     const int n_tiles = j.nq + j.nk + j.nv;
     if (n_tiles == 0) return cudaSuccess;
 
-    auto kern = quant_tiles_kernel<D>;
+    auto kern = quant_tiles_kernel<D, MX>;
     const size_t smem = tiles_smem_bytes<D>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -765,6 +841,15 @@ cudaError_t launch_quant_qkv(const View4& q, const View4& k, const View4& v, int
     return by_head_dim((int)k.size[3], [&](auto d) {
         return launch_quant_d<decltype(d)::value>(&q, &k, &v, blk_q, blk_k, q8, q_scale, k8, k_scale,
                                                   k_mean, v8t, v_scale, ws, s);
+    });
+}
+
+cudaError_t launch_quant_qk_mx(const View4& q, const View4& k, uint8_t* q4, uint8_t* q_sf, uint8_t* k4,
+                               uint8_t* k_sf, float* k_mean, void* ws, cudaStream_t s) {
+    return by_head_dim((int)k.size[3], [&](auto d) {
+        return launch_quant_d<decltype(d)::value, true>(&q, &k, nullptr, 32, 32, nullptr, nullptr, nullptr,
+                                                        nullptr, k_mean, nullptr, nullptr, ws, s, q4, q_sf,
+                                                        k4, k_sf);
     });
 }
 

@@ -386,6 +386,77 @@ sage_status sage_attn_fwd_q16(sage_hadamard h, sage_cview4 q_bf16, int blk_q, co
     return launch_status(sage::launch_attn_fwd(a, static_cast<cudaStream_t>(stream)));
 }
 
+sage_status sage_quant_qk_mx(sage_hadamard h, sage_cview4 q_bf16, sage_cview4 k_bf16, uint8_t* q4,
+                             uint8_t* q_sf, uint8_t* k4, uint8_t* k_sf, float* k_mean, void* ws,
+                             size_t ws_bytes, void* stream) {
+    if (!h || !q_bf16.ptr || !k_bf16.ptr || !q4 || !q_sf || !k4 || !k_sf) return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(q_bf16.size, q_bf16.stride) || !sizes_ok(k_bf16.size, k_bf16.stride))
+        return SAGE_ERR_INVALID_ARG;
+    const int64_t B = q_bf16.size[0], H = q_bf16.size[1], Lq = q_bf16.size[2], D = q_bf16.size[3];
+    const int64_t Hk = k_bf16.size[1], Lk = k_bf16.size[2];
+    if (k_bf16.size[0] != B || k_bf16.size[3] != D) return SAGE_ERR_INVALID_ARG;
+    if (D != h->D) return SAGE_ERR_INVALID_ARG;
+    if (H % Hk != 0) return SAGE_ERR_UNSUPPORTED;
+    if (B * H * sage::round_up(Lq, 128) >= (int64_t(1) << 31) ||
+        B * Hk * sage::round_up(Lk, 128) >= (int64_t(1) << 31))
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(q4, 16) || !aligned(k4, 16) || !aligned(q_sf, 16) || !aligned(k_sf, 16) ||
+        !aligned(k_mean, 4) || !aligned(q_bf16.ptr, 2) || !aligned(k_bf16.ptr, 2))
+        return SAGE_ERR_ALIGNMENT;
+    const size_t need = sage::quant_qk_ws_bytes((int)B, (int)Hk, (int)Lk, (int)D);
+    if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return SAGE_ERR_ALIGNMENT;
+    int dev = -1;
+    if (!current_device(&dev)) return SAGE_ERR_CUDA;
+    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
+    return launch_status(sage::launch_quant_qk_mx(to_view(q_bf16), to_view(k_bf16), q4, q_sf, k4, k_sf,
+                                                  k_mean, ws, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_attn_fwd_mx(const uint8_t* q4, const uint8_t* q_sf, const uint8_t* k4,
+                             const uint8_t* k_sf, const uint8_t* v8_t, const float* v_scale, int B,
+                             int H, int Hk, int Lq, int Lk, int D, float softmax_scale, int causal,
+                             sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!q4 || !q_sf || !k4 || !k_sf || !v8_t || !v_scale || !out_bf16.ptr) return SAGE_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || Hk < 1 || Lq < 1 || Lk < 1 || D < 1) return SAGE_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(out_bf16.size, out_bf16.stride)) return SAGE_ERR_INVALID_ARG;
+    if (out_bf16.size[0] != B || out_bf16.size[1] != H || out_bf16.size[2] != Lq || out_bf16.size[3] != D)
+        return SAGE_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+    if (H % Hk != 0) return SAGE_ERR_UNSUPPORTED;
+    const int64_t nqt = sage::ceil_div(Lq, 128);
+    if ((int64_t)B * H > 65535 || nqt > 65535) return SAGE_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * sage::round_up(Lq, 128) >= (int64_t(1) << 31) ||
+        (int64_t)B * Hk * sage::round_up(Lk, 128) >= (int64_t(1) << 31) ||
+        (int64_t)B * Hk * D >= (int64_t(1) << 31))
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(q4, 16) || !aligned(k4, 16) || !aligned(q_sf, 16) || !aligned(k_sf, 16) ||
+        !aligned(v8_t, 16) || !aligned(v_scale, 4) || !aligned(out_bf16.ptr, 2))
+        return SAGE_ERR_ALIGNMENT;
+    sage::AttnMxArgs a;
+    a.q4 = q4;
+    a.q_sf = q_sf;
+    a.k4 = k4;
+    a.k_sf = k_sf;
+    a.v8t = v8_t;
+    a.v_scale = v_scale;
+    a.B = B;
+    a.H = H;
+    a.Hk = Hk;
+    a.Lq = Lq;
+    a.Lk = Lk;
+    a.D = D;
+    a.softmax_scale = softmax_scale;
+    a.causal = causal ? 1 : 0;
+    a.out = out_bf16.ptr;
+    for (int i = 0; i < 4; ++i) a.out_stride[i] = out_bf16.stride[i];
+    if (!sage::tensor_map_encoder()) return SAGE_ERR_CUDA;
+    return launch_status(sage::launch_attn_mx(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window) {
     if (B < 1 || T < 1 || H < 1 || Hk < 1 || D < 1 || window < 1) return 0;
     return sage::decode_ws_bytes(B, T, H, Hk, D, window);
@@ -456,12 +527,12 @@ sage_status sage_device_error_where(void* stream, int* kernel, int* site) {
     if (kernel) *kernel = 0;
     if (site) *site = 0;
     const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-    // error words of the kernels, in the order of SAGE_KERNEL_* ids 1, 2, 3
-    const unsigned words[3] = {sage::read_clear_attn_error(), sage::read_clear_decode_error(),
-                               sage::read_clear_probe_error()};
+    // error words of the kernels, in the order of SAGE_KERNEL_* ids 1, 2, 3, 4
+    const unsigned words[4] = {sage::read_clear_attn_error(), sage::read_clear_decode_error(),
+                               sage::read_clear_probe_error(), sage::read_clear_attn_mx_error()};
     if (e != cudaSuccess) return SAGE_ERR_CUDA;
     sage_status st = SAGE_OK;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const unsigned code = words[i] & 0xFFu;
         sage_status si = SAGE_OK;
         if (code == sage::kErrTimeoutCode) si = SAGE_ERR_TIMEOUT;

@@ -79,6 +79,10 @@ cudaError_t launch_quant_qkv(const View4& q, const View4& k, const View4& v, int
                              int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
                              uint8_t* v8t, float* v_scale, void* ws, cudaStream_t s);
 
+// Q and K as MXFP4 (E2M1 codes, e8m0 scales per 32 elements): two launches
+cudaError_t launch_quant_qk_mx(const View4& q, const View4& k, uint8_t* q4, uint8_t* q_sf, uint8_t* k4,
+                               uint8_t* k_sf, float* k_mean, void* ws, cudaStream_t s);
+
 // ---- attention forward (attn_fwd.cu)
 struct AttnArgs {
     const int8_t* q8;
@@ -100,6 +104,23 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_fwd(const AttnArgs& a, cudaStream_t s);
 unsigned read_clear_attn_error();
+
+// ---- MXFP4 attention forward (attn_mx.cu)
+struct AttnMxArgs {
+    const uint8_t* q4;
+    const uint8_t* q_sf;
+    const uint8_t* k4;
+    const uint8_t* k_sf;
+    const uint8_t* v8t;
+    const float* v_scale;
+    int B, H, Hk, Lq, Lk, D;
+    float softmax_scale;
+    int causal;
+    void* out;
+    int64_t out_stride[4];
+};
+cudaError_t launch_attn_mx(const AttnMxArgs& a, cudaStream_t s);
+unsigned read_clear_attn_mx_error();
 
 // ---- decode (decode.cu)
 struct DecodeArgs {
