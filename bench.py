@@ -443,6 +443,71 @@ def roofline_object(ops, attn_times, pk, pk_src, traffic):
             "attn_ms_p10_p50_p90": [pct(attn_times, 10), pct(attn_times, 50), pct(attn_times, 90)]}
 
 
+def bench_mx(sage, torch, key, steps, warmup, stream, pk, pk_src):
+    """The MXFP4 variant on one prefill workload: a step is sage_quant_qk_mx
+    + sage_quant_v + sage_attn_fwd_mx on inputs resident in HBM (rotating sets
+    larger than L2). The attention's roofline is the mixed peak of its work:
+    QK^T in FP4 (4 x the bf16 peak, nominal ratio), PV in FP8 (2 x)."""
+    import workloads
+    cfg, q, k, v = workloads.make_prefill_config(key)
+    B, H, Hk, L, D = cfg["B"], cfg["H"], cfg["Hk"], cfg["L"], cfg["D"]
+    h = sage.Hadamard(D)
+    set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + 2 * q.numel() * 2
+    sets = []
+    for _ in range(max(2, int(math.ceil(2 * L2_BYTES / set_bytes)))):
+        out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)
+        sets.append((q.cuda(), k.cuda(), v.cuda(), sage.MxBuffers(B, H, Hk, L, L, D), out))
+
+    def quant(i):
+        qs, ks, vs_, bf, _ = sets[i % len(sets)]
+        sage.sage_quant_qk_mx(h, qs, ks, bf.q4, bf.q_sf, bf.k4, bf.k_sf, bf.k_mean, bf.ws, stream)
+        sage.sage_quant_v(vs_, bf.v8_t, bf.v_scale, bf.ws_v, stream)
+
+    def attn(i):
+        _, _, _, bf, out = sets[i % len(sets)]
+        sage.sage_attn_fwd_mx(bf.q4, bf.q_sf, bf.k4, bf.k_sf, bf.v8_t, bf.v_scale, B, H, Hk, L, L, D,
+                              cfg["softmax_scale"], cfg["causal"], out, None, stream)
+
+    for i in range(warmup):
+        quant(i)
+        attn(i)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        quant(i)
+        ev[i][1].record(stream)
+        attn(i)
+        ev[i][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if sage.sage_device_error(stream) != sage.SAGE_OK:
+        raise RuntimeError("device error in the MXFP4 timing")
+    ms = t0.elapsed_time(t1) / steps
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    q_us = statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3
+    ops = work_ops(cfg)
+    p8 = pk["bf16_tflops"] * INT8_OVER_BF16
+    mixed = 2.0 / (1.0 / (2.0 * p8) + 1.0 / p8)       # half the ops at the FP4 rate, half at FP8
+    achieved = ops / (attn_ms * 1e-3) / 1e12
+    q_bytes = (q.numel() + k.numel()) * (2 + 0.5 + 1.0 / 32) + v.numel() * 3
+    del sets
+    torch.cuda.empty_cache()
+    return {"workload": cfg["name"], "value": ops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "steps": steps,
+            "roofline": {"bound": "tensor", "kernel": "attn_mx", "achieved": achieved, "peak": mixed,
+                         "unit": "TFLOP/s", "frac": achieved / mixed, "attn_ms": attn_ms,
+                         "peak_source": "%s bf16 burst x 4 for the FP4 QK half, x 2 for the FP8 PV half "
+                                        "(nominal ratios)" % pk_src},
+            "quant": {"us_per_call": q_us, "algorithmic_bytes": q_bytes,
+                      "achieved": q_bytes / (q_us * 1e-6) / 1e9, "unit": "GB/s", "peak": pk["hbm_gbs"],
+                      "frac": q_bytes / (q_us * 1e-6) / 1e9 / pk["hbm_gbs"],
+                      "bytes_rule": "Q, K: 2 B read + 0.5 B codes + 1/32 B scale per element; V: 2 + 1",
+                      "launches_per_call": 3}}
+
+
 def run_reference(args):
     import workloads
     rank = int(os.environ.get("RANK", "0"))
@@ -609,6 +674,12 @@ def run_sage(args):
             del epf
             torch.cuda.empty_cache()
 
+    mx = {}
+    if world == 1 and not args.no_extra:
+        for key in ("c4", "c2"):
+            mx[key] = bench_mx(sage, torch, key, max(args.steps, 10) if key == "c4" else 40,
+                               max(args.warmup, 3), stream, pk, pk_src)
+
     dec = None if args.no_decode else bench_decode(sage, torch, stream)
 
     cb = None
@@ -631,6 +702,7 @@ def run_sage(args):
             "e2e": e2e,
             "quant": quant,
             "configs": extra,
+            "mxfp4": mx,
             "decode": dec,
             "gpu_launches": (5 if args.fused_q else 3) * args.steps,
             "clocks": clk.summary(),
