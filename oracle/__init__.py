@@ -83,6 +83,11 @@ def lib():
                                          _f64p, _f64p]
         L.or_decode_quant_q_row.restype = None
         L.or_decode_quant_q_row.argtypes = [_u16p, ctypes.c_int, _u8p, _f32p]
+        L.or_decode_seq_flags.restype = None
+        L.or_decode_seq_flags.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                          _u16p, _f64p]
         L.or_decode_seq.restype = None
         L.or_decode_seq.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -308,10 +313,17 @@ def sage_attention(q, k, v, blk_q, blk_k, softmax_scale, causal, rows=None, thre
 
 # ---------------------------------------------------------------- decode
 
-def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, want_f64=False):
-    """Paged FP8 decode. q: uint16 [B, T, H, D]; kc, vc: uint8
-    [num_pages, Hk, page, D]; ksc, vsc: float32 [num_pages, Hk, page];
-    ptab: int32 [B, max_pages]; ctx: int32 [B]. Returns bf16 bits [B, T, H, D]."""
+KV_PER_TENSOR = 1       # ksc / vsc hold one scale each
+KV_V_TRANSPOSED = 2     # vc is [num_pages, Hk, D, page]
+
+
+def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, want_f64=False,
+           kv_flags=0):
+    """Paged FP8 decode. q: uint16 [B, T, H, D]; kc: uint8 [num_pages, Hk,
+    page, D]; vc: the same, or [num_pages, Hk, D, page] with KV_V_TRANSPOSED;
+    ksc, vsc: float32 [num_pages, Hk, page], or one value each with
+    KV_PER_TENSOR; ptab: int32 [B, max_pages]; ctx: int32 [B]. Returns bf16
+    bits [B, T, H, D]."""
     B, T, H, D = q.shape
     Hk, page = kc.shape[1], kc.shape[2]
     kc = np.ascontiguousarray(kc)
@@ -326,10 +338,10 @@ def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, 
         pt = np.ascontiguousarray(ptab[b], dtype=np.int32)
         oo = np.zeros((T, H, D), dtype=np.uint16)
         of = np.zeros((T, H, D), dtype=np.float64) if want_f64 else None
-        lib().or_decode_seq(_p(qq, _u16p), _p(kc, _u8p), _p(vc, _u8p), _p(ksc, _f32p),
-                            _p(vsc, _f32p), _p(pt, _i32p), int(ctx[b]), T, H, Hk, D, page,
-                            int(window), float(softmax_scale), _p(oo, _u16p),
-                            _p(of, _f64p) if want_f64 else None)
+        lib().or_decode_seq_flags(_p(qq, _u16p), _p(kc, _u8p), _p(vc, _u8p), _p(ksc, _f32p),
+                                  _p(vsc, _f32p), _p(pt, _i32p), int(ctx[b]), T, H, Hk, D, page,
+                                  int(window), float(softmax_scale), int(kv_flags), _p(oo, _u16p),
+                                  _p(of, _f64p) if want_f64 else None)
         out[b] = oo
         if want_f64:
             o64[b] = of

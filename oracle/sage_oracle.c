@@ -665,10 +665,20 @@ void or_decode_quant_q_row(const uint16_t* q, int D, uint8_t* codes, float* scal
     free(qh);
 }
 
-void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
-                   const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
-                   int page, int window, double softmax_scale, uint16_t* out, double* out_f64)
+/* kv_flags (the cache variants of [PA], Performance: "per-tensor and
+ * per-token scales"; Window-family results: "transposed V"):
+ *   bit 0: per-tensor scales -- ksc[0] and vsc[0] scale every cached token;
+ *   bit 1: transposed V -- vc is laid out [num_pages][Hk][D][page]. */
+#define OR_KV_PER_TENSOR 1
+#define OR_KV_V_TRANSPOSED 2
+
+void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
+                         const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
+                         int page, int window, double softmax_scale, int kv_flags, uint16_t* out,
+                         double* out_f64)
 {
+    const int per_tensor = (kv_flags & OR_KV_PER_TENSOR) != 0;
+    const int v_trans = (kv_flags & OR_KV_V_TRANSPOSED) != 0;
     uint8_t* qc = (uint8_t*)malloc((size_t)D);
     double* q8 = (double*)malloc(sizeof(double) * (size_t)D);
     double* o = (double*)malloc(sizeof(double) * (size_t)D);
@@ -692,7 +702,7 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
                 const int64_t tok = (phys * Hk + hk) * page + (j % page);
                 double acc = 0.0;
                 for (int e = 0; e < D; ++e) acc += q8[e] * or_e4m3_decode(kc[tok * D + e]);
-                sv[u] = acc * (double)s * (double)ksc[tok] * (softmax_scale / (double)D);
+                sv[u] = acc * (double)s * (double)ksc[per_tensor ? 0 : tok] * (softmax_scale / (double)D);
                 if (sv[u] > mx) mx = sv[u];
             }
             for (int e = 0; e < D; ++e) o[e] = 0.0;
@@ -705,9 +715,13 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
                 den += pj;
                 /* PV on bf16 operands: the weight p_j * v_scale_j is formed
                    in fp32 and rounded to bf16 (nearest even) */
-                const float wf = (float)pj * vsc[tok];
+                const float wf = (float)pj * vsc[per_tensor ? 0 : tok];
                 double w = (double)or_bf16_to_f32(or_f64_to_bf16((double)wf));
-                for (int e = 0; e < D; ++e) o[e] += w * or_e4m3_decode(vc[tok * D + e]);
+                for (int e = 0; e < D; ++e) {
+                    const int64_t vi = v_trans ? ((phys * Hk + hk) * D + e) * page + (j % page)
+                                               : tok * D + e;
+                    o[e] += w * or_e4m3_decode(vc[vi]);
+                }
             }
             for (int e = 0; e < D; ++e) {
                 double y = o[e] / den;
@@ -719,4 +733,12 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
     free(o);
     free(q8);
     free(qc);
+}
+
+void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
+                   const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
+                   int page, int window, double softmax_scale, uint16_t* out, double* out_f64)
+{
+    or_decode_seq_flags(q, kc, vc, ksc, vsc, ptab, ctx, T, H, Hk, D, page, window, softmax_scale, 0,
+                        out, out_f64);
 }

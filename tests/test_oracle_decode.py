@@ -131,3 +131,26 @@ def test_decode_query_codes_match_torch_float8(oracle_mod):
             assert np.array_equal(codes[idx], ref.view(torch.uint8).numpy())
             # the largest magnitude lands on 448 (code 0x7E, either sign)
             assert ((codes[idx] & 0x7F) == 0x7E).any()
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_decode_cache_variants_match_brute_force(oracle_mod, flags):
+    """Per-tensor scales (one K and one V scale for the whole cache) and the
+    transposed V cache ([num_pages, Hk, D, page]), the variants of the
+    FlyDSL pa_decode page's shape list: the oracle on the variant's layout
+    equals the brute force on the equivalent per-token, untransposed cache."""
+    d = workloads.make_decode(B=2, T=4, H=16, Hk=2, D=128, page=64, ctx_lo=200, ctx_hi=500, seed=31)
+    scale = 1.0 / math.sqrt(128)
+    ksc, vsc, vc = d["k_scale"].numpy(), d["v_scale"].numpy(), d["v_cache"].numpy()
+    if flags & 1:
+        ks1, vs1 = np.float32(0.0123), np.float32(0.0456)
+        d["k_scale"] = torch.full_like(d["k_scale"], float(ks1))
+        d["v_scale"] = torch.full_like(d["v_scale"], float(vs1))
+        ksc, vsc = np.array([ks1], dtype=np.float32), np.array([vs1], dtype=np.float32)
+    if flags & 2:
+        vc = np.ascontiguousarray(vc.transpose(0, 1, 3, 2))
+    out, o64 = oracle_mod.decode(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), vc, ksc, vsc,
+                                 d["page_table"].numpy(), d["ctx_lens"].numpy(), 128, scale,
+                                 want_f64=True, kv_flags=flags)
+    ref = _brute_decode(oracle_mod, d, 128, scale)
+    assert np.abs(o64 - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
