@@ -87,7 +87,9 @@ def lib():
         L.or_decode_seq_flags.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                          _u16p, _f64p]
+                                          _u16p, _f64p, _f64p]
+        L.or_bf16_flip_step.restype = ctypes.c_double
+        L.or_bf16_flip_step.argtypes = [ctypes.c_double, ctypes.c_double]
         L.or_decode_seq.restype = None
         L.or_decode_seq.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -318,35 +320,44 @@ KV_V_TRANSPOSED = 2     # vc is [num_pages, Hk, D, page]
 
 
 def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, want_f64=False,
-           kv_flags=0):
+           kv_flags=0, want_flip=False):
     """Paged FP8 decode. q: uint16 [B, T, H, D]; kc: uint8 [num_pages, Hk,
     page, D]; vc: the same, or [num_pages, Hk, D, page] with KV_V_TRANSPOSED;
     ksc, vsc: float32 [num_pages, Hk, page], or one value each with
     KV_PER_TENSOR; ptab: int32 [B, max_pages]; ctx: int32 [B]. Returns bf16
-    bits [B, T, H, D]."""
+    bits [B, T, H, D] (and the fp64 values, and with want_flip the margin of
+    the PV weights an fp32 evaluation may round to the neighbouring bf16)."""
     B, T, H, D = q.shape
     Hk, page = kc.shape[1], kc.shape[2]
+    want_f64 = want_f64 or want_flip
     kc = np.ascontiguousarray(kc)
     vc = np.ascontiguousarray(vc)
     ksc = np.ascontiguousarray(ksc, dtype=np.float32)
     vsc = np.ascontiguousarray(vsc, dtype=np.float32)
     out = np.zeros((B, T, H, D), dtype=np.uint16)
     o64 = np.zeros((B, T, H, D), dtype=np.float64) if want_f64 else None
+    flip = np.zeros((B, T, H, D), dtype=np.float64) if want_flip else None
 
     def one(b):
         qq = np.ascontiguousarray(q[b])
         pt = np.ascontiguousarray(ptab[b], dtype=np.int32)
         oo = np.zeros((T, H, D), dtype=np.uint16)
         of = np.zeros((T, H, D), dtype=np.float64) if want_f64 else None
+        ff = np.zeros((T, H, D), dtype=np.float64) if want_flip else None
         lib().or_decode_seq_flags(_p(qq, _u16p), _p(kc, _u8p), _p(vc, _u8p), _p(ksc, _f32p),
                                   _p(vsc, _f32p), _p(pt, _i32p), int(ctx[b]), T, H, Hk, D, page,
                                   int(window), float(softmax_scale), int(kv_flags), _p(oo, _u16p),
-                                  _p(of, _f64p) if want_f64 else None)
+                                  _p(of, _f64p) if want_f64 else None,
+                                  _p(ff, _f64p) if want_flip else None)
         out[b] = oo
         if want_f64:
             o64[b] = of
+        if want_flip:
+            flip[b] = ff
 
     _pool_map(one, list(range(B)), threads)
+    if want_flip:
+        return out, o64, flip
     return (out, o64) if want_f64 else out
 
 

@@ -404,6 +404,25 @@ double or_e4m3_flip_step(double v, double delta)
     return st;
 }
 
+/* The same for the bf16 rounding of a value v >= 0 (the decode's PV
+ * weights): the distance to the neighbouring bf16 value when v perturbed
+ * by up to delta (relative) could round there; else 0. */
+double or_bf16_flip_step(double v, double delta)
+{
+    const uint16_t b = or_f64_to_bf16(v);
+    const double here = (double)or_bf16_to_f32(b);
+    double st = 0.0;
+    if (b < 0x7F7F) {
+        const double up = (double)or_bf16_to_f32((uint16_t)(b + 1));
+        if (v * (1.0 + delta) >= 0.5 * (here + up)) st = up - here;
+    }
+    if (b > 0) {
+        const double dn = (double)or_bf16_to_f32((uint16_t)(b - 1));
+        if (v * (1.0 - delta) <= 0.5 * (here + dn) && here - dn > st) st = here - dn;
+    }
+    return st;
+}
+
 /* ------------------------------------------------------------------ */
 /* Quantised attention, one (b,h), selected query rows ([S2TP] order)  */
 /* ------------------------------------------------------------------ */
@@ -672,16 +691,22 @@ void or_decode_quant_q_row(const uint16_t* q, int D, uint8_t* codes, float* scal
 #define OR_KV_PER_TENSOR 1
 #define OR_KV_V_TRANSPOSED 2
 
+/* flip_f64 (optional): per output element, how far an fp32 evaluation of
+ * the weights may land from out_f64 through weights that round to the
+ * neighbouring bf16 value: the sum over the keys whose fp32 weight lies
+ * within or_p_fp32_delta of a bf16 rounding midpoint of step * |v| / sum p
+ * (as or_attn_head's margin for the e4m3 P codes). */
 void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
                          const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
                          int page, int window, double softmax_scale, int kv_flags, uint16_t* out,
-                         double* out_f64)
+                         double* out_f64, double* flip_f64)
 {
     const int per_tensor = (kv_flags & OR_KV_PER_TENSOR) != 0;
     const int v_trans = (kv_flags & OR_KV_V_TRANSPOSED) != 0;
     uint8_t* qc = (uint8_t*)malloc((size_t)D);
     double* q8 = (double*)malloc(sizeof(double) * (size_t)D);
     double* o = (double*)malloc(sizeof(double) * (size_t)D);
+    double* F = (double*)malloc(sizeof(double) * (size_t)D);
     double* sv = (double*)malloc(sizeof(double) * (size_t)(window > 0 ? window : 1));
     const int group = H / Hk;
     for (int t = 0; t < T; ++t)
@@ -705,7 +730,7 @@ void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc
                 sv[u] = acc * (double)s * (double)ksc[per_tensor ? 0 : tok] * (softmax_scale / (double)D);
                 if (sv[u] > mx) mx = sv[u];
             }
-            for (int e = 0; e < D; ++e) o[e] = 0.0;
+            for (int e = 0; e < D; ++e) o[e] = F[e] = 0.0;
             double den = 0.0;
             for (int u = 0; u < n; ++u) {
                 const int j = lo + u;
@@ -717,19 +742,23 @@ void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc
                    in fp32 and rounded to bf16 (nearest even) */
                 const float wf = (float)pj * vsc[per_tensor ? 0 : tok];
                 double w = (double)or_bf16_to_f32(or_f64_to_bf16((double)wf));
+                const double st = flip_f64 ? or_bf16_flip_step((double)wf, or_p_fp32_delta(sv[u], mx)) : 0.0;
                 for (int e = 0; e < D; ++e) {
                     const int64_t vi = v_trans ? ((phys * Hk + hk) * D + e) * page + (j % page)
                                                : tok * D + e;
                     o[e] += w * or_e4m3_decode(vc[vi]);
+                    if (st > 0.0) F[e] += st * fabs(or_e4m3_decode(vc[vi]));
                 }
             }
             for (int e = 0; e < D; ++e) {
                 double y = o[e] / den;
                 out[((int64_t)t * H + h) * D + e] = or_f64_to_bf16(y);
                 if (out_f64) out_f64[((int64_t)t * H + h) * D + e] = y;
+                if (flip_f64) flip_f64[((int64_t)t * H + h) * D + e] = F[e] / den;
             }
         }
     free(sv);
+    free(F);
     free(o);
     free(q8);
     free(qc);
@@ -740,5 +769,5 @@ void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, cons
                    int page, int window, double softmax_scale, uint16_t* out, double* out_f64)
 {
     or_decode_seq_flags(q, kc, vc, ksc, vsc, ptab, ctx, T, H, Hk, D, page, window, softmax_scale, 0,
-                        out, out_f64);
+                        out, out_f64, NULL);
 }
