@@ -285,11 +285,19 @@ sage_status sage_attn_fwd_mx(const uint8_t* q4, const uint8_t* q_sf, const uint8
 /* Bytes of device workspace sage_attn_decode needs (split-KV partials). */
 size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window);
 
+/* Cache variants of sage_attn_decode ("[FlyDSL] [Misc] pa_decode ...",
+ * Performance: FP8 KV with per-tensor and per-token scales; Window-family
+ * results: transposed V), OR-ed into kv_flags. */
+#define SAGE_KV_PER_TENSOR_SCALES 1   /* k_scale / v_scale point to one fp32 each */
+#define SAGE_KV_V_TRANSPOSED 2        /* v_cache is [num_pages, Hk, D, page], page 128 */
+
 /* Paged FP8-KV decode with MTP query tokens and a sliding window.
  *   q_bf16: [B, T, H, D] bf16 view (the T query tokens are the last T
  *   positions of each sequence); k_cache, v_cache: e4m3 codes
- *   [num_pages, Hk, page_size, D] contiguous; k_scale, v_scale: fp32 per
- *   token [num_pages, Hk, page_size]; page_table: int32 [B, max_pages]
+ *   [num_pages, Hk, page_size, D] contiguous (v_cache [num_pages, Hk, D,
+ *   page_size] with SAGE_KV_V_TRANSPOSED); k_scale, v_scale: fp32 per token
+ *   [num_pages, Hk, page_size] (one fp32 each with SAGE_KV_PER_TENSOR_SCALES);
+ *   page_table: int32 [B, max_pages]
  *   logical -> physical page; ctx_lens: int32 [B], T <= ctx <= max_pages *
  *   page_size. The cache holds keys already in the rotated domain.
  * For token t (position p = ctx - T + t) and head h: q_hat = butterfly(q)
@@ -301,13 +309,14 @@ size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window
  * q_scale_out (nullable): their scales s_q, contiguous fp32 [B, T, H] (the
  * codes the QK product used, for callers that reuse them or check them).
  * Supported: D == 128, page_size in {16, 32, 64, 128}, H % Hk == 0,
- * H / Hk <= 16, T * (H / Hk) <= 64, window >= 1. ws: at least
- * sage_attn_decode_workspace(...) bytes. */
+ * H / Hk <= 16, T * (H / Hk) <= 64, window >= 1; SAGE_KV_V_TRANSPOSED
+ * needs page_size 128 (UNSUPPORTED otherwise), unknown kv_flags bits are
+ * INVALID_ARG. ws: at least sage_attn_decode_workspace(...) bytes. */
 sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
                              const uint8_t* v_cache, const float* k_scale, const float* v_scale,
                              const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
                              int H, int Hk, int D, int page_size, int max_pages, int num_pages,
-                             int window, float softmax_scale, sage_view4 out_bf16,
+                             int window, float softmax_scale, int kv_flags, sage_view4 out_bf16,
                              uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
                              void* stream);
 

@@ -39,6 +39,8 @@ SAGE_KERNEL_ATTN = 1
 SAGE_KERNEL_DECODE = 2
 SAGE_KERNEL_PROBE = 3
 SAGE_KERNEL_ATTN_MX = 4
+SAGE_KV_PER_TENSOR_SCALES = 1
+SAGE_KV_V_TRANSPOSED = 2
 
 
 class SageError(RuntimeError):
@@ -104,7 +106,7 @@ def lib():
     L.sage_attn_decode_workspace.argtypes = [i32] * 6
     L.sage_attn_decode.restype = i32
     L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 9 + \
-        [f32, View4, vp, vp, vp, sz, vp]
+        [f32, i32, View4, vp, vp, vp, sz, vp]
     L.sage_device_error.restype = i32
     L.sage_device_error.argtypes = [vp]
     L.sage_device_error_where.restype = i32
@@ -266,14 +268,14 @@ def sage_attn_fwd(q8, q_scale, k8, k_scale, v8_t, v_scale, B, H, Hk, Lq, Lk, D, 
 
 def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_lens, page_size,
                      num_pages, window, softmax_scale, out, ws=None, stream=None, q8_out=None,
-                     q_scale_out=None):
+                     q_scale_out=None, kv_flags=0):
     B, T, H, D = q.shape
     Hk = k_cache.shape[1]
     max_pages = page_table.shape[1]
     _check(lib().sage_attn_decode(h.handle, _view(q, CView4), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(k_scale), _ptr(v_scale), _ptr(page_table), _ptr(ctx_lens),
                                   B, T, H, Hk, D, int(page_size), int(max_pages), int(num_pages),
-                                  int(window), float(softmax_scale), _view(out, View4),
+                                  int(window), float(softmax_scale), int(kv_flags), _view(out, View4),
                                   _ptr(q8_out), _ptr(q_scale_out), _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "sage_attn_decode")

@@ -121,6 +121,8 @@ struct DecParams {
     int64_t os0, os1, os2, os3;
     uint8_t* q8_out;                         // optional: e4m3 query codes [B, T, H, D]
     float* qs_out;                           // optional: query scales [B, T, H]
+    int per_tensor;                          // ksc / vsc hold one scale each
+    int v_trans;                             // V cache [num_pages, Hk, D, page] (page 128)
 };
 
 // The A operand (P') of the PV MMA holds a row's 128 keys in this order:
@@ -237,6 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
         }
+        const float ks_tensor = p.per_tensor ? __ldg(p.ksc) : 0.0f;
+        const float vs_tensor = p.per_tensor ? __ldg(p.vsc) : 0.0f;
         // physical pages of the CTA's logical pages tb * ppt + 32 c + lane,
         // fetched 32 at a time; pages holding no key of [lo, ctx) are not
         // looked up (page 0 stands in; their keys are masked)
@@ -283,8 +287,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // per-token scales of keys 4 lane .. 4 lane + 3, stored by key
-            // parity (index (key & 1) * 64 + key / 2) for the softmax threads
-            {
+            // parity (index (key & 1) * 64 + key / 2) for the softmax threads;
+            // with per-tensor scales the one K and one V scale in every slot
+            if (p.per_tensor) {
+                float* dst = scl + s * 2 * kKeys;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    dst[4 * lane + e] = ks_tensor;
+                    dst[kKeys + 4 * lane + e] = vs_tensor;
+                }
+                mbar_arrive(&bars[Sm::kKvFull + s]);
+            } else {
                 const int kq = 4 * lane;
                 const int pq = __shfl_sync(0xffffffffu, phys, kq / p.page);
                 const int64_t src = ((int64_t)pq * p.Hk + hk) * p.page + (kq % p.page);
@@ -307,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && nt > 0) {
             constexpr uint32_t kIdescQK = umma_idesc(1, 0, kRows, kKeys);              // e4m3 -> f32
             constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, 64) | (1u << 16);    // bf16, B MN-major
+            constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, 64);                // bf16, B K-major
             const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), 128);
             bool ok = mbar_wait(&bars[Sm::kQReady], 0, abort_flag, &g_decode_err, 12);
             for (int i = 0; ok && i <= nt; ++i) {
@@ -335,14 +349,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
                     const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
+                    if (!p.v_trans) {
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf)
+                        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                        for (int st = 0; st < kKeys / 16; ++st)
-                            mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
-                                        umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
-                                        umma_desc_kmajor(vb + hf * (kKeys * 128), 128) + 128 * st,
-                                        kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
+                            for (int st = 0; st < kKeys / 16; ++st)
+                                mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
+                                            umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
+                                            umma_desc_kmajor(vb + hf * (kKeys * 128), 128) + 128 * st,
+                                            kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
+                    } else {
+                        // V^T converted K-major: 64-key atoms of [128 channels][128 B]
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                            for (int st = 0; st < kKeys / 16; ++st)
+                                mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
+                                            umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
+                                            umma_desc_kmajor(vb + (st >> 2) * (kD * 128) + hf * (64 * 128), 128) +
+                                                2 * (st & 3),
+                                            kIdescPVT, (j > 1 || st > 0) ? 1u : 0u);
+                    }
                     mma_commit(&bars[Sm::kPvDone + (j & 1)]);
                 }
             }
@@ -712,6 +739,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = warp_all(mbar_wait(&bars[Sm::kPvDone + bf], ((i - 2) >> 1) & 1, abort_flag,
                                         &g_decode_err, 11));
             if (!ok) break;
+            if (p.v_trans) {
+                // V^T tile [128 channels][128 keys]: lane -> channel row d; its
+                // keys become the row of a K-major bf16 operand in the key order
+                // of P' (per 16 keys: the even keys, then the odd ones)
+                const int d = 32 * cw + lane;
+                const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + d * 128;
+                uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + d * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {       // keys 16c .. 16c + 15
+                    const uint4 u = *reinterpret_cast<const uint4*>(vrow + ((c ^ (d & 7)) << 4));
+                    const uint32_t e0 = e4m3x2_to_bf16x2(u.x, 0x2404u), e1 = e4m3x2_to_bf16x2(u.y, 0x2404u);
+                    const uint32_t e2 = e4m3x2_to_bf16x2(u.z, 0x2404u), e3 = e4m3x2_to_bf16x2(u.w, 0x2404u);
+                    const uint32_t d0 = e4m3x2_to_bf16x2(u.x, 0x3414u), d1 = e4m3x2_to_bf16x2(u.y, 0x3414u);
+                    const uint32_t d2 = e4m3x2_to_bf16x2(u.z, 0x3414u), d3 = e4m3x2_to_bf16x2(u.w, 0x3414u);
+                    uint8_t* atom = dst + (c >> 2) * (kD * 128);
+                    const int g2 = 2 * (c & 3);
+                    *reinterpret_cast<uint4*>(atom + ((g2 ^ (d & 7)) << 4)) = make_uint4(e0, e1, e2, e3);
+                    *reinterpret_cast<uint4*>(atom + (((g2 + 1) ^ (d & 7)) << 4)) = make_uint4(d0, d1, d2, d3);
+                }
+            } else {
             const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + kap * 128;
             uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + pos * 128;
 #pragma unroll
@@ -725,6 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ch = 2 * (c & 3);
                 *reinterpret_cast<uint4*>(half + ((ch ^ (pos & 7)) << 4)) = make_uint4(o0, o1, o2, o3);
                 *reinterpret_cast<uint4*>(half + (((ch + 1) ^ (pos & 7)) << 4)) = make_uint4(o4, o5, o6, o7);
+            }
             }
             fence_proxy_async_smem();               // read by the PV MMAs
             __syncwarp();
@@ -754,6 +802,22 @@ bool encode_cache(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int 
                                 static_cast<cuuint64_t>(num_pages) * Hk};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(page) * kD};
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(page), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The transposed V cache [num_pages, Hk, 128, page = 128] as a 3-D map
+// {128 key bytes, 128 channel rows, num_pages * Hk}; one box = one page of
+// one kv head as [channel][key], 128B swizzle.
+bool encode_cache_vt(CUtensorMap* map, const void* ptr, int num_pages, int Hk) {
+    auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(kD),
+                                static_cast<cuuint64_t>(num_pages) * Hk};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(kD) * kKeys};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kKeys), static_cast<cuuint32_t>(kD), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -845,13 +909,16 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     p.os3 = a.out_stride[3];
     p.q8_out = a.q8_out;
     p.qs_out = a.q_scale_out;
+    p.per_tensor = (a.kv_flags & 1) ? 1 : 0;
+    p.v_trans = (a.kv_flags & 2) ? 1 : 0;
     p.q_vec = (a.q.stride[3] == 1 && a.q.stride[0] % 8 == 0 && a.q.stride[1] % 8 == 0 &&
                a.q.stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.q.ptr) % 16 == 0)
                   ? 1
                   : 0;
     CUtensorMap tk, tv;
     if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size) ||
-        !encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size))
+        !(p.v_trans ? encode_cache_vt(&tv, a.v_cache, a.num_pages, a.Hk)
+                    : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size)))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

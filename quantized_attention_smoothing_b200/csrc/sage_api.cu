@@ -466,7 +466,7 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
                              const uint8_t* v_cache, const float* k_scale, const float* v_scale,
                              const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
                              int H, int Hk, int D, int page_size, int max_pages, int num_pages,
-                             int window, float softmax_scale, sage_view4 out_bf16,
+                             int window, float softmax_scale, int kv_flags, sage_view4 out_bf16,
                              uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
                              void* stream) {
     if (!h || !q_bf16.ptr || !k_cache || !v_cache || !k_scale || !v_scale || !page_table ||
@@ -485,6 +485,8 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
     if (H % Hk != 0 || H / Hk > 16 || T * (H / Hk) > 64) return SAGE_ERR_UNSUPPORTED;
     if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
         return SAGE_ERR_UNSUPPORTED;
+    if (kv_flags & ~(SAGE_KV_PER_TENSOR_SCALES | SAGE_KV_V_TRANSPOSED)) return SAGE_ERR_INVALID_ARG;
+    if ((kv_flags & SAGE_KV_V_TRANSPOSED) && page_size != 128) return SAGE_ERR_UNSUPPORTED;
     if ((int64_t)num_pages * Hk * page_size * D >= (int64_t(1) << 40)) return SAGE_ERR_UNSUPPORTED;
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_scale, 4) ||
         !aligned(v_scale, 4) || !aligned(page_table, 4) || !aligned(ctx_lens, 4) ||
@@ -520,6 +522,7 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
     a.ws = ws;
     a.q8_out = q8_out;
     a.q_scale_out = q_scale_out;
+    a.kv_flags = kv_flags;
     return launch_status(sage::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

@@ -138,6 +138,7 @@ struct DecodeArgs {
     void* ws;
     uint8_t* q8_out;           // optional [B, T, H, D] e4m3 query codes
     float* q_scale_out;        // optional [B, T, H] query scales
+    int kv_flags;              // SAGE_KV_PER_TENSOR_SCALES | SAGE_KV_V_TRANSPOSED
 };
 size_t decode_ws_bytes(int B, int T, int H, int Hk, int D, int window);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

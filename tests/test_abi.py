@@ -145,7 +145,7 @@ def test_decode_validation_without_gpu(L):
     p = ctypes.c_void_p(0x10000)
     q = _cview(size=(2, 4, 16, 128))
     out = _view(0x20000, (2, 4, 16, 128))
-    args = [q, p, p, p, p, p, p, 2, 4, 16, 1, 128, 128, 64, 100, 4096, 0.088, out, None, None, p,
+    args = [q, p, p, p, p, p, p, 2, 4, 16, 1, 128, 128, 64, 100, 4096, 0.088, 0, out, None, None, p,
             1 << 30, None]
     # null handle
     assert L.sage_attn_decode(None, *args) == sage.SAGE_ERR_INVALID_ARG
