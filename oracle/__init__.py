@@ -88,8 +88,6 @@ def lib():
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
                                           _u16p, _f64p, _f64p]
-        L.or_bf16_flip_step.restype = ctypes.c_double
-        L.or_bf16_flip_step.argtypes = [ctypes.c_double, ctypes.c_double]
         L.or_decode_seq.restype = None
         L.or_decode_seq.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,

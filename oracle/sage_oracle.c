@@ -404,25 +404,6 @@ double or_e4m3_flip_step(double v, double delta)
     return st;
 }
 
-/* The same for the bf16 rounding of a value v >= 0 (the decode's PV
- * weights): the distance to the neighbouring bf16 value when v perturbed
- * by up to delta (relative) could round there; else 0. */
-double or_bf16_flip_step(double v, double delta)
-{
-    const uint16_t b = or_f64_to_bf16(v);
-    const double here = (double)or_bf16_to_f32(b);
-    double st = 0.0;
-    if (b < 0x7F7F) {
-        const double up = (double)or_bf16_to_f32((uint16_t)(b + 1));
-        if (v * (1.0 + delta) >= 0.5 * (here + up)) st = up - here;
-    }
-    if (b > 0) {
-        const double dn = (double)or_bf16_to_f32((uint16_t)(b - 1));
-        if (v * (1.0 - delta) <= 0.5 * (here + dn) && here - dn > st) st = here - dn;
-    }
-    return st;
-}
-
 /* ------------------------------------------------------------------ */
 /* Quantised attention, one (b,h), selected query rows ([S2TP] order)  */
 /* ------------------------------------------------------------------ */
@@ -691,11 +672,14 @@ void or_decode_quant_q_row(const uint16_t* q, int D, uint8_t* codes, float* scal
 #define OR_KV_PER_TENSOR 1
 #define OR_KV_V_TRANSPOSED 2
 
-/* flip_f64 (optional): per output element, how far an fp32 evaluation of
- * the weights may land from out_f64 through weights that round to the
- * neighbouring bf16 value: the sum over the keys whose fp32 weight lies
- * within or_p_fp32_delta of a bf16 rounding midpoint of step * |v| / sum p
- * (as or_attn_head's margin for the e4m3 P codes). */
+/* flip_f64 (optional): per output element, how far an implementation may
+ * land from out_f64 through the bf16 rounding of the weights: one that keeps
+ * a running maximum over key tiles and splits rounds each weight p_j vsc_j
+ * at the scale of the maximum it has seen so far and rescales afterwards,
+ * not at the window maximum used here. Both roundings are within half a
+ * bf16 step of the exact weight: half this rounding's step (known) plus at
+ * most 2^-8 of the weight for the other, so the bound is
+ * sum_j (ulp(w_j) / 2 + 2^-8 w_j) |v_j| / sum p. */
 void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
                          const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
                          int page, int window, double softmax_scale, int kv_flags, uint16_t* out,
@@ -741,13 +725,15 @@ void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc
                 /* PV on bf16 operands: the weight p_j * v_scale_j is formed
                    in fp32 and rounded to bf16 (nearest even) */
                 const float wf = (float)pj * vsc[per_tensor ? 0 : tok];
-                double w = (double)or_bf16_to_f32(or_f64_to_bf16((double)wf));
-                const double st = flip_f64 ? or_bf16_flip_step((double)wf, or_p_fp32_delta(sv[u], mx)) : 0.0;
+                const uint16_t wb = or_f64_to_bf16((double)wf);
+                double w = (double)or_bf16_to_f32(wb);
+                const double wmar = flip_f64 ? 0.5 * ((double)or_bf16_to_f32((uint16_t)(wb + 1)) - w) + ldexp(w, -8)
+                                             : 0.0;
                 for (int e = 0; e < D; ++e) {
                     const int64_t vi = v_trans ? ((phys * Hk + hk) * D + e) * page + (j % page)
                                                : tok * D + e;
                     o[e] += w * or_e4m3_decode(vc[vi]);
-                    if (st > 0.0) F[e] += st * fabs(or_e4m3_decode(vc[vi]));
+                    if (flip_f64) F[e] += wmar * fabs(or_e4m3_decode(vc[vi]));
                 }
             }
             for (int e = 0; e < D; ++e) {
