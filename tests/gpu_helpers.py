@@ -8,8 +8,9 @@ oracle reports one, the margin of the P codes that an fp32 evaluation of
 448 p may round the other way (the scores are fp32 before the FP8 cast, and
 a code whose exact value lies within fp32 error of an e4m3 rounding midpoint
 can land on either side; the oracle gives the effect of moving each such
-code by one step) -- for the decode, of the bf16 PV weights p * v_scale that
-may round to the neighbouring bf16 value the same way. The cosine against the oracle must be >= 0.9999 and
+code by one step) -- for the decode, the bound on the bf16 PV weights
+p * v_scale, which a kernel with running maxima rounds at other scales than
+the oracle's window maximum. The cosine against the oracle must be >= 0.9999 and
 against unquantised fp64 attention >= 0.998. Every comparison reports how
 many elements needed the margin.
 """

@@ -126,12 +126,11 @@ def test_decode_dominant_keys(h128):
     """Keys whose k_scale is multiplied by 40, spread over the window, give
     logits far above the running maximum in later tiles of a split (O is
     rescaled in TMEM there) and rows dominated by one key. Both sides round
-    every PV weight w_j = p_j * v_scale_j to bf16 but evaluate p_j in
-    different precisions (fp32 exp2 of fp32 logits against fp64 exp), so a
-    weight within fp32 error of a bf16 rounding midpoint can land one bf16
-    step apart: the oracle's margin gives the effect of exactly those
-    weights. Rows where no single key carries a tenth of the weight must meet
-    the plain bar."""
+    every PV weight w_j = p_j * v_scale_j to bf16, but the kernel rounds it
+    at the running maximum of its tile and split and rescales afterwards,
+    the oracle at the window maximum: the oracle's margin bounds the effect
+    (each weight within half a bf16 step on either side). Rows where no
+    single key carries a tenth of the weight must meet the plain bar."""
     d = workloads.make_decode(B=4, T=4, H=16, Hk=1, D=128, page=128, ctx_lo=3000, ctx_hi=5000,
                               seed=4242)
     ksc = d["k_scale"].clone()
@@ -151,12 +150,12 @@ def test_decode_dominant_keys(h128):
     ulp = bf16_ulp(np.maximum(np.abs(g), np.abs(ref)))
     plain = np.abs(g - ref) - ulp / 2
     # rows where no single key carries a tenth of the weight meet the plain
-    # bar; only rows dominated by a few keys may use the extra term
+    # bar; only rows dominated by a few keys may use the margin
     spread = np.broadcast_to((share < 0.1)[..., None], plain.shape)
     assert float(plain[spread].max()) <= MAX_ABS, float(plain[spread].max())
     n_extra = int((plain > MAX_ABS).sum())
     print("dominant keys: %d of %d rows dominated (a key >= 10%% of the weight); %d of %d "
-          "elements need the bf16 weight-rounding term" % (int((share >= 0.1).sum()), share.size,
+          "elements need the bf16 weight-rounding margin" % (int((share >= 0.1).sum()), share.size,
                                                              n_extra, plain.size))
 
 
@@ -199,41 +198,36 @@ def test_decode_reports_bad_page_ids(h128):
     (3, 2, 8, 2, 100, 900, 512),           # GQA 4, short contexts, T = 2
 ])
 def test_decode_cache_variants(h128, flags, B, T, H, Hk, lo, hi, window):
-    """Per-tensor K/V scales (SAGE_KV_PER_TENSOR_SCALES) and the transposed V
-    cache (SAGE_KV_V_TRANSPOSED, [num_pages, Hk, D, 128]), alone and
-    together, against the oracle on the same layout; with per-tensor scales
-    the output equals the per-token path given the same scale in every slot,
-    bit for bit, and the transposed cache gives the untransposed one's bits."""
+    """Per-tensor K/V scales (SAGE_KV_PER_TENSOR_SCALES: a cache quantised
+    with one amax / 448 scale per tensor) and the transposed V cache
+    (SAGE_KV_V_TRANSPOSED, [num_pages, Hk, D, 128]), alone and together,
+    against the oracle on the same layout; and bit for bit against the
+    default layout given the same data (the per-tensor scale repeated in
+    every per-token slot, V untransposed)."""
     d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=128, page=128, ctx_lo=lo, ctx_hi=hi,
-                              seed=B * 7 + flags)
+                              seed=B * 7 + flags, scale_mode="per_tensor" if flags & 1 else "per_token")
     scale = 1.0 / math.sqrt(128)
     q = d["q"].cuda()
     out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty((16,), dtype=torch.uint8, device="cuda")
     ksc, vsc, vc = d["k_scale"], d["v_scale"], d["v_cache"]
-    if flags & 1:
-        ksc1 = torch.tensor([0.0117], dtype=torch.float32)
-        vsc1 = torch.tensor([0.0391], dtype=torch.float32)
-        d["k_scale"] = torch.full_like(ksc, float(ksc1))
-        d["v_scale"] = torch.full_like(vsc, float(vsc1))
-        ksc, vsc = ksc1, vsc1
+    kfull = ksc.expand(d["k_cache"].shape[:3]).contiguous() if flags & 1 else ksc
+    vfull = vsc.expand(d["k_cache"].shape[:3]).contiguous() if flags & 1 else vsc
     if flags & 2:
         vc = vc.permute(0, 1, 3, 2).contiguous()
     tabs = [d["page_table"].cuda(), d["ctx_lens"].cuda()]
     sage.sage_attn_decode(h128, q, d["k_cache"].cuda(), vc.cuda(), ksc.cuda(), vsc.cuda(), tabs[0], tabs[1],
                           128, d["num_pages"], window, scale, out, ws, kv_flags=flags)
-    # the same data in the default layout (per-token scales, untransposed V)
     ref_out = torch.empty_like(out)
-    sage.sage_attn_decode(h128, q, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(),
-                          d["v_scale"].cuda(), tabs[0], tabs[1], 128, d["num_pages"], window, scale,
-                          ref_out, ws)
+    sage.sage_attn_decode(h128, q, d["k_cache"].cuda(), d["v_cache"].cuda(), kfull.cuda(), vfull.cuda(),
+                          tabs[0], tabs[1], 128, d["num_pages"], window, scale, ref_out, ws)
     torch.cuda.synchronize()
     assert sage.sage_device_error() == sage.SAGE_OK
+    assert torch.equal(out, ref_out)
     _, ref, margin = oracle.decode(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), vc.numpy(),
                                    ksc.numpy(), vsc.numpy(), d["page_table"].numpy(),
                                    d["ctx_lens"].numpy(), window, scale, want_flip=True, kv_flags=flags)
     compare_output(bits(out), (ref, margin), None, label="kv_flags %d %s" % (flags, (B, T, H, Hk)))
-    assert torch.equal(out, ref_out)
 
 
 def test_decode_rejects_bad_kv_flags(h128):

@@ -103,14 +103,16 @@ def make_prefill_config(key, layout="blhd", seed=None):
     return cfg, q, k, v
 
 
-def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, **_unused):
+def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, scale_mode="per_token", **_unused):
     """Paged FP8 decode inputs.
 
     ctx_b ~ U{ctx_lo..ctx_hi}; the pages of all sequences are one random
     permutation of the physical pages. Cached K/V values are N(0, 1) and
-    stored as e4m3 codes with one fp32 scale per token (amax / 448), the cast
-    done by torch's float8_e4m3fn conversion (the cache writer itself is not
-    part of the path). Queries are bf16 N(0, 1), [B, T, H, D].
+    stored as e4m3 codes with one fp32 scale per token (amax / 448), or with
+    scale_mode="per_tensor" one scale for the whole cache (its amax / 448;
+    k_scale and v_scale are then one-element tensors), the cast done by
+    torch's float8_e4m3fn conversion (the cache writer itself is not part of
+    the path). Queries are bf16 N(0, 1), [B, T, H, D].
     Returns a dict of CPU tensors.
     """
     g = torch.Generator().manual_seed(int(seed))
@@ -127,6 +129,10 @@ def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, **_unused):
 
     def cache():
         x = torch.randn((total, Hk, page, D), generator=g)
+        if scale_mode == "per_tensor":
+            scale = (x.abs().amax() / 448.0).reshape(1)
+            codes = (x / scale).to(torch.float8_e4m3fn).view(torch.uint8)
+            return codes.contiguous(), scale.to(torch.float32).contiguous()
         amax = x.abs().amax(dim=-1)
         scale = amax / 448.0
         codes = (x / scale.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
