@@ -61,18 +61,21 @@ constexpr unsigned kErrDecodeRange = kErrRangeCode;   // ctx or page id out of r
 constexpr int kD = 128;
 constexpr int kKeys = 128;                   // keys per tile
 constexpr int kRows = 64;                    // query rows per CTA (M of every MMA)
-constexpr int kStages = 3;                   // K / V / scale ring
+constexpr int kStages = 3;                   // K / V ring
+constexpr int kScStages = 8;                 // per-token scale ring (freed by the softmax alone)
 constexpr int kMaxSplit = 8;                 // CTAs per (sequence, kv head) = cluster size
 constexpr int kSoftWarps = 8;                // warps 0..7
 constexpr int kConvWarp0 = 8;                // warps 8..11
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;                 // warps 14, 15 idle until the merge
 constexpr int kThreads = 512;
-// registers per thread of each warpgroup (setmaxnreg; 256 x 192 + 128 x 64 +
-// 128 x 56 <= 512 x 128, the launch's registers). Only the softmax warps ever
-// grow their share, after the others have shrunk theirs, and no warp grows
-// it again later: a warp that did could take registers another one waits for.
-constexpr int kRegsSoft = 192, kRegsConv = 64, kRegsProd = 56;
+// registers per thread of each warpgroup (setmaxnreg; 256 x 176 + 128 x 96 +
+// 128 x 56 <= 512 x 128, the launch's registers; this split compiles without
+// spills). Only the softmax warps ever grow their share, after the others
+// have shrunk theirs, and no warp grows it again later: a warp that did
+// could take registers another one waits for.
+constexpr int kRegsSoft = 176, kRegsConv = 96, kRegsProd = 56;
+static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kOcPitch = kD + 4;             // fp32 row pitch of the merge area
 
@@ -86,15 +89,16 @@ struct Sm {
     static constexpr int kP = kV + kStages * kKStage;              // [2 bufs] P' (A of PV)
     static constexpr int kVbBuf = 2 * kKeys * 128;                 // two 64-channel halves [128][128 B] bf16
     static constexpr int kVb = kP + 2 * kPBuf;                     // [2 bufs] bf16 V (B of PV)
-    static constexpr int kScale = kVb + 2 * kVbBuf;                // [stage] ks[128] | vs[128] fp32
-    static constexpr int kSq = kScale + kStages * 2 * kKeys * 4;   // [64] fp32 query scales
-    static constexpr int kMeta = kSq + kRows * 4;                  // [stage] int: pages with a bad id
-    static constexpr int kRmax = kMeta + 16;                       // [tile parity][half][64] fp32 row maxima
-    static constexpr int kLsum = kRmax + 2 * 2 * kRows * 4;        // [half][64] fp32 row sums
-    static constexpr int kBar = kLsum + 2 * kRows * 4;
+    static constexpr int kScale = kVb + 2 * kVbBuf;                // [slot] ks[128] | vs[128] fp32
+    static constexpr int kSq = kScale + kScStages * 2 * kKeys * 4; // [64] fp32 query scales
+    static constexpr int kMeta = kSq + kRows * 4;                  // [slot] int: pages with a bad id
+    static constexpr int kGrp = kMeta + kScStages * 4;             // [m | l][tile parity][64] fp32
+    static constexpr int kBar = kGrp + 2 * 2 * kRows * 4;
     // barriers
-    static constexpr int kKvFull = 0, kKvEmpty = 3, kSFull = 6, kSFree = 8, kPReady = 10,
-                         kPvDone = 12, kFinal = 14, kQReady = 15, kRmaxBar = 16, kNumBars = 20;
+    static constexpr int kKvFull = 0, kKvEmpty = kKvFull + kStages, kSFull = kKvEmpty + kStages,
+                         kPReady = kSFull + 2, kPvDone = kPReady + 2, kFinal = kPvDone + 2,
+                         kQReady = kFinal + 1, kScFull = kQReady + 1, kScEmpty = kScFull + kScStages,
+                         kNumBars = kScEmpty + kScStages;
     static constexpr int kMisc = kBar + kNumBars * 8;              // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 16;
     // merge area, over the K stages (free once the last tile is consumed)
@@ -197,13 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         for (int i = 0; i < Sm::kNumBars; ++i) {
-            uint32_t cnt = 1;
-            if (i >= Sm::kKvFull && i < Sm::kKvFull + kStages) cnt = 1 + 32;      // expect_tx + scale copies
-            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + kSoftWarps + 4;  // QK commit + warps
-            if (i >= Sm::kSFree && i < Sm::kSFree + 2) cnt = kSoftWarps;
-            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = kSoftWarps + 4;
+            uint32_t cnt = 1;                                       // expect_tx; commits
+            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + 4;     // QK commit + converters
+            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = 4 + 4;             // softmax group + converters
             if (i == Sm::kQReady) cnt = kSoftWarps;
-            if (i >= Sm::kRmaxBar && i < Sm::kRmaxBar + 4) cnt = 2;                     // the warp pair
+            if (i >= Sm::kScFull && i < Sm::kScFull + kScStages) cnt = 1 + 32;    // bad-page mask + scale copies
+            if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = 4;       // softmax group
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -220,6 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lp = tb * ppt + lane;
         if (lp < (tb + nt) * ppt && lp * p.page < ctx && lp * p.page + p.page > lo)
             pg_first = __ldg(&p.ptab[(int64_t)b * p.max_pages + lp]);
+    }
+    // the softmax warps' query row quarters (contiguous rows), also in flight
+    // across the barrier
+    uint4 qv[4] = {};
+    if (warp < kSoftWarps && p.q_vec && (tid >> 2) < p.R) {
+        const int r = tid >> 2;
+        const uint4* src = reinterpret_cast<const uint4*>(p.q + b * p.qs0 + (r / p.G) * p.qs1 +
+                                                          (hk * p.G + r % p.G) * p.qs2) + 4 * (tid & 3);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) qv[c] = __ldg(src + c);
     }
 
     tc_fence_before();
@@ -248,9 +261,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool bad_l = false;
         int issued = 0;
         for (int i = 0; i < nt; ++i) {
-            const int s = i % kStages;
+            const int s = i % kStages, c = i % kScStages;
             if (!warp_all(mbar_wait(&bars[Sm::kKvEmpty + s], ((i / kStages) & 1) ^ 1, abort_flag,
                                     &g_decode_err, 1)))
+                break;
+            if (!warp_all(mbar_wait(&bars[Sm::kScEmpty + c], ((i / kScStages) & 1) ^ 1, abort_flag,
+                                    &g_decode_err, 7)))
                 break;
             if ((i * ppt) / 32 != chunk) {
                 chunk = (i * ppt) / 32;
@@ -273,7 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool bad = __shfl_sync(0xffffffffu, bad_l ? 1 : 0, slot0 + (lane < ppt ? lane : 0)) != 0 && lane < ppt;
             const unsigned badm = __ballot_sync(0xffffffffu, bad);
             if (lane == 0) {
-                meta[s] = static_cast<int>(badm);
+                meta[c] = static_cast<int>(badm);
+                mbar_arrive(&bars[Sm::kScFull + c]);
                 mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * Sm::kKStage);
             }
             for (int q = 0; q < ppt; ++q) {
@@ -289,89 +306,89 @@ __global__ void __launch_bounds__(kThreads, 1)
             // per-token scales of keys 4 lane .. 4 lane + 3, stored by key
             // parity (index (key & 1) * 64 + key / 2) for the softmax threads;
             // with per-tensor scales the one K and one V scale in every slot
+            float* dst = scl + c * 2 * kKeys;
             if (p.per_tensor) {
-                float* dst = scl + s * 2 * kKeys;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     dst[4 * lane + e] = ks_tensor;
                     dst[kKeys + 4 * lane + e] = vs_tensor;
                 }
-                mbar_arrive(&bars[Sm::kKvFull + s]);
+                mbar_arrive(&bars[Sm::kScFull + c]);
             } else {
                 const int kq = 4 * lane;
                 const int pq = __shfl_sync(0xffffffffu, phys, kq / p.page);
                 const int64_t src = ((int64_t)pq * p.Hk + hk) * p.page + (kq % p.page);
-                float* dst = scl + s * 2 * kKeys;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int key = kq + e, at = (key & 1) * 64 + (key >> 1);
                     cp_async_4(dst + at, p.ksc + src + e);
                     cp_async_4(dst + kKeys + at, p.vsc + src + e);
                 }
-                cp_async_mbar_arrive(&bars[Sm::kKvFull + s]);
+                cp_async_mbar_arrive(&bars[Sm::kScFull + c]);
             }
             issued = i + 1;
         }
         // no copy of this CTA may land after it exits
         for (int i = max(0, issued - kStages); i < issued; ++i)
             mbar_wait_drain(&bars[Sm::kKvFull + i % kStages], (i / kStages) & 1);
+        for (int i = max(0, issued - kScStages); i < issued; ++i)
+            mbar_wait_drain(&bars[Sm::kScFull + i % kScStages], (i / kScStages) & 1);
       } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && nt > 0) {
             constexpr uint32_t kIdescQK = umma_idesc(1, 0, kRows, kKeys);              // e4m3 -> f32
-            constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, 64) | (1u << 16);    // bf16, B MN-major
-            constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, 64);                // bf16, B K-major
+            constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, kD) | (1u << 16);    // bf16, B MN-major
+            constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, kD);                // bf16, B K-major
             const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), 128);
+            // S(i) = Q8 K8(i)^T into S buffer i & 1
+            auto issue_qk = [&](int i) -> bool {
+                const int s = i % kStages;
+                if (!mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2))
+                    return false;
+                tc_fence_after();
+                const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), 128);
+#pragma unroll
+                for (int kk = 0; kk < kD / 32; ++kk)
+                    mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, kk > 0 ? 1u : 0u);
+                mma_commit(&bars[Sm::kSFull + (i & 1)]);
+                mma_commit(&bars[Sm::kKvEmpty + s]);
+                return true;
+            };
+            // order: QK(0), QK(1), then PV(j), QK(j + 2) for j = 0, 1, ...
+            // S(j + 2) is written once the softmax group of tile j is done
+            // with S(j) (its P'(j) implies that), and its commit covers PV(j):
+            // the group's P' buffer and O are free when S(j + 2) is there
             bool ok = mbar_wait(&bars[Sm::kQReady], 0, abort_flag, &g_decode_err, 12);
-            for (int i = 0; ok && i <= nt; ++i) {
-                if (i < nt) {
-                    // S(i) = Q8 K8(i)^T into S buffer i & 1
-                    const int s = i % kStages;
-                    ok = mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2);
-                    if (ok && i >= 2)
-                        ok = mbar_wait(&bars[Sm::kSFree + (i & 1)], ((i - 2) >> 1) & 1, abort_flag,
-                                       &g_decode_err, 3);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), 128);
+            if (ok) ok = issue_qk(0);
+            if (ok && nt > 1) ok = issue_qk(1);
+            for (int j = 0; ok && j < nt; ++j) {
+                // O[j & 1] += P'(j) V(j): 8 steps of 16 keys, all 128 channels
+                ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
+                const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
+                if (!p.v_trans) {
+                    // V MN-major: two 64-channel swizzle atoms [128 keys][128 B], the
+                    // second one kKeys * 128 bytes on (the leading byte offset)
+                    const uint64_t vdesc = umma_desc_kmajor(vb, 128) +
+                                           (static_cast<uint64_t>((kKeys * 128) >> 4) << 16) - (1ull << 16);
 #pragma unroll
-                    for (int kk = 0; kk < kD / 32; ++kk)
-                        mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK,
-                                  kk > 0 ? 1u : 0u);
-                    mma_commit(&bars[Sm::kSFull + (i & 1)]);
-                    mma_commit(&bars[Sm::kKvEmpty + s]);
+                    for (int st = 0; st < kKeys / 16; ++st)
+                        mma_bf16_ss(tmem + kOCol + 128 * (j & 1),
+                                    umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
+                                    vdesc + 128 * st, kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
+                } else {
+                    // V^T converted K-major: 64-key atoms of [128 channels][128 B]
+#pragma unroll
+                    for (int st = 0; st < kKeys / 16; ++st)
+                        mma_bf16_ss(tmem + kOCol + 128 * (j & 1),
+                                    umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
+                                    umma_desc_kmajor(vb + (st >> 2) * (kD * 128), 128) + 2 * (st & 3),
+                                    kIdescPVT, (j > 1 || st > 0) ? 1u : 0u);
                 }
-                if (i >= 1) {
-                    // O[j & 1] += P'(j) V(j): two 64-channel halves x 8 steps of 16 keys
-                    const int j = i - 1;
-                    ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
-                    if (!ok) break;
-                    tc_fence_after();
-                    const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
-                    const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
-                    if (!p.v_trans) {
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-                            for (int st = 0; st < kKeys / 16; ++st)
-                                mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
-                                            umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
-                                            umma_desc_kmajor(vb + hf * (kKeys * 128), 128) + 128 * st,
-                                            kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
-                    } else {
-                        // V^T converted K-major: 64-key atoms of [128 channels][128 B]
-#pragma unroll
-                        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-                            for (int st = 0; st < kKeys / 16; ++st)
-                                mma_bf16_ss(tmem + kOCol + 128 * (j & 1) + 64 * hf,
-                                            umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
-                                            umma_desc_kmajor(vb + (st >> 2) * (kD * 128) + hf * (64 * 128), 128) +
-                                                2 * (st & 3),
-                                            kIdescPVT, (j > 1 || st > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&bars[Sm::kPvDone + (j & 1)]);
-                }
+                mma_commit(&bars[Sm::kPvDone + (j & 1)]);
+                if (j + 2 < nt) ok = issue_qk(j + 2);
             }
             // drain every MMA this thread issued before TMEM is released
             mma_commit(&bars[Sm::kFinal]);
@@ -404,8 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.q_vec) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint4 u = rv ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
-                    const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+                    const uint32_t wd[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};   // zeros past R
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         x[8 * c + 2 * e] = __uint_as_float(wd[e] << 16);
@@ -478,10 +494,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&bars[Sm::kQReady]);
         named_sync(1, kSoftWarps * 32);              // every row's s_q is in shared memory
 
-        // thread: query row r (TMEM lane 32 qw + lr) and the columns
-        // 64 hh + 2k + cpar (k = 0..31) of every tile; warps qw and qw + 4
-        // share their rows and exchange row maxima through shared memory
-        const int qw = warp & 3, hh = warp >> 2;
+        // Group g = warp >> 2 takes the tiles i = g, g + 2, g + 4, ... with
+        // its own running max and sum, accumulated into O[g]; the groups run
+        // side by side and are combined after the last tile. Warp qw = warp &
+        // 3 of a group holds query rows 16 qw .. 16 qw + 15 (TMEM lanes 32 qw
+        // ..) over all 128 columns: thread: row r, register k = column 2k +
+        // cpar (k = 0..63).
+        const int qw = warp & 3, g = warp >> 2;
         const int lr = (lane >> 2) + 8 * (lane & 1);
         const int cpar = (lane >> 1) & 1;
         const int r = 16 * qw + lr;
@@ -492,39 +511,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         // acc = 0, so its logits are 0 either way)
         const float cq = fmaxf(rv ? sq[r] * p.logit_scale_log2 : 0.0f, FLT_MIN);
         const uint64_t cq2 = f2_pack(cq, cq);
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * qw) << 16) + 64 * hh;
-        float* rmax = reinterpret_cast<float*>(sm + Sm::kRmax);
-        float o_fin[32];                              // end-of-split state, merged below
-        float m_fin = -INFINITY;
-        // m_run: running max; m_acc[a]: the max O[a] is expressed against
-        float m_run = -INFINITY;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * qw) << 16);
+        float m_run = -INFINITY;                      // the max O[g] and the sum are expressed against
         uint64_t lsum2 = f2_pack(0.0f, 0.0f);         // running sum as an f32x2 pair
-        float m_acc[2] = {-INFINITY, -INFINITY};
         bool ok = true;
-        for (int i = 0; i < nt; ++i) {
-            const int s = i % kStages, bf = i & 1;
-            ok = warp_all(mbar_wait(&bars[Sm::kSFull + bf], (i >> 1) & 1, abort_flag, &g_decode_err, 5));
+        for (int i = g; i < nt; i += 2) {
+            const int c = i % kScStages;
+            ok = warp_all(mbar_wait(&bars[Sm::kSFull + g], (i >> 1) & 1, abort_flag, &g_decode_err, 5));
             if (ok)
-                ok = warp_all(mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag,
+                ok = warp_all(mbar_wait(&bars[Sm::kScFull + c], (i / kScStages) & 1, abort_flag,
                                         &g_decode_err, 6));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[32];
-            tmem_ld16x32(taddr + 128 * bf, sv);
-            tmem_wait_ld(sv);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[Sm::kSFree + bf]);
+            uint32_t sv[64];
+            tmem_ld16x64(taddr + 128 * g, sv);
+            tmem_wait_ld64(sv);
 
-            const float* ksP = scl + s * 2 * kKeys + cpar * 64 + 32 * hh;   // k_scale of column 64hh + 2k + cpar
+            const float* ksP = scl + c * 2 * kKeys + cpar * 64;   // k_scale of column 2k + cpar
             const float* vsP = ksP + kKeys;
             const int key0 = (tb + i) * kKeys;
-            const int badm = meta[s];
+            const int badm = meta[c];
             // y = acc * k_scale; the logit is y * cq, and cq > 0 keeps the
             // order, so the row max is taken on y
-            float x[32];
+            float x[64];
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
+            for (int k4 = 0; k4 < 16; ++k4) {
                 const float4 kq = *reinterpret_cast<const float4*>(ksP + 4 * k4);
                 const uint64_t a01 = f2_mul(f2_pack(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
                                             f2_pack(kq.x, kq.y));
@@ -538,68 +549,54 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool full = badm == 0 && key0 >= ctx - p.window && key0 + kKeys - 1 <= ctx - p.T;
             if (!rv) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) x[k] = -INFINITY;
+                for (int k = 0; k < 64; ++k) x[k] = -INFINITY;
             } else if (!full) {
-                // the row sees columns [clo, chi] of the tile; register k is
-                // column 64 hh + 2k + cpar
-                const int base = key0 + 64 * hh + cpar;
-                const int clo = pq - p.window + 1 - base, chi = pq - base;
+                // the row sees columns [clo, chi] of the tile
+                const int clo = pq - p.window + 1 - key0 - cpar, chi = pq - key0 - cpar;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) x[k] = (2 * k >= clo && 2 * k <= chi) ? x[k] : -INFINITY;
+                for (int k = 0; k < 64; ++k) x[k] = (2 * k >= clo && 2 * k <= chi) ? x[k] : -INFINITY;
                 if (badm != 0) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if ((badm >> ((64 * hh + 2 * k + cpar) >> p.lg_page)) & 1) x[k] = -INFINITY;
+                    for (int k = 0; k < 64; ++k)
+                        if ((badm >> ((2 * k + cpar) >> p.lg_page)) & 1) x[k] = -INFINITY;
                 }
             }
-            // row max: four chains, a tree, the column partner, the other half
+            // row max: four chains, a tree, the column partner
             float m4[4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) m4[c] = fmax3(x[c], x[c + 4], x[c + 8]);
+            for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmax3(x[q4], x[q4 + 4], x[q4 + 8]);
 #pragma unroll
-            for (int k = 12; k < 28; k += 8)
+            for (int k = 12; k < 60; k += 8)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) m4[c] = fmax3(m4[c], x[k + c], x[k + c + 4]);
+                for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmax3(m4[q4], x[k + q4], x[k + q4 + 4]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) m4[c] = fmaxf(m4[c], x[28 + c]);
+            for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmaxf(m4[q4], x[60 + q4]);
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            float* rm = rmax + (i & 1) * (2 * kRows);
-            if (cpar == 0) rm[hh * kRows + r] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[Sm::kRmaxBar + qw]);
-            ok = warp_all(mbar_wait(&bars[Sm::kRmaxBar + qw], i & 1, abort_flag, &g_decode_err, 13));
-            if (!ok) break;
-            mx = fmaxf(mx, rm[(hh ^ 1) * kRows + r]);
             mx = mx == -INFINITY ? -INFINITY : mx * cq;   // the max of the logits y * cq
             const float m_new = fmaxf(m_run, mx);
-            if (m_run != -INFINITY && m_new != m_run) {
-                const float a = ex2_approx(m_run - m_new);
-                lsum2 = f2_mul(lsum2, f2_pack(a, a));
-            }
+            // O[g] and the sum (tiles i - 2, i - 4, ...) are brought to m_new
+            const bool resc = m_run != -INFINITY && m_new != m_run;
+            const float alpha = resc ? ex2_approx(m_run - m_new) : 1.0f;
+            if (resc) lsum2 = f2_mul(lsum2, f2_pack(alpha, alpha));
             m_run = m_new;
             const float sub = m_new == -INFINITY ? 0.0f : m_new;
             const uint64_t nsub2 = f2_pack(-sub, -sub);
-            // O[bf] (tiles i - 2, i - 4, ...) is brought to m_new before PV(i)
-            const float m_o = m_acc[bf];
-            const bool resc = m_o != -INFINITY && m_o != m_new;
-            const float alpha = resc ? ex2_approx(m_o - m_new) : 1.0f;
-            m_acc[bf] = m_new;
 
-            // P' buffer bf is free: PV(i - 2), its reader, is done -- the MMA
+            // P' buffer g is free: PV(i - 2), its reader, is done -- the MMA
             // thread issues it before QK(i), and the commit that completed
             // S(i) covers every MMA that thread started earlier
-            uint8_t* prow = sm + Sm::kP + bf * Sm::kPBuf + hh * (kRows * 128) + r * 128;
+            uint8_t* prow = sm + Sm::kP + g * Sm::kPBuf + r * 128;
 #pragma unroll
-            for (int i8 = 0; i8 < 4; ++i8) {      // keys 64hh + 16 i8 + cpar + 2m = registers 8 i8 + m
-                const float4 va = *reinterpret_cast<const float4*>(vsP + 8 * i8);
-                const float4 vb = *reinterpret_cast<const float4*>(vsP + 8 * i8 + 4);
+            for (int i16 = 0; i16 < 8; ++i16) {   // keys 16 i16 + cpar + 2m = registers 8 i16 + m
+                const float4 va = *reinterpret_cast<const float4*>(vsP + 8 * i16);
+                const float4 vb = *reinterpret_cast<const float4*>(vsP + 8 * i16 + 4);
                 const float vsv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
                 uint32_t wd[4];
 #pragma unroll
                 for (int m = 0; m < 8; m += 2) {
                     float e0, e1;
-                    f2_unpack(f2_fma(f2_pack(x[8 * i8 + m], x[8 * i8 + m + 1]), cq2, nsub2), e0, e1);
+                    f2_unpack(f2_fma(f2_pack(x[8 * i16 + m], x[8 * i16 + m + 1]), cq2, nsub2), e0, e1);
                     const float p0 = ex2_approx(e0), p1 = ex2_approx(e1);
                     const uint64_t p2 = f2_pack(p0, p1);
                     lsum2 = f2_add(lsum2, p2);
@@ -608,61 +605,83 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __nv_bfloat162 pr = __floats2bfloat162_rn(w0, w1);
                     wd[m / 2] = *reinterpret_cast<const uint32_t*>(&pr);
                 }
-                const int chunk = 2 * i8 + cpar;
-                *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                const int chunk = 2 * (i16 & 3) + cpar;
+                *reinterpret_cast<uint4*>(prow + (i16 >> 2) * (kRows * 128) + ((chunk ^ (r & 7)) << 4)) =
+                    make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
-            // O[bf] *= alpha for the rows whose max rose since tile i - 2 (PV(i - 2),
-            // its last writer, is done, as above); this warp's 64 output
-            // channels
+            // O[g] *= alpha for the rows whose max rose (PV(i - 2), its last
+            // writer, is done, as above), 64 columns at a time
             if (__any_sync(0xffffffffu, resc)) {
                 tc_fence_after();
-                uint32_t o[32];
-                tmem_ld16x32(taddr + kOCol + 128 * bf, o);
-                tmem_wait_ld(o);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                tmem_st16x32(taddr + kOCol + 128 * bf, o);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t o[32];
+                    tmem_ld16x32(taddr + kOCol + 128 * g + 64 * hf, o);
+                    tmem_wait_ld(o);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                    tmem_st16x32(taddr + kOCol + 128 * g + 64 * hf, o);
+                }
                 tmem_wait_st();
             }
             fence_proxy_async_smem();               // P' is read by the PV MMAs
-            tc_fence_before();
+            tc_fence_before();                      // S(i) read: QK(i + 2) may overwrite it
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&bars[Sm::kPReady + bf]);
-                mbar_arrive(&bars[Sm::kKvEmpty + s]);
+                mbar_arrive(&bars[Sm::kPReady + g]);
+                mbar_arrive(&bars[Sm::kScEmpty + c]);
             }
         }
-        bool have = ok && nt > 0;
-        if (have)
-            have = warp_all(mbar_wait(&bars[Sm::kPvDone + ((nt - 1) & 1)], ((nt - 1) >> 1) & 1,
-                                      abort_flag, &g_decode_err, 9));
+        // the group's (m, l) per row, for the combination of O[0] and O[1]
+        {
+            float l0, l1;
+            f2_unpack(lsum2, l0, l1);
+            float lsum = l0 + l1;
+            lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+            float* grp = reinterpret_cast<float*>(sm + Sm::kGrp);
+            if (cpar == 0) {
+                grp[g * kRows + r] = ok ? m_run : -INFINITY;
+                grp[2 * kRows + g * kRows + r] = ok ? lsum : 0.0f;
+            }
+        }
+        named_sync(1, kSoftWarps * 32);
+        // this warp's output channels: 64 g .. 64 g + 63 of its rows;
+        // O = O[0] 2^(m0 - M) + O[1] 2^(m1 - M), l likewise, M = max(m0, m1)
+        float o_fin[32];
+        float m_fin = -INFINITY, l_fin = 0.0f;
+        bool have = nt > 0 && warp_all(mbar_wait(&bars[Sm::kPvDone + ((nt - 1) & 1)], ((nt - 1) >> 1) & 1,
+                                                 abort_flag, &g_decode_err, 9));
+#pragma unroll
+        for (int k = 0; k < 32; ++k) o_fin[k] = 0.0f;
         if (have) {
-            // O = O[0] 2^(m_acc0 - m) + O[1] 2^(m_acc1 - m), m = m_run
+            // (the TMEM loads are warp-wide: every lane takes them, and a row
+            // whose group saw no key, m = -inf, takes none of their values)
+            const float* grp = reinterpret_cast<const float*>(sm + Sm::kGrp);
+            const float m0 = grp[r], m1 = grp[kRows + r];
+            m_fin = fmaxf(m0, m1);
             tc_fence_after();
-            uint32_t o0[32], o1[32];
-            tmem_ld16x32(taddr + kOCol, o0);
-            tmem_wait_ld(o0);
-            const float w0 = m_acc[0] == -INFINITY ? 0.0f : ex2_approx(m_acc[0] - m_run);
+            {
+                const bool use0 = m0 != -INFINITY;
+                const float w0 = use0 ? ex2_approx(m0 - m_fin) : 0.0f;
+                uint32_t o0[32];
+                tmem_ld16x32(taddr + kOCol + 64 * g, o0);
+                tmem_wait_ld(o0);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o_fin[k] = __uint_as_float(o0[k]) * w0;
-            if (nt > 1) {
-                tmem_ld16x32(taddr + kOCol + 128, o1);
-                tmem_wait_ld(o1);
-                const float w1 = m_acc[1] == -INFINITY ? 0.0f : ex2_approx(m_acc[1] - m_run);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) o_fin[k] = fmaf(__uint_as_float(o1[k]), w1, o_fin[k]);
+                for (int k = 0; k < 32; ++k) o_fin[k] = use0 ? __uint_as_float(o0[k]) * w0 : 0.0f;
+                l_fin = use0 ? grp[2 * kRows + r] * w0 : 0.0f;
             }
-            m_fin = m_run;
-        } else {
+            if (nt > 1) {
+                const bool use1 = m1 != -INFINITY;
+                const float w1 = use1 ? ex2_approx(m1 - m_fin) : 0.0f;
+                uint32_t o1[32];
+                tmem_ld16x32(taddr + kOCol + 128 + 64 * g, o1);
+                tmem_wait_ld(o1);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o_fin[k] = 0.0f;
-            lsum2 = f2_pack(0.0f, 0.0f);
+                for (int k = 0; k < 32; ++k)
+                    o_fin[k] = use1 ? fmaf(__uint_as_float(o1[k]), w1, o_fin[k]) : o_fin[k];
+                if (use1) l_fin = fmaf(grp[3 * kRows + r], w1, l_fin);
+            }
         }
-        float l0, l1;
-        f2_unpack(lsum2, l0, l1);
-        float lsum = l0 + l1;
-        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-        if (cpar == 0) reinterpret_cast<float*>(sm + Sm::kLsum)[hh * kRows + r] = lsum;
         // ---- merge the splits of (b, hk) across the cluster (only the
         // softmax warps hold registers enough for it). Every role ends with
         // the same three barriers, reached from its own code: the CTA
@@ -674,11 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             float* oc = reinterpret_cast<float*>(sm + Sm::kOc);
             float2* stat = reinterpret_cast<float2*>(sm + Sm::kStat);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) oc[r * kOcPitch + 64 * hh + 2 * k + cpar] = o_fin[k];
-            if (hh == 0 && cpar == 0) {
-                const float* ls = reinterpret_cast<const float*>(sm + Sm::kLsum);
-                stat[r] = make_float2(m_fin, ls[r] + ls[kRows + r]);
-            }
+            for (int k = 0; k < 32; ++k) oc[r * kOcPitch + 64 * g + 2 * k + cpar] = o_fin[k];
+            if (g == 0 && cpar == 0) stat[r] = make_float2(m_fin, l_fin);
             __syncwarp();
             cluster_arrive_wait();
             // CTA `split` writes rows split, split + nsplit, ...; thread: one
