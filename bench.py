@@ -269,7 +269,7 @@ def bench_decode(sage, torch, stream, copies=8, reps=50):
     caches = [[d[x].cuda() for x in ("k_cache", "v_cache", "k_scale", "v_scale")]
               for _ in range(copies)]
     out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((max(16, sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"])),),
+    ws = torch.zeros((max(16, sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"])),),
                      dtype=torch.uint8, device="cuda")
 
     def call(i):

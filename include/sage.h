@@ -282,7 +282,11 @@ sage_status sage_attn_fwd_mx(const uint8_t* q4, const uint8_t* q_sf, const uint8
                              int H, int Hk, int Lq, int Lk, int D, float softmax_scale, int causal,
                              sage_view4 out_bf16, void* ws, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace sage_attn_decode needs (split-KV partials). */
+/* Bytes of device workspace sage_attn_decode needs on the current device:
+ * the split-KV partials when the keys of a (sequence, kv head) are shared
+ * out among several CTAs (at most one CTA per SM in all), 0 when B * Hk
+ * reaches the SM count. No initial contents are required; concurrent calls
+ * need distinct workspaces. */
 size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window);
 
 /* Cache variants of sage_attn_decode ("[FlyDSL] [Misc] pa_decode ...",
@@ -311,7 +315,10 @@ size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window
  * Supported: D == 128, page_size in {16, 32, 64, 128}, H % Hk == 0,
  * H / Hk <= 16, T * (H / Hk) <= 64, window >= 1; SAGE_KV_V_TRANSPOSED
  * needs page_size 128 (UNSUPPORTED otherwise), unknown kv_flags bits are
- * INVALID_ARG. ws: at least sage_attn_decode_workspace(...) bytes. */
+ * INVALID_ARG. ws: at least sage_attn_decode_workspace(...) bytes, 16-byte
+ * aligned. One kernel launch, or two when the keys of a (sequence, kv head)
+ * are split among CTAs: the split kernel leaves (m, l, O) per CTA in ws and
+ * a merge kernel combines them (log-sum-exp). */
 sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
                              const uint8_t* v_cache, const float* k_scale, const float* v_scale,
                              const int32_t* page_table, const int32_t* ctx_lens, int B, int T,

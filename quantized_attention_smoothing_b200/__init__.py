@@ -272,6 +272,12 @@ def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_l
     B, T, H, D = q.shape
     Hk = k_cache.shape[1]
     max_pages = page_table.shape[1]
+    if ws is None:
+        # the split-KV partials (none when every (sequence, kv head) runs in
+        # one CTA)
+        n = sage_attn_decode_workspace(B, T, H, Hk, D, window)
+        if n > 0:
+            ws = torch.empty((n,), dtype=torch.uint8, device=q.device)
     _check(lib().sage_attn_decode(h.handle, _view(q, CView4), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(k_scale), _ptr(v_scale), _ptr(page_table), _ptr(ctx_lens),
                                   B, T, H, Hk, D, int(page_size), int(max_pages), int(num_pages),

@@ -5,40 +5,44 @@
 // to the FP8 format of the cache (Q here), PV on bf16 operands because a
 // per-token V scale cannot be factored out of the sum).
 //
-// One kernel. The keys of sequence b (the union of its T query tokens'
+// Two kernels. The keys of sequence b (the union of its T query tokens'
 // windows, [lo, ctx)) are cut into 128-key tiles aligned to absolute key
 // positions, so a tile is one page (page 128) or 128 / page whole pages.
-// The tiles of (b, kv head hk) are shared out among up to 8 CTAs that form
-// one thread-block cluster (the size is picked at launch so that the grid
-// runs in one wave); CTA = 16 warps:
-//   warps 0-7  softmax: warps w and w + 4 (w < 4) own query rows 16w ..
-//              16w + 15 (R = T * H/Hk rows, row r = t * G + g, padded to 64)
-//              -- M = 64 MMAs keep those rows in TMEM lanes 32w .. 32w + 15
-//              -- warp w the tile's columns 0-63, warp w + 4 columns 64-127;
+// The tiles of (b, kv head hk) are shared out among up to 16 CTAs of
+// decode_kernel (the count is picked at launch so that the grid runs in one
+// wave, one CTA per SM); CTA = 16 warps:
+//   warps 0-7  softmax, two groups: warps 0-3 take the even tiles, warps 4-7
+//              the odd ones, each group with its own running max and sum
+//              and its own O accumulator; warp w of a group owns query rows
+//              16 (w & 3) .. + 15 (R = T * H/Hk rows, row r = t * G + g,
+//              padded to 64) over all 128 columns -- M = 64 MMAs keep those
+//              rows in TMEM lanes 32 (w & 3) .. + 15;
 //   warps 8-11 V converters: e4m3 V tile -> exact bf16 (integer bit
 //              placement and one bf16 multiply), in the key order of the P
 //              operand;
-//   warp 12    producer: page-table lookups, one TMA box per page for K and
-//              for V, per-token scales by cp.async, all on one mbarrier;
-//   warp 13    TMEM owner and MMA issuer (warps 14, 15 only complete the
-//              producer's warpgroup).
+//   warp 12    K/V producer: page-table lookups, one TMA box per page for K
+//              and for V;
+//   warp 13    TMEM owner and MMA issuer;
+//   warp 14    scale producer: per-token scales by cp.async and the tile's
+//              bad-page mask, on a ring of their own (warp 15 only completes
+//              the producers' warpgroup).
 // Per tile: S = Q8 K8^T (e4m3 tcgen05 MMAs, M=64 N=128, fp32 in TMEM,
-// double-buffered) -> base-2 logits (S * k_scale_j) * s_q * softmax_scale /
-// D, masked to each row's own window -> running max m -> p = 2^(x - m) ->
-// P' = bf16(p * v_scale_j) -> O[i & 1] += P' V (bf16 tcgen05 MMAs, fp32 in
-// TMEM). Even and odd tiles accumulate into two O's: before PV(i), the rows
-// of O[i & 1] whose max rose since tile i - 2 are rescaled by 2^(m_old - m),
-// which needs PV(i - 2) done rather than PV(i - 1); the epilogue adds the two
-// O's at the final max. The query rows are rotated and quantised to e4m3 in
-// the prologue (fp32 butterfly, four threads per row, scale max|q_hat| / 448,
-// the operations of the quantisation kernels). At the end every CTA leaves
-// (m, l, O) of its tiles in shared memory and the CTAs of the cluster merge
-// them (log-sum-exp) through distributed shared memory and write bf16
-// through the caller's strides.
+// double-buffered by tile parity) -> base-2 logits (S * k_scale_j) * s_q *
+// softmax_scale / D, masked to each row's own window -> the group's running
+// max m -> p = 2^(x - m) -> P' = bf16(p * v_scale_j) -> O[i & 1] += P' V
+// (bf16 tcgen05 MMAs, M=64 N=128, fp32 in TMEM). Before PV(i), the rows of
+// O[i & 1] whose group max rose since tile i - 2 are rescaled by 2^(m_old -
+// m); after the last tile the two groups' (m, l, O) are combined. The query
+// rows are rotated and quantised to e4m3 in the prologue (fp32 butterfly,
+// four threads per row, scale max|q_hat| / 448, the operations of the
+// quantisation kernels). A CTA that holds every tile of (b, hk) writes bf16
+// through the caller's strides; otherwise every CTA writes its (m, l, O) to
+// the workspace and decode_merge_kernel, launched after it on the stream,
+// combines the splits (log-sum-exp) and writes bf16.
 //
 // Every mbarrier wait is bounded; on timeout the CTA records an error word,
-// raises its abort flag, drains its own copies and MMAs and still takes part
-// in both cluster barriers.
+// raises its abort flag, drains its own copies and MMAs and still reaches
+// its CTA barriers.
 #include <algorithm>
 #include <cfloat>
 #include <climits>
@@ -63,11 +67,12 @@ constexpr int kKeys = 128;                   // keys per tile
 constexpr int kRows = 64;                    // query rows per CTA (M of every MMA)
 constexpr int kStages = 3;                   // K / V ring
 constexpr int kScStages = 8;                 // per-token scale ring (freed by the softmax alone)
-constexpr int kMaxSplit = 8;                 // CTAs per (sequence, kv head) = cluster size
+constexpr int kMaxSplit = 16;                // CTAs per (sequence, kv head)
 constexpr int kSoftWarps = 8;                // warps 0..7
 constexpr int kConvWarp0 = 8;                // warps 8..11
 constexpr int kTmaWarp = 12;
-constexpr int kMmaWarp = 13;                 // warps 14, 15 idle until the merge
+constexpr int kMmaWarp = 13;
+constexpr int kScaleWarp = 14;               // warp 15 idle until the merge
 constexpr int kThreads = 512;
 // registers per thread of each warpgroup (setmaxnreg; 256 x 176 + 128 x 96 +
 // 128 x 56 <= 512 x 128, the launch's registers; this split compiles without
@@ -78,6 +83,10 @@ constexpr int kRegsSoft = 176, kRegsConv = 96, kRegsProd = 56;
 static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kOcPitch = kD + 4;             // fp32 row pitch of the merge area
+// A scale slot: k_scale then v_scale of the tile's keys, each by key parity
+// (index (key & 1) * kScPar + key / 2); the 4-float pad puts the two parities'
+// 16-byte reads in different banks
+constexpr int kScPar = kKeys / 2 + 4, kScHalf = 2 * kScPar, kScSlot = 2 * kScHalf;
 
 // dynamic shared memory (offsets from a 1024-byte aligned base)
 struct Sm {
@@ -89,8 +98,8 @@ struct Sm {
     static constexpr int kP = kV + kStages * kKStage;              // [2 bufs] P' (A of PV)
     static constexpr int kVbBuf = 2 * kKeys * 128;                 // two 64-channel halves [128][128 B] bf16
     static constexpr int kVb = kP + 2 * kPBuf;                     // [2 bufs] bf16 V (B of PV)
-    static constexpr int kScale = kVb + 2 * kVbBuf;                // [slot] ks[128] | vs[128] fp32
-    static constexpr int kSq = kScale + kScStages * 2 * kKeys * 4; // [64] fp32 query scales
+    static constexpr int kScale = kVb + 2 * kVbBuf;                // [slot] ks | vs fp32, padded
+    static constexpr int kSq = kScale + kScStages * kScSlot * 4;   // [64] fp32 query scales
     static constexpr int kMeta = kSq + kRows * 4;                  // [slot] int: pages with a bad id
     static constexpr int kGrp = kMeta + kScStages * 4;             // [m | l][tile parity][64] fp32
     static constexpr int kBar = kGrp + 2 * 2 * kRows * 4;
@@ -127,6 +136,9 @@ struct DecParams {
     float* qs_out;                           // optional: query scales [B, T, H]
     int per_tensor;                          // ksc / vsc hold one scale each
     int v_trans;                             // V cache [num_pages, Hk, D, page] (page 128)
+    int o_vec;                               // out rows: 4 channels as one 8-byte store
+    float2* ws_stat;                         // nsplit > 1: partial (m, l) [B Hk][nsplit][64]
+    float* ws_o;                             //   and partial O [B Hk][nsplit][64][128] fp32
 };
 
 // The A operand (P') of the PV MMA holds a row's 128 keys in this order:
@@ -158,13 +170,29 @@ __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-// CTA-wide and cluster-wide barriers in their non-aligned forms: the threads
-// may reach them from different code (each thread arrives exactly once).
+// CTA-wide barrier in its non-aligned form: the threads may reach it from
+// different code (each thread arrives exactly once).
 __device__ __forceinline__ void bar_sync_all(int count) {
     asm volatile("bar.sync 0, %0;" ::"r"(count) : "memory");
 }
-__device__ __forceinline__ void cluster_arrive_wait() {
-    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+
+// Output row rr of (b, hk), channels d4 .. d4 + 3: o * inv as bf16 through
+// the caller's strides.
+__device__ __forceinline__ void store_out4(const DecParams& p, int b, int hk, int rr, int d4, float4 o,
+                                           float inv) {
+    const int t = rr / p.G, h = hk * p.G + rr % p.G;
+    __nv_bfloat16* dst = p.out + b * p.os0 + t * p.os1 + h * p.os2 + (int64_t)d4 * p.os3;
+    const __nv_bfloat162 y01 = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+    const __nv_bfloat162 y23 = __floats2bfloat162_rn(o.z * inv, o.w * inv);
+    if (p.o_vec) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(*reinterpret_cast<const uint32_t*>(&y01),
+                                                    *reinterpret_cast<const uint32_t*>(&y23));
+    } else {
+        dst[0] = y01.x;
+        dst[p.os3] = y01.y;
+        dst[2 * p.os3] = y23.x;
+        dst[3 * p.os3] = y23.y;
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -180,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* meta = reinterpret_cast<int*>(sm + Sm::kMeta);
     float* scl = reinterpret_cast<float*>(sm + Sm::kScale);
 
-    const int split = blockIdx.x;                 // == rank in the cluster
+    const int split = blockIdx.x;
     const int bhk = blockIdx.y;
     const int b = bhk / p.Hk, hk = bhk % p.Hk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -219,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the producer's first page-table entries, requested before the barrier
     const int ppt = kKeys / p.page;                  // pages per tile (divides 32)
     int pg_first = 0;
-    if (warp == kTmaWarp) {
+    if (warp == kTmaWarp || warp == kScaleWarp) {
         const int lp = tb * ppt + lane;
         if (lp < (tb + nt) * ppt && lp * p.page < ctx && lp * p.page + p.page > lo)
             pg_first = __ldg(&p.ptab[(int64_t)b * p.max_pages + lp]);
@@ -246,28 +274,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp >= kTmaWarp) {
       reg_dealloc<kRegsProd>();
-      if (warp == kTmaWarp) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
+      if (warp == kTmaWarp || warp == kScaleWarp) {
+        // ------------------------------------------------------------ producers
+        // Both warps look up the physical pages of the CTA's logical pages
+        // tb * ppt + 32 c + lane, 32 at a time (lane j of chunk c holds page
+        // 32 c + j); pages holding no key of [lo, ctx) are not looked up
+        // (page 0 stands in; their keys are masked). Warp 12 loads K and V
+        // by TMA, the lanes of a tile's pages each issuing their own boxes;
+        // warp 14 loads the per-token scales and the tile's bad-page mask.
+        const bool kv = warp == kTmaWarp;
+        if (kv && lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
         }
-        const float ks_tensor = p.per_tensor ? __ldg(p.ksc) : 0.0f;
-        const float vs_tensor = p.per_tensor ? __ldg(p.vsc) : 0.0f;
-        // physical pages of the CTA's logical pages tb * ppt + 32 c + lane,
-        // fetched 32 at a time; pages holding no key of [lo, ctx) are not
-        // looked up (page 0 stands in; their keys are masked)
+        const float ks_tensor = (!kv && p.per_tensor) ? __ldg(p.ksc) : 0.0f;
+        const float vs_tensor = (!kv && p.per_tensor) ? __ldg(p.vsc) : 0.0f;
         int chunk = -1, phys_l = 0;
         bool bad_l = false;
         int issued = 0;
         for (int i = 0; i < nt; ++i) {
             const int s = i % kStages, c = i % kScStages;
-            if (!warp_all(mbar_wait(&bars[Sm::kKvEmpty + s], ((i / kStages) & 1) ^ 1, abort_flag,
-                                    &g_decode_err, 1)))
-                break;
-            if (!warp_all(mbar_wait(&bars[Sm::kScEmpty + c], ((i / kScStages) & 1) ^ 1, abort_flag,
-                                    &g_decode_err, 7)))
-                break;
+            const bool free_slot =
+                kv ? mbar_wait(&bars[Sm::kKvEmpty + s], ((i / kStages) & 1) ^ 1, abort_flag, &g_decode_err, 1)
+                   : mbar_wait(&bars[Sm::kScEmpty + c], ((i / kScStages) & 1) ^ 1, abort_flag, &g_decode_err, 7);
+            if (!warp_all(free_slot)) break;
             if ((i * ppt) / 32 != chunk) {
                 chunk = (i * ppt) / 32;
                 const int lp = tb * ppt + 32 * chunk + lane;
@@ -278,61 +308,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int pg = chunk == 0 ? pg_first : __ldg(&p.ptab[(int64_t)b * p.max_pages + lp]);
                     if (pg < 0 || pg >= p.num_pages) {
                         bad_l = true;
-                        atomicCAS(&g_decode_err, 0u, kErrDecodeRange);
+                        if (kv) atomicCAS(&g_decode_err, 0u, kErrDecodeRange);
                     } else {
                         phys_l = pg;
                     }
                 }
             }
-            const int slot0 = (i * ppt) % 32;             // this tile's pages: lanes slot0 ..
-            const int phys = __shfl_sync(0xffffffffu, phys_l, slot0 + (lane < ppt ? lane : 0));
-            const bool bad = __shfl_sync(0xffffffffu, bad_l ? 1 : 0, slot0 + (lane < ppt ? lane : 0)) != 0 && lane < ppt;
-            const unsigned badm = __ballot_sync(0xffffffffu, bad);
-            if (lane == 0) {
-                meta[c] = static_cast<int>(badm);
-                mbar_arrive(&bars[Sm::kScFull + c]);
-                mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * Sm::kKStage);
-            }
-            for (int q = 0; q < ppt; ++q) {
-                const int pq = __shfl_sync(0xffffffffu, phys, q);
-                if (lane == 0) {
-                    const int z = pq * p.Hk + hk;
-                    tma_load_3d(sm + Sm::kK + s * Sm::kKStage + q * p.page * kD, &tmK,
-                                &bars[Sm::kKvFull + s], 0, 0, z);
-                    tma_load_3d(sm + Sm::kV + s * Sm::kKStage + q * p.page * kD, &tmV,
-                                &bars[Sm::kKvFull + s], 0, 0, z);
+            const int slot0 = (i * ppt) % 32;             // this tile's pages: lanes slot0 .. slot0 + ppt - 1
+            const bool mine = lane >= slot0 && lane < slot0 + ppt;
+            if (kv) {
+                if (lane == slot0) mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * Sm::kKStage);
+                __syncwarp();
+                if (mine) {
+                    const int z = phys_l * p.Hk + hk;
+                    const int q = lane - slot0;
+                    tma_load_3d(sm + Sm::kK + s * Sm::kKStage + q * p.page * kD, &tmK, &bars[Sm::kKvFull + s], 0, 0, z);
+                    tma_load_3d(sm + Sm::kV + s * Sm::kKStage + q * p.page * kD, &tmV, &bars[Sm::kKvFull + s], 0, 0, z);
                 }
-            }
-            // per-token scales of keys 4 lane .. 4 lane + 3, stored by key
-            // parity (index (key & 1) * 64 + key / 2) for the softmax threads;
-            // with per-tensor scales the one K and one V scale in every slot
-            float* dst = scl + c * 2 * kKeys;
-            if (p.per_tensor) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    dst[4 * lane + e] = ks_tensor;
-                    dst[kKeys + 4 * lane + e] = vs_tensor;
-                }
-                mbar_arrive(&bars[Sm::kScFull + c]);
             } else {
-                const int kq = 4 * lane;
-                const int pq = __shfl_sync(0xffffffffu, phys, kq / p.page);
-                const int64_t src = ((int64_t)pq * p.Hk + hk) * p.page + (kq % p.page);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = kq + e, at = (key & 1) * 64 + (key >> 1);
-                    cp_async_4(dst + at, p.ksc + src + e);
-                    cp_async_4(dst + kKeys + at, p.vsc + src + e);
+                const unsigned badm = __ballot_sync(0xffffffffu, mine && bad_l) >> slot0;
+                if (lane == 0) {
+                    meta[c] = static_cast<int>(badm);
+                    mbar_arrive(&bars[Sm::kScFull + c]);
                 }
-                cp_async_mbar_arrive(&bars[Sm::kScFull + c]);
+                // per-token scales of keys 4 lane .. 4 lane + 3, stored by key
+                // parity for the softmax threads; with per-tensor scales the
+                // one K and one V scale in every slot
+                float* dst = scl + c * kScSlot;
+                if (p.per_tensor) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = 4 * lane + e, at = (key & 1) * kScPar + (key >> 1);
+                        dst[at] = ks_tensor;
+                        dst[kScHalf + at] = vs_tensor;
+                    }
+                    mbar_arrive(&bars[Sm::kScFull + c]);
+                } else {
+                    const int kq = 4 * lane;
+                    const int pq = __shfl_sync(0xffffffffu, phys_l, slot0 + kq / p.page);
+                    const int64_t src = ((int64_t)pq * p.Hk + hk) * p.page + (kq % p.page);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = kq + e, at = (key & 1) * kScPar + (key >> 1);
+                        cp_async_4(dst + at, p.ksc + src + e);
+                        cp_async_4(dst + kScHalf + at, p.vsc + src + e);
+                    }
+                    cp_async_mbar_arrive(&bars[Sm::kScFull + c]);
+                }
             }
             issued = i + 1;
         }
         // no copy of this CTA may land after it exits
-        for (int i = max(0, issued - kStages); i < issued; ++i)
-            mbar_wait_drain(&bars[Sm::kKvFull + i % kStages], (i / kStages) & 1);
-        for (int i = max(0, issued - kScStages); i < issued; ++i)
-            mbar_wait_drain(&bars[Sm::kScFull + i % kScStages], (i / kScStages) & 1);
+        if (kv) {
+            for (int i = max(0, issued - kStages); i < issued; ++i)
+                mbar_wait_drain(&bars[Sm::kKvFull + i % kStages], (i / kStages) & 1);
+        } else {
+            for (int i = max(0, issued - kScStages); i < issued; ++i)
+                mbar_wait_drain(&bars[Sm::kScFull + i % kScStages], (i / kScStages) & 1);
+        }
       } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && nt > 0) {
@@ -402,8 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             tmem_dealloc(tmem, 512);
         }
-        cluster_arrive_wait();
-        cluster_arrive_wait();
     } else if (warp < kSoftWarps) {
       reg_alloc<kRegsSoft>();
         // ------------------------------------------------------------ softmax
@@ -467,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (qq == 0) sq[r] = s;
             // the codes and scale also go to the caller's optional outputs
-            // (written once, by the first CTA of the cluster)
+            // (written once, by the first CTA of (b, hk))
             const bool qout = rv && split == 0 && p.q8_out != nullptr;
             const int64_t qtok = ((int64_t)b * p.T + t) * p.H + h;
             if (rv && split == 0 && qq == 0 && p.qs_out != nullptr) p.qs_out[qtok] = s;
@@ -527,8 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16x64(taddr + 128 * g, sv);
             tmem_wait_ld64(sv);
 
-            const float* ksP = scl + c * 2 * kKeys + cpar * 64;   // k_scale of column 2k + cpar
-            const float* vsP = ksP + kKeys;
+            const float* ksP = scl + c * kScSlot + cpar * kScPar;   // k_scale of column 2k + cpar
+            const float* vsP = ksP + kScHalf;
             const int key0 = (tb + i) * kKeys;
             const int badm = meta[c];
             // y = acc * k_scale; the logit is y * cq, and cq > 0 keeps the
@@ -682,11 +713,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (use1) l_fin = fmaf(grp[3 * kRows + r], w1, l_fin);
             }
         }
-        // ---- merge the splits of (b, hk) across the cluster (only the
-        // softmax warps hold registers enough for it). Every role ends with
-        // the same three barriers, reached from its own code: the CTA
-        // barrier (all roles done, the K stages free), then two cluster
-        // barriers around the exchange.
+        // ---- the CTA's (m, l, O) per row, staged row-major over the K stages
+        // (free once every role is past the CTA barrier): the output itself
+        // when the CTA holds every tile of (b, hk), else a partial in the
+        // workspace that the merge kernel combines
         tc_fence_before();
         bar_sync_all(kThreads);
         {
@@ -695,47 +725,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 32; ++k) oc[r * kOcPitch + 64 * g + 2 * k + cpar] = o_fin[k];
             if (g == 0 && cpar == 0) stat[r] = make_float2(m_fin, l_fin);
-            __syncwarp();
-            cluster_arrive_wait();
-            // CTA `split` writes rows split, split + nsplit, ...; thread: one
-            // row and four channels; all remote loads issued before any use
-            for (int idx = tid;; idx += kSoftWarps * 32) {
-                const int rr = split + p.nsplit * (idx >> 5), d4 = 4 * (idx & 31);
-                if (rr >= p.R) break;
-                float2 st[kMaxSplit];
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplit; ++sp)
-                    st[sp] = sp < p.nsplit ? dsmem_ld_f32x2(dsmem_addr(&stat[rr], sp)) : make_float2(-INFINITY, 0.0f);
-                float4 ov[kMaxSplit];
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplit; ++sp)
-                    ov[sp] = sp < p.nsplit ? dsmem_ld_f32x4(dsmem_addr(&oc[rr * kOcPitch + d4], sp))
-                                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                float M = -INFINITY;
-#pragma unroll
-                for (int sp = 0; sp < kMaxSplit; ++sp) M = fmaxf(M, st[sp].x);
-                float den = 0.0f;
-                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                if (M != -INFINITY) {
-#pragma unroll
-                    for (int sp = 0; sp < kMaxSplit; ++sp) {
-                        const float wgt = st[sp].x == -INFINITY ? 0.0f : ex2_approx(st[sp].x - M);
-                        den = fmaf(wgt, st[sp].y, den);
-                        acc.x = fmaf(wgt, ov[sp].x, acc.x);
-                        acc.y = fmaf(wgt, ov[sp].y, acc.y);
-                        acc.z = fmaf(wgt, ov[sp].z, acc.z);
-                        acc.w = fmaf(wgt, ov[sp].w, acc.w);
-                    }
+            named_sync(1, kSoftWarps * 32);
+            if (p.nsplit == 1) {
+                // thread: one row, four channels
+                for (int idx = tid; idx < p.R * 32; idx += kSoftWarps * 32) {
+                    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+                    const float2 st = stat[rr];
+                    store_out4(p, b, hk, rr, d4, *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4),
+                               st.y > 0.0f ? 1.0f / st.y : 0.0f);
                 }
-                const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-                const int t = rr / p.G, h = hk * p.G + rr % p.G;
-                __nv_bfloat16* dst = p.out + b * p.os0 + t * p.os1 + h * p.os2 + (int64_t)d4 * p.os3;
-                const float y[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(int64_t)e * p.os3] = __float2bfloat16_rn(y[e]);
+            } else {
+                // the partial to the workspace, combined by decode_merge_kernel
+                const size_t part = (size_t)bhk * p.nsplit + split;
+                float4* wo = reinterpret_cast<float4*>(p.ws_o + part * kRows * kD);
+                for (int idx = tid; idx < p.R * 32; idx += kSoftWarps * 32) {
+                    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+                    wo[idx] = *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4);
+                }
+                if (tid < p.R) p.ws_stat[part * kRows + tid] = stat[tid];
             }
-            __syncwarp();
-            cluster_arrive_wait();                  // no CTA leaves while others read it
         }
     } else {
       reg_dealloc<kRegsConv>();
@@ -799,9 +807,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before();
         bar_sync_all(kThreads);
-        cluster_arrive_wait();
-        cluster_arrive_wait();
     }
+}
+
+// The splits of (b, hk) combined (log-sum-exp): thread = one query row and
+// four channels; every split's (m, l) and O loaded before any use.
+__global__ void __launch_bounds__(256) decode_merge_kernel(const DecParams p) {
+    const int bhk = blockIdx.x, hk = bhk % p.Hk, b = bhk / p.Hk;
+    const int idx = blockIdx.y * 256 + threadIdx.x;
+    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+    if (rr >= p.R) return;
+    const size_t part0 = (size_t)bhk * p.nsplit;
+    float2 st[kMaxSplit];
+    float4 ov[kMaxSplit];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp) {
+        if (sp < p.nsplit) {
+            st[sp] = __ldcg(p.ws_stat + (part0 + sp) * kRows + rr);
+            ov[sp] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + ((part0 + sp) * kRows + rr) * kD + d4));
+        } else {
+            st[sp] = make_float2(-INFINITY, 0.0f);
+            ov[sp] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp) M = fmaxf(M, st[sp].x);
+    float den = 0.0f;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (M != -INFINITY) {
+#pragma unroll
+        for (int sp = 0; sp < kMaxSplit; ++sp) {
+            const float wgt = st[sp].x == -INFINITY ? 0.0f : ex2_approx(st[sp].x - M);
+            den = fmaf(wgt, st[sp].y, den);
+            acc.x = fmaf(wgt, ov[sp].x, acc.x);
+            acc.y = fmaf(wgt, ov[sp].y, acc.y);
+            acc.z = fmaf(wgt, ov[sp].z, acc.z);
+            acc.w = fmaf(wgt, ov[sp].w, acc.w);
+        }
+    }
+    store_out4(p, b, hk, rr, d4, acc, den > 0.0f ? 1.0f / den : 0.0f);
 }
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -842,29 +887,17 @@ bool encode_cache_vt(CUtensorMap* map, const void* ptr, int num_pages, int Hk) {
 
 constexpr int kSmemBytes = Sm::kBytes + 1024;
 
-// How many clusters of `size` CTAs of decode_kernel fit on the current
-// device at once (queried once per device and size).
-int max_active_clusters(int size) {
+// Streaming multiprocessors of the current device (queried once per device).
+int device_sms() {
     static std::mutex mu;
-    static int cache[64][kMaxSplit + 1] = {};
+    static int cache[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
     std::lock_guard<std::mutex> lock(mu);
-    int& c = cache[dev][size];
+    int& c = cache[dev];
     if (c == 0) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(size, 1);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = kSmemBytes;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = size;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, decode_kernel, &cfg) != cudaSuccess || n < 1) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
             cudaGetLastError();
             n = 1;
         }
@@ -873,17 +906,23 @@ int max_active_clusters(int size) {
     return c;
 }
 
-// CTAs per (sequence, kv head) = cluster size: the one (up to 8) that
-// minimises waves x tiles per CTA for the most 128-key tiles a sequence can
-// span; of equal choices the largest.
-int pick_nsplit(int n_clusters, int T, int window, int page, int max_pages) {
+// The most CTAs per (sequence, kv head): a split grid stays within one wave
+// (one CTA per SM), so that it and the merge are all the work there is.
+int max_split(int n_seq_heads) {
+    return std::max(1, std::min(kMaxSplit, device_sms() / std::max(1, n_seq_heads)));
+}
+
+// CTAs per (sequence, kv head): the one that minimises the most 128-key
+// tiles a CTA gets (for the most tiles a sequence can span) plus the merge,
+// counted as half a tile; of equal choices the smaller.
+int pick_nsplit(int n_seq_heads, int T, int window, int page, int max_pages) {
     const int64_t span = std::min<int64_t>((int64_t)window + T - 1, (int64_t)max_pages * page);
     const int64_t tiles = std::max<int64_t>(1, ceil_div(span, kKeys) + 1);
+    const int cap = max_split(n_seq_heads);
     int best = 1;
     int64_t best_cost = INT64_MAX;
-    for (int sz = static_cast<int>(std::min<int64_t>(kMaxSplit, tiles)); sz >= 1; --sz) {
-        const int64_t waves = ceil_div(n_clusters, max_active_clusters(sz));
-        const int64_t cost = waves * ceil_div(tiles, sz);
+    for (int sz = 1; sz <= std::min<int64_t>(cap, tiles); ++sz) {
+        const int64_t cost = 2 * ceil_div(tiles, sz) + (sz > 1 ? 1 : 0);
         if (cost < best_cost) {
             best_cost = cost;
             best = sz;
@@ -894,7 +933,12 @@ int pick_nsplit(int n_clusters, int T, int window, int page, int max_pages) {
 
 }  // namespace
 
-size_t decode_ws_bytes(int, int, int, int, int, int) { return 0; }
+// Partials for the most splits the launch may pick: (m, l) and O per row.
+size_t decode_ws_bytes(int B, int, int, int Hk, int, int) {
+    const int cap = max_split(B * Hk);
+    if (cap <= 1) return 0;
+    return (size_t)B * Hk * cap * kRows * (sizeof(float2) + kD * sizeof(float));
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     DecParams p;
@@ -939,19 +983,25 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     p.nsplit = pick_nsplit(a.B * a.Hk, a.T, a.window, a.page_size, a.max_pages);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.nsplit, a.B * a.Hk);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = p.nsplit;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel, tk, tv, p);
+    p.o_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 4 == 0 && a.out_stride[1] % 4 == 0 &&
+               a.out_stride[2] % 4 == 0 && reinterpret_cast<uintptr_t>(a.out) % 8 == 0)
+                  ? 1
+                  : 0;
+    p.ws_stat = nullptr;
+    p.ws_o = nullptr;
+    if (p.nsplit > 1) {
+        if (a.ws == nullptr) return cudaErrorInvalidValue;
+        p.ws_stat = static_cast<float2*>(a.ws);
+        p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
+                                          (size_t)a.B * a.Hk * p.nsplit * kRows * sizeof(float2));
+    }
+    decode_kernel<<<dim3(p.nsplit, a.B * a.Hk), kThreads, kSmemBytes, s>>>(tk, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.nsplit == 1) return e;
+    // a plain stream-ordered launch: it measured faster here than one
+    // launched as a programmatic dependent of the split grid
+    decode_merge_kernel<<<dim3(a.B * a.Hk, (p.R * 32 + 255) / 256), 256, 0, s>>>(p);
+    return cudaGetLastError();
 }
 
 unsigned read_clear_decode_error() {

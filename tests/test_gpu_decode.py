@@ -39,7 +39,7 @@ def _run(h, d, window, scale, q_layout="btHd", out_layout="btHd"):
         og = torch.empty((B, H, T, D + 8), dtype=torch.bfloat16, device="cuda").permute(0, 2, 1, 3)[..., :D]
     else:
         og = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((max(16, sage.sage_attn_decode_workspace(B, T, H, d["k_cache"].shape[1], D,
+    ws = torch.zeros((max(16, sage.sage_attn_decode_workspace(B, T, H, d["k_cache"].shape[1], D,
                                                                window)),),
                      dtype=torch.uint8, device="cuda")
     q8 = torch.full((B, T, H, D), 0x7F, dtype=torch.uint8, device="cuda")
@@ -183,7 +183,7 @@ def test_decode_reports_bad_page_ids(h128):
     ptab[1, 2] = d["num_pages"] + 7
     q = d["q"].cuda()
     out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    ws = None                                   # allocated by the binding
     sage.sage_attn_decode(h128, q, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(),
                           d["v_scale"].cuda(), ptab.cuda(), d["ctx_lens"].cuda(), 128, d["num_pages"],
                           4096, 1.0 / math.sqrt(128), out, ws)
@@ -209,7 +209,7 @@ def test_decode_cache_variants(h128, flags, B, T, H, Hk, lo, hi, window):
     scale = 1.0 / math.sqrt(128)
     q = d["q"].cuda()
     out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    ws = None                                   # allocated by the binding
     ksc, vsc, vc = d["k_scale"], d["v_scale"], d["v_cache"]
     kfull = ksc.expand(d["k_cache"].shape[:3]).contiguous() if flags & 1 else ksc
     vfull = vsc.expand(d["k_cache"].shape[:3]).contiguous() if flags & 1 else vsc
