@@ -72,14 +72,15 @@ constexpr int kSoftWarps = 8;                // warps 0..7
 constexpr int kConvWarp0 = 8;                // warps 8..11
 constexpr int kTmaWarp = 12;
 constexpr int kMmaWarp = 13;
-constexpr int kScaleWarp = 14;               // warp 15 idle until the merge
+constexpr int kScaleWarp = 14;
+constexpr int kIdleWarp = 15;                // initialises the barriers, then only completes a warpgroup
 constexpr int kThreads = 512;
-// registers per thread of each warpgroup (setmaxnreg; 256 x 176 + 128 x 96 +
-// 128 x 56 <= 512 x 128, the launch's registers; this split compiles without
+// registers per thread of each warpgroup (setmaxnreg; 256 x 176 + 128 x 80 +
+// 128 x 80 <= 512 x 128, the launch's registers; this split compiles without
 // spills). Only the softmax warps ever grow their share, after the others
 // have shrunk theirs, and no warp grows it again later: a warp that did
 // could take registers another one waits for.
-constexpr int kRegsSoft = 176, kRegsConv = 96, kRegsProd = 56;
+constexpr int kRegsSoft = 176, kRegsConv = 80, kRegsProd = 80;
 static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kOcPitch = kD + 4;             // fp32 row pitch of the merge area
@@ -213,6 +214,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = bhk / p.Hk, hk = bhk % p.Hk;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    // setup that reads no global memory (barriers, TMEM, the tensor maps of
+    // the parameter space) overlaps the preceding kernel in the stream when
+    // this grid is launched as its programmatic dependent; everything after
+    // griddepcontrol.wait sees that kernel's writes
+    if (warp == kIdleWarp) {
+        for (int i = lane; i < Sm::kNumBars; i += 32) {
+            uint32_t cnt = 1;                                       // expect_tx; commits
+            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + 4;     // QK commit + converters
+            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = 4 + 4;             // softmax group + converters
+            if (i == Sm::kQReady) cnt = kSoftWarps;
+            if (i >= Sm::kScFull && i < Sm::kScFull + kScStages) cnt = 1 + 32;    // bad-page mask + scale copies
+            if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = 4;       // softmax group
+            mbar_init(&bars[i], cnt);
+        }
+        if (lane == 0) *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    pdl_wait();
+    pdl_launch_dependents();
+
     int ctx = p.ctx[b];
     const int cap = p.max_pages * p.page;
     if (ctx > cap || ctx < 0) {
@@ -227,23 +256,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tb = t0 + (split * n_all) / p.nsplit;
     const int nt = t0 + ((split + 1) * n_all) / p.nsplit - tb;
 
-    if (tid == 0) {
-        for (int i = 0; i < Sm::kNumBars; ++i) {
-            uint32_t cnt = 1;                                       // expect_tx; commits
-            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + 4;     // QK commit + converters
-            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = 4 + 4;             // softmax group + converters
-            if (i == Sm::kQReady) cnt = kSoftWarps;
-            if (i >= Sm::kScFull && i < Sm::kScFull + kScStages) cnt = 1 + 32;    // bad-page mask + scale copies
-            if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = 4;       // softmax group
-            mbar_init(&bars[i], cnt);
-        }
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
     // the producer's first page-table entries, requested before the barrier
     const int ppt = kKeys / p.page;                  // pages per tile (divides 32)
     int pg_first = 0;
@@ -283,10 +295,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // by TMA, the lanes of a tile's pages each issuing their own boxes;
         // warp 14 loads the per-token scales and the tile's bad-page mask.
         const bool kv = warp == kTmaWarp;
-        if (kv && lane == 0) {
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-        }
         const float ks_tensor = (!kv && p.per_tensor) ? __ldg(p.ksc) : 0.0f;
         const float vs_tensor = (!kv && p.per_tensor) ? __ldg(p.vsc) : 0.0f;
         int chunk = -1, phys_l = 0;
@@ -387,17 +395,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mma_commit(&bars[Sm::kKvEmpty + s]);
                 return true;
             };
-            // order: QK(0), QK(1), then PV(j), QK(j + 2) for j = 0, 1, ...
-            // S(j + 2) is written once the softmax group of tile j is done
-            // with S(j) (its P'(j) implies that), and its commit covers PV(j):
-            // the group's P' buffer and O are free when S(j + 2) is there
+            // order: QK(0), QK(1), then for j = 0, 1, ...: once P'(j) is
+            // there, QK(j + 2) and PV(j) -- QK first when K(j + 2) has
+            // already landed, so that tile j's group can start on tile j + 2
+            // while PV(j) runs. S(j + 2) overwrites S(j), which the group read
+            // before it published P'(j); the group waits for PV(j) itself
+            // before it reuses its P' buffer and O.
             bool ok = mbar_wait(&bars[Sm::kQReady], 0, abort_flag, &g_decode_err, 12);
             if (ok) ok = issue_qk(0);
             if (ok && nt > 1) ok = issue_qk(1);
             for (int j = 0; ok && j < nt; ++j) {
-                // O[j & 1] += P'(j) V(j): 8 steps of 16 keys, all 128 channels
                 ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
                 if (!ok) break;
+                bool qk_next = false;
+                if (j + 2 < nt &&
+                    mbar_test_wait(smem_u32(&bars[Sm::kKvFull + (j + 2) % kStages]), ((j + 2) / kStages) & 1)) {
+                    ok = issue_qk(j + 2);
+                    qk_next = true;
+                }
+                // O[j & 1] += P'(j) V(j): 8 steps of 16 keys, all 128 channels
                 tc_fence_after();
                 const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
                 const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
@@ -421,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     kIdescPVT, (j > 1 || st > 0) ? 1u : 0u);
                 }
                 mma_commit(&bars[Sm::kPvDone + (j & 1)]);
-                if (j + 2 < nt) ok = issue_qk(j + 2);
+                if (ok && j + 2 < nt && !qk_next) ok = issue_qk(j + 2);
             }
             // drain every MMA this thread issued before TMEM is released
             mma_commit(&bars[Sm::kFinal]);
@@ -614,9 +630,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float sub = m_new == -INFINITY ? 0.0f : m_new;
             const uint64_t nsub2 = f2_pack(-sub, -sub);
 
-            // P' buffer g is free: PV(i - 2), its reader, is done -- the MMA
-            // thread issues it before QK(i), and the commit that completed
-            // S(i) covers every MMA that thread started earlier
+            // P' buffer g and O[g] are free once PV(i - 2) is done
+            if (i >= 2) {
+                ok = warp_all(mbar_wait(&bars[Sm::kPvDone + g], ((i - 2) >> 1) & 1, abort_flag,
+                                        &g_decode_err, 15));
+                if (!ok) break;
+                tc_fence_after();
+            }
             uint8_t* prow = sm + Sm::kP + g * Sm::kPBuf + r * 128;
 #pragma unroll
             for (int i16 = 0; i16 < 8; ++i16) {   // keys 16 i16 + cpar + 2m = registers 8 i16 + m
@@ -641,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
             // O[g] *= alpha for the rows whose max rose (PV(i - 2), its last
-            // writer, is done, as above), 64 columns at a time
+            // writer, is done), 64 columns at a time
             if (__any_sync(0xffffffffu, resc)) {
                 tc_fence_after();
 #pragma unroll
@@ -813,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // The splits of (b, hk) combined (log-sum-exp): thread = one query row and
 // four channels; every split's (m, l) and O loaded before any use.
 __global__ void __launch_bounds__(256) decode_merge_kernel(const DecParams p) {
+    pdl_launch_dependents();                 // the next decode may start its setup
     const int bhk = blockIdx.x, hk = bhk % p.Hk, b = bhk / p.Hk;
     const int idx = blockIdx.y * 256 + threadIdx.x;
     const int rr = idx >> 5, d4 = 4 * (idx & 31);
@@ -995,8 +1016,19 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
         p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) +
                                           (size_t)a.B * a.Hk * p.nsplit * kRows * sizeof(float2));
     }
-    decode_kernel<<<dim3(p.nsplit, a.B * a.Hk), kThreads, kSmemBytes, s>>>(tk, tv, p);
-    e = cudaGetLastError();
+    // a programmatic dependent of whatever precedes it on the stream: only
+    // the setup before griddepcontrol.wait overlaps that kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.nsplit, a.B * a.Hk);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_kernel, tk, tv, p);
     if (e != cudaSuccess || p.nsplit == 1) return e;
     // a plain stream-ordered launch: it measured faster here than one
     // launched as a programmatic dependent of the split grid
