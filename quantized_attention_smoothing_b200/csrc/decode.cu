@@ -381,6 +381,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, kD) | (1u << 16);    // bf16, B MN-major
             constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, kD);                // bf16, B K-major
             const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), 128);
+            // descriptors of the P' and V buffers, built once: a step of the
+            // MMA loops only adds a constant to the start-address field
+            // (V MN-major: two 64-channel swizzle atoms [128 keys][128 B], the
+            // second one kKeys * 128 bytes on, the leading byte offset; V^T
+            // converted K-major: 64-key atoms of [128 channels][128 B])
+            const uint64_t vlbo = p.v_trans ? 0ull : (static_cast<uint64_t>((kKeys * 128) >> 4) << 16) - (1ull << 16);
+            const uint64_t pdesc0 = umma_desc_kmajor(smem_u32(sm + Sm::kP), 128);
+            const uint64_t pdesc1 = umma_desc_kmajor(smem_u32(sm + Sm::kP + Sm::kPBuf), 128);
+            const uint64_t vdesc0 = umma_desc_kmajor(smem_u32(sm + Sm::kVb), 128) + vlbo;
+            const uint64_t vdesc1 = umma_desc_kmajor(smem_u32(sm + Sm::kVb + Sm::kVbBuf), 128) + vlbo;
             // S(i) = Q8 K8(i)^T into S buffer i & 1
             auto issue_qk = [&](int i) -> bool {
                 const int s = i % kStages;
@@ -414,27 +424,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     qk_next = true;
                 }
                 // O[j & 1] += P'(j) V(j): 8 steps of 16 keys, all 128 channels
+                // (P' atoms of 64 keys kRows * 128 bytes apart, 32 bytes per
+                // 16 keys inside one; V: 2048 bytes per 16 keys, or V^T atoms
+                // kD * 128 bytes apart and 32 bytes per 16 keys)
                 tc_fence_after();
-                const uint32_t pb = smem_u32(sm + Sm::kP + (j & 1) * Sm::kPBuf);
-                const uint32_t vb = smem_u32(sm + Sm::kVb + (j & 1) * Sm::kVbBuf);
+                const uint64_t pd = (j & 1) ? pdesc1 : pdesc0, vd = (j & 1) ? vdesc1 : vdesc0;
+                const uint32_t odst = tmem + kOCol + 128 * (j & 1);
                 if (!p.v_trans) {
-                    // V MN-major: two 64-channel swizzle atoms [128 keys][128 B], the
-                    // second one kKeys * 128 bytes on (the leading byte offset)
-                    const uint64_t vdesc = umma_desc_kmajor(vb, 128) +
-                                           (static_cast<uint64_t>((kKeys * 128) >> 4) << 16) - (1ull << 16);
 #pragma unroll
                     for (int st = 0; st < kKeys / 16; ++st)
-                        mma_bf16_ss(tmem + kOCol + 128 * (j & 1),
-                                    umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
-                                    vdesc + 128 * st, kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
+                        mma_bf16_ss(odst, pd + (st >> 2) * ((kRows * 128) >> 4) + 2 * (st & 3), vd + 128 * st,
+                                    kIdescPV, (j > 1 || st > 0) ? 1u : 0u);
                 } else {
-                    // V^T converted K-major: 64-key atoms of [128 channels][128 B]
 #pragma unroll
                     for (int st = 0; st < kKeys / 16; ++st)
-                        mma_bf16_ss(tmem + kOCol + 128 * (j & 1),
-                                    umma_desc_kmajor(pb + (st >> 2) * (kRows * 128), 128) + 2 * (st & 3),
-                                    umma_desc_kmajor(vb + (st >> 2) * (kD * 128), 128) + 2 * (st & 3),
-                                    kIdescPVT, (j > 1 || st > 0) ? 1u : 0u);
+                        mma_bf16_ss(odst, pd + (st >> 2) * ((kRows * 128) >> 4) + 2 * (st & 3),
+                                    vd + (st >> 2) * ((kD * 128) >> 4) + 2 * (st & 3), kIdescPVT,
+                                    (j > 1 || st > 0) ? 1u : 0u);
                 }
                 mma_commit(&bars[Sm::kPvDone + (j & 1)]);
                 if (ok && j + 2 < nt && !qk_next) ok = issue_qk(j + 2);
