@@ -312,7 +312,9 @@ size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window
  * receives the e4m3 codes of the rotated queries, contiguous [B, T, H, D];
  * q_scale_out (nullable): their scales s_q, contiguous fp32 [B, T, H] (the
  * codes the QK product used, for callers that reuse them or check them).
- * Supported: D == 128, page_size in {16, 32, 64, 128}, H % Hk == 0,
+ * Supported: D in {64, 128} (D = 256 is UNSUPPORTED: its K/V stages, bf16
+ * V and two O accumulators exceed one CTA's shared and tensor memory in
+ * this pipeline), page_size in {16, 32, 64, 128}, H % Hk == 0,
  * H / Hk <= 16, T * (H / Hk) <= 64, window >= 1; SAGE_KV_V_TRANSPOSED
  * needs page_size 128 (UNSUPPORTED otherwise), unknown kv_flags bits are
  * INVALID_ARG. ws: at least sage_attn_decode_workspace(...) bytes, 16-byte

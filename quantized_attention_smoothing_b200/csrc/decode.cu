@@ -62,7 +62,6 @@ namespace {
 __device__ unsigned g_decode_err;
 constexpr unsigned kErrDecodeRange = kErrRangeCode;   // ctx or page id out of range (clamped / masked)
 
-constexpr int kD = 128;
 constexpr int kKeys = 128;                   // keys per tile
 constexpr int kRows = 64;                    // query rows per CTA (M of every MMA)
 constexpr int kStages = 3;                   // K / V ring
@@ -83,21 +82,42 @@ constexpr int kThreads = 512;
 constexpr int kRegsSoft = 176, kRegsConv = 80, kRegsProd = 80;
 static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kOcPitch = kD + 4;             // fp32 row pitch of the merge area
 // A scale slot: k_scale then v_scale of the tile's keys, each by key parity
 // (index (key & 1) * kScPar + key / 2); the 4-float pad puts the two parities'
 // 16-byte reads in different banks
 constexpr int kScPar = kKeys / 2 + 4, kScHalf = 2 * kScPar, kScSlot = 2 * kScHalf;
 
+// Head size D (64 or 128): an e4m3 row of Q, K or V is D bytes, stored
+// with the swizzle of that span (128B or 64B); a bf16 V row is 2 D bytes,
+// one or two 64-channel 128B-swizzled atoms.
+// The 16-byte chunk c of row r of a D-byte swizzled e4m3 row tile.
+template <int D>
+__device__ __forceinline__ int e4m3_chunk(int c, int r) {
+    return D == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+}
+
+// N registers of 16 TMEM lanes and 2 N columns (shape 16x64b), loaded and
+// waited for: N = 32 or 16.
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld16x32(taddr, r);
+    tmem_wait_ld(r);
+}
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]) {
+    tmem_ld16x16(taddr, r);
+    tmem_wait_ld16(r);
+}
+
 // dynamic shared memory (offsets from a 1024-byte aligned base)
-struct Sm {
-    static constexpr int kQ = 0;                                   // [64][128] e4m3, 128B swizzle
-    static constexpr int kKStage = kKeys * kD;                     // 16 KB
-    static constexpr int kK = kQ + kRows * kD;                     // [stage][128][128] e4m3, 128B swizzle
-    static constexpr int kV = kK + kStages * kKStage;              // [stage][128][128] e4m3, 128B swizzle
+template <int D>
+struct SmL {
+    static constexpr int kOcPitch = D + 4;                         // fp32 row pitch of the merge area
+    static constexpr int kQ = 0;                                   // [64][D] e4m3
+    static constexpr int kKStage = kKeys * D;                      // [128][D] e4m3
+    static constexpr int kK = kQ + kRows * D;                      // [stage][128][D] e4m3
+    static constexpr int kV = kK + kStages * kKStage;              // [stage][128][D] e4m3 (V^T: [D][128])
     static constexpr int kPBuf = 2 * kRows * 128;                  // two 64-key atoms [64][128 B] bf16
     static constexpr int kP = kV + kStages * kKStage;              // [2 bufs] P' (A of PV)
-    static constexpr int kVbBuf = 2 * kKeys * 128;                 // two 64-channel halves [128][128 B] bf16
+    static constexpr int kVbBuf = kKeys * 2 * D;                   // D / 64 channel atoms [128][128 B] bf16
     static constexpr int kVb = kP + 2 * kPBuf;                     // [2 bufs] bf16 V (B of PV)
     static constexpr int kScale = kVb + 2 * kVbBuf;                // [slot] ks | vs fp32, padded
     static constexpr int kSq = kScale + kScStages * kScSlot * 4;   // [64] fp32 query scales
@@ -119,6 +139,7 @@ struct Sm {
     static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0 && kVb % 1024 == 0,
                   "swizzled tiles are 1024-byte aligned");
     static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
+    static_assert(D == 64 || D == 128, "head size");
 };
 
 struct DecParams {
@@ -196,9 +217,17 @@ __device__ __forceinline__ void store_out4(const DecParams& p, int b, int hk, in
     }
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecParams p) {
+    using Sm = SmL<D>;
+    constexpr int kD = D;
+    constexpr int kOcPitch = Sm::kOcPitch;
+    constexpr int kQe = D / 4;                    // query elements per rotating thread (4 per row)
+    constexpr int kQv = D / 32;                   // their 16-byte loads
+    constexpr int kLgQe = D == 128 ? 5 : 4;       // butterfly stages inside a thread
+    constexpr int kOe = D / 4;                    // output registers per epilogue thread (D / 2 columns)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -266,13 +295,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // the softmax warps' query row quarters (contiguous rows), also in flight
     // across the barrier
-    uint4 qv[4] = {};
+    uint4 qv[kQv] = {};
     if (warp < kSoftWarps && p.q_vec && (tid >> 2) < p.R) {
         const int r = tid >> 2;
         const uint4* src = reinterpret_cast<const uint4*>(p.q + b * p.qs0 + (r / p.G) * p.qs1 +
-                                                          (hk * p.G + r % p.G) * p.qs2) + 4 * (tid & 3);
+                                                          (hk * p.G + r % p.G) * p.qs2) + kQv * (tid & 3);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) qv[c] = __ldg(src + c);
+        for (int c = 0; c < kQv; ++c) qv[c] = __ldg(src + c);
     }
 
     tc_fence_before();
@@ -380,13 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdescQK = umma_idesc(1, 0, kRows, kKeys);              // e4m3 -> f32
             constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, kD) | (1u << 16);    // bf16, B MN-major
             constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, kD);                // bf16, B K-major
-            const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), 128);
+            const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), kD);
             // descriptors of the P' and V buffers, built once: a step of the
             // MMA loops only adds a constant to the start-address field
             // (V MN-major: two 64-channel swizzle atoms [128 keys][128 B], the
             // second one kKeys * 128 bytes on, the leading byte offset; V^T
             // converted K-major: 64-key atoms of [128 channels][128 B])
-            const uint64_t vlbo = p.v_trans ? 0ull : (static_cast<uint64_t>((kKeys * 128) >> 4) << 16) - (1ull << 16);
+            const uint64_t vlbo = (p.v_trans || kD == 64) ? 0ull
+                                                          : (static_cast<uint64_t>((kKeys * 128) >> 4) << 16) - (1ull << 16);
             const uint64_t pdesc0 = umma_desc_kmajor(smem_u32(sm + Sm::kP), 128);
             const uint64_t pdesc1 = umma_desc_kmajor(smem_u32(sm + Sm::kP + Sm::kPBuf), 128);
             const uint64_t vdesc0 = umma_desc_kmajor(smem_u32(sm + Sm::kVb), 128) + vlbo;
@@ -397,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2))
                     return false;
                 tc_fence_after();
-                const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), 128);
+                const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), kD);
 #pragma unroll
                 for (int kk = 0; kk < kD / 32; ++kk)
                     mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, kk > 0 ? 1u : 0u);
@@ -429,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // kD * 128 bytes apart and 32 bytes per 16 keys)
                 tc_fence_after();
                 const uint64_t pd = (j & 1) ? pdesc1 : pdesc0, vd = (j & 1) ? vdesc1 : vdesc0;
-                const uint32_t odst = tmem + kOCol + 128 * (j & 1);
+                const uint32_t odst = tmem + kOCol + kD * (j & 1);
                 if (!p.v_trans) {
 #pragma unroll
                     for (int st = 0; st < kKeys / 16; ++st)
@@ -469,11 +499,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int r = tid >> 2, qq = tid & 3;
             const bool rv = r < p.R;
             const int t = rv ? r / p.G : 0, h = rv ? hk * p.G + r % p.G : 0;
-            const uint16_t* src = p.q + b * p.qs0 + t * p.qs1 + h * p.qs2 + (int64_t)(qq * 32) * p.qs3;
-            float x[32];
+            const uint16_t* src = p.q + b * p.qs0 + t * p.qs1 + h * p.qs2 + (int64_t)(qq * kQe) * p.qs3;
+            float x[kQe];
             if (p.q_vec) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < kQv; ++c) {
                     const uint32_t wd[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};   // zeros past R
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -483,34 +513,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
 #pragma unroll
-                for (int d = 0; d < 32; ++d)
+                for (int d = 0; d < kQe; ++d)
                     x[d] = rv ? __uint_as_float(static_cast<uint32_t>(__ldg(src + d * p.qs3)) << 16) : 0.0f;
             }
-            // stages h = 1 .. 16 inside the quarter
+            // stages h = 1 .. D / 8 inside the quarter
 #pragma unroll
-            for (int lg = 0; lg < 5; ++lg) {
+            for (int lg = 0; lg < kLgQe; ++lg) {
                 const int hh = 1 << lg;
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
+                for (int kk = 0; kk < kQe / 2; ++kk) {
                     const int j = ((kk >> lg) << (lg + 1)) + (kk & (hh - 1));
                     const float a = x[j], c = x[j + hh];
                     x[j] = __fadd_rn(a, c);
                     x[j + hh] = __fsub_rn(a, c);
                 }
             }
-            // stages h = 32 and 64 across the row's threads: x[j] +- x[j + h]
+            // stages h = D / 4 and D / 2 across the row's threads: x[j] +- x[j + h]
 #pragma unroll
             for (int st = 1; st <= 2; st <<= 1) {
                 const bool upper = (qq & st) != 0;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+                for (int j = 0; j < kQe; ++j) {
                     const float y = __shfl_xor_sync(0xffffffffu, x[j], st);
                     x[j] = upper ? __fsub_rn(y, x[j]) : __fadd_rn(x[j], y);
                 }
             }
             float amax = 0.0f;
 #pragma unroll
-            for (int d = 0; d < 32; ++d) amax = fmaxf(amax, fabsf(x[d]));
+            for (int d = 0; d < kQe; ++d) amax = fmaxf(amax, fabsf(x[d]));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
             float s = 0.0f, rr = 0.0f;
@@ -524,9 +554,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool qout = rv && split == 0 && p.q8_out != nullptr;
             const int64_t qtok = ((int64_t)b * p.T + t) * p.H + h;
             if (rv && split == 0 && qq == 0 && p.qs_out != nullptr) p.qs_out[qtok] = s;
-            uint8_t* qrow = sm + Sm::kQ + r * 128;
+            uint8_t* qrow = sm + Sm::kQ + r * kD;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {            // 16-byte chunk 2 qq + c of the row
+            for (int c = 0; c < kD / 64; ++c) {      // 16-byte chunk (D / 64) qq + c of the row
                 uint32_t w4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -535,8 +565,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t hi16 = e4m3x2_rn_satfinite(__fmul_rn(x[d + 2], rr), __fmul_rn(x[d + 3], rr));
                     w4[e] = amax != 0.0f ? (lo16 | (hi16 << 16)) : 0u;   // a zero row: +0 codes
                 }
-                const int chunk = 2 * qq + c;
-                *reinterpret_cast<uint4*>(qrow + ((chunk ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                const int chunk = (kD / 64) * qq + c;
+                *reinterpret_cast<uint4*>(qrow + (e4m3_chunk<D>(chunk, r) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 if (qout)
                     *reinterpret_cast<uint4*>(p.q8_out + qtok * kD + 16 * chunk) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -671,13 +701,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (__any_sync(0xffffffffu, resc)) {
                 tc_fence_after();
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < kD / 64; ++hf) {
                     uint32_t o[32];
-                    tmem_ld16x32(taddr + kOCol + 128 * g + 64 * hf, o);
+                    tmem_ld16x32(taddr + kOCol + kD * g + 64 * hf, o);
                     tmem_wait_ld(o);
 #pragma unroll
                     for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                    tmem_st16x32(taddr + kOCol + 128 * g + 64 * hf, o);
+                    tmem_st16x32(taddr + kOCol + kD * g + 64 * hf, o);
                 }
                 tmem_wait_st();
             }
@@ -704,12 +734,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_sync(1, kSoftWarps * 32);
         // this warp's output channels: 64 g .. 64 g + 63 of its rows;
         // O = O[0] 2^(m0 - M) + O[1] 2^(m1 - M), l likewise, M = max(m0, m1)
-        float o_fin[32];
+        float o_fin[kOe];
         float m_fin = -INFINITY, l_fin = 0.0f;
         bool have = nt > 0 && warp_all(mbar_wait(&bars[Sm::kPvDone + ((nt - 1) & 1)], ((nt - 1) >> 1) & 1,
                                                  abort_flag, &g_decode_err, 9));
 #pragma unroll
-        for (int k = 0; k < 32; ++k) o_fin[k] = 0.0f;
+        for (int k = 0; k < kOe; ++k) o_fin[k] = 0.0f;
         if (have) {
             // (the TMEM loads are warp-wide: every lane takes them, and a row
             // whose group saw no key, m = -inf, takes none of their values)
@@ -720,21 +750,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 const bool use0 = m0 != -INFINITY;
                 const float w0 = use0 ? ex2_approx(m0 - m_fin) : 0.0f;
-                uint32_t o0[32];
-                tmem_ld16x32(taddr + kOCol + 64 * g, o0);
-                tmem_wait_ld(o0);
+                uint32_t o0[kOe];
+                tmem_ld16_wait(taddr + kOCol + (kD / 2) * g, o0);
 #pragma unroll
-                for (int k = 0; k < 32; ++k) o_fin[k] = use0 ? __uint_as_float(o0[k]) * w0 : 0.0f;
+                for (int k = 0; k < kOe; ++k) o_fin[k] = use0 ? __uint_as_float(o0[k]) * w0 : 0.0f;
                 l_fin = use0 ? grp[2 * kRows + r] * w0 : 0.0f;
             }
             if (nt > 1) {
                 const bool use1 = m1 != -INFINITY;
                 const float w1 = use1 ? ex2_approx(m1 - m_fin) : 0.0f;
-                uint32_t o1[32];
-                tmem_ld16x32(taddr + kOCol + 128 + 64 * g, o1);
-                tmem_wait_ld(o1);
+                uint32_t o1[kOe];
+                tmem_ld16_wait(taddr + kOCol + kD + (kD / 2) * g, o1);
 #pragma unroll
-                for (int k = 0; k < 32; ++k)
+                for (int k = 0; k < kOe; ++k)
                     o_fin[k] = use1 ? fmaf(__uint_as_float(o1[k]), w1, o_fin[k]) : o_fin[k];
                 if (use1) l_fin = fmaf(grp[3 * kRows + r], w1, l_fin);
             }
@@ -749,13 +777,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             float* oc = reinterpret_cast<float*>(sm + Sm::kOc);
             float2* stat = reinterpret_cast<float2*>(sm + Sm::kStat);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) oc[r * kOcPitch + 64 * g + 2 * k + cpar] = o_fin[k];
+            for (int k = 0; k < kOe; ++k) oc[r * kOcPitch + (kD / 2) * g + 2 * k + cpar] = o_fin[k];
             if (g == 0 && cpar == 0) stat[r] = make_float2(m_fin, l_fin);
             named_sync(1, kSoftWarps * 32);
             if (p.nsplit == 1) {
                 // thread: one row, four channels
-                for (int idx = tid; idx < p.R * 32; idx += kSoftWarps * 32) {
-                    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+                for (int idx = tid; idx < p.R * (kD / 4); idx += kSoftWarps * 32) {
+                    const int rr = idx / (kD / 4), d4 = 4 * (idx % (kD / 4));
                     const float2 st = stat[rr];
                     store_out4(p, b, hk, rr, d4, *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4),
                                st.y > 0.0f ? 1.0f / st.y : 0.0f);
@@ -764,8 +792,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the partial to the workspace, combined by decode_merge_kernel
                 const size_t part = (size_t)bhk * p.nsplit + split;
                 float4* wo = reinterpret_cast<float4*>(p.ws_o + part * kRows * kD);
-                for (int idx = tid; idx < p.R * 32; idx += kSoftWarps * 32) {
-                    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+                for (int idx = tid; idx < p.R * (kD / 4); idx += kSoftWarps * 32) {
+                    const int rr = idx / (kD / 4), d4 = 4 * (idx % (kD / 4));
                     wo[idx] = *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4);
                 }
                 if (tid < p.R) p.ws_stat[part * kRows + tid] = stat[tid];
@@ -790,14 +818,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &g_decode_err, 11));
             if (!ok) break;
             if (p.v_trans) {
-                // V^T tile [128 channels][128 keys]: lane -> channel row d; its
+                // V^T tile [D channels][128 keys]: lane -> channel row d; its
                 // keys become the row of a K-major bf16 operand in the key order
                 // of P' (per 16 keys: the even keys, then the odd ones)
                 const int d = 32 * cw + lane;
                 const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + d * 128;
                 uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + d * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {       // keys 16c .. 16c + 15
+                for (int c = 0; c < 8 && d < kD; ++c) {   // keys 16c .. 16c + 15
                     const uint4 u = *reinterpret_cast<const uint4*>(vrow + ((c ^ (d & 7)) << 4));
                     const uint32_t e0 = e4m3x2_to_bf16x2(u.x, 0x2404u), e1 = e4m3x2_to_bf16x2(u.y, 0x2404u);
                     const uint32_t e2 = e4m3x2_to_bf16x2(u.z, 0x2404u), e3 = e4m3x2_to_bf16x2(u.w, 0x2404u);
@@ -809,11 +837,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4*>(atom + (((g2 + 1) ^ (d & 7)) << 4)) = make_uint4(d0, d1, d2, d3);
                 }
             } else {
-            const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + kap * 128;
+            const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + kap * kD;
             uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + pos * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {           // channels 16c .. 16c + 15
-                const uint4 u = *reinterpret_cast<const uint4*>(vrow + ((c ^ (kap & 7)) << 4));
+            for (int c = 0; c < kD / 16; ++c) {     // channels 16c .. 16c + 15
+                const uint4 u = *reinterpret_cast<const uint4*>(vrow + (e4m3_chunk<D>(c, kap) << 4));
                 const uint32_t o0 = e4m3x2_to_bf16x2(u.x, 0x1404u), o1 = e4m3x2_to_bf16x2(u.x, 0x3424u);
                 const uint32_t o2 = e4m3x2_to_bf16x2(u.y, 0x1404u), o3 = e4m3x2_to_bf16x2(u.y, 0x3424u);
                 const uint32_t o4 = e4m3x2_to_bf16x2(u.z, 0x1404u), o5 = e4m3x2_to_bf16x2(u.z, 0x3424u);
@@ -838,11 +866,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // The splits of (b, hk) combined (log-sum-exp): thread = one query row and
 // four channels; every split's (m, l) and O loaded before any use.
+template <int D>
 __global__ void __launch_bounds__(256) decode_merge_kernel(const DecParams p) {
     pdl_launch_dependents();                 // the next decode may start its setup
     const int bhk = blockIdx.x, hk = bhk % p.Hk, b = bhk / p.Hk;
     const int idx = blockIdx.y * 256 + threadIdx.x;
-    const int rr = idx >> 5, d4 = 4 * (idx & 31);
+    const int rr = idx / (D / 4), d4 = 4 * (idx % (D / 4));
     if (rr >= p.R) return;
     const size_t part0 = (size_t)bhk * p.nsplit;
     float2 st[kMaxSplit];
@@ -851,7 +880,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const DecParams p) {
     for (int sp = 0; sp < kMaxSplit; ++sp) {
         if (sp < p.nsplit) {
             st[sp] = __ldcg(p.ws_stat + (part0 + sp) * kRows + rr);
-            ov[sp] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + ((part0 + sp) * kRows + rr) * kD + d4));
+            ov[sp] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + ((part0 + sp) * kRows + rr) * D + d4));
         } else {
             st[sp] = make_float2(-INFINITY, 0.0f);
             ov[sp] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -881,38 +910,41 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// The cache [num_pages, Hk, page, 128] e4m3 as a 3-D map {128 bytes, page
-// rows, num_pages * Hk}; one box = one page of one kv head, 128B swizzle.
-bool encode_cache(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int page) {
+// The cache [num_pages, Hk, page, D] e4m3 as a 3-D map {D bytes, page
+// rows, num_pages * Hk}; one box = one page of one kv head, with the swizzle
+// of a D-byte row (128B or 64B).
+bool encode_cache(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int page, int D) {
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(page),
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(page),
                                 static_cast<cuuint64_t>(num_pages) * Hk};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(page) * kD};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kD), static_cast<cuuint32_t>(page), 1};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(page) * D};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(page), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The transposed V cache [num_pages, Hk, 128, page = 128] as a 3-D map
-// {128 key bytes, 128 channel rows, num_pages * Hk}; one box = one page of
+// The transposed V cache [num_pages, Hk, D, page = 128] as a 3-D map
+// {128 key bytes, D channel rows, num_pages * Hk}; one box = one page of
 // one kv head as [channel][key], 128B swizzle.
-bool encode_cache_vt(CUtensorMap* map, const void* ptr, int num_pages, int Hk) {
+bool encode_cache_vt(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int D) {
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return false;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(kD),
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(D),
                                 static_cast<cuuint64_t>(num_pages) * Hk};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(kD) * kKeys};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kKeys), static_cast<cuuint32_t>(kD), 1};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kKeys), static_cast<cuuint64_t>(D) * kKeys};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kKeys), static_cast<cuuint32_t>(D), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr int kSmemBytes = Sm::kBytes + 1024;
+template <int D>
+constexpr int smem_bytes() { return SmL<D>::kBytes + 1024; }
 
 // Streaming multiprocessors of the current device (queried once per device).
 int device_sms() {
@@ -961,13 +993,17 @@ int pick_nsplit(int n_seq_heads, int T, int window, int page, int max_pages) {
 }  // namespace
 
 // Partials for the most splits the launch may pick: (m, l) and O per row.
-size_t decode_ws_bytes(int B, int, int, int Hk, int, int) {
+size_t decode_ws_bytes(int B, int, int, int Hk, int D, int) {
     const int cap = max_split(B * Hk);
     if (cap <= 1) return 0;
-    return (size_t)B * Hk * cap * kRows * (sizeof(float2) + kD * sizeof(float));
+    return (size_t)B * Hk * cap * kRows * (sizeof(float2) + D * sizeof(float));
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+namespace {
+
+template <int D>
+cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
+    constexpr int kSmemBytes = smem_bytes<D>();
     DecParams p;
     p.q = static_cast<const uint16_t*>(a.q.ptr);
     p.qs0 = a.q.stride[0];
@@ -1003,11 +1039,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
                   ? 1
                   : 0;
     CUtensorMap tk, tv;
-    if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size) ||
-        !(p.v_trans ? encode_cache_vt(&tv, a.v_cache, a.num_pages, a.Hk)
-                    : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size)))
+    if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size, D) ||
+        !(p.v_trans ? encode_cache_vt(&tv, a.v_cache, a.num_pages, a.Hk, D)
+                    : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size, D)))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     p.nsplit = pick_nsplit(a.B * a.Hk, a.T, a.window, a.page_size, a.max_pages);
     p.o_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 4 == 0 && a.out_stride[1] % 4 == 0 &&
@@ -1034,12 +1070,22 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel, tk, tv, p);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<D>, tk, tv, p);
     if (e != cudaSuccess || p.nsplit == 1) return e;
     // a plain stream-ordered launch: it measured faster here than one
     // launched as a programmatic dependent of the split grid
-    decode_merge_kernel<<<dim3(a.B * a.Hk, (p.R * 32 + 255) / 256), 256, 0, s>>>(p);
+    decode_merge_kernel<D><<<dim3(a.B * a.Hk, (p.R * (D / 4) + 255) / 256), 256, 0, s>>>(p);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+    switch (a.D) {
+        case 64: return launch_decode_d<64>(a, s);
+        case 128: return launch_decode_d<128>(a, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 unsigned read_clear_decode_error() {

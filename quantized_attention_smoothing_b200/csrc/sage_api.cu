@@ -481,7 +481,7 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
     for (int i = 0; i < 4; ++i)
         if (q_bf16.size[i] != want[i] || out_bf16.size[i] != want[i]) return SAGE_ERR_INVALID_ARG;
     if (D != h->D) return SAGE_ERR_INVALID_ARG;
-    if (D != 128) return SAGE_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
     if (H % Hk != 0 || H / Hk > 16 || T * (H / Hk) > 64) return SAGE_ERR_UNSUPPORTED;
     if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
         return SAGE_ERR_UNSUPPORTED;

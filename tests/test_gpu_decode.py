@@ -26,6 +26,13 @@ def h128():
     return sage.Hadamard(128)
 
 
+@pytest.fixture(scope="module")
+def h64():
+    from quantized_attention_smoothing_b200 import build
+    build.build()
+    return sage.Hadamard(64)
+
+
 def _run(h, d, window, scale, q_layout="btHd", out_layout="btHd"):
     q = d["q"]
     B, T, H, D = q.shape
@@ -242,3 +249,50 @@ def test_decode_rejects_bad_kv_flags(h128):
     with pytest.raises(sage.SageError) as e:
         sage.sage_attn_decode(*args, kv_flags=4)
     assert e.value.status == sage.SAGE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,T,H,Hk,page,lo,hi,window", [
+    (16, 4, 16, 1, 128, 4096, 8192, 4096),  # the window-family shape at D = 64
+    (3, 4, 8, 2, 16, 40, 90, 32),           # page 16, window < ctx, R = 16
+    (2, 1, 8, 1, 128, 100, 300, 512),       # T = 1, window >= ctx, R = 8 (padded rows)
+    (2, 2, 16, 2, 64, 257, 700, 256),       # page 64, R = 16
+    (1, 3, 12, 3, 32, 1000, 1000, 300),     # page 32, T = 3, G = 4
+])
+def test_decode_head64(h64, B, T, H, Hk, page, lo, hi, window):
+    """Head size 64 ("[FlyDSL] [Misc] pa_decode ...", Performance: FP8 KV at
+    D64/128/256): 64-byte e4m3 rows (64B swizzle), a 64-channel bf16 V and
+    PV of N = 64; query codes bit-exact and the output within tolerance."""
+    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=64, page=page, ctx_lo=lo, ctx_hi=hi,
+                              seed=B * 3000 + page + window)
+    gpu, ref = _run(h64, d, window, 1.0 / math.sqrt(64))
+    stats = compare_output(gpu, ref, None, label="D64 %s" % ((B, T, H, Hk, page, window),))
+    assert stats["cos_oracle"] >= 0.9999
+
+
+def test_decode_head64_strided_views(h64):
+    d = workloads.make_decode(B=2, T=4, H=16, Hk=1, D=64, page=64, ctx_lo=500, ctx_hi=900, seed=23)
+    gpu, ref = _run(h64, d, 1024, 0.125, q_layout="strided", out_layout="strided")
+    compare_output(gpu, ref, None, label="D64 strided")
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3])
+def test_decode_head64_cache_variants(h64, flags):
+    """Per-tensor scales and the transposed V cache ([num_pages, Hk, 64, 128])
+    at D = 64, against the oracle on the same layout."""
+    d = workloads.make_decode(B=4, T=4, H=16, Hk=1, D=64, page=128, ctx_lo=600, ctx_hi=2000,
+                              seed=70 + flags, scale_mode="per_tensor" if flags & 1 else "per_token")
+    scale, window = 0.125, 1024
+    q = d["q"].cuda()
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    vc = d["v_cache"]
+    if flags & 2:
+        vc = vc.permute(0, 1, 3, 2).contiguous()
+    sage.sage_attn_decode(h64, q, d["k_cache"].cuda(), vc.cuda(), d["k_scale"].cuda(), d["v_scale"].cuda(),
+                          d["page_table"].cuda(), d["ctx_lens"].cuda(), 128, d["num_pages"], window, scale,
+                          out, kv_flags=flags)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    _, ref, margin = oracle.decode(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), vc.numpy(),
+                                   d["k_scale"].numpy(), d["v_scale"].numpy(), d["page_table"].numpy(),
+                                   d["ctx_lens"].numpy(), window, scale, want_flip=True, kv_flags=flags)
+    compare_output(bits(out), (ref, margin), None, label="D64 kv_flags %d" % flags)
