@@ -38,10 +38,15 @@ DECODE = {
     "c5": dict(name="gqa_paged_decode_b16_t4_h16_hk1_d128_p128_w4096", B=16, T=4, H=16, Hk=1,
                D=128, page=128, ctx_lo=4096, ctx_hi=8192, window=4096,
                softmax_scale=1.0 / math.sqrt(128.0)),
+    # the same window-family shape at head size 64 (the pages' decode shape
+    # list runs D 64/128/256)
+    "c5_d64": dict(name="gqa_paged_decode_b16_t4_h16_hk1_d64_p128_w4096", B=16, T=4, H=16, Hk=1,
+                   D=64, page=128, ctx_lo=4096, ctx_hi=8192, window=4096,
+                   softmax_scale=1.0 / math.sqrt(64.0)),
 }
 
 SEED_BASE = 20260000
-CONFIG_INDEX = {"c1": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5}
+CONFIG_INDEX = {"c1": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5, "c5_d64": 6}
 
 
 def seed_for(key):
