@@ -296,3 +296,15 @@ def test_decode_head64_cache_variants(h64, flags):
                                    d["k_scale"].numpy(), d["v_scale"].numpy(), d["page_table"].numpy(),
                                    d["ctx_lens"].numpy(), window, scale, want_flip=True, kv_flags=flags)
     compare_output(bits(out), (ref, margin), None, label="D64 kv_flags %d" % flags)
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_decode_one_split_per_sequence(h128, h64, D):
+    """B * Hk at or above the SM count: every (sequence, kv head) runs in one
+    CTA, which normalises and writes its rows itself (no workspace, no merge
+    launch)."""
+    B = 160
+    assert sage.sage_attn_decode_workspace(B, 2, 8, 1, D, 96) == 0
+    d = workloads.make_decode(B=B, T=2, H=8, Hk=1, D=D, page=16, ctx_lo=20, ctx_hi=300, seed=400 + D)
+    gpu, ref = _run(h128 if D == 128 else h64, d, 96, 1.0 / math.sqrt(D))
+    compare_output(gpu, ref, None, label="one split, D %d" % D)
