@@ -13,6 +13,7 @@ improvements": no forced contiguous copies).
 """
 import ctypes
 import os
+import threading
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -32,7 +33,18 @@ _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
 
 
+_lib_lock = threading.Lock()
+
+
 def lib():
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:                     # worker threads may ask for it at once
+        return _load()
+
+
+def _load():
     global _lib
     if _lib is None:
         path = _build.build()
@@ -92,6 +104,10 @@ def lib():
         L.or_decode_seq.argtypes = [_u16p, _u8p, _u8p, _f32p, _f32p, _i32p, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                     ctypes.c_int, ctypes.c_int, ctypes.c_double, _u16p, _f64p]
+        L.or_decode_seq_mxkv.restype = None
+        L.or_decode_seq_mxkv.argtypes = [_u16p, _u8p, _u8p, _u8p, _u8p, _i32p, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_double, _u16p, _f64p, _f64p]
         _lib = L
     return _lib
 
@@ -347,6 +363,44 @@ def decode(q, kc, vc, ksc, vsc, ptab, ctx, window, softmax_scale, threads=None, 
                                   int(window), float(softmax_scale), int(kv_flags), _p(oo, _u16p),
                                   _p(of, _f64p) if want_f64 else None,
                                   _p(ff, _f64p) if want_flip else None)
+        out[b] = oo
+        if want_f64:
+            o64[b] = of
+        if want_flip:
+            flip[b] = ff
+
+    _pool_map(one, list(range(B)), threads)
+    if want_flip:
+        return out, o64, flip
+    return (out, o64) if want_f64 else out
+
+
+def decode_mxfp4(q, kc, vc, ksf, vsf, ptab, ctx, window, softmax_scale, threads=None, want_f64=False,
+                 want_flip=False):
+    """Paged decode over an MXFP4 cache. q: uint16 [B, T, H, D]; kc, vc:
+    uint8 [num_pages, Hk, page, D / 2] packed E2M1 (element 2i in the low
+    nibble of byte i); ksf, vsf: uint8 e8m0 [num_pages, Hk, page, D / 32];
+    ptab: int32 [B, max_pages]; ctx: int32 [B]. Returns bf16 bits (and the
+    fp64 values, and with want_flip the bf16-weight margin) like decode()."""
+    B, T, H, D = q.shape
+    Hk, page = kc.shape[1], kc.shape[2]
+    want_f64 = want_f64 or want_flip
+    kc, vc = np.ascontiguousarray(kc, dtype=np.uint8), np.ascontiguousarray(vc, dtype=np.uint8)
+    ksf, vsf = np.ascontiguousarray(ksf, dtype=np.uint8), np.ascontiguousarray(vsf, dtype=np.uint8)
+    out = np.zeros((B, T, H, D), dtype=np.uint16)
+    o64 = np.zeros((B, T, H, D), dtype=np.float64) if want_f64 else None
+    flip = np.zeros((B, T, H, D), dtype=np.float64) if want_flip else None
+
+    def one(b):
+        qq = np.ascontiguousarray(q[b])
+        pt = np.ascontiguousarray(ptab[b], dtype=np.int32)
+        oo = np.zeros((T, H, D), dtype=np.uint16)
+        of = np.zeros((T, H, D), dtype=np.float64) if want_f64 else None
+        ff = np.zeros((T, H, D), dtype=np.float64) if want_flip else None
+        lib().or_decode_seq_mxkv(_p(qq, _u16p), _p(kc, _u8p), _p(vc, _u8p), _p(ksf, _u8p), _p(vsf, _u8p),
+                                 _p(pt, _i32p), int(ctx[b]), T, H, Hk, D, page, int(window),
+                                 float(softmax_scale), _p(oo, _u16p), _p(of, _f64p) if want_f64 else None,
+                                 _p(ff, _f64p) if want_flip else None)
         out[b] = oo
         if want_f64:
             o64[b] = of

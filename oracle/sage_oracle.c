@@ -750,6 +750,88 @@ void or_decode_seq_flags(const uint16_t* q, const uint8_t* kc, const uint8_t* vc
     free(qc);
 }
 
+/* Paged decode over an MXFP4 cache ("[FlyDSL] [Misc] pa_decode ...", Changes:
+   uint8 KV is MXFP4, packed float4_e2m1fn_x2 with float8_e8m0fnu scales; the
+   MXFP4 cache's compute type is bf16; Q is quantised to E4M3). kc, vc:
+   [num_pages, Hk, page, D / 2] bytes, element 2i in the low nibble of byte
+   i; ksf, vsf: [num_pages, Hk, page, D / 32] e8m0 bytes, one per 32
+   consecutive channels of a token (value 2^(E - 127); 255 is NaN). A cached
+   element is e2m1(code) * 2^(E - 127), exact. The query is rotated and
+   quantised as for the FP8 cache; S_j = (q8 . k_j) * s_q * softmax_scale / D
+   (the block scales sit inside k_j, no per-token scale); the PV weight is
+   p_j rounded to bf16 (reading: bf16 operands as for the FP8 cache, since the
+   split-KV kernel rounds at its own running maxima and an e4m3 P would
+   round differently from one split to the next). */
+static double or_mx_elem(const uint8_t* codes, const uint8_t* sf, int64_t tok, int D, int e)
+{
+    const uint8_t byte = codes[tok * (D / 2) + e / 2];
+    const uint8_t E = sf[tok * (D / 32) + e / 32];
+    if (E == 255) return NAN;
+    return or_e2m1_decode((uint8_t)((e & 1) ? (byte >> 4) : (byte & 15))) * ldexp(1.0, (int)E - 127);
+}
+
+void or_decode_seq_mxkv(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const uint8_t* ksf,
+                        const uint8_t* vsf, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
+                        int page, int window, double softmax_scale, uint16_t* out, double* out_f64,
+                        double* flip_f64)
+{
+    uint8_t* qc = (uint8_t*)malloc((size_t)D);
+    double* q8 = (double*)malloc(sizeof(double) * (size_t)D);
+    double* o = (double*)malloc(sizeof(double) * (size_t)D);
+    double* F = (double*)malloc(sizeof(double) * (size_t)D);
+    double* sv = (double*)malloc(sizeof(double) * (size_t)(window > 0 ? window : 1));
+    const int group = H / Hk;
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            const int hk = h / group;
+            const uint16_t* qr = q + ((int64_t)t * H + h) * D;
+            float s = 0.0f;
+            or_decode_quant_q_row(qr, D, qc, &s);
+            for (int e = 0; e < D; ++e) q8[e] = or_e4m3_decode(qc[e]);
+            const int p = ctx - T + t;
+            int lo = p - window + 1;
+            if (lo < 0) lo = 0;
+            const int n = p - lo + 1;
+            double mx = -INFINITY;
+            for (int u = 0; u < n; ++u) {
+                const int j = lo + u;
+                const int64_t tok = ((int64_t)ptab[j / page] * Hk + hk) * page + (j % page);
+                double acc = 0.0;
+                for (int e = 0; e < D; ++e) acc += q8[e] * or_mx_elem(kc, ksf, tok, D, e);
+                sv[u] = acc * (double)s * (softmax_scale / (double)D);
+                if (sv[u] > mx) mx = sv[u];
+            }
+            for (int e = 0; e < D; ++e) o[e] = F[e] = 0.0;
+            double den = 0.0;
+            for (int u = 0; u < n; ++u) {
+                const int j = lo + u;
+                const int64_t tok = ((int64_t)ptab[j / page] * Hk + hk) * page + (j % page);
+                double pj = exp(sv[u] - mx);
+                den += pj;
+                const uint16_t wb = or_f64_to_bf16((double)(float)pj);      /* bf16 PV weight */
+                double w = (double)or_bf16_to_f32(wb);
+                const double wmar = flip_f64 ? 0.5 * ((double)or_bf16_to_f32((uint16_t)(wb + 1)) - w) + ldexp(w, -8)
+                                             : 0.0;
+                for (int e = 0; e < D; ++e) {
+                    const double v = or_mx_elem(vc, vsf, tok, D, e);
+                    o[e] += w * v;
+                    if (flip_f64) F[e] += wmar * fabs(v);
+                }
+            }
+            for (int e = 0; e < D; ++e) {
+                double y = o[e] / den;
+                out[((int64_t)t * H + h) * D + e] = or_f64_to_bf16(y);
+                if (out_f64) out_f64[((int64_t)t * H + h) * D + e] = y;
+                if (flip_f64) flip_f64[((int64_t)t * H + h) * D + e] = F[e] / den;
+            }
+        }
+    free(sv);
+    free(F);
+    free(o);
+    free(q8);
+    free(qc);
+}
+
 void or_decode_seq(const uint16_t* q, const uint8_t* kc, const uint8_t* vc, const float* ksc,
                    const float* vsc, const int32_t* ptab, int ctx, int T, int H, int Hk, int D,
                    int page, int window, double softmax_scale, uint16_t* out, double* out_f64)

@@ -216,3 +216,59 @@ def test_decode_weight_margin_bounds_rounding_at_another_scale(oracle_mod):
     assert (dev > 1e-4).sum() > 0
     bad = _fp32_weight_decode(oracle_mod, d, 256, scale, 2.0 ** -5, rng)
     assert float((np.abs(bad - y) - margin).max()) > 1e-4
+
+
+# OCP MX E2M1 magnitudes by the code's low three bits (bit 3 is the sign)
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _mx_dequant(codes, sf, D):
+    """Packed E2M1 [..., D/2] (element 2i in the low nibble of byte i) with
+    e8m0 scales [..., D/32] -> float64 [..., D]."""
+    nib = np.stack([codes & 15, codes >> 4], axis=-1).reshape(codes.shape[:-1] + (D,))
+    val = np.where(nib & 8, -_E2M1[nib & 7], _E2M1[nib & 7])
+    return val * np.repeat(np.exp2(sf.astype(np.float64) - 127.0), 32, axis=-1)
+
+
+@pytest.mark.parametrize("B,T,H,Hk,D,window", [(2, 4, 16, 2, 128, 256), (3, 1, 8, 1, 64, 1000)])
+def test_decode_mxfp4_cache_matches_brute_force(oracle_mod, B, T, H, Hk, D, window):
+    """The MXFP4-cache decode (packed E2M1 K/V with an e8m0 scale per 32
+    channels of a token) equals a brute force over the dequantised un-paged
+    cache: the format's value table and 2^(E - 127), scipy's Hadamard matrix,
+    torch's float8 cast of the rotated query and torch's bfloat16 cast of the
+    PV weights p_j."""
+    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=D, page=128, ctx_lo=150, ctx_hi=600, seed=60 + D,
+                              kv_format="mxfp4")
+    scale = 1.0 / math.sqrt(D)
+    out, o64 = oracle_mod.decode_mxfp4(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), d["v_cache"].numpy(),
+                                       d["k_scale"].numpy(), d["v_scale"].numpy(), d["page_table"].numpy(),
+                                       d["ctx_lens"].numpy(), window, scale, want_f64=True)
+    q = d["q"].float().numpy()
+    Hmat = scipy.linalg.hadamard(D).astype(np.float64)
+    kdq = _mx_dequant(d["k_cache"].numpy(), d["k_scale"].numpy(), D)
+    vdq = _mx_dequant(d["v_cache"].numpy(), d["v_scale"].numpy(), D)
+    ref = np.zeros((B, T, H, D))
+    for b in range(B):
+        ctx = int(d["ctx_lens"][b])
+        toks = np.arange(ctx)
+        phys = d["page_table"][b].numpy()[toks // 128]
+        for h in range(H):
+            hk = h // (H // Hk)
+            K, V = kdq[phys, hk, toks % 128], vdq[phys, hk, toks % 128]
+            for t in range(T):
+                qh = q[b, t, h] @ Hmat
+                a = np.float32(np.abs(qh).max())
+                s = a / np.float32(448.0)
+                q8 = torch.from_numpy((qh * (np.float32(448.0) / a)).astype(np.float32)).to(torch.float8_e4m3fn)
+                q8 = q8.to(torch.float64).numpy()
+                p = ctx - T + t
+                sl = slice(max(0, p - window + 1), p + 1)
+                logits = (K[sl] @ q8) * float(s) * (scale / D)
+                w = np.exp(logits - logits.max())
+                wb = torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+                ref[b, t, h] = (wb @ V[sl]) / w.sum()
+    assert np.abs(o64 - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    assert np.array_equal(out, oracle_mod.f64_to_bf16(o64))
+    # the block scales matter: with every scale taken as 1 the outputs move
+    flat = _mx_dequant(d["k_cache"].numpy(), np.full_like(d["k_scale"].numpy(), 127), D)
+    assert not np.allclose(flat, kdq)

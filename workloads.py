@@ -108,7 +108,8 @@ def make_prefill_config(key, layout="blhd", seed=None):
     return cfg, q, k, v
 
 
-def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, scale_mode="per_token", **_unused):
+def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, scale_mode="per_token", kv_format="fp8",
+                **_unused):
     """Paged FP8 decode inputs.
 
     ctx_b ~ U{ctx_lo..ctx_hi}; the pages of all sequences are one random
@@ -118,6 +119,10 @@ def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, scale_mode="per_toke
     k_scale and v_scale are then one-element tensors), the cast done by
     torch's float8_e4m3fn conversion (the cache writer itself is not part of
     the path). Queries are bf16 N(0, 1), [B, T, H, D].
+    kv_format="mxfp4": an MXFP4 cache instead, drawn directly in its storage
+    format: uniform random E2M1 codes packed two per byte [num_pages, Hk,
+    page, D / 2] and e8m0 block scales [num_pages, Hk, page, D / 32] (uint8,
+    in k_scale / v_scale) uniform in 2^-3 .. 2^1.
     Returns a dict of CPU tensors.
     """
     g = torch.Generator().manual_seed(int(seed))
@@ -143,8 +148,13 @@ def make_decode(B, T, H, Hk, D, page, ctx_lo, ctx_hi, seed, scale_mode="per_toke
         codes = (x / scale.unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
         return codes.contiguous(), scale.to(torch.float32).contiguous()
 
-    kc, ksc = cache()
-    vc, vsc = cache()
+    def cache_mx():
+        codes = torch.randint(0, 256, (total, Hk, page, D // 2), generator=g, dtype=torch.int32)
+        sf = 127 + torch.randint(-3, 2, (total, Hk, page, D // 32), generator=g, dtype=torch.int32)
+        return codes.to(torch.uint8).contiguous(), sf.to(torch.uint8).contiguous()
+
+    kc, ksc = cache_mx() if kv_format == "mxfp4" else cache()
+    vc, vsc = cache_mx() if kv_format == "mxfp4" else cache()
     q = torch.randn((B, T, H, D), generator=g).to(torch.bfloat16)
     return dict(q=q, k_cache=kc, v_cache=vc, k_scale=ksc, v_scale=vsc, page_table=ptab,
                 ctx_lens=ctx.to(torch.int32), num_pages=total, max_pages=max_pages)
