@@ -29,6 +29,7 @@
  *                        batch-first plan grid", Changes), bf16 output.
  *   sage_attn_decode     paged FP8-KV decode (same page: window-family
  *                        workload, per-token FP8 K/V scales, MTP, GQA).
+ *   sage_attn_decode_mxfp4  the same decode over an MXFP4 KV cache.
  *
  * Conventions shared by every entry point
  *   - All tensor pointers are DEVICE pointers on the device that is current
@@ -328,6 +329,33 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
                              int window, float softmax_scale, int kv_flags, sage_view4 out_bf16,
                              uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
                              void* stream);
+
+/* Paged decode over an MXFP4 cache ("[FlyDSL] [Misc] pa_decode ...",
+ * Changes: a uint8 cache is MXFP4, packed E2M1 with e8m0 scales, and the
+ * query is quantised to E4M3 for it; Performance: MXFP4 KV, GQA 16, page
+ * 128, batch 1 / 32 / 256, ctx 2k / 32k).
+ *   k_cache, v_cache: E2M1 codes [num_pages, Hk, page_size, D / 2] bytes,
+ *   contiguous, element 2i in the low nibble of byte i and 2i + 1 in the
+ *   high one (nibble: sign, two exponent bits, one mantissa bit: 0, 0.5, 1,
+ *   1.5, 2, 3, 4, 6); k_sf, v_sf: e8m0 block scales [num_pages, Hk,
+ *   page_size, D / 32] bytes, contiguous, 16-byte aligned: element e of a
+ *   token is code(e) * 2^(sf[e / 32] - 127). Everything else is as for
+ *   sage_attn_decode (same query quantisation, windows, q8_out /
+ *   q_scale_out, workspace and launches) with k_scale = v_scale = 1: S_j =
+ *   (q8 . k_j) * s_q * softmax_scale / D; out = sum_j p_j v_j -> bf16, the
+ *   weights p_j rounded to bf16 before the PV product. The dequantised K and
+ *   V are exact in bf16 for scale codes 0 .. 252; codes 253 .. 255
+ *   (values beyond the bf16 range, and NaN) are outside the contract and
+ *   read as 252, so the unused slots of the pages a window touches may hold
+ *   any bytes. Supported: D = 128 (other D: UNSUPPORTED), page_size in
+ *   {16, 32, 64, 128}, H % Hk == 0, H / Hk <= 16, T * (H / Hk) <= 64. */
+sage_status sage_attn_decode_mxfp4(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
+                                   const uint8_t* v_cache, const uint8_t* k_sf, const uint8_t* v_sf,
+                                   const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
+                                   int H, int Hk, int D, int page_size, int max_pages, int num_pages,
+                                   int window, float softmax_scale, sage_view4 out_bf16,
+                                   uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
+                                   void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* sage_status_string(sage_status s);

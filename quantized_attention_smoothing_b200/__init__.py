@@ -32,7 +32,7 @@ EXPORTS = (
     "sage_quant_qkv",
     "sage_attn_fwd_workspace", "sage_attn_fwd", "sage_attn_fwd_q16", "sage_attn_decode_workspace",
     "sage_attn_decode", "sage_status_string", "sage_device_error", "sage_device_error_where",
-    "sage_wait_probe", "sage_quant_qk_mx", "sage_attn_fwd_mx",
+    "sage_wait_probe", "sage_quant_qk_mx", "sage_attn_fwd_mx", "sage_attn_decode_mxfp4",
 )
 
 SAGE_KERNEL_ATTN = 1
@@ -107,6 +107,9 @@ def lib():
     L.sage_attn_decode.restype = i32
     L.sage_attn_decode.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 9 + \
         [f32, i32, View4, vp, vp, vp, sz, vp]
+    L.sage_attn_decode_mxfp4.restype = i32
+    L.sage_attn_decode_mxfp4.argtypes = [vp, CView4, vp, vp, vp, vp, vp, vp] + [i32] * 9 + \
+        [f32, View4, vp, vp, vp, sz, vp]
     L.sage_device_error.restype = i32
     L.sage_device_error.argtypes = [vp]
     L.sage_device_error_where.restype = i32
@@ -285,6 +288,28 @@ def sage_attn_decode(h, q, k_cache, v_cache, k_scale, v_scale, page_table, ctx_l
                                   _ptr(q8_out), _ptr(q_scale_out), _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(),
                                   _stream(stream)), "sage_attn_decode")
+
+
+def sage_attn_decode_mxfp4(h, q, k_cache, v_cache, k_sf, v_sf, page_table, ctx_lens, page_size,
+                           num_pages, window, softmax_scale, out, ws=None, stream=None, q8_out=None,
+                           q_scale_out=None):
+    """Paged decode over an MXFP4 cache: k_cache / v_cache uint8 [num_pages,
+    Hk, page, D / 2] (two E2M1 codes a byte), k_sf / v_sf uint8 e8m0
+    [num_pages, Hk, page, D / 32]."""
+    B, T, H, D = q.shape
+    Hk = k_cache.shape[1]
+    max_pages = page_table.shape[1]
+    if ws is None:
+        n = sage_attn_decode_workspace(B, T, H, Hk, D, window)
+        if n > 0:
+            ws = torch.empty((n,), dtype=torch.uint8, device=q.device)
+    _check(lib().sage_attn_decode_mxfp4(h.handle, _view(q, CView4), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(k_sf), _ptr(v_sf), _ptr(page_table), _ptr(ctx_lens),
+                                        B, T, H, Hk, D, int(page_size), int(max_pages), int(num_pages),
+                                        int(window), float(softmax_scale), _view(out, View4),
+                                        _ptr(q8_out), _ptr(q_scale_out), _ptr(ws),
+                                        0 if ws is None else ws.numel() * ws.element_size(),
+                                        _stream(stream)), "sage_attn_decode_mxfp4")
 
 
 def sage_quant_qk_mx(h, q, k, q4, q_sf, k4, k_sf, k_mean=None, ws=None, stream=None):

@@ -81,6 +81,10 @@ constexpr int kThreads = 512;
 // could take registers another one waits for.
 constexpr int kRegsSoft = 176, kRegsConv = 80, kRegsProd = 80;
 static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
+// the MXFP4 cache's converters (K and V, 16 bf16 pairs per block) take more
+// (this split, too, compiles without spills)
+constexpr int kRegsSoftMx = 168, kRegsConvMx = 96, kRegsProdMx = 80;
+static_assert(2 * 128 * kRegsSoftMx + 128 * kRegsConvMx + 128 * kRegsProdMx <= 512 * 128, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 // A scale slot: k_scale then v_scale of the tile's keys, each by key parity
 // (index (key & 1) * kScPar + key / 2); the 4-float pad puts the two parities'
@@ -139,16 +143,25 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
     tmem_wait_ld16(r);
 }
 
-// dynamic shared memory (offsets from a 1024-byte aligned base)
-template <int D>
+constexpr int al1024(int x) { return (x + 1023) & ~1023; }
+
+// dynamic shared memory (offsets from a 1024-byte aligned base). MX: the
+// cache holds E2M1 codes with e8m0 block scales (head size 128), the query
+// rows are bf16 and K is converted to bf16 before QK.
+template <int D, bool MX = false>
 struct SmL {
     static constexpr int kOcPitch = D + 4;                         // fp32 row pitch of the merge area
-    static constexpr int kQ = 0;                                   // [64][D] e4m3
-    static constexpr int kKStage = kKeys * D;                      // [128][D] e4m3
-    static constexpr int kK = kQ + kRows * D;                      // [stage][128][D] e4m3
-    static constexpr int kV = kK + kStages * kKStage;              // [stage][128][D] e4m3 (V^T: [D][128])
+    static constexpr int kQ = 0;                                   // [64][D] e4m3, MX: bf16 [2 atoms][64][128 B]
+    static constexpr int kKStage = MX ? kKeys * D / 2 : kKeys * D; // codes of one tile: [128][D] e4m3 | [128][D / 2] E2M1
+    static constexpr int kK = kQ + (MX ? 2 : 1) * kRows * D;       // [stage] K codes
+    static constexpr int kV = kK + kStages * kKStage;              // [stage] V codes (V^T: [D][128])
+    static constexpr int kSfStage = MX ? kKeys * D / 32 : 0;       // MX: e8m0 block scales of one tile [128][D / 32]
+    static constexpr int kKsf = kV + kStages * kKStage;
+    static constexpr int kVsf = kKsf + kStages * kSfStage;
+    static constexpr int kKbBuf = MX ? kKeys * 2 * D : 0;          // MX: bf16 K, D / 64 channel atoms [128][128 B]
+    static constexpr int kKb = MX ? al1024(kVsf + kStages * kSfStage) : kVsf;
     static constexpr int kPBuf = 2 * kRows * 128;                  // two 64-key atoms [64][128 B] bf16
-    static constexpr int kP = kV + kStages * kKStage;              // [2 bufs] P' (A of PV)
+    static constexpr int kP = kKb + kKbBuf;                        // [2 bufs] P' (A of PV)
     static constexpr int kVbBuf = kKeys * 2 * D;                   // D / 64 channel atoms [128][128 B] bf16
     static constexpr int kVb = kP + 2 * kPBuf;                     // [2 bufs] bf16 V (B of PV)
     static constexpr int kScale = kVb + 2 * kVbBuf;                // [slot] ks | vs fp32, padded
@@ -160,18 +173,22 @@ struct SmL {
     static constexpr int kKvFull = 0, kKvEmpty = kKvFull + kStages, kSFull = kKvEmpty + kStages,
                          kPReady = kSFull + 2, kPvDone = kPReady + 2, kFinal = kPvDone + 2,
                          kQReady = kFinal + 1, kScFull = kQReady + 1, kScEmpty = kScFull + kScStages,
-                         kNumBars = kScEmpty + kScStages;
+                         kKbReady = kScEmpty + kScStages, kKbFree = kKbReady + 1,
+                         kNumBars = kKbFree + 1;
     static constexpr int kMisc = kBar + kNumBars * 8;              // TMEM base, abort flag
     static constexpr int kBytes = kMisc + 16;
-    // merge area, over the K stages (free once the last tile is consumed)
+    // merge area, over the K (and, MX, V) code stages (free once the last
+    // tile is consumed)
     static constexpr int kOc = kK;                                 // [64][kOcPitch] fp32
     static constexpr int kStat = kOc + kRows * kOcPitch * 4;       // [64] (m, l)
     static_assert(kOcPitch % 4 == 0, "merge rows are 16-byte aligned");
-    static_assert(kStat + kRows * 8 <= kV, "merge area fits in the K stages");
-    static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0 && kVb % 1024 == 0,
+    static_assert(kStat + kRows * 8 <= (MX ? kKsf : kV), "merge area fits in the code stages");
+    static_assert(kK % 1024 == 0 && kV % 1024 == 0 && kP % 1024 == 0 && kVb % 1024 == 0 &&
+                      kKb % 1024 == 0 && kKsf % 16 == 0,
                   "swizzled tiles are 1024-byte aligned");
     static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
     static_assert(D == 64 || D == 128, "head size");
+    static_assert(!MX || D == 128, "the MXFP4 cache is read at head size 128");
 };
 
 struct DecParams {
@@ -191,6 +208,8 @@ struct DecParams {
     int per_tensor;                          // ksc / vsc hold one scale each
     int v_trans;                             // V cache [num_pages, Hk, D, page] (page 128)
     int o_vec;                               // out rows: 4 channels as one 8-byte store
+    const uint8_t* ksf8;                     // MX: e8m0 block scales [num_pages, Hk, page, D / 32]
+    const uint8_t* vsf8;
     float2* ws_stat;                         // nsplit > 1: partial (m, l) [B Hk][nsplit][64]
     float* ws_o;                             //   and partial O [B Hk][nsplit][64][128] fp32
 };
@@ -215,6 +234,57 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w, uint32_t sel) {
     uint32_t r;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7B807B80u));   // 2^120
     return r;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// The e4m3 codes byte m of `a` and byte m of `b` as one bf16 pair (low half
+// from `a`), exactly, as in e4m3x2_to_bf16x2; m = 0..3.
+template <int m>
+__device__ __forceinline__ uint32_t e4m3_pick_to_bf16x2(uint32_t a, uint32_t b) {
+    const uint32_t t = __byte_perm(a, b, (m << 4) | ((4 + m) << 12));   // bytes 1 and 3; 0, 2 unused
+    return bf16x2_mul(((t >> 4) & 0x07F007F0u) | (t & 0x80008000u), 0x7B807B80u);
+}
+
+// Eight E2M1 codes (OCP MX: sign, two exponent bits, one mantissa bit),
+// nibble i of `w` (bits 4i .. 4i + 3) holding element i, as four bf16 pairs:
+// pair m = (element m, element m + 4), each times the bf16 pair `c2`.
+// A code's three magnitude bits placed at bf16 bits 6..8 and its sign at bit
+// 15 read as a bf16 of value x * 2^-126 (exponent field = the code's, a
+// zero-exponent code a bf16 subnormal), so c2 = 2^(E - 1) gives x * 2^(E -
+// 127) in one exact product while that is a bf16 value.
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t c2, uint32_t* o) {
+    const uint32_t a0 = w << 6, a1 = w << 2, a2 = w >> 2, a3 = w >> 6;
+    const uint32_t s0 = w << 12, s1 = w << 8, s2 = w << 4, s3 = w;
+    o[0] = bf16x2_mul((a0 & 0x01C001C0u) | (s0 & 0x80008000u), c2);
+    o[1] = bf16x2_mul((a1 & 0x01C001C0u) | (s1 & 0x80008000u), c2);
+    o[2] = bf16x2_mul((a2 & 0x01C001C0u) | (s2 & 0x80008000u), c2);
+    o[3] = bf16x2_mul((a3 & 0x01C001C0u) | (s3 & 0x80008000u), c2);
+}
+
+// One MX block (32 E2M1 codes, 16 bytes: elements 8g .. 8g + 7 in word g)
+// times 2^(E - 127), E its e8m0 scale code, as 16 bf16 pairs: pair 4g + m =
+// (element 8g + m, element 8g + m + 4). E is read as min(E, 252), the largest
+// exponent whose values (up to 6 * 2^125) are finite in bf16, so that cache
+// bytes the window masks (slots past ctx) cannot turn a zero weight into a
+// NaN; a larger E (and E = 255, NaN) lies outside the contract.
+__device__ __forceinline__ void e2m1_block_to_bf16(uint4 u, uint32_t E, uint32_t (&o)[16]) {
+    E = min(E, 252u);
+    const uint32_t lo = E <= 128u ? E + 126u : 253u;                  // 2^(E - 1), or 2^126 then 2^(E - 127)
+    const uint32_t c2 = (lo << 7) | (lo << 23);
+    e2m1x8_to_bf16(u.x, c2, o);
+    e2m1x8_to_bf16(u.y, c2, o + 4);
+    e2m1x8_to_bf16(u.z, c2, o + 8);
+    e2m1x8_to_bf16(u.w, c2, o + 12);
+    if (E > 128u) {
+        const uint32_t c3 = (E << 7) | (E << 23);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = bf16x2_mul(o[k], c3);
+    }
 }
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
@@ -249,11 +319,11 @@ __device__ __forceinline__ void store_out4(const DecParams& p, int b, int hk, in
     }
 }
 
-template <int D>
+template <int D, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecParams p) {
-    using Sm = SmL<D>;
+    using Sm = SmL<D, MX>;
     constexpr int kD = D;
     constexpr int kOcPitch = Sm::kOcPitch;
     constexpr int kQe = D / 4;                    // query elements per rotating thread (4 per row)
@@ -282,11 +352,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kIdleWarp) {
         for (int i = lane; i < Sm::kNumBars; i += 32) {
             uint32_t cnt = 1;                                       // expect_tx; commits
-            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = 1 + 4;     // QK commit + converters
+            if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = MX ? 4 : 1 + 4;  // (QK commit +) converters
             if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = 4 + 4;             // softmax group + converters
             if (i == Sm::kQReady) cnt = kSoftWarps;
             if (i >= Sm::kScFull && i < Sm::kScFull + kScStages) cnt = 1 + 32;    // bad-page mask + scale copies
             if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = 4;       // softmax group
+            if (i == Sm::kKbReady) cnt = 4;                                       // converters (MX)
             mbar_init(&bars[i], cnt);
         }
         if (lane == 0) *abort_flag = 0;
@@ -346,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
     if (warp >= kTmaWarp) {
-      reg_dealloc<kRegsProd>();
+      reg_dealloc<MX ? kRegsProdMx : kRegsProd>();
       if (warp == kTmaWarp || warp == kScaleWarp) {
         // ------------------------------------------------------------ producers
         // Both warps look up the physical pages of the CTA's logical pages
@@ -356,8 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // by TMA, the lanes of a tile's pages each issuing their own boxes;
         // warp 14 loads the per-token scales and the tile's bad-page mask.
         const bool kv = warp == kTmaWarp;
-        const float ks_tensor = (!kv && p.per_tensor) ? __ldg(p.ksc) : 0.0f;
-        const float vs_tensor = (!kv && p.per_tensor) ? __ldg(p.vsc) : 0.0f;
+        // MX: the block scales are applied in the conversion, so every key's
+        // k_scale and v_scale are 1
+        const bool per_tensor = MX || p.per_tensor;
+        const float ks_tensor = MX ? 1.0f : (!kv && per_tensor) ? __ldg(p.ksc) : 0.0f;
+        const float vs_tensor = MX ? 1.0f : (!kv && per_tensor) ? __ldg(p.vsc) : 0.0f;
         int chunk = -1, phys_l = 0;
         bool bad_l = false;
         int issued = 0;
@@ -386,13 +460,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot0 = (i * ppt) % 32;             // this tile's pages: lanes slot0 .. slot0 + ppt - 1
             const bool mine = lane >= slot0 && lane < slot0 + ppt;
             if (kv) {
-                if (lane == slot0) mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * Sm::kKStage);
+                if (lane == slot0)
+                    mbar_arrive_expect_tx(&bars[Sm::kKvFull + s], 2 * (Sm::kKStage + Sm::kSfStage));
                 __syncwarp();
                 if (mine) {
                     const int z = phys_l * p.Hk + hk;
                     const int q = lane - slot0;
-                    tma_load_3d(sm + Sm::kK + s * Sm::kKStage + q * p.page * kD, &tmK, &bars[Sm::kKvFull + s], 0, 0, z);
-                    tma_load_3d(sm + Sm::kV + s * Sm::kKStage + q * p.page * kD, &tmV, &bars[Sm::kKvFull + s], 0, 0, z);
+                    constexpr int kRowB = Sm::kKStage / kKeys;      // code bytes per key
+                    tma_load_3d(sm + Sm::kK + s * Sm::kKStage + q * p.page * kRowB, &tmK, &bars[Sm::kKvFull + s], 0, 0, z);
+                    tma_load_3d(sm + Sm::kV + s * Sm::kKStage + q * p.page * kRowB, &tmV, &bars[Sm::kKvFull + s], 0, 0, z);
+                    if constexpr (MX) {
+                        // the page's block scales, contiguous [page][D / 32]
+                        constexpr int kSfB = kD / 32;
+                        const int64_t off = (int64_t)z * p.page * kSfB;
+                        bulk_load(sm + Sm::kKsf + s * Sm::kSfStage + q * p.page * kSfB, p.ksf8 + off,
+                                  p.page * kSfB, &bars[Sm::kKvFull + s]);
+                        bulk_load(sm + Sm::kVsf + s * Sm::kSfStage + q * p.page * kSfB, p.vsf8 + off,
+                                  p.page * kSfB, &bars[Sm::kKvFull + s]);
+                    }
                 }
             } else {
                 const unsigned badm = __ballot_sync(0xffffffffu, mine && bad_l) >> slot0;
@@ -404,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // parity for the softmax threads; with per-tensor scales the
                 // one K and one V scale in every slot
                 float* dst = scl + c * kScSlot;
-                if (p.per_tensor) {
+                if (per_tensor) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int key = 4 * lane + e, at = (key & 1) * kScPar + (key >> 1);
@@ -438,10 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && nt > 0) {
-            constexpr uint32_t kIdescQK = umma_idesc(1, 0, kRows, kKeys);              // e4m3 -> f32
+            constexpr uint32_t kIdescQK = umma_idesc(1, MX ? 1 : 0, kRows, kKeys);     // e4m3 | bf16 -> f32
             constexpr uint32_t kIdescPV = umma_idesc(1, 1, kRows, kD) | (1u << 16);    // bf16, B MN-major
             constexpr uint32_t kIdescPVT = umma_idesc(1, 1, kRows, kD);                // bf16, B K-major
-            const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), kD);
+            const uint64_t qdesc = umma_desc_kmajor(smem_u32(sm + Sm::kQ), MX ? 128 : kD);
             // descriptors of the P' and V buffers, built once: a step of the
             // MMA loops only adds a constant to the start-address field
             // (V MN-major: two 64-channel swizzle atoms [128 keys][128 B], the
@@ -453,18 +538,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t pdesc1 = umma_desc_kmajor(smem_u32(sm + Sm::kP + Sm::kPBuf), 128);
             const uint64_t vdesc0 = umma_desc_kmajor(smem_u32(sm + Sm::kVb), 128) + vlbo;
             const uint64_t vdesc1 = umma_desc_kmajor(smem_u32(sm + Sm::kVb + Sm::kVbBuf), 128) + vlbo;
-            // S(i) = Q8 K8(i)^T into S buffer i & 1
+            // S(i) = Q8 K8(i)^T into S buffer i & 1 (MX: bf16 Q and the
+            // converters' bf16 K(i), two 64-channel atoms each, 16 channels a
+            // step; the converters reuse the K buffer once this QK is done)
             auto issue_qk = [&](int i) -> bool {
                 const int s = i % kStages;
-                if (!mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2))
-                    return false;
-                tc_fence_after();
-                const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), kD);
+                if constexpr (MX) {
+                    if (!mbar_wait(&bars[Sm::kKbReady], i & 1, abort_flag, &g_decode_err, 2)) return false;
+                    tc_fence_after();
+                    const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kKb), 128);
 #pragma unroll
-                for (int kk = 0; kk < kD / 32; ++kk)
-                    mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, kk > 0 ? 1u : 0u);
-                mma_commit(&bars[Sm::kSFull + (i & 1)]);
-                mma_commit(&bars[Sm::kKvEmpty + s]);
+                    for (int st = 0; st < kD / 16; ++st)
+                        mma_bf16_ss(tmem + 128 * (i & 1), qdesc + (st >> 2) * ((kRows * 128) >> 4) + 2 * (st & 3),
+                                    kdesc + (st >> 2) * ((kKeys * 128) >> 4) + 2 * (st & 3), kIdescQK,
+                                    st > 0 ? 1u : 0u);
+                    mma_commit(&bars[Sm::kSFull + (i & 1)]);
+                    mma_commit(&bars[Sm::kKbFree]);
+                } else {
+                    if (!mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 2))
+                        return false;
+                    tc_fence_after();
+                    const uint64_t kdesc = umma_desc_kmajor(smem_u32(sm + Sm::kK + s * Sm::kKStage), kD);
+#pragma unroll
+                    for (int kk = 0; kk < kD / 32; ++kk)
+                        mma_f8_ss(tmem + 128 * (i & 1), qdesc + 2 * kk, kdesc + 2 * kk, kIdescQK, kk > 0 ? 1u : 0u);
+                    mma_commit(&bars[Sm::kSFull + (i & 1)]);
+                    mma_commit(&bars[Sm::kKvEmpty + s]);
+                }
                 return true;
             };
             // order: QK(0), QK(1), then for j = 0, 1, ...: once P'(j) is
@@ -481,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 bool qk_next = false;
                 if (j + 2 < nt &&
-                    mbar_test_wait(smem_u32(&bars[Sm::kKvFull + (j + 2) % kStages]), ((j + 2) / kStages) & 1)) {
+                    (MX ? mbar_test_wait(smem_u32(&bars[Sm::kKbReady]), (j + 2) & 1)
+                        : mbar_test_wait(smem_u32(&bars[Sm::kKvFull + (j + 2) % kStages]), ((j + 2) / kStages) & 1))) {
                     ok = issue_qk(j + 2);
                     qk_next = true;
                 }
@@ -520,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_dealloc(tmem, 512);
         }
     } else if (warp < kSoftWarps) {
-      reg_alloc<kRegsSoft>();
+      reg_alloc<MX ? kRegsSoftMx : kRegsSoft>();
         // ------------------------------------------------------------ softmax
         // ---- query rows: rotate and quantise to e4m3, four threads per row
         // (thread qq holds elements [32 qq, 32 qq + 32)), written as the
@@ -598,7 +699,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     w4[e] = amax != 0.0f ? (lo16 | (hi16 << 16)) : 0u;   // a zero row: +0 codes
                 }
                 const int chunk = (kD / 64) * qq + c;
-                *reinterpret_cast<uint4*>(qrow + (e4m3_chunk<D>(chunk, r) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                if constexpr (MX) {
+                    // the codes' exact bf16 values (A of a bf16 QK), eight
+                    // channels per 16-byte chunk in the order in which the
+                    // converters lay out K: pair m = (channel m, m + 4)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int k8 = 2 * chunk + hh;
+                        const uint32_t wa = w4[2 * hh], wb = w4[2 * hh + 1];
+                        *reinterpret_cast<uint4*>(sm + Sm::kQ + (k8 >> 3) * (kRows * 128) + r * 128 +
+                                                  (((k8 & 7) ^ (r & 7)) << 4)) =
+                            make_uint4(e4m3_pick_to_bf16x2<0>(wa, wb), e4m3_pick_to_bf16x2<1>(wa, wb),
+                                       e4m3_pick_to_bf16x2<2>(wa, wb), e4m3_pick_to_bf16x2<3>(wa, wb));
+                    }
+                } else {
+                    *reinterpret_cast<uint4*>(qrow + (e4m3_chunk<D>(chunk, r) << 4)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
                 if (qout)
                     *reinterpret_cast<uint4*>(p.q8_out + qtok * kD + 16 * chunk) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -808,8 +925,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
             float* oc = reinterpret_cast<float*>(sm + Sm::kOc);
             float2* stat = reinterpret_cast<float2*>(sm + Sm::kStat);
+            // (MX: TMEM column 8 u + 2 m + c holds channel 8 u + m + 4 c, the
+            // order of the converted V rows)
 #pragma unroll
-            for (int k = 0; k < kOe; ++k) oc[r * kOcPitch + (kD / 2) * g + 2 * k + cpar] = o_fin[k];
+            for (int k = 0; k < kOe; ++k)
+                oc[r * kOcPitch + (kD / 2) * g + (MX ? 8 * (k >> 2) + (k & 3) + 4 * cpar : 2 * k + cpar)] = o_fin[k];
             if (g == 0 && cpar == 0) stat[r] = make_float2(m_fin, l_fin);
             named_sync(1, kSoftWarps * 32);
             if (p.nsplit == 1) {
@@ -832,7 +952,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-      reg_dealloc<kRegsConv>();
+      reg_dealloc<MX ? kRegsConvMx : kRegsConv>();
         // ------------------------------------------------------------ V converters
         // lane -> V row kap of the tile (warp cw: rows 32 cw .. 32 cw + 31),
         // chosen so that the eight lanes of a quarter-warp read eight
@@ -842,6 +962,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kap = 32 * cw + 16 * (q8 >> 1) + 2 * e8 + ((e8 >> 2) ^ (q8 & 1));
         const int pos = pv_position(kap);
         bool ok = true;
+        if constexpr (MX) {
+        // MX: K(i) to the one bf16 K buffer (once QK(i - 1) has read it),
+        // lane -> key 32 cw + lane in key order; then V(i) to bf16 buffer
+        // i & 1 as below. A code row is 64 bytes (64B-swizzled by the TMA),
+        // one 16-byte chunk per 32-channel block, its e8m0 scales 4 bytes.
+        for (int i = 0; i < nt; ++i) {
+            const int s = i % kStages, bf = i & 1;
+            ok = warp_all(mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 10));
+            if (ok && i >= 1)
+                ok = warp_all(mbar_wait(&bars[Sm::kKbFree], (i - 1) & 1, abort_flag, &g_decode_err, 16));
+            if (!ok) break;
+            {
+                const int key = 32 * cw + lane;
+                const uint8_t* krow = sm + Sm::kK + s * Sm::kKStage + key * 64;
+                const uint32_t esc = *reinterpret_cast<const uint32_t*>(sm + Sm::kKsf + s * Sm::kSfStage + key * 4);
+                uint8_t* dst = sm + Sm::kKb + key * 128;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t o[16];
+                    e2m1_block_to_bf16(*reinterpret_cast<const uint4*>(krow + (e4m3_chunk<64>(blk, key) << 4)),
+                                       (esc >> (8 * blk)) & 0xFFu, o);
+                    uint8_t* atom = dst + (blk >> 1) * (kKeys * 128);
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq)
+                        *reinterpret_cast<uint4*>(atom + (((4 * (blk & 1) + gq) ^ (key & 7)) << 4)) =
+                            make_uint4(o[4 * gq], o[4 * gq + 1], o[4 * gq + 2], o[4 * gq + 3]);
+                }
+            }
+            fence_proxy_async_smem();               // read by the QK MMAs
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[Sm::kKbReady]);
+            if (i >= 2)
+                ok = warp_all(mbar_wait(&bars[Sm::kPvDone + bf], ((i - 2) >> 1) & 1, abort_flag,
+                                        &g_decode_err, 11));
+            if (!ok) break;
+            {
+                const uint8_t* vrow = sm + Sm::kV + s * Sm::kKStage + kap * 64;
+                const uint32_t esc = *reinterpret_cast<const uint32_t*>(sm + Sm::kVsf + s * Sm::kSfStage + kap * 4);
+                uint8_t* dst = sm + Sm::kVb + bf * Sm::kVbBuf + pos * 128;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    uint32_t o[16];
+                    e2m1_block_to_bf16(*reinterpret_cast<const uint4*>(vrow + (e4m3_chunk<64>(blk, kap) << 4)),
+                                       (esc >> (8 * blk)) & 0xFFu, o);
+                    uint8_t* atom = dst + (blk >> 1) * (kKeys * 128);
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq)
+                        *reinterpret_cast<uint4*>(atom + (((4 * (blk & 1) + gq) ^ (pos & 7)) << 4)) =
+                            make_uint4(o[4 * gq], o[4 * gq + 1], o[4 * gq + 2], o[4 * gq + 3]);
+                }
+            }
+            fence_proxy_async_smem();               // read by the PV MMAs
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[Sm::kPReady + bf]);
+                mbar_arrive(&bars[Sm::kKvEmpty + s]);
+            }
+        }
+        } else {
         for (int i = 0; i < nt; ++i) {
             const int s = i % kStages, bf = i & 1;
             ok = warp_all(mbar_wait(&bars[Sm::kKvFull + s], (i / kStages) & 1, abort_flag, &g_decode_err, 10));
@@ -890,6 +1069,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bars[Sm::kPReady + bf]);
                 mbar_arrive(&bars[Sm::kKvEmpty + s]);
             }
+        }
         }
         tc_fence_before();
         bar_sync_all(kThreads);
@@ -975,8 +1155,24 @@ bool encode_cache_vt(CUtensorMap* map, const void* ptr, int num_pages, int Hk, i
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
-constexpr int smem_bytes() { return SmL<D>::kBytes + 1024; }
+// The MXFP4 cache codes [num_pages, Hk, page, D / 2] bytes (two E2M1 codes a
+// byte) as a 3-D map {D / 2 bytes, page rows, num_pages * Hk}; one box = one
+// page of one kv head, 64B swizzle (D = 128: 64-byte rows).
+bool encode_cache_mx(CUtensorMap* map, const void* ptr, int num_pages, int Hk, int page, int D) {
+    auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+    if (!enc || D != 128) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D / 2), static_cast<cuuint64_t>(page),
+                                static_cast<cuuint64_t>(num_pages) * Hk};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D / 2), static_cast<cuuint64_t>(page) * (D / 2)};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(D / 2), static_cast<cuuint32_t>(page), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool MX>
+constexpr int smem_bytes() { return SmL<D, MX>::kBytes + 1024; }
 
 // Streaming multiprocessors of the current device (queried once per device).
 int device_sms() {
@@ -1033,9 +1229,9 @@ size_t decode_ws_bytes(int B, int, int, int Hk, int D, int) {
 
 namespace {
 
-template <int D>
+template <int D, bool MX>
 cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
-    constexpr int kSmemBytes = smem_bytes<D>();
+    constexpr int kSmemBytes = smem_bytes<D, MX>();
     DecParams p;
     p.q = static_cast<const uint16_t*>(a.q.ptr);
     p.qs0 = a.q.stride[0];
@@ -1065,17 +1261,24 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
     p.q8_out = a.q8_out;
     p.qs_out = a.q_scale_out;
     p.per_tensor = (a.kv_flags & 1) ? 1 : 0;
-    p.v_trans = (a.kv_flags & 2) ? 1 : 0;
+    p.v_trans = (!MX && (a.kv_flags & 2)) ? 1 : 0;
+    p.ksf8 = a.k_sf;
+    p.vsf8 = a.v_sf;
     p.q_vec = (a.q.stride[3] == 1 && a.q.stride[0] % 8 == 0 && a.q.stride[1] % 8 == 0 &&
                a.q.stride[2] % 8 == 0 && reinterpret_cast<uintptr_t>(a.q.ptr) % 16 == 0)
                   ? 1
                   : 0;
     CUtensorMap tk, tv;
-    if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size, D) ||
-        !(p.v_trans ? encode_cache_vt(&tv, a.v_cache, a.num_pages, a.Hk, D)
-                    : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size, D)))
+    if (MX) {
+        if (!encode_cache_mx(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size, D) ||
+            !encode_cache_mx(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size, D))
+            return cudaErrorInvalidValue;
+    } else if (!encode_cache(&tk, a.k_cache, a.num_pages, a.Hk, a.page_size, D) ||
+               !(p.v_trans ? encode_cache_vt(&tv, a.v_cache, a.num_pages, a.Hk, D)
+                           : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size, D))) {
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    }
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     p.nsplit = pick_nsplit(a.B * a.Hk, a.T, a.window, a.page_size, a.max_pages);
     p.o_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 4 == 0 && a.out_stride[1] % 4 == 0 &&
@@ -1102,7 +1305,7 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<D>, tk, tv, p);
+    e = cudaLaunchKernelEx(&cfg, decode_kernel<D, MX>, tk, tv, p);
     if (e != cudaSuccess || p.nsplit == 1) return e;
     // a plain stream-ordered launch: it measured faster here than one
     // launched as a programmatic dependent of the split grid
@@ -1113,9 +1316,10 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
+    if (a.mx) return a.D == 128 ? launch_decode_d<128, true>(a, s) : cudaErrorInvalidValue;
     switch (a.D) {
-        case 64: return launch_decode_d<64>(a, s);
-        case 128: return launch_decode_d<128>(a, s);
+        case 64: return launch_decode_d<64, false>(a, s);
+        case 128: return launch_decode_d<128, false>(a, s);
         default: return cudaErrorInvalidValue;
     }
 }

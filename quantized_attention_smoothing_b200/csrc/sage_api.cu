@@ -72,6 +72,59 @@ bool current_device(int* dev) { return cudaGetDevice(dev) == cudaSuccess; }
 
 sage_status launch_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
 
+// Checks shared by the decode entry points and the DecodeArgs they fill
+// (everything but the cache formats).
+sage_status decode_args(sage_hadamard h, sage_cview4 q_bf16, const int32_t* page_table,
+                        const int32_t* ctx_lens, int B, int T, int H, int Hk, int D, int page_size,
+                        int max_pages, int num_pages, int window, float softmax_scale,
+                        sage_view4 out_bf16, uint8_t* q8_out, float* q_scale_out, void* ws,
+                        size_t ws_bytes, sage::DecodeArgs* a) {
+    if (!h || !q_bf16.ptr || !page_table || !ctx_lens || !out_bf16.ptr) return SAGE_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || Hk < 1 || D < 1 || page_size < 1 || max_pages < 1 ||
+        num_pages < 1 || window < 1 || !std::isfinite(softmax_scale))
+        return SAGE_ERR_INVALID_ARG;
+    if (!sizes_ok(q_bf16.size, q_bf16.stride) || !sizes_ok(out_bf16.size, out_bf16.stride))
+        return SAGE_ERR_INVALID_ARG;
+    const int64_t want[4] = {B, T, H, D};
+    for (int i = 0; i < 4; ++i)
+        if (q_bf16.size[i] != want[i] || out_bf16.size[i] != want[i]) return SAGE_ERR_INVALID_ARG;
+    if (D != h->D) return SAGE_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+    if (H % Hk != 0 || H / Hk > 16 || T * (H / Hk) > 64) return SAGE_ERR_UNSUPPORTED;
+    if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
+        return SAGE_ERR_UNSUPPORTED;
+    if ((int64_t)num_pages * Hk * page_size * D >= (int64_t(1) << 40)) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(page_table, 4) || !aligned(ctx_lens, 4) || !aligned(q_bf16.ptr, 2) ||
+        !aligned(out_bf16.ptr, 2) || !aligned(q8_out, 16) || !aligned(q_scale_out, 4))
+        return SAGE_ERR_ALIGNMENT;
+    const size_t need = sage::decode_ws_bytes(B, T, H, Hk, D, window);
+    if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return SAGE_ERR_ALIGNMENT;
+    int dev = -1;
+    if (!current_device(&dev)) return SAGE_ERR_CUDA;
+    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
+    a->q = to_view(q_bf16);
+    a->page_table = page_table;
+    a->ctx_lens = ctx_lens;
+    a->B = B;
+    a->T = T;
+    a->H = H;
+    a->Hk = Hk;
+    a->D = D;
+    a->page_size = page_size;
+    a->max_pages = max_pages;
+    a->num_pages = num_pages;
+    a->window = window;
+    a->softmax_scale = softmax_scale;
+    a->out = out_bf16.ptr;
+    for (int i = 0; i < 4; ++i) a->out_stride[i] = out_bf16.stride[i];
+    a->ws = ws;
+    a->q8_out = q8_out;
+    a->q_scale_out = q_scale_out;
+    return SAGE_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -469,60 +522,48 @@ sage_status sage_attn_decode(sage_hadamard h, sage_cview4 q_bf16, const uint8_t*
                              int window, float softmax_scale, int kv_flags, sage_view4 out_bf16,
                              uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
                              void* stream) {
-    if (!h || !q_bf16.ptr || !k_cache || !v_cache || !k_scale || !v_scale || !page_table ||
-        !ctx_lens || !out_bf16.ptr)
-        return SAGE_ERR_INVALID_ARG;
-    if (B < 1 || T < 1 || H < 1 || Hk < 1 || D < 1 || page_size < 1 || max_pages < 1 ||
-        num_pages < 1 || window < 1 || !std::isfinite(softmax_scale))
-        return SAGE_ERR_INVALID_ARG;
-    if (!sizes_ok(q_bf16.size, q_bf16.stride) || !sizes_ok(out_bf16.size, out_bf16.stride))
-        return SAGE_ERR_INVALID_ARG;
-    const int64_t want[4] = {B, T, H, D};
-    for (int i = 0; i < 4; ++i)
-        if (q_bf16.size[i] != want[i] || out_bf16.size[i] != want[i]) return SAGE_ERR_INVALID_ARG;
-    if (D != h->D) return SAGE_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
-    if (H % Hk != 0 || H / Hk > 16 || T * (H / Hk) > 64) return SAGE_ERR_UNSUPPORTED;
-    if (page_size != 16 && page_size != 32 && page_size != 64 && page_size != 128)
-        return SAGE_ERR_UNSUPPORTED;
+    if (!k_cache || !v_cache || !k_scale || !v_scale) return SAGE_ERR_INVALID_ARG;
     if (kv_flags & ~(SAGE_KV_PER_TENSOR_SCALES | SAGE_KV_V_TRANSPOSED)) return SAGE_ERR_INVALID_ARG;
-    if ((kv_flags & SAGE_KV_V_TRANSPOSED) && page_size != 128) return SAGE_ERR_UNSUPPORTED;
-    if ((int64_t)num_pages * Hk * page_size * D >= (int64_t(1) << 40)) return SAGE_ERR_UNSUPPORTED;
-    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_scale, 4) ||
-        !aligned(v_scale, 4) || !aligned(page_table, 4) || !aligned(ctx_lens, 4) ||
-        !aligned(q_bf16.ptr, 2) || !aligned(out_bf16.ptr, 2) || !aligned(q8_out, 16) ||
-        !aligned(q_scale_out, 4))
-        return SAGE_ERR_ALIGNMENT;
-    const size_t need = sage::decode_ws_bytes(B, T, H, Hk, D, window);
-    if (need > 0 && (!ws || ws_bytes < need)) return SAGE_ERR_WORKSPACE;
-    if (!aligned(ws, 16)) return SAGE_ERR_ALIGNMENT;
-    int dev = -1;
-    if (!current_device(&dev)) return SAGE_ERR_CUDA;
-    if (dev != h->device) return SAGE_ERR_INVALID_ARG;
     sage::DecodeArgs a;
-    a.q = to_view(q_bf16);
+    sage_status st = decode_args(h, q_bf16, page_table, ctx_lens, B, T, H, Hk, D, page_size, max_pages,
+                                 num_pages, window, softmax_scale, out_bf16, q8_out, q_scale_out, ws,
+                                 ws_bytes, &a);
+    if (st != SAGE_OK) return st;
+    if ((kv_flags & SAGE_KV_V_TRANSPOSED) && page_size != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+        return SAGE_ERR_ALIGNMENT;
     a.k_cache = k_cache;
     a.v_cache = v_cache;
     a.k_scale = k_scale;
     a.v_scale = v_scale;
-    a.page_table = page_table;
-    a.ctx_lens = ctx_lens;
-    a.B = B;
-    a.T = T;
-    a.H = H;
-    a.Hk = Hk;
-    a.D = D;
-    a.page_size = page_size;
-    a.max_pages = max_pages;
-    a.num_pages = num_pages;
-    a.window = window;
-    a.softmax_scale = softmax_scale;
-    a.out = out_bf16.ptr;
-    for (int i = 0; i < 4; ++i) a.out_stride[i] = out_bf16.stride[i];
-    a.ws = ws;
-    a.q8_out = q8_out;
-    a.q_scale_out = q_scale_out;
     a.kv_flags = kv_flags;
+    return launch_status(sage::launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_attn_decode_mxfp4(sage_hadamard h, sage_cview4 q_bf16, const uint8_t* k_cache,
+                                   const uint8_t* v_cache, const uint8_t* k_sf, const uint8_t* v_sf,
+                                   const int32_t* page_table, const int32_t* ctx_lens, int B, int T,
+                                   int H, int Hk, int D, int page_size, int max_pages, int num_pages,
+                                   int window, float softmax_scale, sage_view4 out_bf16,
+                                   uint8_t* q8_out, float* q_scale_out, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    if (!k_cache || !v_cache || !k_sf || !v_sf) return SAGE_ERR_INVALID_ARG;
+    sage::DecodeArgs a;
+    sage_status st = decode_args(h, q_bf16, page_table, ctx_lens, B, T, H, Hk, D, page_size, max_pages,
+                                 num_pages, window, softmax_scale, out_bf16, q8_out, q_scale_out, ws,
+                                 ws_bytes, &a);
+    if (st != SAGE_OK) return st;
+    if (D != 128) return SAGE_ERR_UNSUPPORTED;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(k_sf, 16) || !aligned(v_sf, 16))
+        return SAGE_ERR_ALIGNMENT;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.k_scale = nullptr;
+    a.v_scale = nullptr;
+    a.kv_flags = 0;
+    a.mx = 1;
+    a.k_sf = k_sf;
+    a.v_sf = v_sf;
     return launch_status(sage::launch_decode(a, static_cast<cudaStream_t>(stream)));
 }
 

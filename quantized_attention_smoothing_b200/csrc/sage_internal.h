@@ -139,6 +139,9 @@ struct DecodeArgs {
     uint8_t* q8_out;           // optional [B, T, H, D] e4m3 query codes
     float* q_scale_out;        // optional [B, T, H] query scales
     int kv_flags;              // SAGE_KV_PER_TENSOR_SCALES | SAGE_KV_V_TRANSPOSED
+    int mx = 0;                // k_cache / v_cache: E2M1 codes [.., page, D / 2] with
+    const uint8_t* k_sf = nullptr;   // e8m0 block scales [num_pages, Hk, page, D / 32]
+    const uint8_t* v_sf = nullptr;
 };
 size_t decode_ws_bytes(int B, int T, int H, int Hk, int D, int window);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);

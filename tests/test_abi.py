@@ -157,3 +157,25 @@ def test_decode_validation_without_gpu(L):
         sage.sage_attn_decode(FakeHandle(), qt, qt, qt, qt, qt, qt, qt, 128, 100, 4096, 0.088, qt,
                               None, stream=0)
     assert e.value.status == sage.SAGE_ERR_INVALID_ARG
+
+
+def test_decode_mxfp4_marshalling_without_gpu(L):
+    """The MXFP4-cache decode entry point: argument count of the binding and
+    the null-handle refusal (nothing else is reachable without a device)."""
+    p = ctypes.c_void_p(0x10000)
+    q = _cview(size=(2, 1, 16, 128))
+    out = _view(0x20000, (2, 1, 16, 128))
+    args = [q, p, p, p, p, p, p, 2, 1, 16, 1, 128, 128, 64, 100, 4096, 0.088, out, None, None, p,
+            1 << 30, None]
+    assert L.sage_attn_decode_mxfp4(None, *args) == sage.SAGE_ERR_INVALID_ARG
+    torch = __import__("torch")
+
+    class FakeHandle:
+        handle = None
+    qt = torch.zeros((2, 1, 16, 128), dtype=torch.bfloat16)
+    u8 = torch.zeros((4, 1, 128, 64), dtype=torch.uint8)
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_attn_decode_mxfp4(FakeHandle(), qt, u8, u8, u8, u8, torch.zeros((2, 4), dtype=torch.int32),
+                                    torch.zeros(2, dtype=torch.int32), 128, 4, 4096, 0.088, qt,
+                                    ws=u8, stream=0)
+    assert e.value.status == sage.SAGE_ERR_INVALID_ARG
