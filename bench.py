@@ -9,7 +9,10 @@ B=1 H=40 L=32760 D=128 (Q blocks 128 tokens, K blocks 64), the largest of the
 single-GPU workloads. Metric: TOPS = 4 B H L^2 D / step time (halved for
 causal). The line also carries the B1 H24 L4096 and the causal B2 H32 L8192
 workloads under "configs", each with its attention roofline and its
-quantisation bandwidth, and the paged FP8 decode under "decode".
+quantisation bandwidth, and the paged decode: the MTP4 / GQA16 / window-4096
+workload over the FP8 cache ("decode", head size 128; "decode_d64") and
+over an MXFP4 cache ("decode_mxfp4"), and the batch-32 / ctx-32k / T-1
+workload over both ("decode_long").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sage|reference]
                     [--workload c2|c3|c4]
@@ -256,19 +259,27 @@ def cpu_baseline(cfg, seconds):
 
 
 def bench_decode(sage, torch, stream, copies=8, reps=50, key="c5"):
-    """Paged FP8 decode on the MTP4 / GQA16 / window-4096 workload (head size
-    128, or 64 with key "c5_d64"): one call = the split kernel and the merge
-    kernel; `copies` cache copies rotate so the working set exceeds L2;
-    calls are captured in a CUDA graph and replayed."""
+    """Paged decode on one of the decode workloads: the MTP4 / GQA16 /
+    window-4096 one over the FP8 cache (head size 128, or 64 with key
+    "c5_d64") or over an MXFP4 cache ("c5_mx"), and the batch-32 / ctx-32k /
+    T 1 one over either cache ("c7", "c7_mx"). One call = the split kernel
+    and the merge kernel; cache copies rotate so that the working set
+    exceeds L2 (8, or 2 when one copy is larger than L2); calls are captured
+    in a CUDA graph and replayed."""
     import workloads
     cfg, d = workloads.make_decode_config(key)
+    mx = cfg.get("kv_format") == "mxfp4"
     B, T, H, D = d["q"].shape
     Hk, page = d["k_cache"].shape[1], d["k_cache"].shape[2]
     h = sage.Hadamard(D)
     q = d["q"].cuda()
     tabs = [d[x].cuda() for x in ("page_table", "ctx_lens")]
+    copy_bytes = sum(d[x].numel() * d[x].element_size() for x in ("k_cache", "v_cache", "k_scale", "v_scale"))
+    if copy_bytes > 128 << 20:
+        copies = 2
     caches = [[d[x].cuda() for x in ("k_cache", "v_cache", "k_scale", "v_scale")]
               for _ in range(copies)]
+    run = sage.sage_attn_decode_mxfp4 if mx else sage.sage_attn_decode
     out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
     ws = torch.zeros((max(16, sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"])),),
                      dtype=torch.uint8, device="cuda")
@@ -276,8 +287,8 @@ def bench_decode(sage, torch, stream, copies=8, reps=50, key="c5"):
     def call(i):
         kc, vc, ksc, vsc = caches[i % copies]
         # torch's current stream: the side stream below, or the capture stream
-        sage.sage_attn_decode(h, q, kc, vc, ksc, vsc, tabs[0], tabs[1], page, d["num_pages"],
-                              cfg["window"], cfg["softmax_scale"], out, ws, None)
+        run(h, q, kc, vc, ksc, vsc, tabs[0], tabs[1], page, d["num_pages"], cfg["window"],
+            cfg["softmax_scale"], out, ws, None)
 
     side = torch.cuda.Stream()
     with torch.cuda.stream(side):
@@ -308,7 +319,10 @@ def bench_decode(sage, torch, stream, copies=8, reps=50, key="c5"):
     times.sort()
     ctx = d["ctx_lens"].tolist()
     keys = sum(min(c, cfg["window"] + T - 1) for c in ctx)
-    algo = keys * Hk * (2 * D + 8) + 2 * q.numel() * 2 + tabs[0].numel() * 4 + tabs[1].numel() * 4
+    # K and V rows of the keys read: D e4m3 codes and one fp32 scale each, or
+    # (MXFP4) D / 2 code bytes and D / 32 e8m0 scale bytes each
+    row = (D // 2 + D // 32) if mx else (D + 4)
+    algo = keys * Hk * 2 * row + 2 * q.numel() * 2 + tabs[0].numel() * 4 + tabs[1].numel() * 4
     pk, pk_src = peaks()
     gbs = algo / (ms * 1e-3) / 1e9
     del g
@@ -318,6 +332,7 @@ def bench_decode(sage, torch, stream, copies=8, reps=50, key="c5"):
             "achieved": gbs, "unit": "GB/s", "peak": pk["hbm_gbs"], "frac": gbs / pk["hbm_gbs"],
             "peak_source": pk_src + " copy bandwidth (burst)",
             "launches_per_call": 2 if sage.sage_attn_decode_workspace(B, T, H, Hk, D, cfg["window"]) > 0 else 1,
+            "kv_format": "mxfp4" if mx else "fp8",
             "timing": "median of 5 replays of a CUDA graph of %d calls over %d rotating cache copies"
                       % (reps, copies)}
 
@@ -684,6 +699,11 @@ def run_sage(args):
 
     dec = None if args.no_decode else bench_decode(sage, torch, stream)
     dec64 = None if args.no_decode or world > 1 else bench_decode(sage, torch, stream, key="c5_d64")
+    dec_mx = None if args.no_decode or world > 1 else bench_decode(sage, torch, stream, key="c5_mx")
+    dec_long = None
+    if not args.no_decode and world == 1:
+        dec_long = {"fp8": bench_decode(sage, torch, stream, key="c7"),
+                    "mxfp4": bench_decode(sage, torch, stream, key="c7_mx")}
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -708,6 +728,8 @@ def run_sage(args):
             "mxfp4": mx,
             "decode": dec,
             "decode_d64": dec64,
+            "decode_mxfp4": dec_mx,
+            "decode_long": dec_long,
             "gpu_launches": (5 if args.fused_q else 3) * args.steps,
             "clocks": clk.summary(),
         }
@@ -722,7 +744,7 @@ def main():
         import torch
         import quantized_attention_smoothing_b200 as sage
         s = torch.cuda.current_stream()
-        print(json.dumps({"c5": bench_decode(sage, torch, s), "c5_d64": bench_decode(sage, torch, s, key="c5_d64")}))
+        print(json.dumps({k: bench_decode(sage, torch, s, key=k) for k in ("c5", "c5_d64", "c5_mx", "c7", "c7_mx")}))
         return
     if args.impl == "reference":
         run_reference(args)

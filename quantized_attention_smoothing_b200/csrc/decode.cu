@@ -74,17 +74,22 @@ constexpr int kMmaWarp = 13;
 constexpr int kScaleWarp = 14;
 constexpr int kIdleWarp = 15;                // initialises the barriers, then only completes a warpgroup
 constexpr int kThreads = 512;
-// registers per thread of each warpgroup (setmaxnreg; 256 x 176 + 128 x 80 +
+// registers per thread of each warpgroup (setmaxnreg; 256 x 168 + 128 x 96 +
 // 128 x 80 <= 512 x 128, the launch's registers; this split compiles without
-// spills). Only the softmax warps ever grow their share, after the others
-// have shrunk theirs, and no warp grows it again later: a warp that did
-// could take registers another one waits for.
-constexpr int kRegsSoft = 176, kRegsConv = 80, kRegsProd = 80;
+// spills at both head sizes). Only the softmax warps ever grow their share,
+// after the others have shrunk theirs, and no warp grows it again later: a
+// warp that did could take registers another one waits for.
+constexpr int kRegsSoft = 168, kRegsConv = 96, kRegsProd = 80;
 static_assert(2 * 128 * kRegsSoft + 128 * kRegsConv + 128 * kRegsProd <= 512 * 128, "register split");
-// the MXFP4 cache's converters (K and V, 16 bf16 pairs per block) take more
-// (this split, too, compiles without spills)
-constexpr int kRegsSoftMx = 168, kRegsConvMx = 96, kRegsProdMx = 80;
-static_assert(2 * 128 * kRegsSoftMx + 128 * kRegsConvMx + 128 * kRegsProdMx <= 512 * 128, "register split");
+// the MXFP4 cache's kernels: the split that compiles without spills for
+// each row-repeat count (the converters do K and V there)
+template <bool MX, int NREP> struct RegSplit {
+    static constexpr int soft = kRegsSoft, conv = kRegsConv, prod = kRegsProd;
+};
+template <int NREP> struct RegSplit<true, NREP> {
+    static constexpr int soft = 168, conv = NREP == 2 ? 80 : 96, prod = NREP == 2 ? 96 : 80;
+    static_assert(2 * 128 * soft + 128 * conv + 128 * prod <= 512 * 128, "register split");
+};
 constexpr float kLog2e = 1.4426950408889634f;
 // A scale slot: k_scale then v_scale of the tile's keys, each by key parity
 // (index (key & 1) * kScPar + key / 2); the 4-float pad puts the two parities'
@@ -144,6 +149,15 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16]
 }
 
 constexpr int al1024(int x) { return (x + 1023) & ~1023; }
+
+// N registers of 16 TMEM lanes and 2 N columns (shape 16x64b), loaded and
+// waited for: N = 64, 32 or 16.
+__device__ __forceinline__ void tmem_ld16_cols(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_ld16x64(taddr, r);
+    tmem_wait_ld64(r);
+}
+__device__ __forceinline__ void tmem_ld16_cols(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld16_wait(taddr, r); }
+__device__ __forceinline__ void tmem_ld16_cols(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16_wait(taddr, r); }
 
 // dynamic shared memory (offsets from a 1024-byte aligned base). MX: the
 // cache holds E2M1 codes with e8m0 block scales (head size 128), the query
@@ -319,11 +333,22 @@ __device__ __forceinline__ void store_out4(const DecParams& p, int b, int hk, in
     }
 }
 
-template <int D, bool MX>
+// NREP (1, 2, 4): the R <= 64 / NREP query rows are repeated NREP times in
+// the 64 rows of the QK A operand, row r holding query row r % (64 / NREP),
+// and warp qw of a softmax group takes the 128 / NREP key columns of its
+// 16 rows that begin at (qw / (4 / NREP)) * 128 / NREP: with few query rows
+// (one query token: R = H / Hk) every softmax warp then holds a share of the
+// logits instead of one warp holding them all. Each A row keeps its own
+// running max, sum and O rows; the NREP rows of a query row are combined
+// (log-sum-exp) with the two groups' when the CTA's result is written.
+template <int D, bool MX, int NREP>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecParams p) {
     using Sm = SmL<D, MX>;
+    static_assert(NREP == 1 || NREP == 2 || NREP == 4, "row repeats");
+    constexpr int kPeriod = kRows / NREP;         // query rows per repeat of the A operand
+    constexpr int kNC = 64 / NREP;                // S registers per softmax thread (2 kNC columns a row)
     constexpr int kD = D;
     constexpr int kOcPitch = Sm::kOcPitch;
     constexpr int kQe = D / 4;                    // query elements per rotating thread (4 per row)
@@ -349,14 +374,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the parameter space) overlaps the preceding kernel in the stream when
     // this grid is launched as its programmatic dependent; everything after
     // griddepcontrol.wait sees that kernel's writes
+    // softmax warps per group that hold query rows (the others, whose 16
+    // rows are all padding, take no part in the tile loop)
+    const int n_act = NREP > 1 ? 4 : min(4, (p.R + 15) >> 4);
     if (warp == kIdleWarp) {
         for (int i = lane; i < Sm::kNumBars; i += 32) {
             uint32_t cnt = 1;                                       // expect_tx; commits
             if (i >= Sm::kKvEmpty && i < Sm::kKvEmpty + kStages) cnt = MX ? 4 : 1 + 4;  // (QK commit +) converters
-            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = 4 + 4;             // softmax group + converters
+            if (i >= Sm::kPReady && i < Sm::kPReady + 2) cnt = n_act + 4;         // softmax group + converters
             if (i == Sm::kQReady) cnt = kSoftWarps;
             if (i >= Sm::kScFull && i < Sm::kScFull + kScStages) cnt = 1 + 32;    // bad-page mask + scale copies
-            if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = 4;       // softmax group
+            if (i >= Sm::kScEmpty && i < Sm::kScEmpty + kScStages) cnt = n_act;   // softmax group
             if (i == Sm::kKbReady) cnt = 4;                                       // converters (MX)
             mbar_init(&bars[i], cnt);
         }
@@ -399,8 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the softmax warps' query row quarters (contiguous rows), also in flight
     // across the barrier
     uint4 qv[kQv] = {};
-    if (warp < kSoftWarps && p.q_vec && (tid >> 2) < p.R) {
-        const int r = tid >> 2;
+    if (warp < kSoftWarps && p.q_vec && ((tid >> 2) % kPeriod) < p.R) {
+        const int r = (tid >> 2) % kPeriod;
         const uint4* src = reinterpret_cast<const uint4*>(p.q + b * p.qs0 + (r / p.G) * p.qs1 +
                                                           (hk * p.G + r % p.G) * p.qs2) + kQv * (tid & 3);
 #pragma unroll
@@ -417,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
     if (warp >= kTmaWarp) {
-      reg_dealloc<MX ? kRegsProdMx : kRegsProd>();
+      reg_dealloc<RegSplit<MX, NREP>::prod>();
       if (warp == kTmaWarp || warp == kScaleWarp) {
         // ------------------------------------------------------------ producers
         // Both warps look up the physical pages of the CTA's logical pages
@@ -572,17 +600,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // already landed, so that tile j's group can start on tile j + 2
             // while PV(j) runs. S(j + 2) overwrites S(j), which the group read
             // before it published P'(j); the group waits for PV(j) itself
-            // before it reuses its P' buffer and O.
+            // before it reuses its P' buffer and O. (Issuing QK(j + 2) as soon
+            // as the group has read S(j) measured slower.)
+            auto k_there = [&](int i) -> bool {
+                return MX ? mbar_test_wait(smem_u32(&bars[Sm::kKbReady]), i & 1)
+                          : mbar_test_wait(smem_u32(&bars[Sm::kKvFull + i % kStages]), (i / kStages) & 1);
+            };
             bool ok = mbar_wait(&bars[Sm::kQReady], 0, abort_flag, &g_decode_err, 12);
             if (ok) ok = issue_qk(0);
             if (ok && nt > 1) ok = issue_qk(1);
             for (int j = 0; ok && j < nt; ++j) {
+                bool qk_next = false;
                 ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
                 if (!ok) break;
-                bool qk_next = false;
-                if (j + 2 < nt &&
-                    (MX ? mbar_test_wait(smem_u32(&bars[Sm::kKbReady]), (j + 2) & 1)
-                        : mbar_test_wait(smem_u32(&bars[Sm::kKvFull + (j + 2) % kStages]), ((j + 2) / kStages) & 1))) {
+                if (j + 2 < nt && k_there(j + 2)) {
                     ok = issue_qk(j + 2);
                     qk_next = true;
                 }
@@ -621,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_dealloc(tmem, 512);
         }
     } else if (warp < kSoftWarps) {
-      reg_alloc<MX ? kRegsSoftMx : kRegsSoft>();
+      reg_alloc<RegSplit<MX, NREP>::soft>();
         // ------------------------------------------------------------ softmax
         // ---- query rows: rotate and quantise to e4m3, four threads per row
         // (thread qq holds elements [32 qq, 32 qq + 32)), written as the
@@ -629,9 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // runs the whole sequence, shuffles included; rows past R load zeros,
         // which gives them zero codes and a zero scale.
         {
-            const int r = tid >> 2, qq = tid & 3;
-            const bool rv = r < p.R;
-            const int t = rv ? r / p.G : 0, h = rv ? hk * p.G + r % p.G : 0;
+            const int r = tid >> 2, qq = tid & 3;          // A row r holds query row rq
+            const int rq = r % kPeriod;
+            const bool rv = rq < p.R;
+            const int t = rv ? rq / p.G : 0, h = rv ? hk * p.G + rq % p.G : 0;
             const uint16_t* src = p.q + b * p.qs0 + t * p.qs1 + h * p.qs2 + (int64_t)(qq * kQe) * p.qs3;
             float x[kQe];
             if (p.q_vec) {
@@ -684,9 +716,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (qq == 0) sq[r] = s;
             // the codes and scale also go to the caller's optional outputs
             // (written once, by the first CTA of (b, hk))
-            const bool qout = rv && split == 0 && p.q8_out != nullptr;
+            const bool qout = rv && r == rq && split == 0 && p.q8_out != nullptr;
             const int64_t qtok = ((int64_t)b * p.T + t) * p.H + h;
-            if (rv && split == 0 && qq == 0 && p.qs_out != nullptr) p.qs_out[qtok] = s;
+            if (rv && r == rq && split == 0 && qq == 0 && p.qs_out != nullptr) p.qs_out[qtok] = s;
             uint8_t* qrow = sm + Sm::kQ + r * kD;
 #pragma unroll
             for (int c = 0; c < kD / 64; ++c) {      // 16-byte chunk (D / 64) qq + c of the row
@@ -720,7 +752,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4*>(p.q8_out + qtok * kD + 16 * chunk) =
                         make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
-            fence_proxy_async_smem();                // the QK MMAs read these rows
+            if constexpr (NREP > 1) {
+                // a warp writes only its own key columns of P'; the others
+                // of its rows stay zero
+                uint4* pz = reinterpret_cast<uint4*>(sm + Sm::kP);
+                for (int z = tid; z < 2 * Sm::kPBuf / 16; z += kSoftWarps * 32) pz[z] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();                // the QK / PV MMAs read these rows
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Sm::kQReady]);
@@ -729,15 +767,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Group g = warp >> 2 takes the tiles i = g, g + 2, g + 4, ... with
         // its own running max and sum, accumulated into O[g]; the groups run
         // side by side and are combined after the last tile. Warp qw = warp &
-        // 3 of a group holds query rows 16 qw .. 16 qw + 15 (TMEM lanes 32 qw
-        // ..) over all 128 columns: thread: row r, register k = column 2k +
-        // cpar (k = 0..63).
+        // 3 of a group holds A rows 16 qw .. 16 qw + 15 (TMEM lanes 32 qw ..)
+        // over the 2 kNC columns that begin at cb: thread: row r, register k
+        // = column cb + 2k + cpar (k = 0 .. kNC - 1).
         const int qw = warp & 3, g = warp >> 2;
         const int lr = (lane >> 2) + 8 * (lane & 1);
         const int cpar = (lane >> 1) & 1;
         const int r = 16 * qw + lr;
-        const bool rv = r < p.R;
-        const int pq = rv ? ctx - p.T + r / p.G : -1;     // the row's query position
+        const int rq = r % kPeriod;                       // its query row
+        const int cb = (qw / (4 / NREP)) * (2 * kNC);
+        const bool rv = rq < p.R;
+        const int pq = rv ? ctx - p.T + rq / p.G : -1;    // the row's query position
         // base-2 logit of a key = (acc * k_scale) * cq; cq kept >= FLT_MIN so
         // that a masked key (-inf) times cq stays -inf (a zero query row has
         // acc = 0, so its logits are 0 either way)
@@ -747,7 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_run = -INFINITY;                      // the max O[g] and the sum are expressed against
         uint64_t lsum2 = f2_pack(0.0f, 0.0f);         // running sum as an f32x2 pair
         bool ok = true;
-        for (int i = g; i < nt; i += 2) {
+        const int nt_mine = (NREP > 1 || 16 * qw < p.R) ? nt : 0;   // a warp of padding rows only sits out
+        for (int i = g; i < nt_mine; i += 2) {
             const int c = i % kScStages;
             ok = warp_all(mbar_wait(&bars[Sm::kSFull + g], (i >> 1) & 1, abort_flag, &g_decode_err, 5));
             if (ok)
@@ -755,19 +796,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         &g_decode_err, 6));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[64];
-            tmem_ld16x64(taddr + 128 * g, sv);
-            tmem_wait_ld64(sv);
+            uint32_t sv[kNC];
+            tmem_ld16_cols(taddr + 128 * g + cb, sv);
 
-            const float* ksP = scl + c * kScSlot + cpar * kScPar;   // k_scale of column 2k + cpar
+            const float* ksP = scl + c * kScSlot + cpar * kScPar + cb / 2;   // k_scale of column cb + 2k + cpar
             const float* vsP = ksP + kScHalf;
             const int key0 = (tb + i) * kKeys;
+            const int kc0 = key0 + cb;                  // the key of register 0 (cpar 0)
             const int badm = meta[c];
             // y = acc * k_scale; the logit is y * cq, and cq > 0 keeps the
             // order, so the row max is taken on y
-            float x[64];
+            float x[kNC];
 #pragma unroll
-            for (int k4 = 0; k4 < 16; ++k4) {
+            for (int k4 = 0; k4 < kNC / 4; ++k4) {
                 const float4 kq = *reinterpret_cast<const float4*>(ksP + 4 * k4);
                 const uint64_t a01 = f2_mul(f2_pack(__uint_as_float(sv[4 * k4]), __uint_as_float(sv[4 * k4 + 1])),
                                             f2_pack(kq.x, kq.y));
@@ -781,16 +822,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool full = badm == 0 && key0 >= ctx - p.window && key0 + kKeys - 1 <= ctx - p.T;
             if (!rv) {
 #pragma unroll
-                for (int k = 0; k < 64; ++k) x[k] = -INFINITY;
+                for (int k = 0; k < kNC; ++k) x[k] = -INFINITY;
             } else if (!full) {
-                // the row sees columns [clo, chi] of the tile
-                const int clo = pq - p.window + 1 - key0 - cpar, chi = pq - key0 - cpar;
+                // the row sees keys [kc0 + clo, kc0 + chi] of this thread's
+                const int clo = pq - p.window + 1 - kc0 - cpar, chi = pq - kc0 - cpar;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) x[k] = (2 * k >= clo && 2 * k <= chi) ? x[k] : -INFINITY;
+                for (int k = 0; k < kNC; ++k) x[k] = (2 * k >= clo && 2 * k <= chi) ? x[k] : -INFINITY;
                 if (badm != 0) {
 #pragma unroll
-                    for (int k = 0; k < 64; ++k)
-                        if ((badm >> ((2 * k + cpar) >> p.lg_page)) & 1) x[k] = -INFINITY;
+                    for (int k = 0; k < kNC; ++k)
+                        if ((badm >> ((cb + 2 * k + cpar) >> p.lg_page)) & 1) x[k] = -INFINITY;
                 }
             }
             // row max: four chains, a tree, the column partner
@@ -798,11 +839,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmax3(x[q4], x[q4 + 4], x[q4 + 8]);
 #pragma unroll
-            for (int k = 12; k < 60; k += 8)
+            for (int k = 12; k + 8 <= kNC - 4; k += 8)
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmax3(m4[q4], x[k + q4], x[k + q4 + 4]);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmaxf(m4[q4], x[60 + q4]);
+            for (int q4 = 0; q4 < 4; ++q4) m4[q4] = fmaxf(m4[q4], x[kNC - 4 + q4]);
             float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             mx = mx == -INFINITY ? -INFINITY : mx * cq;   // the max of the logits y * cq
@@ -824,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint8_t* prow = sm + Sm::kP + g * Sm::kPBuf + r * 128;
 #pragma unroll
-            for (int i16 = 0; i16 < 8; ++i16) {   // keys 16 i16 + cpar + 2m = registers 8 i16 + m
+            for (int i16 = 0; i16 < kNC / 8; ++i16) {   // keys cb + 16 i16 + cpar + 2m = registers 8 i16 + m
                 const float4 va = *reinterpret_cast<const float4*>(vsP + 8 * i16);
                 const float4 vb = *reinterpret_cast<const float4*>(vsP + 8 * i16 + 4);
                 const float vsv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
@@ -841,8 +882,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __nv_bfloat162 pr = __floats2bfloat162_rn(w0, w1);
                     wd[m / 2] = *reinterpret_cast<const uint32_t*>(&pr);
                 }
-                const int chunk = 2 * (i16 & 3) + cpar;
-                *reinterpret_cast<uint4*>(prow + (i16 >> 2) * (kRows * 128) + ((chunk ^ (r & 7)) << 4)) =
+                const int kb = cb / 16 + i16;            // 16-key block of the tile
+                const int chunk = 2 * (kb & 3) + cpar;
+                *reinterpret_cast<uint4*>(prow + (kb >> 2) * (kRows * 128) + ((chunk ^ (r & 7)) << 4)) =
                     make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
             // O[g] *= alpha for the rows whose max rose (PV(i - 2), its last
@@ -932,13 +974,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 oc[r * kOcPitch + (kD / 2) * g + (MX ? 8 * (k >> 2) + (k & 3) + 4 * cpar : 2 * k + cpar)] = o_fin[k];
             if (g == 0 && cpar == 0) stat[r] = make_float2(m_fin, l_fin);
             named_sync(1, kSoftWarps * 32);
+            // query row rr: its NREP A rows rr + u kPeriod combined
+            auto row_stat = [&](int rr) -> float2 {
+                if constexpr (NREP == 1) {
+                    return stat[rr];
+                } else {
+                    float M = -INFINITY, L = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < NREP; ++u) M = fmaxf(M, stat[rr + u * kPeriod].x);
+#pragma unroll
+                    for (int u = 0; u < NREP; ++u) {
+                        const float2 su = stat[rr + u * kPeriod];
+                        if (su.x != -INFINITY) L = fmaf(ex2_approx(su.x - M), su.y, L);
+                    }
+                    return make_float2(M, L);
+                }
+            };
+            auto row_o4 = [&](int rr, int d4, float M) -> float4 {
+                if constexpr (NREP == 1) {
+                    return *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4);
+                } else {
+                    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+                    for (int u = 0; u < NREP; ++u) {
+                        const float mu = stat[rr + u * kPeriod].x;
+                        if (mu == -INFINITY) continue;
+                        const float w = ex2_approx(mu - M);
+                        const float4 o = *reinterpret_cast<const float4*>(oc + (rr + u * kPeriod) * kOcPitch + d4);
+                        acc.x = fmaf(w, o.x, acc.x);
+                        acc.y = fmaf(w, o.y, acc.y);
+                        acc.z = fmaf(w, o.z, acc.z);
+                        acc.w = fmaf(w, o.w, acc.w);
+                    }
+                    return acc;
+                }
+            };
             if (p.nsplit == 1) {
                 // thread: one row, four channels
                 for (int idx = tid; idx < p.R * (kD / 4); idx += kSoftWarps * 32) {
                     const int rr = idx / (kD / 4), d4 = 4 * (idx % (kD / 4));
-                    const float2 st = stat[rr];
-                    store_out4(p, b, hk, rr, d4, *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4),
-                               st.y > 0.0f ? 1.0f / st.y : 0.0f);
+                    const float2 st = row_stat(rr);
+                    store_out4(p, b, hk, rr, d4, row_o4(rr, d4, st.x), st.y > 0.0f ? 1.0f / st.y : 0.0f);
                 }
             } else {
                 // the partial to the workspace, combined by decode_merge_kernel
@@ -946,13 +1022,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float4* wo = reinterpret_cast<float4*>(p.ws_o + part * kRows * kD);
                 for (int idx = tid; idx < p.R * (kD / 4); idx += kSoftWarps * 32) {
                     const int rr = idx / (kD / 4), d4 = 4 * (idx % (kD / 4));
-                    wo[idx] = *reinterpret_cast<const float4*>(oc + rr * kOcPitch + d4);
+                    wo[idx] = row_o4(rr, d4, row_stat(rr).x);
                 }
-                if (tid < p.R) p.ws_stat[part * kRows + tid] = stat[tid];
+                if (tid < p.R) p.ws_stat[part * kRows + tid] = row_stat(tid);
             }
         }
     } else {
-      reg_dealloc<MX ? kRegsConvMx : kRegsConv>();
+      reg_dealloc<RegSplit<MX, NREP>::conv>();
         // ------------------------------------------------------------ V converters
         // lane -> V row kap of the tile (warp cw: rows 32 cw .. 32 cw + 31),
         // chosen so that the eight lanes of a quarter-warp read eight
@@ -1174,6 +1250,9 @@ bool encode_cache_mx(CUtensorMap* map, const void* ptr, int num_pages, int Hk, i
 template <int D, bool MX>
 constexpr int smem_bytes() { return SmL<D, MX>::kBytes + 1024; }
 
+// Repeats of the query rows in the QK A operand for R query rows.
+int pick_nrep(int R) { return R <= 16 ? 4 : (R <= 32 ? 2 : 1); }
+
 // Streaming multiprocessors of the current device (queried once per device).
 int device_sms() {
     static std::mutex mu;
@@ -1278,7 +1357,9 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
                            : encode_cache(&tv, a.v_cache, a.num_pages, a.Hk, a.page_size, D))) {
         return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const int nrep = pick_nrep(p.R);
+    auto kern = nrep == 4 ? decode_kernel<D, MX, 4> : (nrep == 2 ? decode_kernel<D, MX, 2> : decode_kernel<D, MX, 1>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     p.nsplit = pick_nsplit(a.B * a.Hk, a.T, a.window, a.page_size, a.max_pages);
     p.o_vec = (a.out_stride[3] == 1 && a.out_stride[0] % 4 == 0 && a.out_stride[1] % 4 == 0 &&
@@ -1305,7 +1386,7 @@ cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_kernel<D, MX>, tk, tv, p);
+    e = cudaLaunchKernelEx(&cfg, kern, tk, tv, p);
     if (e != cudaSuccess || p.nsplit == 1) return e;
     // a plain stream-ordered launch: it measured faster here than one
     // launched as a programmatic dependent of the split grid

@@ -112,6 +112,8 @@ def test_decode_window_family_workload(h128):
     (1, 3, 12, 3, 128, 1000, 1000, 300), # T = 3, G = 4
     (2, 4, 16, 2, 16, 5000, 6000, 8192), # page 16, long window: page ids refetched 32 at a time
     (40, 2, 8, 1, 128, 1500, 2500, 4096),# 40 clusters: more than one wave of them
+    (2, 3, 16, 1, 64, 700, 1200, 1024),  # R = 48: one softmax warp per group sits out
+    (3, 1, 16, 1, 128, 3000, 5000, 8192),# R = 16, T = 1: the query rows repeated four times
 ])
 def test_decode_shapes(h128, B, T, H, Hk, page, lo, hi, window):
     d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=128, page=page, ctx_lo=lo, ctx_hi=hi,
@@ -257,6 +259,7 @@ def test_decode_rejects_bad_kv_flags(h128):
     (2, 1, 8, 1, 128, 100, 300, 512),       # T = 1, window >= ctx, R = 8 (padded rows)
     (2, 2, 16, 2, 64, 257, 700, 256),       # page 64, R = 16
     (1, 3, 12, 3, 32, 1000, 1000, 300),     # page 32, T = 3, G = 4
+    (2, 2, 16, 1, 128, 600, 1500, 512),     # R = 32: the query rows repeated twice
 ])
 def test_decode_head64(h64, B, T, H, Hk, page, lo, hi, window):
     """Head size 64 ("[FlyDSL] [Misc] pa_decode ...", Performance: FP8 KV at

@@ -85,6 +85,8 @@ def _mx(B, T, H, Hk, page, lo, hi, seed):
     (1, 3, 12, 3, 32, 1000, 1000, 300),         # page 32, T = 3, G = 4
     (4, 4, 16, 1, 32, 4, 30, 4096),             # tiny contexts
     (160, 2, 8, 1, 16, 20, 300, 96),            # B * Hk >= the SM count: one CTA per sequence
+    (3, 3, 8, 1, 64, 300, 900, 512),            # R = 24: the query rows repeated twice
+    (2, 3, 16, 1, 128, 700, 1200, 1024),        # R = 48: one softmax warp per group sits out
 ])
 def test_decode_mx_shapes(h128, B, T, H, Hk, page, lo, hi, window):
     d = _mx(B, T, H, Hk, page, lo, hi, seed=B * 500 + page + window % 9973)
@@ -174,3 +176,31 @@ def test_decode_mx_refusals(h128):
         sage.sage_attn_decode_mxfp4(h64, q64, kc, vc, ksf, vsf, *tabs, 64, d["num_pages"], 128, 0.1, o64)
     assert e.value.status == sage.SAGE_ERR_UNSUPPORTED
     assert sage.sage_device_error() == sage.SAGE_OK
+
+
+@pytest.mark.parametrize("key", ["c7_mx", "c7", "c5_mx"])
+def test_decode_bench_workloads_sampled(h128, key):
+    """The decode workloads the bench times, at full size and in the bench's
+    launch configuration (the whole batch in one call, the binding's split
+    choice and workspace): the first and last sequences' rows against the
+    oracle (which runs on those two sequences alone)."""
+    cfg, d = workloads.make_decode_config(key)
+    mx = cfg.get("kv_format") == "mxfp4"
+    q = d["q"]
+    B, T, H, D = q.shape
+    qg = q.cuda()
+    og = torch.empty((B, T, H, D), dtype=torch.bfloat16, device="cuda")
+    run = sage.sage_attn_decode_mxfp4 if mx else sage.sage_attn_decode
+    run(h128, qg, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(), d["v_scale"].cuda(),
+        d["page_table"].cuda(), d["ctx_lens"].cuda(), d["k_cache"].shape[2], d["num_pages"], cfg["window"],
+        cfg["softmax_scale"], og)
+    torch.cuda.synchronize()
+    assert sage.sage_device_error() == sage.SAGE_OK
+    pick = [0, B - 1]
+    qb = workloads.bits_u16(q)[pick]
+    fn = oracle.decode_mxfp4 if mx else oracle.decode
+    _, ref, margin = fn(qb, d["k_cache"].numpy(), d["v_cache"].numpy(), d["k_scale"].numpy(),
+                        d["v_scale"].numpy(), d["page_table"].numpy()[pick], d["ctx_lens"].numpy()[pick],
+                        cfg["window"], cfg["softmax_scale"], want_flip=True)
+    stats = compare_output(bits(og[pick].contiguous()), (ref, margin), None, label=key + " sampled")
+    assert stats["cos_oracle"] >= 0.9999

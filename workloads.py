@@ -43,10 +43,23 @@ DECODE = {
     "c5_d64": dict(name="gqa_paged_decode_b16_t4_h16_hk1_d64_p128_w4096", B=16, T=4, H=16, Hk=1,
                    D=64, page=128, ctx_lo=4096, ctx_hi=8192, window=4096,
                    softmax_scale=1.0 / math.sqrt(64.0)),
+    # the window-family shape over an MXFP4 cache
+    "c5_mx": dict(name="gqa_paged_decode_mxfp4_b16_t4_h16_hk1_d128_p128_w4096", B=16, T=4, H=16,
+                  Hk=1, D=128, page=128, ctx_lo=4096, ctx_hi=8192, window=4096,
+                  softmax_scale=1.0 / math.sqrt(128.0), kv_format="mxfp4"),
+    # the pages' MXFP4 KV shape list (GQA 16, page 128, batch 1/32/256, ctx
+    # 2k/32k) at batch 32 and ctx 32k, every key in the window, one query
+    # token; and the same shape over the FP8 cache (per-token scales)
+    "c7_mx": dict(name="gqa_paged_decode_mxfp4_b32_t1_h16_hk1_d128_p128_c32768", B=32, T=1, H=16,
+                  Hk=1, D=128, page=128, ctx_lo=32768, ctx_hi=32768, window=32768,
+                  softmax_scale=1.0 / math.sqrt(128.0), kv_format="mxfp4"),
+    "c7": dict(name="gqa_paged_decode_b32_t1_h16_hk1_d128_p128_c32768", B=32, T=1, H=16, Hk=1,
+               D=128, page=128, ctx_lo=32768, ctx_hi=32768, window=32768,
+               softmax_scale=1.0 / math.sqrt(128.0)),
 }
 
 SEED_BASE = 20260000
-CONFIG_INDEX = {"c1": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5, "c5_d64": 6}
+CONFIG_INDEX = {"c1": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5, "c5_d64": 6, "c5_mx": 7, "c7": 8, "c7_mx": 9}
 
 
 def seed_for(key):
