@@ -596,12 +596,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             // order: QK(0), QK(1), then for j = 0, 1, ...: once P'(j) is
-            // there, QK(j + 2) and PV(j) -- QK first when K(j + 2) has
-            // already landed, so that tile j's group can start on tile j + 2
-            // while PV(j) runs. S(j + 2) overwrites S(j), which the group read
-            // before it published P'(j); the group waits for PV(j) itself
-            // before it reuses its P' buffer and O. (Issuing QK(j + 2) as soon
-            // as the group has read S(j) measured slower.)
+            // there, QK(j + 2) and PV(j). S(j + 2) overwrites S(j), which the
+            // group read before it published P'(j); the group waits for PV(j)
+            // itself before it reuses its P' buffer and O. (Measured slower:
+            // issuing QK(j + 2) as soon as the group has read S(j); polling
+            // for whichever of QK and PV can go next; the MX softmax groups
+            // converting K of their own tiles.)
             auto k_there = [&](int i) -> bool {
                 return MX ? mbar_test_wait(smem_u32(&bars[Sm::kKbReady]), i & 1)
                           : mbar_test_wait(smem_u32(&bars[Sm::kKvFull + i % kStages]), (i / kStages) & 1);
@@ -613,7 +613,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bool qk_next = false;
                 ok = mbar_wait(&bars[Sm::kPReady + (j & 1)], (j >> 1) & 1, abort_flag, &g_decode_err, 4);
                 if (!ok) break;
-                if (j + 2 < nt && k_there(j + 2)) {
+                // (FP8: PV first, measured faster -- the converters wait for it
+                // before they reuse its V buffer; MX: QK first, which frees the
+                // one bf16 K buffer the converters wait for)
+                if (MX && j + 2 < nt && k_there(j + 2)) {
                     ok = issue_qk(j + 2);
                     qk_next = true;
                 }
