@@ -13,13 +13,15 @@
 // wave, one CTA per SM); CTA = 16 warps:
 //   warps 0-7  softmax, two groups: warps 0-3 take the even tiles, warps 4-7
 //              the odd ones, each group with its own running max and sum
-//              and its own O accumulator; warp w of a group owns query rows
-//              16 (w & 3) .. + 15 (R = T * H/Hk rows, row r = t * G + g,
-//              padded to 64) over all 128 columns -- M = 64 MMAs keep those
-//              rows in TMEM lanes 32 (w & 3) .. + 15;
+//              and its own O accumulator; warp w of a group owns A rows
+//              16 (w & 3) .. + 15 of the QK operand (R = T * H/Hk query
+//              rows, row r = t * G + g, padded to 64; with R <= 32 the rows
+//              repeated NREP = 2 or 4 times, and the warp takes 128 / NREP
+//              of the key columns) -- M = 64 MMAs keep those rows in TMEM
+//              lanes 32 (w & 3) .. + 15;
 //   warps 8-11 V converters: e4m3 V tile -> exact bf16 (integer bit
 //              placement and one bf16 multiply), in the key order of the P
-//              operand;
+//              operand (an MXFP4 cache: K and V tiles -> exact bf16);
 //   warp 12    K/V producer: page-table lookups, one TMA box per page for K
 //              and for V;
 //   warp 13    TMEM owner and MMA issuer;
@@ -39,6 +41,12 @@
 // through the caller's strides; otherwise every CTA writes its (m, l, O) to
 // the workspace and decode_merge_kernel, launched after it on the stream,
 // combines the splits (log-sum-exp) and writes bf16.
+//
+// The MXFP4 cache (same page, Changes: a uint8 cache is MXFP4, E4M3 for the
+// query): E2M1 codes with one e8m0 exponent per 32 elements, converted to
+// exact bf16 in shared memory (K into one buffer that each QK frees, V as
+// above); QK is then a bf16 MMA on the query codes widened to bf16, and the
+// key and value scales are 1.
 //
 // Every mbarrier wait is bounded; on timeout the CTA records an error word,
 // raises its abort flag, drains its own copies and MMAs and still reaches
