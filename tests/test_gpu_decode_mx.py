@@ -155,6 +155,24 @@ def test_decode_mx_large_block_exponents(h128):
     compare_output(gpu, ref, None, label="mx large exponents")
 
 
+def test_decode_mx_reports_bad_page_ids(h128):
+    """A page-table entry outside [0, num_pages) for a page inside the window
+    is not dereferenced (neither its codes nor its scale blocks): its keys are
+    left out, the output stays finite and sage_device_error reports
+    SAGE_ERR_INVALID_ARG (then clears it)."""
+    d = _mx(2, 4, 16, 1, 128, 600, 900, seed=5)
+    ptab = d["page_table"].clone()
+    ptab[1, 2] = d["num_pages"] + 7
+    q = d["q"].cuda()
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    sage.sage_attn_decode_mxfp4(h128, q, d["k_cache"].cuda(), d["v_cache"].cuda(), d["k_scale"].cuda(),
+                                d["v_scale"].cuda(), ptab.cuda(), d["ctx_lens"].cuda(), 128, d["num_pages"],
+                                4096, 1.0 / math.sqrt(128), out)
+    assert sage.sage_device_error() == sage.SAGE_ERR_INVALID_ARG
+    assert sage.sage_device_error() == sage.SAGE_OK
+    assert torch.isfinite(out.float()).all()
+
+
 def test_decode_mx_refusals(h128):
     d = _mx(1, 1, 8, 1, 64, 100, 200, seed=1)
     q = d["q"].cuda()
