@@ -10,7 +10,13 @@ oracle by the GPU tests):
   right by 4 (sign kept) is a bf16 whose value times 2^120 is the code's
   value, subnormal codes included;
 * attention: the FMA-pipe exp2 that takes every 8th key pair keeps its
-  stated relative error bound."""
+  stated relative error bound;
+* decode over an MXFP4 cache: an E2M1 code's three magnitude bits placed at
+  bf16 bits 6..8 and its sign at bit 15 read as a bf16 of value x * 2^-126,
+  and one bf16 product by 2^(E - 1) (E <= 128; else by 2^126 and then by
+  2^(E - 127)) is exactly x * 2^(E - 127) for every block exponent E the
+  kernel accepts (0 .. 252); a word of eight codes becomes the four pairs
+  (element m, element m + 4), the order the bf16 query rows are given too."""
 import numpy as np
 import torch
 
@@ -35,6 +41,71 @@ def test_e4m3_code_to_bf16_by_shift_and_scale():
     # the scaled values are bf16-representable and the subnormal codes (exponent field 0)
     # land on bf16 subnormals, which the multiply keeps
     assert (np.abs(as_f32[np.abs(ref) > 0]) < 2.0 ** -126).any()
+
+
+def _e2m1_value(n):
+    """The OCP MX E2M1 value of 4-bit code n (sign, two exponent bits with
+    bias 1, one mantissa bit; exponent 0 is subnormal), from the format's
+    definition."""
+    sign = -1.0 if n & 8 else 1.0
+    e, m = (n >> 1) & 3, n & 1
+    return sign * (0.5 * m if e == 0 else 2.0 ** (e - 1) * (1.0 + 0.5 * m))
+
+
+def _bf16_bits_value(bits):
+    return float(np.array([bits << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def _exact_in_bf16(x):
+    t = torch.tensor([x], dtype=torch.float64)
+    return t.to(torch.bfloat16).to(torch.float64).item() == x
+
+
+def test_e2m1_code_to_bf16_by_bit_placement_and_block_scale():
+    for n in range(16):
+        bits = ((n & 8) << 12) | ((n & 7) << 6)
+        x = _e2m1_value(n)
+        placed = _bf16_bits_value(bits)
+        assert placed * 2.0 ** 126 == x, n
+        for E in range(0, 253):
+            if E <= 128:
+                c = 2.0 ** (E - 1)                   # one product
+                assert _exact_in_bf16(c)
+                y = placed * c
+            else:
+                c1, c2 = 2.0 ** 126, 2.0 ** (E - 127)
+                assert _exact_in_bf16(c1) and _exact_in_bf16(c2)
+                y1 = placed * c1
+                assert _exact_in_bf16(y1)
+                y = y1 * c2
+            # each product is the exact value and a bf16 value, so the bf16
+            # multiply rounds nothing (nonzero codes stay nonzero)
+            assert y == x * 2.0 ** (E - 127), (n, E)
+            assert _exact_in_bf16(y), (n, E)
+    # the largest exponent read: 6 * 2^125 is still finite in bf16
+    assert _exact_in_bf16(6.0 * 2.0 ** 125)
+
+
+def test_e2m1_word_to_bf16_pairs_and_query_order():
+    rng = np.random.default_rng(3)
+    for w in [int(v) for v in rng.integers(0, 2 ** 32, size=200, dtype=np.uint64)] + [0xFFFFFFFF, 0x89ABCDEF]:
+        nib = [(w >> (4 * i)) & 15 for i in range(8)]
+        for m in range(4):
+            a = (w << (6 - 4 * m)) if m < 2 else (w >> (4 * m - 6))
+            sgn = (w << (12 - 4 * m)) & 0xFFFFFFFF
+            bits = ((a & 0x01C001C0) | (sgn & 0x80008000)) & 0xFFFFFFFF
+            lo, hi = _bf16_bits_value(bits & 0xFFFF), _bf16_bits_value(bits >> 16)
+            assert lo * 2.0 ** 126 == _e2m1_value(nib[m]), (hex(w), m)
+            assert hi * 2.0 ** 126 == _e2m1_value(nib[m + 4]), (hex(w), m)
+    # the bf16 query rows: pair m of 8 e4m3 codes (bytes of words a, b) =
+    # (code m, code m + 4), bytes m of a and b picked into bytes 1 and 3
+    def byte_perm(x, y, sel):
+        src = [(x >> (8 * i)) & 255 for i in range(4)] + [(y >> (8 * i)) & 255 for i in range(4)]
+        return sum(src[(sel >> (4 * i)) & 7] << (8 * i) for i in range(4))
+    for a, b in [(0x03020100, 0x07060504), (0xF1E2D3C4, 0x8A9BACBD)]:
+        for m in range(4):
+            t = byte_perm(a, b, (m << 4) | ((4 + m) << 12))
+            assert (t >> 8) & 255 == (a >> (8 * m)) & 255 and (t >> 24) & 255 == (b >> (8 * m)) & 255
 
 
 def _poly_coefficients():
