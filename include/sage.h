@@ -304,7 +304,12 @@ size_t sage_attn_decode_workspace(int B, int T, int H, int Hk, int D, int window
  *   [num_pages, Hk, page_size] (one fp32 each with SAGE_KV_PER_TENSOR_SCALES);
  *   page_table: int32 [B, max_pages]
  *   logical -> physical page; ctx_lens: int32 [B], T <= ctx <= max_pages *
- *   page_size. The cache holds keys already in the rotated domain.
+ *   page_size. The cache holds keys already in the rotated domain. The
+ *   kernel reads whole 128-key tiles and gives the keys outside a window a
+ *   weight of exactly zero, multiplied by their v_scale: the per-token
+ *   v_scale of every slot of the pages a window touches, and of page 0
+ *   (it stands in for the pages of a tile that hold no window key), must be
+ *   finite; codes and k_scale there may hold any bytes.
  * For token t (position p = ctx - T + t) and head h: q_hat = butterfly(q)
  * (fp32), per-(t, h) e4m3 quantisation with scale max|q_hat| / 448; keys j in
  * [max(0, p - window + 1), p]; S_j = (q8 . k8_j) * s_q * k_scale_j *
