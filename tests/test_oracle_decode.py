@@ -230,14 +230,15 @@ def _mx_dequant(codes, sf, D):
     return val * np.repeat(np.exp2(sf.astype(np.float64) - 127.0), 32, axis=-1)
 
 
-@pytest.mark.parametrize("B,T,H,Hk,D,window", [(2, 4, 16, 2, 128, 256), (3, 1, 8, 1, 64, 1000)])
-def test_decode_mxfp4_cache_matches_brute_force(oracle_mod, B, T, H, Hk, D, window):
+@pytest.mark.parametrize("B,T,H,Hk,D,window,page", [(2, 4, 16, 2, 128, 256, 128), (3, 1, 8, 1, 64, 1000, 128),
+                                                    (2, 2, 8, 2, 128, 100, 16)])
+def test_decode_mxfp4_cache_matches_brute_force(oracle_mod, B, T, H, Hk, D, window, page):
     """The MXFP4-cache decode (packed E2M1 K/V with an e8m0 scale per 32
     channels of a token) equals a brute force over the dequantised un-paged
     cache: the format's value table and 2^(E - 127), scipy's Hadamard matrix,
     torch's float8 cast of the rotated query and torch's bfloat16 cast of the
     PV weights p_j."""
-    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=D, page=128, ctx_lo=150, ctx_hi=600, seed=60 + D,
+    d = workloads.make_decode(B=B, T=T, H=H, Hk=Hk, D=D, page=page, ctx_lo=150, ctx_hi=600, seed=60 + D + page,
                               kv_format="mxfp4")
     scale = 1.0 / math.sqrt(D)
     out, o64 = oracle_mod.decode_mxfp4(workloads.bits_u16(d["q"]), d["k_cache"].numpy(), d["v_cache"].numpy(),
@@ -251,10 +252,10 @@ def test_decode_mxfp4_cache_matches_brute_force(oracle_mod, B, T, H, Hk, D, wind
     for b in range(B):
         ctx = int(d["ctx_lens"][b])
         toks = np.arange(ctx)
-        phys = d["page_table"][b].numpy()[toks // 128]
+        phys = d["page_table"][b].numpy()[toks // page]
         for h in range(H):
             hk = h // (H // Hk)
-            K, V = kdq[phys, hk, toks % 128], vdq[phys, hk, toks % 128]
+            K, V = kdq[phys, hk, toks % page], vdq[phys, hk, toks % page]
             for t in range(T):
                 qh = q[b, t, h] @ Hmat
                 a = np.float32(np.abs(qh).max())
